@@ -1,0 +1,213 @@
+/*
+ * gear.h -- C ABI of the GEAR KV-cache codec for NVIDIA B200 (sm_100a).
+ *
+ * GEAR compresses a KV-cache matrix X (tokens x head_dim) into three parts
+ * (GEAR: Efficient KV Cache Compression for LLM Inference, Q3 "How does the
+ * paper solve the problem?"; GEAR: An Efficient KV Cache Compression Recipe
+ * for Near-Lossless Generative Inference of LLM, Abstract):
+ *   S  - a sparse set holding the largest-magnitude entries in full precision
+ *        ("S = Filter_s(X)", Cites: SqueezeLLM entry);
+ *   D  - a uniform, group-wise, per-token b-bit quantization of the rest
+ *        (Cites: FlexGen entry, "Per-token group-wise quantization");
+ *   L.Rf^T - a rank-r approximation of the quantization residual, computed by
+ *        power iteration (Q3 "low-rank approximation"; Cites: PowerSGD entry),
+ * so that X ~ D + L.Rf^T with the outlier slots overwritten by S.
+ * New tokens go to a small full-precision streaming buffer that is compressed
+ * when it fills (Q3 "Streaming strategy").
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or torch-owned)
+ *    unless stated. The library never allocates device memory: caches and
+ *    workspaces are carved from buffers the caller owns and sizes with the
+ *    *_bytes() queries.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it. Argument validation runs on the
+ *    host before any launch; on any non-OK status nothing was enqueued.
+ *  - Element types: GEAR_F16 / GEAR_BF16 / GEAR_F32 for KV, queries, buffer
+ *    and outlier values. Quantization metadata is fp32. Low-rank factors L are
+ *    fp16 for 16-bit caches and fp32 for fp32 caches; Rf is always fp32.
+ *  - Shapes are row-major, innermost dimension last, densely packed.
+ *  - One "unit" is one (batch b, kv-head h) matrix; units are indexed
+ *    u = b*H + h. Every unit of a cache holds the same number of tokens.
+ */
+#ifndef GEAR_H_
+#define GEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GEAR_OK = 0,
+  GEAR_ERR_INVALID_ARG = 1,  /* null pointer, bad shape/param, misalignment */
+  GEAR_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d != 128)   */
+  GEAR_ERR_CAPACITY = 3,     /* would exceed n_max / nblk_max of the cache   */
+  GEAR_ERR_CUDA = 4,         /* a CUDA runtime call failed                   */
+  GEAR_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up           */
+  GEAR_ERR_WORKSPACE = 6     /* workspace pointer null or too small          */
+} gear_status;
+
+typedef enum { GEAR_F16 = 0, GEAR_BF16 = 1, GEAR_F32 = 2 } gear_dtype;
+
+/* Codec parameters -- the pages' statement of the problem.
+ *  bits         b in {2, 4, 8}: code width of the quantized backbone
+ *               (Q3: "ultra-low-precision quantization (for example, 4-bit)").
+ *  group_size   g: channels per quantization group; g divides d and g*b is a
+ *               multiple of 32 (Cites: FlexGen entry, fine-grained grouping).
+ *  outlier_frac s in [0, 0.5]: fraction of each token's entries kept exactly;
+ *               k = ceil(s*d - 1e-9) outliers per token (Cites: ZeroQuant
+ *               entry, "sparsity ratio s at 2%").
+ *  rank         r in [0, 16], r <= min(n, d): rank of the residual factors of
+ *               a block written by gear_encode (ZeroQuant entry: r = 4 for
+ *               prefill inputs).
+ *  power_iters  T >= 1 when any rank > 0: power-iteration count, T counting
+ *               (P, Q) update pairs (Cites: PowerSGD entry).
+ *  buffer_len   n_b >= 1: streaming-buffer length (Q3 "Streaming strategy").
+ *  buffer_rank  r_buf in [0, 16], r_buf <= min(n_b, d): rank of each flushed
+ *               buffer block (ZeroQuant entry: "rank to 2 for each group of
+ *               n_b new tokens in decoding phase").
+ *  seed         seeds the power-iteration start matrix Q0 (d x r): entry
+ *               (i, j) is the (i*r + j)-th output of the splitmix64 stream
+ *               whose state starts at `seed` (Steele, Lea & Flood, OOPSLA
+ *               2014), top 24 bits mapped to [-1, 1) as u*2^-23 - 1. */
+typedef struct gear_params {
+  int32_t bits;
+  int32_t group_size;
+  float outlier_frac;
+  int32_t rank;
+  int32_t power_iters;
+  int32_t buffer_len;
+  int32_t buffer_rank;
+  int32_t reserved0;
+  uint64_t seed;
+} gear_params;
+
+/* Compressed cache for ONE tensor (K or V) of one layer: B x H units, each with
+ * up to n_max compressed tokens plus an n_b-token full-precision buffer.
+ *
+ * Filled by gear_cache_init(); the caller then treats it as opaque except for
+ * reading the counters. The struct lives in HOST memory; the arrays it points
+ * to live in the caller's device buffer, laid out in this order, each array
+ * starting on a 256-byte boundary:
+ *
+ *   codes  uint32 [U][n_max][W]      W = d*b/32. Channel c of a token is bits
+ *                                    [(c*b)%32, (c*b)%32 + b) of word c*b/32.
+ *   meta   float  [U][n_max][G][2]   G = d/g; (scale, zero) of each group,
+ *                                    zero = group minimum over non-outliers.
+ *   oidx   uint8  [U][n_max][k]      outlier channels, ascending.
+ *   oval   dtype  [U][n_max][k]      outlier values, bit-exact input copies.
+ *   lfac   f16|f32[U][n_max][r_max]  L rows, stored as L * 2^e_blk.
+ *   rfac   float  [U][nblk_max][r_max][d]  Rf columns, stored as Rf * 2^-e_blk.
+ *   buf    dtype  [U][n_b][d]        streaming buffer (full precision).
+ *
+ * with U = B*H, k = outliers per token, r_max = max(rank, buffer_rank) and
+ * e_blk = floor(log2(block_len) / 2) (the factor keeps fp16 L rows near unit
+ * magnitude; L * Rf^T is unchanged). Blocks: block 0 holds tokens
+ * [0, blk0_len) with rank blk0_rank; block i >= 1 holds the n_b tokens
+ * [blk0_len + (i-1)*n_b, blk0_len + i*n_b) with rank buffer_rank. */
+typedef struct gear_cache {
+  /* geometry and parameters (written by gear_cache_init) */
+  int32_t B, H, d, n_max, nblk_max;
+  int32_t dtype;      /* gear_dtype */
+  gear_params p;
+  int32_t k, G, W, r_max;
+  /* device arrays carved from the caller's buffer (not owned) */
+  uint32_t* codes;
+  float* meta;
+  uint8_t* oidx;
+  void* oval;
+  void* lfac;
+  float* rfac;
+  void* buf;
+  /* host-side counters, advanced by gear_encode / gear_append_buffer */
+  int32_t n_comp;     /* compressed tokens per unit                  */
+  int32_t n_buf;      /* tokens currently in the streaming buffer    */
+  int32_t n_blk;      /* compressed blocks                           */
+  int32_t blk0_len;   /* tokens in block 0 (0 while n_blk == 0)      */
+  int32_t blk0_rank;  /* rank of block 0                             */
+  int32_t reserved1;
+} gear_cache;
+
+/* Number of outliers kept per token: k = ceil(s*d - 1e-9), computed in double
+ * (so s = 2% at d = 128 keeps 3 entries, s = 5% keeps 7). */
+int32_t gear_num_outliers(float outlier_frac, int32_t d);
+
+/* Checks a parameter set (the limits listed at gear_params). */
+gear_status gear_validate_params(const gear_params* p, int32_t d);
+
+/* Bytes of device memory a cache with this geometry needs (0 on bad args). */
+size_t gear_cache_bytes(const gear_params* p, int32_t B, int32_t H, int32_t d,
+                        int32_t n_max, int32_t nblk_max, gear_dtype dtype);
+
+/* Lays a cache out in [dev, dev + bytes). `dev` must be 256-byte aligned and
+ * bytes >= gear_cache_bytes(...). Sets counters to zero. Writes no device
+ * memory. Errors: INVALID_ARG (null, misaligned, bad params), UNSUPPORTED
+ * (d != 128), CAPACITY (bytes too small). */
+gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int32_t H,
+                            int32_t d, int32_t n_max, int32_t nblk_max, gear_dtype dtype,
+                            void* dev, size_t bytes);
+
+/* Workspace bytes gear_encode needs to encode n tokens per unit of c. */
+size_t gear_encode_workspace_bytes(const gear_cache* c, int32_t n);
+
+/* Encodes kv [B][H][n][d] (cache dtype, 16-byte aligned) as block 0 of an empty
+ * cache, with rank p.rank: outliers, per-token group-wise quantization and the
+ * rank-r power-iteration factors of the residual (Q3; Cites: SqueezeLLM,
+ * FlexGen and PowerSGD entries). Requires c->n_comp == 0 and n_buf == 0,
+ * 1 <= n <= n_max, rank <= n. On success sets n_comp = n, n_blk = 1.
+ * Errors: INVALID_ARG, CAPACITY, WORKSPACE, CUDA. */
+gear_status gear_encode(gear_cache* c, const void* kv, int32_t n,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes gear_decode_attn needs for these caches and Hq query heads. */
+size_t gear_decode_workspace_bytes(const gear_cache* k, const gear_cache* v, int32_t Hq);
+
+/* One decode step of attention over the compressed caches plus buffers:
+ *   out[b][j] = sum_t softmax_t(scale * q[b][j] . Khat[b][h][t]) Vhat[b][h][t]
+ * over the n_comp compressed tokens (Khat/Vhat = dequantized codes + L.Rf^T,
+ * outlier slots replaced by their exact values) followed by the n_buf buffer
+ * tokens, with h = j / (Hq / H) (grouped-query sharing).
+ *   q    [B][Hq][d], cache dtype.       out  [B][Hq][d], out_dtype
+ *   out_dtype is the cache dtype or GEAR_F32.
+ * k and v must have identical geometry and counters; Hq % H == 0.
+ * Errors: INVALID_ARG, WORKSPACE, CUDA. */
+gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const void* q,
+                             int32_t Hq, float softmax_scale, void* out, gear_dtype out_dtype,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes gear_append_buffer needs (covers the flush encode). */
+size_t gear_append_workspace_bytes(const gear_cache* k);
+
+/* Appends one token per unit, k_new/v_new [B][H][d] (cache dtype). If the
+ * buffer already holds n_b tokens, they are first compressed as a new block
+ * of rank buffer_rank (same codec as gear_encode) appended after the
+ * compressed tokens, and the buffer is emptied (Q3 "Streaming strategy":
+ * compression is triggered when the buffer fills). Then the new token is
+ * written to buffer slot n_buf. Errors: INVALID_ARG, CAPACITY, WORKSPACE, CUDA. */
+gear_status gear_append_buffer(gear_cache* k, gear_cache* v, const void* k_new,
+                               const void* v_new, void* workspace, size_t ws_bytes,
+                               void* stream);
+
+/* Debug/test export: writes the reconstruction of every token of c,
+ * out_f32 [B][H][n_comp + n_buf][d] fp32 (compressed tokens first, then the
+ * buffer). Errors: INVALID_ARG, CUDA. */
+gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream);
+
+/* Reads (host, synchronous) and clears the device-side error word that
+ * kernels set instead of trapping (GEAR_ERR_* value, 0 if none). */
+gear_status gear_get_device_status(int32_t* status);
+
+/* Static description of a status code. */
+const char* gear_status_string(gear_status s);
+
+/* Library version as "major.minor.patch". */
+const char* gear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GEAR_H_ */
