@@ -1,0 +1,341 @@
+// api.cu -- the C ABI of libgear (declared in include/gear.h).
+//
+// Host-side validation, cache layout, workspace sizing and launch sequencing.
+// Every entry point validates on the host first and enqueues nothing on error.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "encode.cuh"
+
+namespace gear {
+__device__ int32_t g_device_status = 0;
+
+static int current_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+static int esize(int dt) { return dt == GEAR_F32 ? 4 : 2; }
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Layout {
+  size_t codes, meta, oidx, oval, lfac, rfac, buf, total;
+};
+
+static Layout cache_layout(const gear_params* p, int B, int H, int d, int n_max, int nblk_max, int dt) {
+  Layout L;
+  const size_t U = (size_t)B * H;
+  const int k = gear_num_outliers(p->outlier_frac, d);
+  const int G = d / p->group_size;
+  const int W = d * p->bits / 32;
+  const int rmax = p->rank > p->buffer_rank ? p->rank : p->buffer_rank;
+  const int rm = rmax > 0 ? rmax : 1;
+  size_t off = 0;
+  L.codes = off; off = align256(off + U * n_max * W * 4);
+  L.meta = off;  off = align256(off + U * n_max * G * 8);
+  L.oidx = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1));
+  L.oval = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1) * esize(dt));
+  L.lfac = off;  off = align256(off + U * n_max * rm * (dt == GEAR_F32 ? 4 : 2));
+  L.rfac = off;  off = align256(off + U * nblk_max * rm * (size_t)d * 4);
+  L.buf = off;   off = align256(off + U * (size_t)p->buffer_len * d * esize(dt));
+  L.total = off;
+  return L;
+}
+
+static int e_of_len(int len) {
+  // floor(log2(len) / 2)
+  int lg = 0;
+  while ((2 << lg) <= len) ++lg;
+  return lg / 2;
+}
+
+static gear_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GEAR_OK : GEAR_ERR_CUDA; }
+
+static bool cache_ok(const gear_cache* c) {
+  return c && c->codes && c->meta && c->rfac && c->buf && c->d == 128 && c->B > 0 && c->H > 0;
+}
+
+// encode n tokens per unit of `kv` into c as block `blk` at token offset t_off
+static gear_status encode_block(gear_cache* c, const void* kv, int n, int t_off, int blk, int rank, void* ws,
+                                size_t ws_bytes, cudaStream_t st) {
+  EncodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kv = kv;
+  a.U = c->B * c->H;
+  a.n = n;
+  a.dtype = c->dtype;
+  a.bits = c->p.bits;
+  a.g = c->p.group_size;
+  a.k = c->k;
+  a.r = rank;
+  a.T = c->p.power_iters;
+  a.seed = c->p.seed;
+  a.t_off = t_off;
+  a.blk = blk;
+  a.e_blk = e_of_len(n);
+  a.n_max = c->n_max;
+  a.nblk_max = c->nblk_max;
+  a.W = c->W;
+  a.G = c->G;
+  a.r_max = c->r_max;
+  a.codes = c->codes;
+  a.meta = c->meta;
+  a.oidx = c->oidx;
+  a.oval = c->oval;
+  a.lfac = c->lfac;
+  a.rfac = c->rfac;
+  a.tpu = (n + 127) / 128;
+  a.total_tiles = (int64_t)a.U * a.tpu;
+  const int sms = current_sm_count();
+  a.grid_e1 = encode_grid(a, sms);
+  a.maxc = encode_maxc(a.total_tiles, a.grid_e1, a.tpu);
+  const size_t gbytes = align256((size_t)a.U * a.maxc * 128 * 128 * 4);
+  const size_t zbytes = align256((size_t)a.U * 128 * 16 * 4);
+  if (!ws || ws_bytes < gbytes + zbytes || !aligned(ws, 256)) return GEAR_ERR_WORKSPACE;
+  a.gram = reinterpret_cast<float*>(ws);
+  a.zbuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gbytes);
+  return cuda_status(encode_launch(a, sms, st));
+}
+
+static size_t encode_ws_bytes(const gear_cache* c, int n) {
+  if (!c || n <= 0) return 0;
+  EncodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.U = c->B * c->H;
+  a.tpu = (n + 127) / 128;
+  a.total_tiles = (int64_t)a.U * a.tpu;
+  const int grid = encode_grid(a, current_sm_count());
+  const int maxc = encode_maxc(a.total_tiles, grid, a.tpu);
+  return align256((size_t)a.U * maxc * 128 * 128 * 4) + align256((size_t)a.U * 128 * 16 * 4);
+}
+
+// ------------------------------------------------------------------ append
+template <typename T>
+__global__ void append_rows(T* __restrict__ kbuf, T* __restrict__ vbuf, const T* __restrict__ kn,
+                            const T* __restrict__ vn, int U, int n_b, int slot) {
+  const int u = blockIdx.x, c = threadIdx.x;
+  if (u >= U) return;
+  kbuf[((size_t)u * n_b + slot) * 128 + c] = kn[(size_t)u * 128 + c];
+  vbuf[((size_t)u * n_b + slot) * 128 + c] = vn[(size_t)u * 128 + c];
+}
+
+}  // namespace gear
+
+using namespace gear;
+
+extern "C" {
+
+int32_t gear_num_outliers(float outlier_frac, int32_t d) {
+  double v = (double)outlier_frac * (double)d - 1e-9;
+  if (!(v > 0.0)) return 0;
+  int32_t k = (int32_t)ceil(v);
+  return k > d ? d : k;
+}
+
+gear_status gear_validate_params(const gear_params* p, int32_t d) {
+  if (!p) return GEAR_ERR_INVALID_ARG;
+  if (p->bits != 2 && p->bits != 4 && p->bits != 8) return GEAR_ERR_INVALID_ARG;
+  if (p->group_size <= 0 || d <= 0 || d % p->group_size != 0 || (p->group_size * p->bits) % 32 != 0)
+    return GEAR_ERR_INVALID_ARG;
+  if (!(p->outlier_frac >= 0.0f && p->outlier_frac <= 0.5f)) return GEAR_ERR_INVALID_ARG;
+  if (p->rank < 0 || p->rank > 16 || p->rank > d) return GEAR_ERR_INVALID_ARG;
+  if (p->buffer_len < 1) return GEAR_ERR_INVALID_ARG;
+  if (p->buffer_rank < 0 || p->buffer_rank > 16 || p->buffer_rank > d || p->buffer_rank > p->buffer_len)
+    return GEAR_ERR_INVALID_ARG;
+  if ((p->rank > 0 || p->buffer_rank > 0) && p->power_iters < 1) return GEAR_ERR_INVALID_ARG;
+  if (p->power_iters < 0) return GEAR_ERR_INVALID_ARG;
+  if (d != 128) return GEAR_ERR_UNSUPPORTED;
+  if (p->group_size < 32) return GEAR_ERR_UNSUPPORTED;
+  if (gear_num_outliers(p->outlier_frac, d) > 16) return GEAR_ERR_UNSUPPORTED;
+  return GEAR_OK;
+}
+
+size_t gear_cache_bytes(const gear_params* p, int32_t B, int32_t H, int32_t d, int32_t n_max, int32_t nblk_max,
+                        gear_dtype dtype) {
+  if (gear_validate_params(p, d) != GEAR_OK) return 0;
+  if (B <= 0 || H <= 0 || n_max <= 0 || nblk_max <= 0 || dtype < GEAR_F16 || dtype > GEAR_F32) return 0;
+  return cache_layout(p, B, H, d, n_max, nblk_max, dtype).total;
+}
+
+gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int32_t H, int32_t d, int32_t n_max,
+                            int32_t nblk_max, gear_dtype dtype, void* dev, size_t bytes) {
+  if (!c || !p || !dev) return GEAR_ERR_INVALID_ARG;
+  gear_status s = gear_validate_params(p, d);
+  if (s != GEAR_OK) return s;
+  if (B <= 0 || H <= 0 || n_max <= 0 || nblk_max <= 0 || dtype < GEAR_F16 || dtype > GEAR_F32)
+    return GEAR_ERR_INVALID_ARG;
+  if (!aligned(dev, 256)) return GEAR_ERR_INVALID_ARG;
+  if ((size_t)B * H * n_max >= ((size_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
+  Layout L = cache_layout(p, B, H, d, n_max, nblk_max, dtype);
+  if (bytes < L.total) return GEAR_ERR_CAPACITY;
+  memset(c, 0, sizeof(*c));
+  c->B = B; c->H = H; c->d = d; c->n_max = n_max; c->nblk_max = nblk_max; c->dtype = dtype;
+  c->p = *p;
+  c->k = gear_num_outliers(p->outlier_frac, d);
+  c->G = d / p->group_size;
+  c->W = d * p->bits / 32;
+  int rmax = p->rank > p->buffer_rank ? p->rank : p->buffer_rank;
+  c->r_max = rmax > 0 ? rmax : 1;
+  uint8_t* base = reinterpret_cast<uint8_t*>(dev);
+  c->codes = reinterpret_cast<uint32_t*>(base + L.codes);
+  c->meta = reinterpret_cast<float*>(base + L.meta);
+  c->oidx = base + L.oidx;
+  c->oval = base + L.oval;
+  c->lfac = base + L.lfac;
+  c->rfac = reinterpret_cast<float*>(base + L.rfac);
+  c->buf = base + L.buf;
+  return GEAR_OK;
+}
+
+size_t gear_encode_workspace_bytes(const gear_cache* c, int32_t n) { return encode_ws_bytes(c, n); }
+
+gear_status gear_encode(gear_cache* c, const void* kv, int32_t n, void* workspace, size_t ws_bytes, void* stream) {
+  if (!cache_ok(c) || !kv) return GEAR_ERR_INVALID_ARG;
+  if (!aligned(kv, 16)) return GEAR_ERR_INVALID_ARG;
+  if (n < 1) return GEAR_ERR_INVALID_ARG;
+  if (c->n_comp != 0 || c->n_buf != 0 || c->n_blk != 0) return GEAR_ERR_INVALID_ARG;
+  if (c->p.rank > n) return GEAR_ERR_INVALID_ARG;
+  if (n > c->n_max || c->nblk_max < 1) return GEAR_ERR_CAPACITY;
+  if ((int64_t)c->B * c->H * n >= ((int64_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
+  gear_status s = encode_block(c, kv, n, 0, 0, c->p.rank, workspace, ws_bytes, (cudaStream_t)stream);
+  if (s != GEAR_OK) return s;
+  c->n_comp = n;
+  c->n_blk = 1;
+  c->blk0_len = n;
+  c->blk0_rank = c->p.rank;
+  return GEAR_OK;
+}
+
+static gear_status decode_args(const gear_cache* k, const gear_cache* v, int32_t Hq, DecodeArgs& a) {
+  if (!cache_ok(k) || !cache_ok(v)) return GEAR_ERR_INVALID_ARG;
+  if (k->B != v->B || k->H != v->H || k->dtype != v->dtype || k->n_comp != v->n_comp || k->n_buf != v->n_buf ||
+      k->n_blk != v->n_blk || k->blk0_len != v->blk0_len || k->n_max != v->n_max || k->nblk_max != v->nblk_max ||
+      memcmp(&k->p, &v->p, sizeof(gear_params)) != 0)
+    return GEAR_ERR_INVALID_ARG;
+  if (Hq <= 0 || Hq % k->H != 0 || Hq / k->H > 8) return GEAR_ERR_INVALID_ARG;
+  if (k->n_comp + k->n_buf == 0) return GEAR_ERR_INVALID_ARG;
+  memset(&a, 0, sizeof(a));
+  a.K = CacheView{k->codes, k->meta, k->oidx, k->oval, k->lfac, k->rfac, k->buf};
+  a.V = CacheView{v->codes, v->meta, v->oidx, v->oval, v->lfac, v->rfac, v->buf};
+  a.dtype = k->dtype;
+  a.B = k->B; a.H = k->H; a.Hq = Hq; a.hq = Hq / k->H;
+  a.bits = k->p.bits; a.g = k->p.group_size; a.G = k->G; a.W = k->W; a.k = k->k; a.r_max = k->r_max;
+  a.n_max = k->n_max; a.nblk_max = k->nblk_max; a.n_b = k->p.buffer_len;
+  a.n_comp = k->n_comp; a.n_buf = k->n_buf;
+  a.blk0_len = k->blk0_len; a.blk0_rank = k->blk0_rank; a.buffer_rank = k->p.buffer_rank;
+  decode_plan(a, current_sm_count());
+  return GEAR_OK;
+}
+
+size_t gear_decode_workspace_bytes(const gear_cache* k, const gear_cache* v, int32_t Hq) {
+  DecodeArgs a;
+  if (decode_args(k, v, Hq, a) != GEAR_OK) return 0;
+  return decode_workspace_bytes(a.B, a.Hq, a.nsplit);
+}
+
+gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq, float softmax_scale,
+                             void* out, gear_dtype out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  DecodeArgs a;
+  gear_status s = decode_args(k, v, Hq, a);
+  if (s != GEAR_OK) return s;
+  if (!q || !out) return GEAR_ERR_INVALID_ARG;
+  if (out_dtype != k->dtype && out_dtype != GEAR_F32) return GEAR_ERR_INVALID_ARG;
+  if (!isfinite(softmax_scale)) return GEAR_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < decode_workspace_bytes(a.B, a.Hq, a.nsplit) || !aligned(workspace, 16))
+    return GEAR_ERR_WORKSPACE;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.q = q;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  a.part = reinterpret_cast<float*>(workspace);
+  return cuda_status(decode_launch(a, (cudaStream_t)stream));
+}
+
+size_t gear_append_workspace_bytes(const gear_cache* k) {
+  if (!cache_ok(k)) return 0;
+  return encode_ws_bytes(k, k->p.buffer_len);
+}
+
+gear_status gear_append_buffer(gear_cache* k, gear_cache* v, const void* k_new, const void* v_new, void* workspace,
+                               size_t ws_bytes, void* stream) {
+  if (!cache_ok(k) || !cache_ok(v) || !k_new || !v_new) return GEAR_ERR_INVALID_ARG;
+  if (k->B != v->B || k->H != v->H || k->dtype != v->dtype || k->n_comp != v->n_comp || k->n_buf != v->n_buf ||
+      k->n_blk != v->n_blk || memcmp(&k->p, &v->p, sizeof(gear_params)) != 0)
+    return GEAR_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int n_b = k->p.buffer_len;
+  const bool flush = k->n_buf == n_b;
+  if (flush) {
+    if (k->n_comp + n_b > k->n_max || k->n_blk + 1 > k->nblk_max) return GEAR_ERR_CAPACITY;
+    if (ws_bytes < encode_ws_bytes(k, n_b)) return GEAR_ERR_WORKSPACE;
+    gear_cache* cs[2] = {k, v};
+    for (gear_cache* c : cs) {
+      gear_status s = encode_block(c, c->buf, n_b, c->n_comp, c->n_blk, c->p.buffer_rank, workspace, ws_bytes, st);
+      if (s != GEAR_OK) return s;
+    }
+    for (gear_cache* c : cs) {
+      if (c->n_blk == 0) { c->blk0_len = n_b; c->blk0_rank = c->p.buffer_rank; }
+      c->n_comp += n_b;
+      c->n_blk += 1;
+      c->n_buf = 0;
+    }
+  }
+  const int U = k->B * k->H;
+  if (k->dtype == GEAR_F32)
+    append_rows<float><<<U, 128, 0, st>>>((float*)k->buf, (float*)v->buf, (const float*)k_new, (const float*)v_new, U,
+                                          n_b, k->n_buf);
+  else
+    append_rows<uint16_t><<<U, 128, 0, st>>>((uint16_t*)k->buf, (uint16_t*)v->buf, (const uint16_t*)k_new,
+                                             (const uint16_t*)v_new, U, n_b, k->n_buf);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return GEAR_ERR_CUDA;
+  k->n_buf += 1;
+  v->n_buf += 1;
+  return GEAR_OK;
+}
+
+gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream) {
+  if (!cache_ok(c) || !out_f32) return GEAR_ERR_INVALID_ARG;
+  DenseArgs a;
+  memset(&a, 0, sizeof(a));
+  a.C = CacheView{c->codes, c->meta, c->oidx, c->oval, c->lfac, c->rfac, c->buf};
+  a.dtype = c->dtype;
+  a.U = c->B * c->H;
+  a.bits = c->p.bits; a.g = c->p.group_size; a.G = c->G; a.W = c->W; a.k = c->k; a.r_max = c->r_max;
+  a.n_max = c->n_max; a.nblk_max = c->nblk_max; a.n_b = c->p.buffer_len;
+  a.n_comp = c->n_comp; a.n_buf = c->n_buf;
+  a.blk0_len = c->blk0_len; a.blk0_rank = c->blk0_rank; a.buffer_rank = c->p.buffer_rank;
+  a.out = out_f32;
+  return cuda_status(dense_launch(a, (cudaStream_t)stream));
+}
+
+gear_status gear_get_device_status(int32_t* status) {
+  if (!status) return GEAR_ERR_INVALID_ARG;
+  int32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return GEAR_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return GEAR_ERR_CUDA;
+  *status = v;
+  return GEAR_OK;
+}
+
+const char* gear_status_string(gear_status s) {
+  switch (s) {
+    case GEAR_OK: return "ok";
+    case GEAR_ERR_INVALID_ARG: return "invalid argument";
+    case GEAR_ERR_UNSUPPORTED: return "unsupported configuration";
+    case GEAR_ERR_CAPACITY: return "cache capacity exceeded";
+    case GEAR_ERR_CUDA: return "CUDA runtime error";
+    case GEAR_ERR_TIMEOUT: return "device-side wait timed out";
+    case GEAR_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* gear_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,887 @@
+// encode.cu -- GEAR encoder on B200: outliers, group-wise quantization and the
+// power-iteration factors of the quantization residual.
+//
+// Method (GEAR: Efficient KV Cache Compression for LLM Inference, Q3; GEAR: An
+// Efficient KV Cache Compression Recipe ..., Cites: SqueezeLLM, FlexGen and
+// PowerSGD entries): per token keep the k largest-|x| entries exactly, quantize
+// the rest group-wise to b bits (min-max, zero = group minimum), and approximate
+// the residual R = X - Dhat of each (batch, head) block with rank-r factors
+// from T steps of power iteration started at a seeded matrix Q0.
+//
+// B200 design. Power iteration only ever touches R through R Q and R^T P, so
+// with the d x d Gram matrix M = R^T R (d = 128):
+//     P~_t = R Q_{t-1},  P~_t^T P~_t = Q_{t-1}^T M Q_{t-1},  R^T P~_t = M Q_{t-1}.
+// Orthonormalizing P~_t by Cholesky-QR of that r x r Gram therefore needs only
+// M, and the whole iteration runs on a 128 x 128 matrix. That turns the
+// token-long reductions into ONE dense contraction per tile (R_tile^T R_tile,
+// tensor cores) and leaves a single extra look at each token at the end
+// (L = R Z). Three kernels:
+//   E1 encode_quant_gram  persistent, warp-specialized: TMA loads 128-token
+//       tiles, 8 quantizer warps compute outliers / codes / metadata (written
+//       straight to the cache) and the residual split as bf16 hi + lo, one
+//       thread issues tcgen05.mma accumulating hi^T [hi | lo] (M=128, N=256) in
+//       tensor memory; per (CTA, unit) segment the partial Gram is written out.
+//   E2 encode_power      one CTA per unit: sums the partials in fp64, runs T
+//       power steps with Cholesky-QR, writes Rf and Z = Q_{T-1} C_T^-1.
+//   E3 encode_lowrank    L = R Z for every token, R rebuilt from the codes.
+#include <cuda.h>
+
+#include <cfloat>
+
+#include "common.cuh"
+#include "encode.cuh"
+
+namespace gear {
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  return (uint64_t)__float_as_uint(a) | ((uint64_t)__float_as_uint(b) << 32);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// round-to-nearest-even of q in [0, 2^22) by the 1.5 * 2^23 addend: the sum's
+// unit in the last place is 1, so the addition itself rounds q to an integer
+// (ties to even) and the low mantissa bits of the sum hold it.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+// Element loads/stores of the KV dtype as 16-bit patterns.
+template <typename T>
+struct Elem16;
+template <>
+struct Elem16<__half> {
+  static constexpr uint16_t kNaN = 0x7E00;
+  __device__ static __half2 hmin(__half2 a, __half2 b) { return __hmin2(a, b); }
+  __device__ static __half2 hmax(__half2 a, __half2 b) { return __hmax2(a, b); }
+  __device__ static float2 to_f2(uint32_t v) { return __half22float2(*reinterpret_cast<__half2*>(&v)); }
+  __device__ static float lo(uint32_t v) { return __half2float(__ushort_as_half((uint16_t)v)); }
+  __device__ static uint32_t from_f(float f) { return __half_as_ushort(__float2half_rn(f)); }
+};
+template <>
+struct Elem16<__nv_bfloat16> {
+  static constexpr uint16_t kNaN = 0x7FC0;
+  __device__ static __nv_bfloat162 hmin(__nv_bfloat162 a, __nv_bfloat162 b) { return __hmin2(a, b); }
+  __device__ static __nv_bfloat162 hmax(__nv_bfloat162 a, __nv_bfloat162 b) { return __hmax2(a, b); }
+  __device__ static float2 to_f2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+  }
+  __device__ static float lo(uint32_t v) { return __uint_as_float(v << 16); }
+  __device__ static uint32_t from_f(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+};
+
+template <typename T>
+__device__ __forceinline__ uint32_t pair_min(uint32_t a, uint32_t b) {
+  using V2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
+  V2 r = Elem16<T>::hmin(*reinterpret_cast<V2*>(&a), *reinterpret_cast<V2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+template <typename T>
+__device__ __forceinline__ uint32_t pair_max(uint32_t a, uint32_t b) {
+  using V2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
+  V2 r = Elem16<T>::hmax(*reinterpret_cast<V2*>(&a), *reinterpret_cast<V2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Correctly rounded a / s for the code decision. When 2^-100 <= s <= 2^100
+// (so s and y = RN(1/s) are normal), the quotient is refined from the
+// correctly rounded reciprocal with one exact remainder (Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990: q1 = RN(q0 + r y), r = a - s q0, equals RN(a/s) whenever
+// q0 is within one ulp and a/s is normal). Only rint(q) is used and only
+// q >= 1/4 can round to a non-zero code, where all operands are normal.
+// Otherwise the correctly rounded division intrinsic is used.
+__device__ __forceinline__ uint64_t div_pair(uint64_t a, float s, float y, bool fast) {
+  if (fast) {
+    uint64_t y2 = f2_pack(y, y);
+    uint64_t s2n = f2_pack(-s, -s);
+    uint64_t q0 = f2_mul(a, y2);
+    uint64_t r = f2_fma(q0, s2n, a);
+    return f2_fma(r, y2, q0);
+  }
+  return f2_pack(__fdiv_rn(f2_lo(a), s), __fdiv_rn(f2_hi(a), s));
+}
+
+// ================================================================ E1 ======
+// Shared-memory map of E1 (dynamic, 1024-byte aligned):
+//   X stages  kNX x kXBytes   TMA tiles, [box][128 rows][128 B] swizzle-128B
+//   R stages  kNR x 64 KiB    residual hi (32 KiB) then lo (32 KiB), each two
+//                             64-channel blocks of [128 tokens][128 B], swz-128B
+//   barriers, tensor-memory slot, abort flag
+constexpr int kTile = 128;       // tokens per tile
+constexpr int kQThreads = 256;   // quantizer threads (2 per token)
+constexpr int kE1Threads = 64 + kQThreads;
+constexpr int kNR = 2;
+constexpr uint32_t kRBytes = 65536;
+
+template <typename T>
+struct E1Cfg {
+  static constexpr int kNX = sizeof(T) == 4 ? 1 : 2;
+  static constexpr uint32_t kXBytes = kTile * 128 * sizeof(T);
+  static constexpr int kBoxCols = 128 / sizeof(T);            // 128-byte rows
+  static constexpr int kBoxes = 128 / kBoxCols;
+  static constexpr uint32_t kBarOff = kNX * kXBytes + kNR * kRBytes;
+  static constexpr uint32_t kSmem = kBarOff + 256 + 1024;     // + alignment slack
+};
+
+struct E1Bars {
+  uint64_t x_full[2], x_empty[2], r_full[kNR], r_empty[kNR], acc_full, acc_empty;
+  uint32_t tmem_slot;
+  int32_t abort_flag;
+};
+
+// byte offset of 16-byte chunk j of row t inside a swizzle-128B box
+__device__ __forceinline__ uint32_t swz(int t, int j) { return (uint32_t)(t * 128 + ((j ^ (t & 7)) << 4)); }
+
+__device__ __forceinline__ int64_t seg_first_cta(int64_t tile, int64_t grid, int64_t total) {
+  return ((tile + 1) * grid - 1) / total;
+}
+
+// One quantizer thread: half h (channels 64h .. 64h+63) of token t of the tile.
+// Writes codes/meta/outliers of the token to the cache and the residual split
+// into the R stage. `valid` is false for tile rows past the unit's last token.
+template <typename T, int BITS, int KMAX>
+__device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, uint8_t* rs, int t, int h,
+                                              bool valid, int u, int tok) {
+  constexpr int kCodesPerWord = 32 / BITS;
+  constexpr int kWordsHalf = 64 * BITS / 32;
+  const float levels = (float)((1 << BITS) - 1);
+  const int k = a.k;
+
+  // ---------------- load the half row --------------------------------------
+  // 16-bit: 8 chunks of 8 channels (4 packed pairs each); fp32: 16 chunks of 4.
+  constexpr int kChunks = sizeof(T) == 4 ? 16 : 8;
+  uint32_t xr[32 * (sizeof(T) / 2)];  // 32 pairs (16-bit) or 64 floats (fp32)
+  auto chunk_addr = [&](int j) -> uint8_t* {
+    if constexpr (sizeof(T) == 4) {
+      int box = 2 * h + (j >> 3);
+      return xs + box * 16384 + swz(t, j & 7);
+    } else {
+      return xs + h * 16384 + swz(t, j);
+    }
+  };
+#pragma unroll
+  for (int j = 0; j < kChunks; ++j) {
+    uint4 v = *reinterpret_cast<const uint4*>(chunk_addr(j));
+    xr[4 * j + 0] = v.x; xr[4 * j + 1] = v.y; xr[4 * j + 2] = v.z; xr[4 * j + 3] = v.w;
+  }
+
+  // ---------------- outliers: top-k keys (|x|, then lower channel) ---------
+  // key = |x| bits << 7 | (127 - c): larger key = larger |x|, ties to the lower
+  // channel. Each thread keeps the top KMAX of its 64 keys with a branch-free
+  // insertion network, then merges its partner's list (lane ^ 1).
+  uint64_t top[KMAX > 0 ? KMAX : 1];
+  int cidx[KMAX > 0 ? KMAX : 1];
+  uint32_t oval_bits[KMAX > 0 ? KMAX : 1];
+  if constexpr (KMAX > 0) {
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) top[i] = 0;
+    const uint32_t tb0 = 127u - 64u * h;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+      uint64_t key;
+      if constexpr (sizeof(T) == 4) {
+        key = ((uint64_t)(xr[e] & 0x7FFFFFFFu) << 7) | (tb0 - e);
+      } else {
+        uint32_t p = xr[e >> 1];
+        uint32_t ab = (e & 1) ? ((p >> 16) & 0x7FFFu) : (p & 0x7FFFu);
+        key = (uint64_t)((ab << 7) | (tb0 - e));
+      }
+      if (!valid) key = 0;
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i) {
+        uint64_t hi = key > top[i] ? key : top[i];
+        key = key > top[i] ? top[i] : key;
+        top[i] = hi;
+      }
+    }
+    // snapshot the partner's list before either lane modifies its own
+    uint64_t other[KMAX];
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) other[i] = __shfl_xor_sync(0xFFFFFFFFu, top[i], 1);
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) {
+      uint64_t key = other[i];
+#pragma unroll
+      for (int m = 0; m < KMAX; ++m) {
+        uint64_t hi = key > top[m] ? key : top[m];
+        key = key > top[m] ? top[m] : key;
+        top[m] = hi;
+      }
+    }
+    // read the k outlier values (both threads read all k), then patch own half
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) {
+      int c = 127 - (int)(top[i] & 127u);
+      cidx[i] = c;
+      oval_bits[i] = 0;
+      if (i < k && valid) {
+        int hh = c >> 6, cl = c & 63;
+        uint8_t* p;
+        if constexpr (sizeof(T) == 4) {
+          p = xs + (2 * hh + (cl >> 5)) * 16384 + swz(t, (cl & 31) >> 2) + (cl & 3) * 4;
+          oval_bits[i] = *reinterpret_cast<uint32_t*>(p);
+        } else {
+          p = xs + hh * 16384 + swz(t, cl >> 3) + (cl & 7) * 2;
+          oval_bits[i] = *reinterpret_cast<uint16_t*>(p);
+        }
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) {
+      int c = cidx[i];
+      if (i < k && valid && (c >> 6) == h) {
+        int cl = c & 63;
+        if constexpr (sizeof(T) == 4) {
+          uint8_t* p = xs + (2 * h + (cl >> 5)) * 16384 + swz(t, (cl & 31) >> 2) + (cl & 3) * 4;
+          *reinterpret_cast<uint32_t*>(p) = 0x7FC00000u;
+        } else {
+          uint8_t* p = xs + h * 16384 + swz(t, cl >> 3) + (cl & 7) * 2;
+          *reinterpret_cast<uint16_t*>(p) = Elem16<T>::kNaN;
+        }
+      }
+    }
+    __syncwarp();
+    // reload: outlier slots now hold NaN, which min/max ignore
+#pragma unroll
+    for (int j = 0; j < kChunks; ++j) {
+      uint4 v = *reinterpret_cast<const uint4*>(chunk_addr(j));
+      xr[4 * j + 0] = v.x; xr[4 * j + 1] = v.y; xr[4 * j + 2] = v.z; xr[4 * j + 3] = v.w;
+    }
+  }
+
+  // ---------------- group min / max over non-outliers ----------------------
+  // Two 32-channel sub-halves; combined for g >= 64, and with the partner for
+  // g = 128. NaN (outlier) operands are ignored by min/max.
+  float mn[2], mx[2];
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int sh = 0; sh < 2; ++sh) {
+      float lo = __uint_as_float(0x7FC00000u), hi = lo;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        float v = __uint_as_float(xr[32 * sh + e]);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+      }
+      mn[sh] = lo; mx[sh] = hi;
+    }
+  } else {
+#pragma unroll
+    for (int sh = 0; sh < 2; ++sh) {
+      uint32_t lo2 = xr[16 * sh], hi2 = xr[16 * sh];
+#pragma unroll
+      for (int p = 1; p < 16; ++p) {
+        lo2 = pair_min<T>(lo2, xr[16 * sh + p]);
+        hi2 = pair_max<T>(hi2, xr[16 * sh + p]);
+      }
+      float2 l = Elem16<T>::to_f2(lo2), u2 = Elem16<T>::to_f2(hi2);
+      mn[sh] = fminf(l.x, l.y);
+      mx[sh] = fmaxf(u2.x, u2.y);
+    }
+  }
+  if (a.g >= 64) {
+    mn[0] = mn[1] = fminf(mn[0], mn[1]);
+    mx[0] = mx[1] = fmaxf(mx[0], mx[1]);
+  }
+  if (a.g == 128) {
+    float om = __shfl_xor_sync(0xFFFFFFFFu, mn[0], 1), oM = __shfl_xor_sync(0xFFFFFFFFu, mx[0], 1);
+    mn[0] = mn[1] = fminf(mn[0], om);
+    mx[0] = mx[1] = fmaxf(mx[0], oM);
+  }
+  float scale[2], y[2];
+  bool fast[2];
+#pragma unroll
+  for (int sh = 0; sh < 2; ++sh) {
+    if (isnan(mn[sh])) { mn[sh] = 0.0f; mx[sh] = 0.0f; }   // group made of outliers only
+    mn[sh] = __fadd_rn(mn[sh], 0.0f);                      // -0 -> +0
+    mx[sh] = __fadd_rn(mx[sh], 0.0f);
+    scale[sh] = __fdiv_rn(__fsub_rn(mx[sh], mn[sh]), levels);
+    fast[sh] = scale[sh] >= 0x1p-100f && scale[sh] <= 0x1p100f;
+    y[sh] = __frcp_rn(scale[sh]);
+  }
+
+  // ---------------- quantize, pack, residual split -------------------------
+  uint32_t words[kWordsHalf];
+#pragma unroll
+  for (int w = 0; w < kWordsHalf; ++w) words[w] = 0u;
+  uint32_t hi_out[32], lo_out[32];  // packed bf16 pairs of R (hi) and R - hi (lo)
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    const int sh = p >> 4;
+    float x0, x1;
+    if constexpr (sizeof(T) == 4) {
+      x0 = fmaxf(__uint_as_float(xr[2 * p]), mn[sh]);       // NaN -> zero point
+      x1 = fmaxf(__uint_as_float(xr[2 * p + 1]), mn[sh]);
+    } else {
+      uint32_t m2 = Elem16<T>::from_f(mn[sh]);
+      m2 |= m2 << 16;
+      float2 f = Elem16<T>::to_f2(pair_max<T>(xr[p], m2));  // NaN -> zero point
+      x0 = f.x; x1 = f.y;
+    }
+    uint64_t xv = f2_pack(x0, x1);
+    uint64_t mnv = f2_pack(mn[sh], mn[sh]);
+    uint64_t av = f2_sub(xv, mnv);
+    uint64_t q = div_pair(av, scale[sh], y[sh], fast[sh]);
+    if (scale[sh] == 0.0f) q = 0;
+    uint64_t tq = f2_add(q, f2_pack(kRoundMagic, kRoundMagic));
+    uint64_t cf = f2_sub(tq, f2_pack(kRoundMagic, kRoundMagic));
+    uint64_t dh = f2_fma(cf, f2_pack(scale[sh], scale[sh]), mnv);
+    uint64_t rv = f2_sub(xv, dh);
+    if (!valid) rv = 0;
+    // pack: word += bits(tq) << (b * e); the constant part of bits(tq) is
+    // removed once per word below
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+      const int e = 2 * p + e2;
+      uint32_t bits = e2 ? (uint32_t)(tq >> 32) : (uint32_t)tq;
+      words[e / kCodesPerWord] += bits << (BITS * (e % kCodesPerWord));
+    }
+    // residual split: hi = bf16(R), lo = bf16(R - hi)
+    float r0 = f2_lo(rv), r1 = f2_hi(rv);
+    __nv_bfloat162 hb = __floats2bfloat162_rn(r0, r1);
+    uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb);
+    uint64_t hv = f2_pack(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u));
+    uint64_t lv = f2_sub(rv, hv);
+    __nv_bfloat162 lb = __floats2bfloat162_rn(f2_lo(lv), f2_hi(lv));
+    hi_out[p] = hbits;
+    lo_out[p] = *reinterpret_cast<uint32_t*>(&lb);
+  }
+  {
+    uint32_t magic_sum = 0;
+#pragma unroll
+    for (int e = 0; e < kCodesPerWord; ++e) magic_sum += kRoundMagicBits << (BITS * e);
+#pragma unroll
+    for (int w = 0; w < kWordsHalf; ++w) words[w] -= magic_sum;
+  }
+
+  // ---------------- residual to the R stage (MN-major swizzle-128B) --------
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint8_t* ph = rs + h * 16384 + swz(t, j);
+    *reinterpret_cast<uint4*>(ph) = make_uint4(hi_out[4 * j], hi_out[4 * j + 1], hi_out[4 * j + 2], hi_out[4 * j + 3]);
+    *reinterpret_cast<uint4*>(ph + 32768) =
+        make_uint4(lo_out[4 * j], lo_out[4 * j + 1], lo_out[4 * j + 2], lo_out[4 * j + 3]);
+  }
+
+  // ---------------- cache outputs -------------------------------------------
+  if (valid) {
+    const size_t row = (size_t)u * a.n_max + (size_t)(a.t_off + tok);
+    uint32_t* cw = a.codes + row * a.W + h * kWordsHalf;
+#pragma unroll
+    for (int w = 0; w < kWordsHalf; w += 4)
+      *reinterpret_cast<uint4*>(cw + w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
+    // meta: (scale, zero) per group; this thread owns groups in its half
+    float2* meta = reinterpret_cast<float2*>(a.meta) + row * a.G;
+    const int gsz = a.g;
+    if (gsz == 32) {
+      meta[2 * h] = make_float2(scale[0], mn[0]);
+      meta[2 * h + 1] = make_float2(scale[1], mn[1]);
+    } else if (gsz == 64) {
+      meta[h] = make_float2(scale[0], mn[0]);
+    } else if (h == 0) {
+      meta[0] = make_float2(scale[0], mn[0]);
+    }
+    if constexpr (KMAX > 0) {
+      if (h == 0 && k > 0) {
+        // ascending channel order: selection by rank among the k channels
+        uint8_t* oi = a.oidx + row * k;
+#pragma unroll
+        for (int i = 0; i < KMAX; ++i) {
+          if (i < k) {
+            int rank = 0;
+#pragma unroll
+            for (int m = 0; m < KMAX; ++m) rank += (m < k && cidx[m] < cidx[i]) ? 1 : 0;
+            oi[rank] = (uint8_t)cidx[i];
+            if constexpr (sizeof(T) == 4)
+              reinterpret_cast<uint32_t*>(a.oval)[row * k + rank] = oval_bits[i];
+            else
+              reinterpret_cast<uint16_t*>(a.oval)[row * k + rank] = (uint16_t)oval_bits[i];
+          }
+        }
+      }
+    }
+  }
+}
+
+template <typename T, int BITS, int KMAX>
+__global__ void __launch_bounds__(kE1Threads, 1)
+    encode_quant_gram(const __grid_constant__ CUtensorMap tmap, const EncodeArgs a) {
+  using C = E1Cfg<T>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xst = smem;
+  uint8_t* rst = smem + C::kNX * C::kXBytes;
+  E1Bars* bars = reinterpret_cast<E1Bars*>(smem + C::kBarOff);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = a.total_tiles;
+  const int64_t grid = gridDim.x;
+  const int64_t t_begin = (int64_t)blockIdx.x * total / grid;
+  const int64_t t_end = ((int64_t)blockIdx.x + 1) * total / grid;
+  const int ntiles = (int)(t_end - t_begin);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kNX; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 8); }
+    for (int s = 0; s < kNR; ++s) { mbar_init(&bars->r_full[s], 8); mbar_init(&bars->r_empty[s], 1); }
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, 8);
+    bars->abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) tmem_alloc(&bars->tmem_slot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_slot;
+
+  auto is_seg_start = [&](int64_t i) { return i == t_begin || (i % a.tpu) == 0; };
+  auto is_seg_end = [&](int64_t i) { return i + 1 == t_end || ((i + 1) % a.tpu) == 0; };
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int last_it[2] = {-1, -1};
+      prefetch_tensormap(&tmap);
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % C::kNX;
+        if (!mbar_wait(&bars->x_empty[s], ((it / C::kNX) & 1) ^ 1)) { bars->abort_flag = 1; break; }
+        const int64_t tile = t_begin + it;
+        const int u = (int)(tile / a.tpu);
+        const int t0 = (int)(tile % a.tpu) * kTile;
+        const int32_t row0 = u * a.n + t0;
+        mbar_arrive_expect_tx(&bars->x_full[s], C::kXBytes);
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_2d(xst + s * C::kXBytes + b * 16384, &tmap, &bars->x_full[s], b * C::kBoxCols, row0);
+        last_it[s] = it;
+      }
+      // every issued load must have landed before the CTA may exit
+      for (int s = 0; s < C::kNX; ++s)
+        if (last_it[s] >= 0) mbar_wait(&bars->x_full[s], (last_it[s] / C::kNX) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_f16(128, 256, true, true, true);
+      int seg = 0;
+      for (int it = 0; it < ntiles; ++it) {
+        const int64_t tile = t_begin + it;
+        const int sr = it % kNR;
+        bool ok = mbar_wait(&bars->r_full[sr], (it / kNR) & 1);
+        const bool first = is_seg_start(tile);
+        if (ok && first) ok = mbar_wait(&bars->acc_empty, (seg & 1) ^ 1);
+        if (!ok) { bars->abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t base = smem_u32(rst + sr * kRBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          uint64_t ad = smem_desc_sw128(base + kk * 2048, 16384, 1024);
+          uint64_t bd = smem_desc_sw128(base + kk * 2048, 16384, 1024);
+          tc_mma_f16(tmem, ad, bd, kIdesc, (first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(&bars->r_empty[sr]);
+        if (is_seg_end(tile)) { tc_commit(&bars->acc_full); ++seg; }
+      }
+    }
+  } else {
+    // ------------------------------------------------ quantizer warps
+    const int qid = threadIdx.x - 64;
+    const int t = qid >> 1, h = qid & 1;
+    const int qw = warp - 2;
+    int seg = 0;
+    for (int it = 0; it < ntiles; ++it) {
+      const int64_t tile = t_begin + it;
+      const int u = (int)(tile / a.tpu);
+      const int t0 = (int)(tile % a.tpu) * kTile;
+      const int s = it % C::kNX, sr = it % kNR;
+      bool ok = mbar_wait(&bars->x_full[s], (it / C::kNX) & 1);
+      ok = ok && mbar_wait(&bars->r_empty[sr], ((it / kNR) & 1) ^ 1);
+      if (!ok || bars->abort_flag) { bars->abort_flag = 1; break; }
+      quantize_half<T, BITS, KMAX>(a, xst + s * C::kXBytes, rst + sr * kRBytes, t, h, t0 + t < a.n, u, t0 + t);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) { mbar_arrive(&bars->r_full[sr]); mbar_arrive(&bars->x_empty[s]); }
+      if (is_seg_end(tile)) {
+        // ---------------- epilogue: partial Gram of this (CTA, unit) segment
+        if (!mbar_wait(&bars->acc_full, seg & 1)) { bars->abort_flag = 1; break; }
+        tc_fence_after();
+        const int quarter = warp & 3;
+        const int ch = quarter * 32 + lane;
+        const int col0 = (qw < 4) ? 0 : 64;
+        const int64_t slot = (int64_t)blockIdx.x - seg_first_cta((int64_t)u * a.tpu, grid, total);
+        float* dst = a.gram + (((int64_t)u * a.maxc + slot) * 128 + ch) * 128;
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 32) {
+          uint32_t d1[32], d2[32];
+          const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+          tmem_ld_32x32b_x32(lane_addr + col0 + cc, d1);
+          tmem_ld_32x32b_x32(lane_addr + 128 + col0 + cc, d2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 v;
+            v.x = __uint_as_float(d1[j + 0]) + 2.0f * __uint_as_float(d2[j + 0]);
+            v.y = __uint_as_float(d1[j + 1]) + 2.0f * __uint_as_float(d2[j + 1]);
+            v.z = __uint_as_float(d1[j + 2]) + 2.0f * __uint_as_float(d2[j + 2]);
+            v.w = __uint_as_float(d1[j + 3]) + 2.0f * __uint_as_float(d2[j + 3]);
+            *reinterpret_cast<float4*>(dst + col0 + cc + j) = v;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->acc_empty);
+        ++seg;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ================================================================ E2 ======
+// Per unit: M = sym(sum of partial Grams) in fp64, then T power steps with
+// Cholesky-QR on the r x r Gram. Outputs Rf (cache, scaled 2^-e) and
+// Z = Q_{T-1} C_T^-1 scaled 2^e (workspace) so that E3's R Z is the stored L.
+constexpr int kE2Threads = 256;
+constexpr int kMStride = 129;  // padded row (doubles) for conflict-free column reads
+
+__device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t i) {
+  // output number i (0-based) of the splitmix64 stream whose state starts at seed
+  uint64_t z = seed + (i + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__global__ void __launch_bounds__(kE2Threads) encode_power(const EncodeArgs a) {
+  extern __shared__ double sm2[];
+  double* M = sm2;                          // [128][129]
+  double* Q = M + 128 * kMStride;           // [128][16]
+  double* Wm = Q + 128 * 16;                // [128][16]
+  double* Gm = Wm + 128 * 16;               // [16][16]
+  double* Xi = Gm + 256;                    // [16][16] inverse Cholesky factor
+  const int u = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int r = a.r;
+  const int64_t total = a.total_tiles, grid = a.grid_e1;
+  const int64_t c0 = seg_first_cta((int64_t)u * a.tpu, grid, total);
+  const int64_t c1 = seg_first_cta((int64_t)u * a.tpu + a.tpu - 1, grid, total);
+  const int nseg = (int)(c1 - c0 + 1);
+
+  // sum partials in a fixed order
+  for (int e = tid; e < 128 * 128; e += kE2Threads) {
+    double acc = 0.0;
+    const float* src = a.gram + (int64_t)u * a.maxc * 16384 + e;
+    for (int s = 0; s < nseg; ++s) acc += (double)src[(int64_t)s * 16384];
+    M[(e >> 7) * kMStride + (e & 127)] = acc;
+  }
+  // Q0 from the seed
+  for (int e = tid; e < 128 * r; e += kE2Threads) {
+    uint64_t z = splitmix64_at(a.seed, (uint64_t)e);
+    Q[(e / r) * 16 + (e % r)] = (double)(uint32_t)(z >> 40) * 0x1p-23 - 1.0;
+  }
+  __syncthreads();
+  for (int e = tid; e < 128 * 128; e += kE2Threads) {
+    int i = e >> 7, j = e & 127;
+    if (i < j) {
+      double m = 0.5 * (M[i * kMStride + j] + M[j * kMStride + i]);
+      M[i * kMStride + j] = m;
+      M[j * kMStride + i] = m;
+    }
+  }
+  __syncthreads();
+
+  for (int it = 0; it < a.T; ++it) {
+    // W = M Q
+    for (int e = tid; e < 128 * r; e += kE2Threads) {
+      int i = e / r, j = e % r;
+      double acc = 0.0;
+      for (int c = 0; c < 128; ++c) acc += M[c * kMStride + i] * Q[c * 16 + j];
+      Wm[i * 16 + j] = acc;
+    }
+    __syncthreads();
+    // G = Q^T W
+    for (int e = tid; e < r * r; e += kE2Threads) {
+      int p = e / r, q = e % r;
+      double acc = 0.0;
+      for (int i = 0; i < 128; ++i) acc += Q[i * 16 + p] * Wm[i * 16 + q];
+      Gm[p * 16 + q] = acc;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      // Cholesky G = C^T C (upper C) with column dropping, then X = C^-1 so
+      // that P~ X has orthonormal (or zero) columns.
+      double Cm[16][16];
+      bool nz[16];
+      for (int j = 0; j < r; ++j) {
+        for (int m = 0; m < j; ++m) {
+          double v = 0.0;
+          if (nz[m]) {
+            v = Gm[m * 16 + j];
+            for (int i = 0; i < m; ++i) v -= Cm[i][m] * Cm[i][j];
+            v /= Cm[m][m];
+          }
+          Cm[m][j] = v;
+        }
+        double gjj = Gm[j * 16 + j];
+        double piv = gjj;
+        for (int m = 0; m < j; ++m) piv -= Cm[m][j] * Cm[m][j];
+        nz[j] = gjj > 0.0 && piv > 1e-10 * gjj;
+        Cm[j][j] = nz[j] ? sqrt(piv) : 0.0;
+      }
+      for (int j = 0; j < r; ++j) {
+        for (int i = 0; i < r; ++i) Xi[i * 16 + j] = 0.0;
+        if (!nz[j]) continue;
+        // column j of C^-1: (e_j - sum_{m<j} C[m][j] X[:, m]) / C[j][j]
+        for (int i = 0; i < r; ++i) {
+          double v = (i == j) ? 1.0 : 0.0;
+          for (int m = 0; m < j; ++m) v -= Cm[m][j] * Xi[i * 16 + m];
+          Xi[i * 16 + j] = v / Cm[j][j];
+        }
+      }
+    }
+    __syncthreads();
+    const bool last = (it + 1 == a.T);
+    // next Q = W X, or on the last step Z = Q X and Rf = W X
+    double zq[16], wq[16];
+    const int i = tid;
+    if (i < 128) {
+      for (int j = 0; j < r; ++j) {
+        double sq = 0.0, sw = 0.0;
+        for (int m = 0; m < r; ++m) {
+          sq += Q[i * 16 + m] * Xi[m * 16 + j];
+          sw += Wm[i * 16 + m] * Xi[m * 16 + j];
+        }
+        zq[j] = sq;
+        wq[j] = sw;
+      }
+    }
+    __syncthreads();
+    if (i < 128) {
+      if (!last) {
+        for (int j = 0; j < r; ++j) Q[i * 16 + j] = wq[j];
+      } else {
+        const double sL = ldexp(1.0, a.e_blk), sR = ldexp(1.0, -a.e_blk);
+        for (int j = 0; j < 16; ++j)
+          a.zbuf[((int64_t)u * 128 + i) * 16 + j] = j < r ? (float)(zq[j] * sL) : 0.0f;
+        for (int j = 0; j < a.r_max; ++j)
+          a.rfac[(((int64_t)u * a.nblk_max + a.blk) * a.r_max + j) * 128 + i] = j < r ? (float)(wq[j] * sR) : 0.0f;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ================================================================ E3 ======
+// L rows: L_t = R_t Z, with R rebuilt from the stored codes and zero points:
+// R = x - fma(code, scale, zero) on every slot, then the outlier slots'
+// contribution (x_o - zero) Z[c_o] is removed again. One tile of 128 tokens
+// per CTA, two threads per token.
+constexpr int kE3Threads = 256;
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kE3Threads) encode_lowrank(const EncodeArgs a) {
+  __shared__ float Zs[128][16];
+  const int u = blockIdx.y;
+  const int r = a.r;
+  for (int e = threadIdx.x; e < 128 * 16; e += kE3Threads)
+    Zs[e >> 4][e & 15] = a.zbuf[((int64_t)u * 128 + (e >> 4)) * 16 + (e & 15)];
+  __syncthreads();
+  const int t = blockIdx.x * kTile + (threadIdx.x >> 1);
+  const int h = threadIdx.x & 1;
+  if (t >= a.n) return;
+  const size_t row = (size_t)u * a.n_max + (size_t)(a.t_off + t);
+  const uint8_t* xin = reinterpret_cast<const uint8_t*>(a.kv) + ((size_t)u * a.n + t) * 128 * sizeof(T);
+  constexpr int kWordsHalf = 64 * BITS / 32;
+  constexpr int kCodesPerWord = 32 / BITS;
+  const uint32_t* cw = a.codes + row * a.W + h * kWordsHalf;
+  uint32_t words[kWordsHalf];
+#pragma unroll
+  for (int w = 0; w < kWordsHalf; w += 4) {
+    uint4 v = *reinterpret_cast<const uint4*>(cw + w);
+    words[w] = v.x; words[w + 1] = v.y; words[w + 2] = v.z; words[w + 3] = v.w;
+  }
+  const float2* meta = reinterpret_cast<const float2*>(a.meta) + row * a.G;
+  float acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+  constexpr int kVec = 16 / sizeof(T);
+#pragma unroll
+  for (int j = 0; j < 64 / kVec; ++j) {
+    uint4 v = *reinterpret_cast<const uint4*>(xin + (h * 64 + j * kVec) * sizeof(T));
+    uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < kVec; ++e) {
+      const int cl = j * kVec + e;            // channel within the half
+      const int c = h * 64 + cl;
+      float x;
+      if constexpr (sizeof(T) == 4) x = __uint_as_float(vv[e]);
+      else x = Elem16<T>::lo(sizeof(T) == 2 ? (e & 1 ? vv[e >> 1] >> 16 : vv[e >> 1] & 0xFFFFu) : 0u);
+      const float2 sz = meta[c / a.g];
+      const uint32_t code = (words[cl / kCodesPerWord] >> (BITS * (cl % kCodesPerWord))) & ((1u << BITS) - 1u);
+      const float dh = __fmaf_rn((float)code, sz.x, sz.y);
+      const float rr = __fsub_rn(x, dh);
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < r) acc[q] = __fmaf_rn(rr, Zs[c][q], acc[q]);
+    }
+  }
+  // outlier slots: their residual is zero; remove what the loop added
+  const int k = a.k;
+  for (int i = 0; i < k; ++i) {
+    const int c = a.oidx[row * k + i];
+    if ((c >> 6) != h) continue;
+    float x;
+    if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(a.oval)[row * k + i];
+    else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(a.oval)[row * k + i]);
+    const float2 sz = meta[c / a.g];
+    const float rr = __fsub_rn(x, __fmaf_rn(0.0f, sz.x, sz.y));
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (q < r) acc[q] = __fmaf_rn(-rr, Zs[c][q], acc[q]);
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], 1);
+  if (h == 0) {
+    for (int q = 0; q < a.r_max; ++q) {
+      const float v = q < r ? acc[q] : 0.0f;
+      if constexpr (sizeof(T) == 4)
+        reinterpret_cast<float*>(a.lfac)[row * a.r_max + q] = v;
+      else
+        reinterpret_cast<__half*>(a.lfac)[row * a.r_max + q] = __float2half_rn(v);
+    }
+  }
+}
+
+// ================================================================ host =====
+template <typename T, int BITS, int KMAX>
+static cudaError_t launch_e1(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
+  auto kern = encode_quant_gram<T, BITS, KMAX>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, E1Cfg<T>::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kE1Threads, E1Cfg<T>::kSmem, st>>>(map, a);
+  return cudaGetLastError();
+}
+
+template <typename T, int BITS>
+static cudaError_t launch_e1_k(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
+  if (a.k == 0) return launch_e1<T, BITS, 0>(map, a, grid, st);
+  if (a.k <= 4) return launch_e1<T, BITS, 4>(map, a, grid, st);
+  if (a.k <= 8) return launch_e1<T, BITS, 8>(map, a, grid, st);
+  return launch_e1<T, BITS, 16>(map, a, grid, st);
+}
+
+template <typename T>
+static cudaError_t launch_e1_b(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
+  switch (a.bits) {
+    case 2: return launch_e1_k<T, 2>(map, a, grid, st);
+    case 4: return launch_e1_k<T, 4>(map, a, grid, st);
+    default: return launch_e1_k<T, 8>(map, a, grid, st);
+  }
+}
+
+template <typename T>
+static cudaError_t launch_e3_b(const EncodeArgs& a, cudaStream_t st) {
+  dim3 grid(a.tpu, a.U);
+  switch (a.bits) {
+    case 2: encode_lowrank<T, 2><<<grid, kE3Threads, 0, st>>>(a); break;
+    case 4: encode_lowrank<T, 4><<<grid, kE3Threads, 0, st>>>(a); break;
+    default: encode_lowrank<T, 8><<<grid, kE3Threads, 0, st>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode_tiled() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  }
+  return fn;
+}
+
+int encode_grid(const EncodeArgs& a, int num_sms) {
+  int64_t total = a.total_tiles;
+  return (int)(total < num_sms ? total : num_sms);
+}
+
+int encode_maxc(int64_t total_tiles, int grid, int tpu) {
+  int64_t tmin = total_tiles / grid;
+  if (tmin < 1) tmin = 1;
+  int64_t m = (tpu - 1 + tmin - 1) / tmin + 1;
+  if (m > tpu) m = tpu;
+  if (m > grid) m = grid;
+  return (int)m;
+}
+
+cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
+  const int esz = a.dtype == GEAR_F32 ? 4 : 2;
+  PFN_encodeTiled enc = get_encode_tiled();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)a.U * (cuuint64_t)a.n};
+  const cuuint64_t strides[1] = {(cuuint64_t)128 * esz};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)kTile};
+  const cuuint32_t estr[2] = {1, 1};
+  CUtensorMapDataType dt = a.dtype == GEAR_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                           : a.dtype == GEAR_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult cr = enc(&map, dt, 2, const_cast<void*>(a.kv), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+  const int grid = a.grid_e1;
+  cudaError_t e;
+  if (a.dtype == GEAR_F16) e = launch_e1_b<__half>(map, a, grid, st);
+  else if (a.dtype == GEAR_BF16) e = launch_e1_b<__nv_bfloat16>(map, a, grid, st);
+  else e = launch_e1_b<float>(map, a, grid, st);
+  if (e != cudaSuccess) return e;
+  if (a.r == 0) return cudaSuccess;
+
+  const size_t sm2 = (128 * kMStride + 128 * 16 * 2 + 256 * 2) * sizeof(double);
+  e = cudaFuncSetAttribute(encode_power, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+  if (e != cudaSuccess) return e;
+  encode_power<<<a.U, kE2Threads, sm2, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.dtype == GEAR_F16) return launch_e3_b<__half>(a, st);
+  if (a.dtype == GEAR_BF16) return launch_e3_b<__nv_bfloat16>(a, st);
+  return launch_e3_b<float>(a, st);
+}
+
+}  // namespace gear

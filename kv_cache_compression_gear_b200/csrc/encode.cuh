@@ -1,0 +1,40 @@
+// encode.cuh -- argument block and host entry of the GEAR encoder kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gear {
+
+struct EncodeArgs {
+  // input block: U units of n tokens, row-major [U][n][128], cache dtype
+  const void* kv;
+  int32_t U, n;
+  int32_t dtype;     // gear_dtype
+  // codec
+  int32_t bits, g, k, r, T;
+  uint64_t seed;
+  // destination in the cache: tokens [t_off, t_off + n) of block `blk`
+  int32_t t_off, blk, e_blk;
+  int32_t n_max, nblk_max, W, G, r_max;
+  uint32_t* codes;
+  float* meta;
+  uint8_t* oidx;
+  void* oval;
+  void* lfac;
+  float* rfac;
+  // workspace: partial Grams [U][maxc][128][128] and Z [U][128][16]
+  float* gram;
+  float* zbuf;
+  // tiling of E1
+  int32_t tpu;           // 128-token tiles per unit
+  int64_t total_tiles;   // U * tpu
+  int32_t grid_e1;       // persistent CTAs of E1
+  int32_t maxc;          // partial-Gram slots per unit
+};
+
+int encode_grid(const EncodeArgs& a, int num_sms);
+int encode_maxc(int64_t total_tiles, int grid, int tpu);
+cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st);
+
+}  // namespace gear

@@ -1,0 +1,222 @@
+"""ctypes binding of libgear (include/gear.h), with torch for memory and streams.
+
+This module only marshals arguments: every step of the codec and of the
+attention runs in the CUDA kernels of libgear.so. The C entry points are
+re-exported under their own names (gear_encode, gear_decode_attn, ...); the
+``Cache`` class wraps one compressed tensor whose device memory is a torch
+uint8 buffer. Importing fails loudly if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgear.so")
+
+GEAR_OK, GEAR_ERR_INVALID_ARG, GEAR_ERR_UNSUPPORTED, GEAR_ERR_CAPACITY = 0, 1, 2, 3
+GEAR_ERR_CUDA, GEAR_ERR_TIMEOUT, GEAR_ERR_WORKSPACE = 4, 5, 6
+GEAR_F16, GEAR_BF16, GEAR_F32 = 0, 1, 2
+
+_DT = {torch.float16: GEAR_F16, torch.bfloat16: GEAR_BF16, torch.float32: GEAR_F32}
+_TORCH = {v: k for k, v in _DT.items()}
+
+
+class GearParams(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("outlier_frac", ctypes.c_float),
+                ("rank", ctypes.c_int32), ("power_iters", ctypes.c_int32), ("buffer_len", ctypes.c_int32),
+                ("buffer_rank", ctypes.c_int32), ("reserved0", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+
+
+class GearCacheStruct(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d", ctypes.c_int32), ("n_max", ctypes.c_int32),
+                ("nblk_max", ctypes.c_int32), ("dtype", ctypes.c_int32), ("p", GearParams),
+                ("k", ctypes.c_int32), ("G", ctypes.c_int32), ("W", ctypes.c_int32), ("r_max", ctypes.c_int32),
+                ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("oidx", ctypes.c_void_p),
+                ("oval", ctypes.c_void_p), ("lfac", ctypes.c_void_p), ("rfac", ctypes.c_void_p),
+                ("buf", ctypes.c_void_p), ("n_comp", ctypes.c_int32), ("n_buf", ctypes.c_int32),
+                ("n_blk", ctypes.c_int32), ("blk0_len", ctypes.c_int32), ("blk0_rank", ctypes.c_int32),
+                ("reserved1", ctypes.c_int32)]
+
+
+class GearError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libgear.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    P, S = ctypes.c_void_p, ctypes.c_size_t
+    i32 = ctypes.c_int32
+    pp = ctypes.POINTER(GearParams)
+    pc = ctypes.POINTER(GearCacheStruct)
+    sig = {
+        "gear_num_outliers": (i32, [ctypes.c_float, i32]),
+        "gear_validate_params": (i32, [pp, i32]),
+        "gear_cache_bytes": (S, [pp, i32, i32, i32, i32, i32, i32]),
+        "gear_cache_init": (i32, [pc, pp, i32, i32, i32, i32, i32, i32, P, S]),
+        "gear_encode_workspace_bytes": (S, [pc, i32]),
+        "gear_encode": (i32, [pc, P, i32, P, S, P]),
+        "gear_decode_workspace_bytes": (S, [pc, pc, i32]),
+        "gear_decode_attn": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P, S, P]),
+        "gear_append_workspace_bytes": (S, [pc]),
+        "gear_append_buffer": (i32, [pc, pc, P, P, P, S, P]),
+        "gear_decode_dense": (i32, [pc, P, P]),
+        "gear_get_device_status": (i32, [ctypes.POINTER(i32)]),
+        "gear_status_string": (ctypes.c_char_p, [i32]),
+        "gear_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L, list(sig)
+
+
+lib, EXPORTS = _load()
+for _name in EXPORTS:
+    globals()[_name] = getattr(lib, _name)
+
+
+def status_string(s: int) -> str:
+    return lib.gear_status_string(s).decode()
+
+
+def _check(status: int, what: str):
+    if status != GEAR_OK:
+        raise GearError(status, what)
+
+
+def _stream_ptr(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_params(bits=4, group_size=64, outlier_frac=0.02, rank=4, power_iters=3, buffer_len=20, buffer_rank=2,
+                seed=0) -> GearParams:
+    return GearParams(bits, group_size, outlier_frac, rank, power_iters, buffer_len, buffer_rank, 0, seed)
+
+
+class _Workspace:
+    """Grow-only device scratch buffer owned by torch."""
+
+    def __init__(self):
+        self.buf = None
+
+    def get(self, nbytes: int, device) -> tuple[int, int]:
+        if nbytes == 0:
+            return 0, 0
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != torch.device(device):
+            self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        p = self.buf.data_ptr()
+        p = (p + 255) & ~255
+        return p, nbytes
+
+
+_ws = _Workspace()
+
+
+class Cache:
+    """One compressed tensor (K or V) of shape [B][H][*][128] on a CUDA device."""
+
+    def __init__(self, params: GearParams, B: int, H: int, n_max: int, nblk_max: int, dtype: torch.dtype,
+                 device="cuda", d: int = 128):
+        self.params = params
+        self.dtype = dtype
+        self.device = torch.device(device)
+        nbytes = lib.gear_cache_bytes(ctypes.byref(params), B, H, d, n_max, nblk_max, _DT[dtype])
+        if nbytes == 0:
+            _check(lib.gear_validate_params(ctypes.byref(params), d) or GEAR_ERR_INVALID_ARG, "gear_cache_bytes")
+        self.mem = torch.empty(nbytes + 256, dtype=torch.uint8, device=self.device)
+        base = (self.mem.data_ptr() + 255) & ~255
+        self.c = GearCacheStruct()
+        _check(lib.gear_cache_init(ctypes.byref(self.c), ctypes.byref(params), B, H, d, n_max, nblk_max, _DT[dtype],
+                                   ctypes.c_void_p(base), nbytes), "gear_cache_init")
+
+    # counters
+    @property
+    def n_comp(self) -> int:
+        return self.c.n_comp
+
+    @property
+    def n_buf(self) -> int:
+        return self.c.n_buf
+
+    @property
+    def n_blk(self) -> int:
+        return self.c.n_blk
+
+    def encode(self, kv: torch.Tensor, stream=None):
+        assert kv.is_cuda and kv.dtype == self.dtype and kv.is_contiguous()
+        B, H, n, d = kv.shape
+        nbytes = lib.gear_encode_workspace_bytes(ctypes.byref(self.c), n)
+        wp, wn = _ws.get(nbytes, kv.device)
+        _check(lib.gear_encode(ctypes.byref(self.c), ctypes.c_void_p(kv.data_ptr()), n, ctypes.c_void_p(wp), wn,
+                               _stream_ptr(stream)), "gear_encode")
+
+    def dense(self, stream=None) -> torch.Tensor:
+        c = self.c
+        out = torch.empty((c.B, c.H, c.n_comp + c.n_buf, c.d), dtype=torch.float32, device=self.device)
+        _check(lib.gear_decode_dense(ctypes.byref(c), ctypes.c_void_p(out.data_ptr()), _stream_ptr(stream)),
+               "gear_decode_dense")
+        return out
+
+    # raw views of the stored arrays (for tests)
+    def _view(self, ptr, count, dtype):
+        off = ptr - self.mem.data_ptr()
+        nbytes = count * torch.empty((), dtype=dtype).element_size()
+        return self.mem[off:off + nbytes].view(dtype)
+
+    def arrays(self) -> dict:
+        c = self.c
+        U = c.B * c.H
+        n = c.n_max
+        ld = torch.float32 if self.dtype == torch.float32 else torch.float16
+        k = max(c.k, 1)
+        return {
+            "codes": self._view(c.codes, U * n * c.W, torch.int32).view(U, n, c.W),
+            "meta": self._view(c.meta, U * n * c.G * 2, torch.float32).view(U, n, c.G, 2),
+            "oidx": self._view(c.oidx, U * n * k, torch.uint8).view(U, n, k),
+            "oval": self._view(c.oval, U * n * k, self.dtype).view(U, n, k),
+            "lfac": self._view(c.lfac, U * n * c.r_max, ld).view(U, n, c.r_max),
+            "rfac": self._view(c.rfac, U * c.nblk_max * c.r_max * c.d, torch.float32).view(U, c.nblk_max, c.r_max,
+                                                                                          c.d),
+            "buf": self._view(c.buf, U * c.p.buffer_len * c.d, self.dtype).view(U, c.p.buffer_len, c.d),
+        }
+
+
+def decode_attn(kc: Cache, vc: Cache, q: torch.Tensor, softmax_scale: float, out_dtype=None, out=None,
+                stream=None) -> torch.Tensor:
+    assert q.is_cuda and q.dtype == kc.dtype and q.is_contiguous()
+    B, Hq, d = q.shape
+    od = out_dtype or kc.dtype
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=od, device=q.device)
+    nbytes = lib.gear_decode_workspace_bytes(ctypes.byref(kc.c), ctypes.byref(vc.c), Hq)
+    if nbytes == 0:
+        raise GearError(GEAR_ERR_INVALID_ARG, "gear_decode_workspace_bytes")
+    wp, wn = _ws.get(nbytes, q.device)
+    _check(lib.gear_decode_attn(ctypes.byref(kc.c), ctypes.byref(vc.c), ctypes.c_void_p(q.data_ptr()), Hq,
+                                ctypes.c_float(softmax_scale), ctypes.c_void_p(out.data_ptr()), _DT[od],
+                                ctypes.c_void_p(wp), wn, _stream_ptr(stream)), "gear_decode_attn")
+    return out
+
+
+def append_buffer(kc: Cache, vc: Cache, k_new: torch.Tensor, v_new: torch.Tensor, stream=None):
+    assert k_new.is_cuda and k_new.dtype == kc.dtype and k_new.is_contiguous() and v_new.is_contiguous()
+    nbytes = lib.gear_append_workspace_bytes(ctypes.byref(kc.c))
+    wp, wn = _ws.get(nbytes, k_new.device)
+    _check(lib.gear_append_buffer(ctypes.byref(kc.c), ctypes.byref(vc.c), ctypes.c_void_p(k_new.data_ptr()),
+                                  ctypes.c_void_p(v_new.data_ptr()), ctypes.c_void_p(wp), wn, _stream_ptr(stream)),
+           "gear_append_buffer")
+
+
+def device_status() -> int:
+    v = ctypes.c_int32(0)
+    _check(lib.gear_get_device_status(ctypes.byref(v)), "gear_get_device_status")
+    return v.value

@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI (no GPU): the library loads and exports every
+function include/gear.h declares, the ctypes structs match the C layout, and
+invalid arguments are rejected on the host before anything is enqueued."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gear.h")
+
+
+@pytest.fixture(scope="module")
+def gear():
+    from kv_cache_compression_gear_b200 import build
+    build.build()
+    import kv_cache_compression_gear_b200 as g
+    return g
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gear_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_function(gear):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(gear.lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", gear.gear.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (gear_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_struct_layout_matches_c(gear):
+    prog = r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "gear.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu %zu\n", sizeof(gear_params), sizeof(gear_cache),
+         offsetof(gear_cache, p), offsetof(gear_cache, codes), offsetof(gear_cache, buf),
+         offsetof(gear_cache, n_comp), offsetof(gear_params, seed));
+  return 0;
+}'''
+    with tempfile.TemporaryDirectory() as td:
+        c = os.path.join(td, "t.c")
+        open(c, "w").write(prog)
+        exe = os.path.join(td, "t")
+        subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe])
+        vals = [int(v) for v in subprocess.check_output([exe]).split()]
+    G, P = gear.GearCacheStruct, gear.GearParams
+    assert vals == [ctypes.sizeof(P), ctypes.sizeof(G), G.p.offset, G.codes.offset, G.buf.offset,
+                    G.n_comp.offset, P.seed.offset]
+
+
+def test_num_outliers_and_validation(gear):
+    L = gear.lib
+    assert L.gear_num_outliers(ctypes.c_float(0.02), 128) == 3
+    assert L.gear_num_outliers(ctypes.c_float(0.05), 128) == 7
+    assert L.gear_num_outliers(ctypes.c_float(0.0), 128) == 0
+    ok = gear.make_params()
+    assert L.gear_validate_params(ctypes.byref(ok), 128) == 0
+    bad = [dict(bits=3), dict(group_size=48), dict(group_size=8, bits=2), dict(outlier_frac=-0.1),
+           dict(outlier_frac=0.6), dict(rank=-1), dict(rank=17), dict(power_iters=0), dict(buffer_len=0),
+           dict(buffer_rank=21)]
+    for kw in bad:
+        p = gear.make_params(**kw)
+        assert L.gear_validate_params(ctypes.byref(p), 128) == gear.gear.GEAR_ERR_INVALID_ARG, kw
+    assert L.gear_validate_params(ctypes.byref(ok), 64) == gear.gear.GEAR_ERR_UNSUPPORTED
+    p = gear.make_params(group_size=16, bits=2)   # valid, but groups below 32 channels are not implemented
+    assert L.gear_validate_params(ctypes.byref(p), 128) == gear.gear.GEAR_ERR_UNSUPPORTED
+    p = gear.make_params(outlier_frac=0.2)   # k = 26 > 16
+    assert L.gear_validate_params(ctypes.byref(p), 128) == gear.gear.GEAR_ERR_UNSUPPORTED
+    assert L.gear_validate_params(None, 128) == gear.gear.GEAR_ERR_INVALID_ARG
+
+
+def test_cache_layout_and_host_errors(gear):
+    L = gear.lib
+    p = gear.make_params()
+    nbytes = L.gear_cache_bytes(ctypes.byref(p), 1, 32, 128, 4096, 1, 0)
+    # codes 64 B + meta 16 B + 3 idx + 3 fp16 values + 4 fp16 L per token
+    per_tok = 64 + 16 + 3 + 6 + 8
+    assert per_tok * 32 * 4096 <= nbytes <= per_tok * 32 * 4096 + 32 * 20 * 256 + 32 * 4 * 512 + 8 * 256
+    c = gear.GearCacheStruct()
+    fake = ctypes.c_void_p(1 << 40)  # never dereferenced on the host
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(p), 1, 32, 128, 4096, 1, 0, fake, nbytes - 1) == \
+        gear.gear.GEAR_ERR_CAPACITY
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(p), 1, 32, 128, 4096, 1, 0,
+                             ctypes.c_void_p((1 << 40) + 8), nbytes) == gear.gear.GEAR_ERR_INVALID_ARG
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(p), 1, 32, 128, 4096, 1, 0, fake, nbytes) == 0
+    assert (c.k, c.G, c.W, c.r_max) == (3, 2, 16, 4)
+    assert c.codes == 1 << 40 and c.n_comp == 0
+    offs = [c.codes, c.meta, c.oidx, c.oval, c.lfac, c.rfac, c.buf]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert c.buf + 32 * 20 * 128 * 2 <= (1 << 40) + nbytes
+    # argument errors return before touching the device
+    E = gear.gear
+    assert L.gear_encode(ctypes.byref(c), None, 10, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_encode(ctypes.byref(c), ctypes.c_void_p(4096 + 8), 10, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_encode(ctypes.byref(c), ctypes.c_void_p(4096), 0, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_encode(ctypes.byref(c), ctypes.c_void_p(4096), 5000, None, 0, None) == E.GEAR_ERR_CAPACITY
+    assert L.gear_encode(ctypes.byref(c), ctypes.c_void_p(4096), 2, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_decode_attn(ctypes.byref(c), ctypes.byref(c), ctypes.c_void_p(4096), 32, ctypes.c_float(0.1),
+                              ctypes.c_void_p(4096), 0, None, 0, None) == E.GEAR_ERR_INVALID_ARG  # empty cache
+    assert L.gear_decode_dense(ctypes.byref(c), None, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_status_string(6) == b"workspace missing or too small"
+    assert L.gear_version() == b"0.1.0"

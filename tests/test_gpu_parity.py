@@ -1,0 +1,267 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs. Codes, scales, zero points and outliers are compared bit for
+bit; the low-rank term, the reconstruction and attention within stated
+tolerances (see gpu_helpers)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.gpu_helpers import (TORCH_DT, compare_dense, compare_unit, gpu_block, oracle_params, seeded_kv,
+                               to_dev)
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import kv_cache_compression_gear_b200 as gear
+else:
+    gear = None
+
+
+def _tol_out(dtype: str) -> float:
+    return 8e-3 if dtype == "bf16" else 1e-3
+
+
+def _encode_both(x: np.ndarray, dtype: str, p, n_max=None, nblk_max=4):
+    B, H, n, d = x.shape
+    kc = gear.Cache(p, B, H, n_max or n, nblk_max, TORCH_DT[dtype])
+    kc.encode(to_dev(x, dtype))
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    op = oracle_params(p)
+    units = [oracle.encode_unit(x[b, h], op) for b in range(B) for h in range(H)]
+    return kc, units, op
+
+
+# ------------------------------------------------------------------ encode
+ENC_CASES = [
+    # dtype, B, H, n, bits, g, s, r, T
+    ("f16", 1, 2, 1, 4, 64, 0.02, 1, 3),
+    ("f16", 1, 2, 2, 4, 64, 0.02, 2, 3),
+    ("f16", 2, 1, 7, 4, 64, 0.02, 4, 3),
+    ("f16", 1, 3, 33, 2, 32, 0.05, 4, 2),
+    ("f16", 1, 2, 128, 4, 64, 0.02, 4, 3),
+    ("f16", 1, 2, 129, 8, 64, 0.02, 4, 3),
+    ("f16", 2, 2, 300, 4, 32, 0.02, 8, 3),
+    ("f16", 1, 3, 1000, 4, 128, 0.02, 4, 3),
+    ("f16", 1, 2, 257, 4, 64, 0.0, 0, 1),
+    ("f16", 1, 2, 257, 4, 64, 0.1, 16, 2),
+    ("bf16", 1, 2, 300, 4, 64, 0.02, 4, 3),
+    ("bf16", 2, 2, 77, 2, 64, 0.05, 2, 1),
+    ("f32", 1, 1, 256, 4, 64, 0.02, 4, 3),
+    ("f32", 1, 2, 130, 8, 32, 0.05, 3, 2),
+]
+
+
+@pytest.mark.parametrize("dtype,B,H,n,bits,g,s,r,T", ENC_CASES)
+def test_encode_matches_oracle(dtype, B, H, n, bits, g, s, r, T):
+    p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, power_iters=T, seed=1234 + n)
+    x = seeded_kv(7 + n + bits, 1, (B, H, n, 128), dtype, channel_scale=True)
+    kc, units, op = _encode_both(x, dtype, p)
+    dense = kc.dense().cpu().numpy()
+    for u, o in enumerate(units):
+        gb = gpu_block(kc, u, 0, n, 0, r)
+        compare_unit(gb, o, p, f"unit {u}")
+        compare_dense(dense[u // H, u % H], oracle.reconstruct_unit(o, op), o.scale, g, f"unit {u}")
+
+
+def test_encode_ties_and_constant_groups():
+    # many exact ties in |x| (integers), constant groups, signed zeros
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.05, rank=4, seed=3)
+    rng = np.random.default_rng(5)
+    x = rng.integers(-4, 5, size=(1, 2, 200, 128)).astype(np.float32)
+    x[0, 0, 3, :64] = 2.0
+    x[0, 0, 4, :] = 0.0
+    x[0, 1, 5, ::2] = -0.0
+    kc, units, op = _encode_both(x, "f16", p)
+    for u, o in enumerate(units):
+        compare_unit(gpu_block(kc, u, 0, 200, 0, 4), o, p, f"unit {u}")
+
+
+def test_encode_rank_deficient_residual():
+    # (a) 8-bit codes with a group range of exactly 255: scale 1, every entry is
+    # reproduced, the residual is zero and all factors must be zero
+    p = gear.make_params(bits=8, group_size=64, outlier_frac=0.0, rank=4, seed=9)
+    rng = np.random.default_rng(2)
+    x = rng.integers(0, 256, size=(1, 1, 64, 128)).astype(np.float32)
+    x[..., 0::64] = 0.0
+    x[..., 1::64] = 255.0
+    kc, units, op = _encode_both(x, "f16", p)
+    g = gpu_block(kc, 0, 0, 64, 0, 4)
+    compare_unit(g, units[0], p)
+    assert not units[0].resid.any()
+    assert not g["L"].any() and not g["Rf"].any()
+    # (b) identical rows: the residual has rank 1, so three of four columns drop
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.02, rank=4, seed=9)
+    x = np.tile(seeded_kv(4, 1, (1, 128), "f16"), (1, 1, 64, 1))
+    kc, units, op = _encode_both(x, "f16", p)
+    g = gpu_block(kc, 0, 0, 64, 0, 4)
+    compare_unit(g, units[0], p)
+    R = units[0].resid.astype(np.float64)
+    assert np.abs(g["L"] @ g["Rf"].T - R).max() <= 1e-3 * np.abs(R).max()
+
+
+# ------------------------------------------------------------ decode + append
+def _build_caches(dtype, B, H, n0, p, nappend, seed, n_max=None, nblk_max=None):
+    xk = seeded_kv(seed, 1, (B, H, n0, 128), dtype, channel_scale=True)
+    xv = seeded_kv(seed, 2, (B, H, n0, 128), dtype)
+    n_max = n_max or n0 + nappend + 1
+    nblk_max = nblk_max or 2 + nappend // p.buffer_len
+    kc = gear.Cache(p, B, H, n_max, nblk_max, TORCH_DT[dtype])
+    vc = gear.Cache(p, B, H, n_max, nblk_max, TORCH_DT[dtype])
+    op = oracle_params(p)
+    ok, ov = oracle.Cache(op, B, H, 128), oracle.Cache(op, B, H, 128)
+    if n0:
+        kc.encode(to_dev(xk, dtype))
+        vc.encode(to_dev(xv, dtype))
+        ok.encode(xk)
+        ov.encode(xv)
+    for i in range(nappend):
+        rk = seeded_kv(seed + 100 + i, 3, (B, H, 128), dtype)
+        rv = seeded_kv(seed + 100 + i, 4, (B, H, 128), dtype)
+        gear.append_buffer(kc, vc, to_dev(rk, dtype), to_dev(rv, dtype))
+        ok.append(rk)
+        ov.append(rv)
+    torch.cuda.synchronize()
+    return kc, vc, ok, ov
+
+
+DEC_CASES = [
+    # dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf
+    ("f16", 2, 2, 2, 300, 0, 4, 64, 0.02, 4, 20, 2),
+    ("f16", 1, 2, 8, 200, 5, 4, 64, 0.02, 4, 20, 2),
+    ("f16", 2, 1, 4, 130, 45, 2, 32, 0.05, 8, 20, 2),
+    ("f16", 1, 2, 2, 0, 7, 4, 64, 0.02, 4, 3, 1),
+    ("f16", 1, 2, 2, 1000, 21, 4, 128, 0.0, 0, 20, 0),
+    ("bf16", 1, 2, 8, 257, 20, 4, 64, 0.02, 4, 20, 2),
+    ("f32", 1, 1, 1, 256, 0, 4, 64, 0.02, 4, 20, 2),
+    ("f32", 1, 2, 4, 64, 9, 8, 32, 0.05, 2, 4, 2),
+]
+
+
+@pytest.mark.parametrize("dtype,B,H,Hq,n0,nappend,bits,g,s,r,n_b,r_buf", DEC_CASES)
+def test_decode_and_append_match_oracle(dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf):
+    p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, buffer_len=n_b, buffer_rank=r_buf,
+                         power_iters=3, seed=77)
+    kc, vc, ok, ov = _build_caches(dtype, B, H, n0, p, nappend, seed=11 + n0)
+    assert kc.n_comp == ok.n_comp and kc.n_buf == len(ok.buffer) and kc.n_blk == len(ok.blocks)
+    q = seeded_kv(99 + n0, 5, (B, Hq, 128), dtype)
+    tau = 1.0 / math.sqrt(128)
+    od = oracle.decode_attn(ok, ov, q, tau)
+    vmax = np.abs(ov.dense()).max()
+    for out_dt in [TORCH_DT[dtype], torch.float32]:
+        out = gear.decode_attn(kc, vc, to_dev(q, dtype), tau, out_dtype=out_dt).float().cpu().numpy()
+        err = np.abs(out - od).max()
+        assert err <= _tol_out(dtype) * vmax, f"attention error {err:.3e} vs {_tol_out(dtype) * vmax:.3e}"
+    # flushed blocks equal the oracle's blocks
+    t0 = ok.blocks[0][0].codes.shape[0] if n0 else 0
+    for bi, blk in enumerate(ok.blocks):
+        if n0 and bi == 0:
+            continue
+        for u, o in enumerate(blk):
+            compare_unit(gpu_block(kc, u, t0, t0 + n_b, bi, r_buf), o, p, f"K block {bi} unit {u}")
+        t0 += n_b
+    assert gear.device_status() == 0
+
+
+# ------------------------------------------------------ full-size workloads
+def _workload_encode_check(w: wl.Workload, units_to_check, layer=0):
+    p = gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
+                         buffer_len=w.buffer_len, buffer_rank=w.buffer_rank, seed=w.seed)
+    op = oracle_params(p)
+    out = {}
+    for which in ["k", "v"]:
+        x = wl.kv_tensor_torch(w, which, layer, "cuda")
+        c = gear.Cache(p, w.B, w.H, w.n + 64, 4, TORCH_DT[w.dtype])
+        c.encode(x)
+        torch.cuda.synchronize()
+        del x
+        for (b, h) in units_to_check:
+            xo = wl.kv_unit_np(w, which, layer, b, h)
+            o = oracle.encode_unit(xo, op)
+            compare_unit(gpu_block(c, b * w.H + h, 0, w.n, 0, w.rank), o, p, f"{w.name} {which} ({b},{h})")
+        out[which] = c
+    assert gear.device_status() == 0
+    return p, out
+
+
+def test_full_llama7b_layer_encode():
+    w = wl.WORKLOADS["llama7b_layer_encode"]
+    _workload_encode_check(w, [(0, 0), (0, 13), (0, 31)])
+
+
+def test_full_twobit_b64_encode_and_decode():
+    w = wl.WORKLOADS["twobit_b64_ctx8192"]
+    p, caches = _workload_encode_check(w, [(0, 0), (37, 5), (63, 31)])
+    q = wl.rows_torch(w, wl.S_Q, 0, 0, w.Hq, "cuda")
+    tau = 1.0 / math.sqrt(128)
+    out = gear.decode_attn(caches["k"], caches["v"], q, tau, out_dtype=torch.float32).cpu().numpy()
+    qn = wl.rows_np(w, wl.S_Q, 0, 0, w.Hq)
+    op = oracle_params(p)
+    for (b, h) in [(5, 7), (63, 0)]:
+        K = oracle.reconstruct_unit(oracle.encode_unit(wl.kv_unit_np(w, "k", 0, b, h), op), op)
+        Vu = oracle.encode_unit(wl.kv_unit_np(w, "v", 0, b, h), op)
+        V = oracle.reconstruct_unit(Vu, op)
+        ref = oracle.attention(qn[b, h], K, V, tau)
+        assert np.abs(out[b, h] - ref).max() <= 1e-3 * np.abs(V).max()
+
+
+def test_full_decode_b16_with_buffer_and_flush():
+    w = wl.WORKLOADS["decode_b16_ctx8192"]
+    p = gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
+                         buffer_len=w.buffer_len, buffer_rank=w.buffer_rank, seed=w.seed)
+    op = oracle_params(p)
+    kc = gear.Cache(p, w.B, w.H, w.n + 64, 4, TORCH_DT[w.dtype])
+    vc = gear.Cache(p, w.B, w.H, w.n + 64, 4, TORCH_DT[w.dtype])
+    kc.encode(wl.kv_tensor_torch(w, "k", 0, "cuda"))
+    vc.encode(wl.kv_tensor_torch(w, "v", 0, "cuda"))
+    for i in range(w.buffer_fill):
+        gear.append_buffer(kc, vc, wl.rows_torch(w, wl.S_KBUF, 0, i, w.H, "cuda"),
+                           wl.rows_torch(w, wl.S_VBUF, 0, i, w.H, "cuda"))
+    q = wl.rows_torch(w, wl.S_Q, 0, 0, w.Hq, "cuda")
+    tau = 1.0 / math.sqrt(128)
+    out = gear.decode_attn(kc, vc, q, tau, out_dtype=torch.float32).cpu().numpy()
+    # one more token: flushes the full buffer as block 1
+    gear.append_buffer(kc, vc, wl.rows_torch(w, wl.S_KNEW, 0, 0, w.H, "cuda"),
+                       wl.rows_torch(w, wl.S_VNEW, 0, 0, w.H, "cuda"))
+    out2 = gear.decode_attn(kc, vc, q, tau, out_dtype=torch.float32).cpu().numpy()
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    qn = wl.rows_np(w, wl.S_Q, 0, 0, w.Hq)
+    for (b, h) in [(0, 0), (9, 17), (15, 31)]:
+        ok, ov = oracle.Cache(op, 1, 1, 128), oracle.Cache(op, 1, 1, 128)
+        ok.encode(wl.kv_unit_np(w, "k", 0, b, h)[None, None])
+        ov.encode(wl.kv_unit_np(w, "v", 0, b, h)[None, None])
+        for i in range(w.buffer_fill):
+            ok.append(wl.rows_np(w, wl.S_KBUF, 0, i, w.H)[b:b + 1, h:h + 1])
+            ov.append(wl.rows_np(w, wl.S_VBUF, 0, i, w.H)[b:b + 1, h:h + 1])
+        ref = oracle.decode_attn(ok, ov, qn[b:b + 1, h:h + 1], tau)[0, 0]
+        vmax = np.abs(ov.dense()).max()
+        assert np.abs(out[b, h] - ref).max() <= 1e-3 * vmax
+        ok.append(wl.rows_np(w, wl.S_KNEW, 0, 0, w.H)[b:b + 1, h:h + 1])
+        ov.append(wl.rows_np(w, wl.S_VNEW, 0, 0, w.H)[b:b + 1, h:h + 1])
+        ref2 = oracle.decode_attn(ok, ov, qn[b:b + 1, h:h + 1], tau)[0, 0]
+        assert np.abs(out2[b, h] - ref2).max() <= 1e-3 * np.abs(ov.dense()).max()
+        compare_unit(gpu_block(kc, b * w.H + h, w.n, w.n + w.buffer_len, 1, w.buffer_rank), ok.blocks[1][0], p,
+                     f"flushed K block ({b},{h})")
+
+
+def test_full_llama3_gqa_layer():
+    w = wl.WORKLOADS["llama3_8b_gqa"]
+    layer = 17
+    p, caches = _workload_encode_check(w, [(0, 0), (7, 7)], layer=layer)
+    q = wl.rows_torch(w, wl.S_Q, layer, 0, w.Hq, "cuda")
+    tau = 1.0 / math.sqrt(128)
+    out = gear.decode_attn(caches["k"], caches["v"], q, tau, out_dtype=torch.float32).cpu().numpy()
+    qn = wl.rows_np(w, wl.S_Q, layer, 0, w.Hq)
+    op = oracle_params(p)
+    b, h = 3, 5
+    K = oracle.reconstruct_unit(oracle.encode_unit(wl.kv_unit_np(w, "k", layer, b, h), op), op)
+    V = oracle.reconstruct_unit(oracle.encode_unit(wl.kv_unit_np(w, "v", layer, b, h), op), op)
+    hq = w.Hq // w.H
+    for j in range(h * hq, (h + 1) * hq):
+        ref = oracle.attention(qn[b, j], K, V, tau)
+        assert np.abs(out[b, j] - ref).max() <= 8e-3 * np.abs(V).max()

@@ -200,24 +200,32 @@ def kv_unit_np(w: Workload, which: str, layer: int, b: int, h: int, n: int | Non
 
 
 def kv_tensor_torch(w: Workload, which: str, layer: int, device, n: int | None = None):
-    """[B][H][n][d] tensor in the workload dtype, generated on `device`."""
+    """[B][H][n][d] tensor in the workload dtype, generated on `device` in chunks
+    of whole units (bounded temporaries)."""
     import torch
     n = w.n if n is None else n
     stream = S_K if which == "k" else S_V
-    base = layer * w.B * w.H * n * w.d
-    idx = base + torch.arange(w.B * w.H * n * w.d, device=device, dtype=torch.int64)
-    x = normal_torch(w.seed, stream, idx).view(w.B, w.H, n, w.d)
-    del idx
-    if which == "k":
-        sig = torch.from_numpy(channel_sigma(w, layer)).to(device)
-        x.mul_(sig[None, :, None, :])
-        sp = spike_positions(w)
-        sp = sp[sp < n * w.d]
-        if sp.size:
-            xs = x.view(w.B * w.H, n * w.d)
-            spt = torch.from_numpy(sp).to(device)
-            xs[:, spt] *= 10.0
-    return x.to(torch_dtype(w.dtype))
+    out = torch.empty((w.B * w.H, n, w.d), dtype=torch_dtype(w.dtype), device=device)
+    sig = torch.from_numpy(channel_sigma(w, layer)).to(device) if which == "k" else None
+    sp = spike_positions(w) if which == "k" else np.zeros(0, np.int64)
+    sp = sp[sp < n * w.d]
+    spt = torch.from_numpy(sp).to(device) if sp.size else None
+    per_unit = n * w.d
+    step = max(1, (1 << 26) // per_unit)
+    base0 = layer * w.B * w.H * per_unit
+    for u0 in range(0, w.B * w.H, step):
+        u1 = min(w.B * w.H, u0 + step)
+        idx = base0 + u0 * per_unit + torch.arange((u1 - u0) * per_unit, device=device, dtype=torch.int64)
+        x = normal_torch(w.seed, stream, idx).view(u1 - u0, n, w.d)
+        del idx
+        if sig is not None:
+            h = torch.arange(u0, u1, device=device) % w.H
+            x.mul_(sig[h][:, None, :])
+            if spt is not None:
+                xs = x.view(u1 - u0, n * w.d)
+                xs[:, spt] *= 10.0
+        out[u0:u1] = x.to(out.dtype)
+    return out.view(w.B, w.H, n, w.d)
 
 
 def rows_np(w: Workload, stream: int, layer: int, step: int, heads: int) -> np.ndarray:
