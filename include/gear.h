@@ -178,6 +178,27 @@ gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const voi
                              int32_t Hq, float softmax_scale, void* out, gear_dtype out_dtype,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* Decode attention that allocates nothing. The GEAR paper has no counterpart
+ * of this entry point: it exists for callers that cannot call cudaMalloc or
+ * hand the library a workspace -- for example a plugin inside a host framework
+ * that owns all device memory and offers plugins no allocator, or a decode loop
+ * whose device memory budget is fixed when the process starts.
+ * Same computation, arguments, layouts and errors as gear_decode_attn, except
+ * that the split-K partial results go to a scratch array inside the library: a
+ * file-scope __device__ array of 4 MiB that every GPU which loads the library
+ * holds until the process exits. The caller still passes q and out.
+ * Limit: returns GEAR_ERR_WORKSPACE, enqueuing nothing, when the partials would
+ * not fit, i.e. when gear_decode_workspace_bytes(k, v, Hq) > 4 MiB (each of the
+ * B * Hq query rows needs 520 bytes per split).
+ * Set-up: the first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress and caches it; make that first call before any stream
+ * capture. All calls share the one array and it keeps the last call's contents:
+ * calls that overlap on the GPU (different streams, or threads) race and
+ * corrupt each other's results, so serialize them. Every call writes each
+ * scratch entry before reading it, so nothing needs clearing. */
+gear_status gear_decode_attn_noalloc(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq,
+                                     float softmax_scale, void* out, gear_dtype out_dtype, void* stream);
+
 /* Workspace bytes gear_append_buffer needs (covers the flush encode). */
 size_t gear_append_workspace_bytes(const gear_cache* k);
 

@@ -5,6 +5,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "decode.cuh"
 #include "encode.cuh"
@@ -339,3 +341,51 @@ const char* gear_status_string(gear_status s) {
 const char* gear_version(void) { return "0.1.0"; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-alloc decode
+// Decode attention for callers that cannot call cudaMalloc. The split-K
+// partial results live in a fixed array inside this library instead of a
+// caller-provided workspace. The array is a file-scope __device__ variable, so
+// every GPU that loads the library holds it (4 MiB) until the process exits.
+// Host code cannot pass the array's name to a kernel (in host code it is a
+// host-side stand-in), so its device address is looked up once per device
+// with cudaGetSymbolAddress and cached.
+namespace gear {
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+static std::mutex g_noalloc_mu;
+static float* g_noalloc_ptr[256];
+
+// Device address of the scratch array on the current device (nullptr on error).
+static float* noalloc_scratch_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    g_noalloc_ptr[dev] = reinterpret_cast<float*>(p);
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace gear
+
+extern "C" gear_status gear_decode_attn_noalloc(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq,
+                                                float softmax_scale, void* out, gear_dtype out_dtype, void* stream) {
+  DecodeArgs a;
+  gear_status s = decode_args(k, v, Hq, a);
+  if (s != GEAR_OK) return s;
+  if (!q || !out) return GEAR_ERR_INVALID_ARG;
+  if (out_dtype != k->dtype && out_dtype != GEAR_F32) return GEAR_ERR_INVALID_ARG;
+  if (!isfinite(softmax_scale)) return GEAR_ERR_INVALID_ARG;
+  if (decode_workspace_bytes(a.B, a.Hq, a.nsplit) > kNoAllocScratchBytes) return GEAR_ERR_WORKSPACE;
+  float* scratch = noalloc_scratch_for_current_device();
+  if (!scratch) return GEAR_ERR_CUDA;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.q = q;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  a.part = scratch;  // every split writes all of its partial row: nothing needs clearing
+  return cuda_status(decode_launch(a, (cudaStream_t)stream));
+}

@@ -64,6 +64,7 @@ def _load():
         "gear_encode": (i32, [pc, P, i32, P, S, P]),
         "gear_decode_workspace_bytes": (S, [pc, pc, i32]),
         "gear_decode_attn": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P, S, P]),
+        "gear_decode_attn_noalloc": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P]),
         "gear_append_workspace_bytes": (S, [pc]),
         "gear_append_buffer": (i32, [pc, pc, P, P, P, S, P]),
         "gear_decode_dense": (i32, [pc, P, P]),
