@@ -2,18 +2,18 @@
  * gear.h -- C ABI of the GEAR KV-cache codec for NVIDIA B200 (sm_100a).
  *
  * GEAR compresses a KV-cache matrix X (tokens x head_dim) into three parts
- * (GEAR: Efficient KV Cache Compression for LLM Inference, Q3 "How does the
- * paper solve the problem?"; GEAR: An Efficient KV Cache Compression Recipe
- * for Near-Lossless Generative Inference of LLM, Abstract):
- *   S  - a sparse set holding the largest-magnitude entries in full precision
- *        ("S = Filter_s(X)", Cites: SqueezeLLM entry);
+ * (GEAR: Efficient KV Cache Compression for LLM Inference, Q3 on the method;
+ * GEAR: An Efficient KV Cache Compression Recipe for Near-Lossless Generative
+ * Inference of LLM, Abstract):
+ *   S  - a sparse set holding the largest-magnitude entries exactly
+ *        (S = Filter_s(X); Cites list, SqueezeLLM entry);
  *   D  - a uniform, group-wise, per-token b-bit quantization of the rest
- *        (Cites: FlexGen entry, "Per-token group-wise quantization");
+ *        (Cites list, FlexGen entry);
  *   L.Rf^T - a rank-r approximation of the quantization residual, computed by
- *        power iteration (Q3 "low-rank approximation"; Cites: PowerSGD entry),
+ *        power iteration (Q3, low-rank part; Cites list, PowerSGD entry),
  * so that X ~ D + L.Rf^T with the outlier slots overwritten by S.
  * New tokens go to a small full-precision streaming buffer that is compressed
- * when it fills (Q3 "Streaming strategy").
+ * when it fills (Q3, streaming strategy).
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or torch-owned)
@@ -54,21 +54,21 @@ typedef enum { GEAR_F16 = 0, GEAR_BF16 = 1, GEAR_F32 = 2 } gear_dtype;
 
 /* Codec parameters -- the pages' statement of the problem.
  *  bits         b in {2, 4, 8}: code width of the quantized backbone
- *               (Q3: "ultra-low-precision quantization (for example, 4-bit)").
+ *               (Q3: very low precision such as 4 bits).
  *  group_size   g: channels per quantization group; g divides d and g*b is a
  *               multiple of 32 (Cites: FlexGen entry, fine-grained grouping).
  *  outlier_frac s in [0, 0.5]: fraction of each token's entries kept exactly;
- *               k = ceil(s*d - 1e-9) outliers per token (Cites: ZeroQuant
- *               entry, "sparsity ratio s at 2%").
+ *               k = ceil(s*d - 1e-9) outliers per token (Cites list,
+ *               ZeroQuant entry: the paper fixes s at 2 %).
  *  rank         r in [0, 16], r <= min(n, d): rank of the residual factors of
- *               a block written by gear_encode (ZeroQuant entry: r = 4 for
- *               prefill inputs).
+ *               a block written by gear_encode (ZeroQuant entry: the paper
+ *               uses 4 for prefill inputs).
  *  power_iters  T >= 1 when any rank > 0: power-iteration count, T counting
- *               (P, Q) update pairs (Cites: PowerSGD entry).
- *  buffer_len   n_b >= 1: streaming-buffer length (Q3 "Streaming strategy").
+ *               (P, Q) update pairs (Cites list, PowerSGD entry).
+ *  buffer_len   n_b >= 1: streaming-buffer length (Q3, streaming strategy).
  *  buffer_rank  r_buf in [0, 16], r_buf <= min(n_b, d): rank of each flushed
- *               buffer block (ZeroQuant entry: "rank to 2 for each group of
- *               n_b new tokens in decoding phase").
+ *               buffer block (ZeroQuant entry: the paper gives every group of
+ *               n_b decoded tokens rank 2).
  *  seed         seeds the power-iteration start matrix Q0 (d x r): entry
  *               (i, j) is the (i*r + j)-th output of the splitmix64 stream
  *               whose state starts at `seed` (Steele, Lea & Flood, OOPSLA
@@ -205,8 +205,8 @@ size_t gear_append_workspace_bytes(const gear_cache* k);
 /* Appends one token per unit, k_new/v_new [B][H][d] (cache dtype). If the
  * buffer already holds n_b tokens, they are first compressed as a new block
  * of rank buffer_rank (same codec as gear_encode) appended after the
- * compressed tokens, and the buffer is emptied (Q3 "Streaming strategy":
- * compression is triggered when the buffer fills). Then the new token is
+ * compressed tokens, and the buffer is emptied (Q3, streaming strategy: the
+ * buffer is compressed once it is full). Then the new token is
  * written to buffer slot n_buf. Errors: INVALID_ARG, CAPACITY, WORKSPACE, CUDA. */
 gear_status gear_append_buffer(gear_cache* k, gear_cache* v, const void* k_new,
                                const void* v_new, void* workspace, size_t ws_bytes,

@@ -2,7 +2,7 @@
 //
 // One query token per sequence attends to the n_comp compressed tokens and
 // the n_buf full-precision buffer tokens of its kv head (GEAR: Efficient KV
-// Cache Compression for LLM Inference, Q3 "Streaming strategy"; the compressed
+// Cache Compression for LLM Inference, Q3, streaming strategy; the compressed
 // entries are consumed as D + L Rf^T with the sparse outliers restored).
 // The reconstruction is never materialized: for a key token t of block b
 //   q . Khat_t = sum_g [ scale_tg * (sum_{c in g} code_tc q_c) + zero_tg * sum_{c in g} q_c ]

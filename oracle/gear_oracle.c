@@ -8,11 +8,11 @@
  * description, step by step, in the order the pages give it.
  *
  * Pages (cited by title and section):
- *   [summary] "GEAR: Efficient KV Cache Compression for LLM Inference",
- *             Q3 "How does the paper solve the problem?"
- *   [cites]   "GEAR: An Efficient KV Cache Compression Recipe for
- *             Near-Lossless Generative Inference of LLM", section "Cites"
- *             (verbatim sentences of the paper, listed under the cited work).
+ *   [summary] GEAR: Efficient KV Cache Compression for LLM Inference,
+ *             question Q3 (how the method works);
+ *   [cites]   GEAR: An Efficient KV Cache Compression Recipe for
+ *             Near-Lossless Generative Inference of LLM, the Cites list (the
+ *             paper's own sentences, filed under the work each one cites).
  *
  * Precision: the quantization decisions (outlier choice, min/max, scale,
  * codes, dequantized value, residual) are taken in IEEE binary32 with
@@ -28,10 +28,10 @@
 
 /* ------------------------------------------------------------------------ */
 /* Step 1: outlier extraction.                                               */
-/* [cites] SqueezeLLM entry: the largest-magnitude entries are kept "in full  */
-/* precision with a sparse matrix S = Filter_s(X)"; [cites] ZeroQuant entry:  */
-/* "we fix the sparsity ratio s at 2%". Reading: Filter_s acts per token and  */
-/* keeps k = ceil(s*d) entries (at least a fraction s is kept).               */
+/* [cites] SqueezeLLM entry: the entries of largest magnitude stay exact, held */
+/* as a sparse matrix S = Filter_s(X); [cites] ZeroQuant entry: the sparsity   */
+/* ratio s is fixed at 2 %. Reading: Filter_s acts per token and keeps         */
+/* k = ceil(s*d) entries (at least a fraction s is kept).                     */
 /* ------------------------------------------------------------------------ */
 int32_t oracle_num_outliers(float s, int32_t d) {
   double v = (double)s * (double)d - 1e-9;
@@ -62,10 +62,11 @@ void oracle_select_outliers(const float* x, int32_t d, int32_t k, int32_t* idx_o
 
 /* ------------------------------------------------------------------------ */
 /* Step 2: uniform group-wise quantization of the extracted matrix.          */
-/* [summary] Q3: "ultra-low-precision quantization (for example, 4-bit) to   */
-/* most KV cache entries"; [cites] SqueezeLLM entry: "we perform the          */
-/* quantization on the extracted matrix"; [cites] FlexGen entry: "quantizes   */
-/* KV cache per-token with fine-grained grouping". Reading: asymmetric        */
+/* [summary] Q3: the bulk of the entries, which have similar magnitudes, are  */
+/* quantized to very few bits (4, for instance); [cites] SqueezeLLM entry:    */
+/* the quantizer runs on the matrix left once the outliers are taken out;     */
+/* [cites] FlexGen entry: the quantizer groups channels finely within each    */
+/* token. Reading: asymmetric                                                 */
 /* min-max quantization (zero point = group minimum) over the non-outlier     */
 /* entries of each group of g channels of a token:                            */
 /*   scale = (mx - mn) / (2^b - 1)                                            */
@@ -94,6 +95,11 @@ void oracle_quantize_token(const float* x, int32_t d, int32_t bits, int32_t g,
       if (x[c] < mn) mn = x[c];
       if (x[c] > mx) mx = x[c];
     }
+    /* Reading: the zero point and the maximum are stored with -0 replaced by
+       +0 (v + 0.0f under round-to-nearest), so they do not depend on the order
+       in which +0 and -0 occur in the group. */
+    mn = mn + 0.0f;
+    mx = mx + 0.0f;
     float scale = (mx - mn) / (float)levels;
     scale_out[grp] = scale;
     zero_out[grp] = mn;
@@ -143,9 +149,9 @@ void oracle_start_matrix(uint64_t seed, int32_t d, int32_t r, double* q0) {
 
 /* ------------------------------------------------------------------------ */
 /* Step 5: low-rank approximation of the residual by power iteration.       */
-/* [summary] Q3: "Use a low-rank matrix to approximate the residual error    */
-/* introduced by quantization ... via singular value decomposition";        */
-/* [cites] PowerSGD entry (the power-iteration compressor the method cites). */
+/* [summary] Q3: a low-rank matrix, found by singular value decomposition,   */
+/* models the error that quantization leaves; [cites] PowerSGD entry: the   */
+/* method cites the power-iteration compressor, used here for the SVD.      */
 /* For t = 1..T:  P = orthonormalize(R Q),  Q = R^T P;  L = P_T, Rf = Q_T.   */
 /* Orthonormalization: modified Gram-Schmidt in binary64; a column whose     */
 /* norm after removing the earlier columns is at most 1e-10 of its norm      */
@@ -230,9 +236,9 @@ void oracle_encode_unit(const float* X, int32_t n, int32_t d, int32_t bits, int3
 
 /* ------------------------------------------------------------------------ */
 /* Step 6: reconstruction, X ~ D + L Rf^T with the outlier slots holding    */
-/* their exact values ([cites] LoftQ and Zafrir et al. entries: the         */
-/* low-rank part captures the coherent error, the sparse part "rectifies    */
-/* the incoherency existing in individual outliers").                        */
+/* their exact values ([cites] LoftQ and Zafrir et al. entries: the low-rank */
+/* part carries the error shared across entries, the sparse part fixes the  */
+/* individual outliers).                                                     */
 /* ------------------------------------------------------------------------ */
 void oracle_reconstruct_unit(int32_t n, int32_t d, int32_t bits, int32_t g, int32_t k,
                              int32_t r, const uint32_t* codes, const float* scale,

@@ -144,6 +144,19 @@ def test_quantization_invariants(bits, g, s):
     assert np.array_equal(u.resid[~out_mask], (x - dh32)[~out_mask])
 
 
+def test_signed_zero_minimum_is_stored_as_positive_zero():
+    # a group whose minimum is zero, with -0 before +0 and the reverse
+    x = np.abs(RNG.standard_normal((2, 128)).astype(np.float32)) + 0.5
+    x[0, 3], x[0, 9] = -0.0, 0.0
+    x[1, 3], x[1, 9] = 0.0, -0.0
+    x[:, 64:] = -0.0                      # second group all -0: scale and zero +0
+    p = Params(bits=4, group_size=64, outlier_frac=0.0, rank=0)
+    u = oracle.encode_unit(x, p)
+    assert np.all(u.zero.view(np.uint32) == 0)
+    assert np.all(u.scale[:, 1].view(np.uint32) == 0)
+    assert np.all(unpack_codes(u.codes, 128, 4)[:, [3, 9]] == 0)
+
+
 def test_all_outlier_group():
     # g = 32 with s = 0.5: k = 64 outliers can cover a whole group
     x = np.zeros((1, 128), np.float32)
