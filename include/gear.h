@@ -89,7 +89,7 @@ typedef struct gear_params {
  * up to n_max compressed tokens plus an n_b-token full-precision buffer.
  *
  * Filled by gear_cache_init(); the caller then treats it as opaque except for
- * reading the counters. The struct lives in HOST memory; the arrays it points
+ * reading the counters. n_max is stored rounded up to a multiple of 32 tokens. The struct lives in HOST memory; the arrays it points
  * to live in the caller's device buffer, laid out in this order, each array
  * starting on a 256-byte boundary:
  *

@@ -15,9 +15,12 @@ namespace gear {
 __device__ int32_t g_device_status = 0;
 
 static int current_sm_count() {
+  static int cached[256];
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 256 && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  if (dev >= 0 && dev < 256) cached[dev] = n;
   return n;
 }
 
@@ -29,8 +32,13 @@ struct Layout {
   size_t codes, meta, oidx, oval, lfac, rfac, buf, total;
 };
 
+// token capacity per unit, rounded up so that every 32-token tile of every
+// per-token array starts on a 16-byte boundary
+static int round_nmax(int n_max) { return (n_max + 31) & ~31; }
+
 static Layout cache_layout(const gear_params* p, int B, int H, int d, int n_max, int nblk_max, int dt) {
   Layout L;
+  n_max = round_nmax(n_max);
   const size_t U = (size_t)B * H;
   const int k = gear_num_outliers(p->outlier_frac, d);
   const int G = d / p->group_size;
@@ -172,11 +180,11 @@ gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int3
   if (B <= 0 || H <= 0 || n_max <= 0 || nblk_max <= 0 || dtype < GEAR_F16 || dtype > GEAR_F32)
     return GEAR_ERR_INVALID_ARG;
   if (!aligned(dev, 256)) return GEAR_ERR_INVALID_ARG;
-  if ((size_t)B * H * n_max >= ((size_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
+  if ((size_t)B * H * round_nmax(n_max) >= ((size_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
   Layout L = cache_layout(p, B, H, d, n_max, nblk_max, dtype);
   if (bytes < L.total) return GEAR_ERR_CAPACITY;
   memset(c, 0, sizeof(*c));
-  c->B = B; c->H = H; c->d = d; c->n_max = n_max; c->nblk_max = nblk_max; c->dtype = dtype;
+  c->B = B; c->H = H; c->d = d; c->n_max = round_nmax(n_max); c->nblk_max = nblk_max; c->dtype = dtype;
   c->p = *p;
   c->k = gear_num_outliers(p->outlier_frac, d);
   c->G = d / p->group_size;

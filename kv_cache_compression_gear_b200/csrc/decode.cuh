@@ -17,6 +17,11 @@ struct CacheView {
   const void* buf;
 };
 
+// Byte offsets of one tensor's 32-token tile in shared memory.
+struct TileLayout {
+  int32_t codes, meta, oidx, oval, lf, bytes;
+};
+
 struct DecodeArgs {
   CacheView K, V;
   int32_t dtype;          // cache dtype
@@ -30,9 +35,12 @@ struct DecodeArgs {
   void* out;              // [B][Hq][128] out dtype
   int32_t out_dtype;
   float* part;            // [B][Hq][nsplit][130] partial (m, l, acc[128])
-  int32_t chunk;          // compressed tokens per split
-  int32_t nsplit_comp;    // splits over compressed tokens
+  int32_t chunk;          // compressed tokens per split (whole 32-token tiles)
+  int32_t nsplit_comp;    // splits over compressed tokens, per unit
   int32_t nsplit;         // + 1 if the buffer is non-empty
+  int32_t total_splits;   // units * nsplit: one warp each
+  int32_t warp_bytes;     // shared memory per warp
+  TileLayout tl;
 };
 
 struct DenseArgs {

@@ -190,7 +190,8 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
   // key = |x| bits << 7 | (127 - c): larger key = larger |x|, ties to the lower
   // channel. Each thread keeps the top KMAX of its 64 keys with a branch-free
   // insertion network, then merges its partner's list (lane ^ 1).
-  uint64_t top[KMAX > 0 ? KMAX : 1];
+  using Key = typename std::conditional<sizeof(T) == 4, uint64_t, uint32_t>::type;
+  Key top[KMAX > 0 ? KMAX : 1];
   int cidx[KMAX > 0 ? KMAX : 1];
   uint32_t oval_bits[KMAX > 0 ? KMAX : 1];
   if constexpr (KMAX > 0) {
@@ -199,32 +200,32 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     const uint32_t tb0 = 127u - 64u * h;
 #pragma unroll
     for (int e = 0; e < 64; ++e) {
-      uint64_t key;
+      Key key;
       if constexpr (sizeof(T) == 4) {
         key = ((uint64_t)(xr[e] & 0x7FFFFFFFu) << 7) | (tb0 - e);
       } else {
         uint32_t p = xr[e >> 1];
         uint32_t ab = (e & 1) ? ((p >> 16) & 0x7FFFu) : (p & 0x7FFFu);
-        key = (uint64_t)((ab << 7) | (tb0 - e));
+        key = (ab << 7) | (tb0 - e);
       }
       if (!valid) key = 0;
 #pragma unroll
       for (int i = 0; i < KMAX; ++i) {
-        uint64_t hi = key > top[i] ? key : top[i];
+        Key hi = key > top[i] ? key : top[i];
         key = key > top[i] ? top[i] : key;
         top[i] = hi;
       }
     }
     // snapshot the partner's list before either lane modifies its own
-    uint64_t other[KMAX];
+    Key other[KMAX];
 #pragma unroll
     for (int i = 0; i < KMAX; ++i) other[i] = __shfl_xor_sync(0xFFFFFFFFu, top[i], 1);
 #pragma unroll
     for (int i = 0; i < KMAX; ++i) {
-      uint64_t key = other[i];
+      Key key = other[i];
 #pragma unroll
       for (int m = 0; m < KMAX; ++m) {
-        uint64_t hi = key > top[m] ? key : top[m];
+        Key hi = key > top[m] ? key : top[m];
         key = key > top[m] ? top[m] : key;
         top[m] = hi;
       }
@@ -566,11 +567,14 @@ __global__ void __launch_bounds__(kE1Threads, 1)
 }
 
 // ================================================================ E2 ======
-// Per unit: M = sym(sum of partial Grams) in fp64, then T power steps with
+// Per unit: M = sym(sum of partial Grams), then T power steps with
 // Cholesky-QR on the r x r Gram. Outputs Rf (cache, scaled 2^-e) and
 // Z = Q_{T-1} C_T^-1 scaled 2^e (workspace) so that E3's R Z is the stored L.
+// The partials arrive by 64 KiB bulk asynchronous copies, two in flight, and
+// are summed in a fixed order (deterministic); M is kept in fp32 (the
+// partials carry about 17 significant bits), products accumulate in fp64.
 constexpr int kE2Threads = 256;
-constexpr int kMStride = 129;  // padded row (doubles) for conflict-free column reads
+constexpr int kMStride = 132;  // padded fp32 row of M
 
 __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t i) {
   // output number i (0-based) of the splitmix64 stream whose state starts at seed
@@ -580,119 +584,207 @@ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t i) {
   return z ^ (z >> 31);
 }
 
-__global__ void __launch_bounds__(kE2Threads) encode_power(const EncodeArgs a) {
-  extern __shared__ double sm2[];
-  double* M = sm2;                          // [128][129]
-  double* Q = M + 128 * kMStride;           // [128][16]
-  double* Wm = Q + 128 * 16;                // [128][16]
-  double* Gm = Wm + 128 * 16;               // [16][16]
-  double* Xi = Gm + 256;                    // [16][16] inverse Cholesky factor
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int RM>
+struct E2Smem {
+  float M[128 * kMStride];
+  double Q[128 * RM];
+  uint64_t bar[2];
+  union {
+    float stage[2][16384];   // partial Grams in flight (phase 1)
+    struct {                 // power-iteration scratch (phase 2)
+      double Wp[2 * 128 * RM];
+      double red[4 * RM * RM];
+      double Xi[RM * RM];
+    } it;
+  } u;
+};
+
+template <int RM>
+__global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a) {
+  extern __shared__ __align__(128) uint8_t sm2raw[];
+  E2Smem<RM>& S = *reinterpret_cast<E2Smem<RM>*>(sm2raw);
   const int u = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = a.r;
   const int64_t total = a.total_tiles, grid = a.grid_e1;
   const int64_t c0 = seg_first_cta((int64_t)u * a.tpu, grid, total);
   const int64_t c1 = seg_first_cta((int64_t)u * a.tpu + a.tpu - 1, grid, total);
   const int nseg = (int)(c1 - c0 + 1);
+  const float* part = a.gram + (int64_t)u * a.maxc * 16384;
 
-  // sum partials in a fixed order
-  for (int e = tid; e < 128 * 128; e += kE2Threads) {
-    double acc = 0.0;
-    const float* src = a.gram + (int64_t)u * a.maxc * 16384 + e;
-    for (int s = 0; s < nseg; ++s) acc += (double)src[(int64_t)s * 16384];
-    M[(e >> 7) * kMStride + (e & 127)] = acc;
-  }
-  // Q0 from the seed
-  for (int e = tid; e < 128 * r; e += kE2Threads) {
-    uint64_t z = splitmix64_at(a.seed, (uint64_t)e);
-    Q[(e / r) * 16 + (e % r)] = (double)(uint32_t)(z >> 40) * 0x1p-23 - 1.0;
-  }
-  __syncthreads();
-  for (int e = tid; e < 128 * 128; e += kE2Threads) {
-    int i = e >> 7, j = e & 127;
-    if (i < j) {
-      double m = 0.5 * (M[i * kMStride + j] + M[j * kMStride + i]);
-      M[i * kMStride + j] = m;
-      M[j * kMStride + i] = m;
+  if (tid == 0) {
+    mbar_init(&S.bar[0], 1);
+    mbar_init(&S.bar[1], 1);
+    fence_mbarrier_init();
+    for (int sg = 0; sg < 2 && sg < nseg; ++sg) {
+      mbar_arrive_expect_tx(&S.bar[sg], 65536);
+      bulk_load(S.u.stage[sg], part + (int64_t)sg * 16384, 65536, &S.bar[sg]);
     }
   }
+  // Q0 from the seed (columns r .. RM-1 stay zero)
+  for (int e = tid; e < 128 * RM; e += kE2Threads) {
+    const int i = e / RM, j = e % RM;
+    double v = 0.0;
+    if (j < r) {
+      const uint64_t z = splitmix64_at(a.seed, (uint64_t)(i * r + j));
+      v = (double)(uint32_t)(z >> 40) * 0x1p-23 - 1.0;
+    }
+    S.Q[e] = v;
+  }
   __syncthreads();
-
-  for (int it = 0; it < a.T; ++it) {
-    // W = M Q
-    for (int e = tid; e < 128 * r; e += kE2Threads) {
-      int i = e / r, j = e % r;
-      double acc = 0.0;
-      for (int c = 0; c < 128; ++c) acc += M[c * kMStride + i] * Q[c * 16 + j];
-      Wm[i * 16 + j] = acc;
+  bool ok = true;
+  for (int sg = 0; sg < nseg; ++sg) {
+    const int b = sg & 1;
+    ok = mbar_wait(&S.bar[b], (sg >> 1) & 1) && ok;
+    for (int e4 = tid; e4 < 4096; e4 += kE2Threads) {
+      const float4 v = reinterpret_cast<const float4*>(S.u.stage[b])[e4];
+      float* dst = &S.M[(e4 >> 5) * kMStride + ((e4 & 31) << 2)];
+      if (sg == 0) {
+        dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+      } else {
+        dst[0] += v.x; dst[1] += v.y; dst[2] += v.z; dst[3] += v.w;
+      }
     }
     __syncthreads();
-    // G = Q^T W
-    for (int e = tid; e < r * r; e += kE2Threads) {
-      int p = e / r, q = e % r;
-      double acc = 0.0;
-      for (int i = 0; i < 128; ++i) acc += Q[i * 16 + p] * Wm[i * 16 + q];
-      Gm[p * 16 + q] = acc;
+    if (tid == 0 && sg + 2 < nseg) {
+      mbar_arrive_expect_tx(&S.bar[b], 65536);
+      bulk_load(S.u.stage[b], part + (int64_t)(sg + 2) * 16384, 65536, &S.bar[b]);
+    }
+  }
+  (void)ok;
+  for (int e = tid; e < 128 * 128; e += kE2Threads) {
+    const int i = e >> 7, j = e & 127;
+    if (i < j) {
+      const float mv = 0.5f * (S.M[i * kMStride + j] + S.M[j * kMStride + i]);
+      S.M[i * kMStride + j] = mv;
+      S.M[j * kMStride + i] = mv;
+    }
+  }
+  __syncthreads();
+
+  const int i = tid & 127, half = tid >> 7;
+  for (int step = 0; step < a.T; ++step) {
+    // W = M Q: two threads per row, each over 64 of the 128 channels
+    {
+      double w[RM];
+#pragma unroll
+      for (int j = 0; j < RM; ++j) w[j] = 0.0;
+#pragma unroll 8
+      for (int c = half * 64; c < half * 64 + 64; ++c) {
+        const double mv = (double)S.M[c * kMStride + i];
+#pragma unroll
+        for (int j = 0; j < RM; ++j) w[j] = fma(mv, S.Q[c * RM + j], w[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < RM; ++j) S.u.it.Wp[(half * 128 + i) * RM + j] = w[j];
+    }
+    __syncthreads();
+    // G = Q^T W (upper triangle), reduced by warp then across warps
+    if (tid < 128) {
+      double w[RM], qv[RM];
+#pragma unroll
+      for (int j = 0; j < RM; ++j) {
+        w[j] = S.u.it.Wp[i * RM + j] + S.u.it.Wp[(128 + i) * RM + j];
+        qv[j] = S.Q[i * RM + j];
+      }
+#pragma unroll
+      for (int j = 0; j < RM; ++j) S.u.it.Wp[i * RM + j] = w[j];
+#pragma unroll
+      for (int p = 0; p < RM; ++p)
+#pragma unroll
+        for (int q = p; q < RM; ++q) {
+          double v = qv[p] * w[q];
+          for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+          if (lane == 0) S.u.it.red[(warp * RM + p) * RM + q] = v;
+        }
     }
     __syncthreads();
     if (tid == 0) {
       // Cholesky G = C^T C (upper C) with column dropping, then X = C^-1 so
-      // that P~ X has orthonormal (or zero) columns.
-      double Cm[16][16];
-      bool nz[16];
-      for (int j = 0; j < r; ++j) {
-        for (int m = 0; m < j; ++m) {
-          double v = 0.0;
-          if (nz[m]) {
-            v = Gm[m * 16 + j];
-            for (int i = 0; i < m; ++i) v -= Cm[i][m] * Cm[i][j];
-            v /= Cm[m][m];
-          }
-          Cm[m][j] = v;
+      // that P~ X has orthonormal (or zero) columns. All indices are
+      // compile-time, so C and X stay in registers.
+      double C[RM][RM], X[RM][RM];
+      bool nz[RM];
+#pragma unroll
+      for (int p = 0; p < RM; ++p)
+#pragma unroll
+        for (int q = 0; q < RM; ++q) {
+          double g = 0.0;
+          if (p <= q) g = S.u.it.red[p * RM + q] + S.u.it.red[(RM + p) * RM + q] + S.u.it.red[(2 * RM + p) * RM + q] +
+                          S.u.it.red[(3 * RM + p) * RM + q];
+          C[p][q] = g;
+          X[p][q] = 0.0;
         }
-        double gjj = Gm[j * 16 + j];
+#pragma unroll
+      for (int j = 0; j < RM; ++j) {
+        const double gjj = C[j][j];
+#pragma unroll
+        for (int m2 = 0; m2 < j; ++m2) {
+          double v = C[m2][j];
+#pragma unroll
+          for (int i2 = 0; i2 < m2; ++i2) v -= C[i2][m2] * C[i2][j];
+          C[m2][j] = nz[m2] ? v / C[m2][m2] : 0.0;
+        }
         double piv = gjj;
-        for (int m = 0; m < j; ++m) piv -= Cm[m][j] * Cm[m][j];
-        nz[j] = gjj > 0.0 && piv > 1e-10 * gjj;
-        Cm[j][j] = nz[j] ? sqrt(piv) : 0.0;
+#pragma unroll
+        for (int m2 = 0; m2 < j; ++m2) piv -= C[m2][j] * C[m2][j];
+        nz[j] = j < r && gjj > 0.0 && piv > 1e-10 * gjj;
+        C[j][j] = nz[j] ? sqrt(piv) : 1.0;
       }
-      for (int j = 0; j < r; ++j) {
-        for (int i = 0; i < r; ++i) Xi[i * 16 + j] = 0.0;
-        if (!nz[j]) continue;
-        // column j of C^-1: (e_j - sum_{m<j} C[m][j] X[:, m]) / C[j][j]
-        for (int i = 0; i < r; ++i) {
-          double v = (i == j) ? 1.0 : 0.0;
-          for (int m = 0; m < j; ++m) v -= Cm[m][j] * Xi[i * 16 + m];
-          Xi[i * 16 + j] = v / Cm[j][j];
+#pragma unroll
+      for (int j = 0; j < RM; ++j) {
+        const double inv = nz[j] ? 1.0 / C[j][j] : 0.0;
+#pragma unroll
+        for (int i2 = 0; i2 <= j; ++i2) {
+          double v = (i2 == j) ? 1.0 : 0.0;
+#pragma unroll
+          for (int m2 = 0; m2 < j; ++m2) v -= C[m2][j] * X[i2][m2];
+          X[i2][j] = v * inv;
         }
       }
+#pragma unroll
+      for (int p = 0; p < RM; ++p)
+#pragma unroll
+        for (int q = 0; q < RM; ++q) S.u.it.Xi[p * RM + q] = X[p][q];
     }
     __syncthreads();
-    const bool last = (it + 1 == a.T);
-    // next Q = W X, or on the last step Z = Q X and Rf = W X
-    double zq[16], wq[16];
-    const int i = tid;
-    if (i < 128) {
-      for (int j = 0; j < r; ++j) {
-        double sq = 0.0, sw = 0.0;
-        for (int m = 0; m < r; ++m) {
-          sq += Q[i * 16 + m] * Xi[m * 16 + j];
-          sw += Wm[i * 16 + m] * Xi[m * 16 + j];
+    const bool last = (step + 1 == a.T);
+    if (tid < 128) {
+      double zq[RM], wq[RM];
+#pragma unroll
+      for (int j = 0; j < RM; ++j) {
+        double sq = 0.0, swv = 0.0;
+#pragma unroll
+        for (int m2 = 0; m2 < RM; ++m2) {
+          sq = fma(S.Q[i * RM + m2], S.u.it.Xi[m2 * RM + j], sq);
+          swv = fma(S.u.it.Wp[i * RM + m2], S.u.it.Xi[m2 * RM + j], swv);
         }
         zq[j] = sq;
-        wq[j] = sw;
+        wq[j] = swv;
       }
-    }
-    __syncthreads();
-    if (i < 128) {
       if (!last) {
-        for (int j = 0; j < r; ++j) Q[i * 16 + j] = wq[j];
+        // row i is read and written by this thread only
+#pragma unroll
+        for (int j = 0; j < RM; ++j) S.Q[i * RM + j] = wq[j];
       } else {
         const double sL = ldexp(1.0, a.e_blk), sR = ldexp(1.0, -a.e_blk);
-        for (int j = 0; j < 16; ++j)
-          a.zbuf[((int64_t)u * 128 + i) * 16 + j] = j < r ? (float)(zq[j] * sL) : 0.0f;
-        for (int j = 0; j < a.r_max; ++j)
-          a.rfac[(((int64_t)u * a.nblk_max + a.blk) * a.r_max + j) * 128 + i] = j < r ? (float)(wq[j] * sR) : 0.0f;
+        float* zrow = a.zbuf + ((int64_t)u * 128 + i) * 16;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) zrow[j] = (j < RM && j < r) ? (float)(zq[j < RM ? j : 0] * sL) : 0.0f;
+        for (int j = 0; j < a.r_max; ++j) {
+          double wv = 0.0;
+#pragma unroll
+          for (int jj = 0; jj < RM; ++jj) if (jj == j) wv = wq[jj];
+          a.rfac[(((int64_t)u * a.nblk_max + a.blk) * a.r_max + j) * 128 + i] = j < r ? (float)(wv * sR) : 0.0f;
+        }
       }
     }
     __syncthreads();
@@ -702,80 +794,107 @@ __global__ void __launch_bounds__(kE2Threads) encode_power(const EncodeArgs a) {
 // ================================================================ E3 ======
 // L rows: L_t = R_t Z, with R rebuilt from the stored codes and zero points:
 // R = x - fma(code, scale, zero) on every slot, then the outlier slots'
-// contribution (x_o - zero) Z[c_o] is removed again. One tile of 128 tokens
-// per CTA, two threads per token.
-constexpr int kE3Threads = 256;
+// contribution (x_o - zero) Z[c_o] is removed again. Each thread takes two
+// tokens (t, t + 64) of a 128-token tile, so every Z entry, duplicated in
+// shared memory, feeds one packed two-token FMA.
+constexpr int kE3Threads = 64;
 
-template <typename T, int BITS>
+template <typename T, int BITS, int RMAX>
 __global__ void __launch_bounds__(kE3Threads) encode_lowrank(const EncodeArgs a) {
-  __shared__ float Zs[128][16];
+  __shared__ __align__(16) float Zd[128][RMAX][2];
   const int u = blockIdx.y;
-  const int r = a.r;
-  for (int e = threadIdx.x; e < 128 * 16; e += kE3Threads)
-    Zs[e >> 4][e & 15] = a.zbuf[((int64_t)u * 128 + (e >> 4)) * 16 + (e & 15)];
-  __syncthreads();
-  const int t = blockIdx.x * kTile + (threadIdx.x >> 1);
-  const int h = threadIdx.x & 1;
-  if (t >= a.n) return;
-  const size_t row = (size_t)u * a.n_max + (size_t)(a.t_off + t);
-  const uint8_t* xin = reinterpret_cast<const uint8_t*>(a.kv) + ((size_t)u * a.n + t) * 128 * sizeof(T);
-  constexpr int kWordsHalf = 64 * BITS / 32;
-  constexpr int kCodesPerWord = 32 / BITS;
-  const uint32_t* cw = a.codes + row * a.W + h * kWordsHalf;
-  uint32_t words[kWordsHalf];
-#pragma unroll
-  for (int w = 0; w < kWordsHalf; w += 4) {
-    uint4 v = *reinterpret_cast<const uint4*>(cw + w);
-    words[w] = v.x; words[w + 1] = v.y; words[w + 2] = v.z; words[w + 3] = v.w;
+  for (int e = threadIdx.x; e < 128 * RMAX; e += kE3Threads) {
+    const float z = a.zbuf[((int64_t)u * 128 + e / RMAX) * 16 + e % RMAX];
+    Zd[e / RMAX][e % RMAX][0] = z;
+    Zd[e / RMAX][e % RMAX][1] = z;
   }
-  const float2* meta = reinterpret_cast<const float2*>(a.meta) + row * a.G;
-  float acc[16];
+  __syncthreads();
+  constexpr int kCpw = 32 / BITS;
+  const int ta = blockIdx.x * kTile + threadIdx.x;
+  const int tb = ta + 64;
+  const bool va = ta < a.n, vb = tb < a.n;
+  if (!va) return;
+  const int tbx = vb ? tb : ta;   // a missing second token repeats the first
+  const size_t rowa = (size_t)u * a.n_max + (size_t)(a.t_off + ta);
+  const size_t rowb = (size_t)u * a.n_max + (size_t)(a.t_off + tbx);
+  const uint8_t* xa = reinterpret_cast<const uint8_t*>(a.kv) + ((size_t)u * a.n + ta) * 128 * sizeof(T);
+  const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.kv) + ((size_t)u * a.n + tbx) * 128 * sizeof(T);
+  const float2* ma = reinterpret_cast<const float2*>(a.meta) + rowa * a.G;
+  const float2* mb = reinterpret_cast<const float2*>(a.meta) + rowb * a.G;
+  uint64_t acc[RMAX];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-  constexpr int kVec = 16 / sizeof(T);
+  for (int j = 0; j < RMAX; ++j) acc[j] = 0;
+  const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
+  constexpr int kVec = 16 / sizeof(T);   // elements per 16-byte load
+#pragma unroll 2
+  for (int c0 = 0; c0 < 128; c0 += 8) {
+    // 8 channels of both tokens
+    float xv[2][8];
 #pragma unroll
-  for (int j = 0; j < 64 / kVec; ++j) {
-    uint4 v = *reinterpret_cast<const uint4*>(xin + (h * 64 + j * kVec) * sizeof(T));
-    uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+    for (int q = 0; q < 8 / kVec; ++q) {
+      const uint4 va4 = *reinterpret_cast<const uint4*>(xa + (c0 + q * kVec) * sizeof(T));
+      const uint4 vb4 = *reinterpret_cast<const uint4*>(xb + (c0 + q * kVec) * sizeof(T));
+      const uint32_t wa[4] = {va4.x, va4.y, va4.z, va4.w}, wb[4] = {vb4.x, vb4.y, vb4.z, vb4.w};
 #pragma unroll
-    for (int e = 0; e < kVec; ++e) {
-      const int cl = j * kVec + e;            // channel within the half
-      const int c = h * 64 + cl;
-      float x;
-      if constexpr (sizeof(T) == 4) x = __uint_as_float(vv[e]);
-      else x = Elem16<T>::lo(sizeof(T) == 2 ? (e & 1 ? vv[e >> 1] >> 16 : vv[e >> 1] & 0xFFFFu) : 0u);
-      const float2 sz = meta[c / a.g];
-      const uint32_t code = (words[cl / kCodesPerWord] >> (BITS * (cl % kCodesPerWord))) & ((1u << BITS) - 1u);
-      const float dh = __fmaf_rn((float)code, sz.x, sz.y);
-      const float rr = __fsub_rn(x, dh);
+      for (int e = 0; e < kVec; ++e) {
+        if constexpr (sizeof(T) == 4) {
+          xv[0][q * kVec + e] = __uint_as_float(wa[e]);
+          xv[1][q * kVec + e] = __uint_as_float(wb[e]);
+        } else {
+          const uint32_t pa = wa[e >> 1], pb = wb[e >> 1];
+          xv[0][q * kVec + e] = Elem16<T>::lo((e & 1) ? (pa >> 16) : (pa & 0xFFFFu));
+          xv[1][q * kVec + e] = Elem16<T>::lo((e & 1) ? (pb >> 16) : (pb & 0xFFFFu));
+        }
+      }
+    }
+    const float2 sa = ma[c0 >> lg], sb = mb[c0 >> lg];
+    const uint64_t sc2 = f2_pack(sa.x, sb.x), zr2 = f2_pack(sa.y, sb.y);
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (q < r) acc[q] = __fmaf_rn(rr, Zs[c][q], acc[q]);
+    for (int e = 0; e < 8; ++e) {
+      const int c = c0 + e;
+      const uint32_t wa = a.codes[rowa * a.W + c / kCpw], wb = a.codes[rowb * a.W + c / kCpw];
+      const uint32_t sh = BITS * (c % kCpw), msk = (1u << BITS) - 1u;
+      const uint64_t cf = f2_sub(f2_pack(__uint_as_float(((wa >> sh) & msk) | 0x4B000000u),
+                                         __uint_as_float(((wb >> sh) & msk) | 0x4B000000u)),
+                                 f2_pack(8388608.0f, 8388608.0f));
+      const uint64_t dh = f2_fma(cf, sc2, zr2);
+      const uint64_t rr = f2_sub(f2_pack(xv[0][e], xv[1][e]), dh);
+#pragma unroll
+      for (int j = 0; j < RMAX; j += 2) {
+        const float4 z = *reinterpret_cast<const float4*>(&Zd[c][j][0]);
+        acc[j] = f2_fma(rr, f2_pack(z.x, z.y), acc[j]);
+        acc[j + 1] = f2_fma(rr, f2_pack(z.z, z.w), acc[j + 1]);
+      }
     }
   }
   // outlier slots: their residual is zero; remove what the loop added
   const int k = a.k;
-  for (int i = 0; i < k; ++i) {
-    const int c = a.oidx[row * k + i];
-    if ((c >> 6) != h) continue;
-    float x;
-    if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(a.oval)[row * k + i];
-    else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(a.oval)[row * k + i]);
-    const float2 sz = meta[c / a.g];
-    const float rr = __fsub_rn(x, __fmaf_rn(0.0f, sz.x, sz.y));
+  for (int side = 0; side < 2; ++side) {
+    const size_t row = side ? rowb : rowa;
+    const float2* mt = side ? mb : ma;
+    for (int i = 0; i < k; ++i) {
+      const int c = a.oidx[row * k + i];
+      float x;
+      if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(a.oval)[row * k + i];
+      else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(a.oval)[row * k + i]);
+      const float rr = __fsub_rn(x, __fmaf_rn(0.0f, mt[c >> lg].x, mt[c >> lg].y));
 #pragma unroll
-    for (int q = 0; q < 16; ++q)
-      if (q < r) acc[q] = __fmaf_rn(-rr, Zs[c][q], acc[q]);
+      for (int j = 0; j < RMAX; ++j) {
+        const uint64_t mask = side ? f2_pack(0.0f, rr * Zd[c][j][0]) : f2_pack(rr * Zd[c][j][0], 0.0f);
+        acc[j] = f2_sub(acc[j], mask);
+      }
+    }
   }
-#pragma unroll
-  for (int q = 0; q < 16; ++q) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], 1);
-  if (h == 0) {
+  for (int side = 0; side < (vb ? 2 : 1); ++side) {
+    const size_t row = side ? rowb : rowa;
     for (int q = 0; q < a.r_max; ++q) {
-      const float v = q < r ? acc[q] : 0.0f;
-      if constexpr (sizeof(T) == 4)
-        reinterpret_cast<float*>(a.lfac)[row * a.r_max + q] = v;
-      else
-        reinterpret_cast<__half*>(a.lfac)[row * a.r_max + q] = __float2half_rn(v);
+      float v = 0.0f;
+#pragma unroll
+      for (int j = 0; j < RMAX; ++j)
+        if (j == q) v = side ? f2_hi(acc[j]) : f2_lo(acc[j]);
+      if (q >= a.r) v = 0.0f;
+      if constexpr (sizeof(T) == 4) reinterpret_cast<float*>(a.lfac)[row * a.r_max + q] = v;
+      else reinterpret_cast<__half*>(a.lfac)[row * a.r_max + q] = __float2half_rn(v);
     }
   }
 }
@@ -784,8 +903,12 @@ __global__ void __launch_bounds__(kE3Threads) encode_lowrank(const EncodeArgs a)
 template <typename T, int BITS, int KMAX>
 static cudaError_t launch_e1(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
   auto kern = encode_quant_gram<T, BITS, KMAX>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, E1Cfg<T>::kSmem);
-  if (e != cudaSuccess) return e;
+  static bool configured = false;   // the attribute persists for the process
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, E1Cfg<T>::kSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
   kern<<<grid, kE1Threads, E1Cfg<T>::kSmem, st>>>(map, a);
   return cudaGetLastError();
 }
@@ -793,6 +916,7 @@ static cudaError_t launch_e1(const CUtensorMap& map, const EncodeArgs& a, int gr
 template <typename T, int BITS>
 static cudaError_t launch_e1_k(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
   if (a.k == 0) return launch_e1<T, BITS, 0>(map, a, grid, st);
+  if (a.k == 3) return launch_e1<T, BITS, 3>(map, a, grid, st);
   if (a.k <= 4) return launch_e1<T, BITS, 4>(map, a, grid, st);
   if (a.k <= 8) return launch_e1<T, BITS, 8>(map, a, grid, st);
   return launch_e1<T, BITS, 16>(map, a, grid, st);
@@ -807,13 +931,20 @@ static cudaError_t launch_e1_b(const CUtensorMap& map, const EncodeArgs& a, int 
   }
 }
 
+template <typename T, int BITS>
+static void launch_e3_r(const EncodeArgs& a, dim3 grid, cudaStream_t st) {
+  if (a.r <= 4) encode_lowrank<T, BITS, 4><<<grid, kE3Threads, 0, st>>>(a);
+  else if (a.r <= 8) encode_lowrank<T, BITS, 8><<<grid, kE3Threads, 0, st>>>(a);
+  else encode_lowrank<T, BITS, 16><<<grid, kE3Threads, 0, st>>>(a);
+}
+
 template <typename T>
 static cudaError_t launch_e3_b(const EncodeArgs& a, cudaStream_t st) {
   dim3 grid(a.tpu, a.U);
   switch (a.bits) {
-    case 2: encode_lowrank<T, 2><<<grid, kE3Threads, 0, st>>>(a); break;
-    case 4: encode_lowrank<T, 4><<<grid, kE3Threads, 0, st>>>(a); break;
-    default: encode_lowrank<T, 8><<<grid, kE3Threads, 0, st>>>(a); break;
+    case 2: launch_e3_r<T, 2>(a, grid, st); break;
+    case 4: launch_e3_r<T, 4>(a, grid, st); break;
+    default: launch_e3_r<T, 8>(a, grid, st); break;
   }
   return cudaGetLastError();
 }
@@ -873,11 +1004,20 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if (a.r == 0) return cudaSuccess;
 
-  const size_t sm2 = (128 * kMStride + 128 * 16 * 2 + 256 * 2) * sizeof(double);
-  e = cudaFuncSetAttribute(encode_power, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-  if (e != cudaSuccess) return e;
-  encode_power<<<a.U, kE2Threads, sm2, st>>>(a);
-  e = cudaGetLastError();
+  {
+    const int RM = a.r <= 4 ? 4 : (a.r <= 8 ? 8 : 16);
+    const size_t sm2 = RM == 4 ? sizeof(E2Smem<4>) : (RM == 8 ? sizeof(E2Smem<8>) : sizeof(E2Smem<16>));
+    auto kern = RM == 4 ? encode_power<4> : (RM == 8 ? encode_power<8> : encode_power<16>);
+    static bool configured[3] = {false, false, false};
+    const int ci = RM == 4 ? 0 : (RM == 8 ? 1 : 2);
+    if (!configured[ci]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+      if (e != cudaSuccess) return e;
+      configured[ci] = true;
+    }
+    kern<<<a.U, kE2Threads, sm2, st>>>(a);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   if (a.dtype == GEAR_F16) return launch_e3_b<__half>(a, st);
   if (a.dtype == GEAR_BF16) return launch_e3_b<__nv_bfloat16>(a, st);
