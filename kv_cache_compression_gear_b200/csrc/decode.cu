@@ -91,57 +91,66 @@ struct CodeFloats {
   }
 };
 
-template <int BITS>
-__device__ __forceinline__ void stage_codes_async(const uint32_t* codes, uint8_t* dst, size_t row0, int lane) {
-  constexpr int W = 4 * BITS;           // code words per token (d = 128)
-  constexpr int kCpr = W / 4;           // 16-byte chunks per token row
-  constexpr int kStride = (W + 4) * 4;  // padded row in shared memory
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(codes + row0 * W);
-#pragma unroll
-  for (int ci = lane; ci < kDTile * kCpr; ci += 32) {
-    const int t = ci / kCpr, jj = ci % kCpr;
-    cp_async16(dst + t * kStride + jj * 16, src + (size_t)t * W * 4 + jj * 16);
-  }
-}
-
-// Stage one tensor's tokens [t0, t0 + nt) of unit u into `dst` (layout a.tl).
-// Whole, 32-aligned tiles use 16-byte asynchronous copies; others plain loads.
+// Stages 32-token tiles of one compressed tensor of one split. The per-token
+// arrays of the split's first token are located once; a tile then only adds
+// its token offset. Whole, 32-aligned tiles use 16-byte asynchronous copies
+// (every region of such a tile is a multiple of 16 bytes and 16-byte
+// aligned); other tiles (block tails) use plain loads.
 template <typename T, int BITS>
-__device__ __forceinline__ void stage_tensor(const DecodeArgs& a, const CacheView& cv, uint8_t* dst, int u, int t0,
-                                             int nt, bool async, int lane) {
-  constexpr int W = 4 * BITS;
-  constexpr int kStride = (W + 4) * 4;
-  const TileLayout& L = a.tl;
-  const size_t row0 = (size_t)u * a.n_max + t0;
-  const int G = a.G, k = a.k, rm = a.r_max;
-  constexpr int lsz = sizeof(T) == 4 ? 4 : 2;
-  if (async) {
-    stage_codes_async<BITS>(cv.codes, dst + L.codes, row0, lane);
-    const uint8_t* m = reinterpret_cast<const uint8_t*>(cv.meta) + row0 * G * 8;
-    for (int off = lane * 16; off < kDTile * G * 8; off += 512) cp_async16(dst + L.meta + off, m + off);
-    if (k > 0) {
-      const uint8_t* oi = cv.oidx + row0 * k;
-      for (int off = lane * 16; off < kDTile * k; off += 512) cp_async16(dst + L.oidx + off, oi + off);
-      const uint8_t* ov = reinterpret_cast<const uint8_t*>(cv.oval) + row0 * k * sizeof(T);
-      for (int off = lane * 16; off < (int)(kDTile * k * sizeof(T)); off += 512) cp_async16(dst + L.oval + off, ov + off);
-    }
-    const uint8_t* lf = reinterpret_cast<const uint8_t*>(cv.lfac) + row0 * rm * lsz;
-    for (int off = lane * 16; off < kDTile * rm * lsz; off += 512) cp_async16(dst + L.lf + off, lf + off);
-  } else {
-    for (int e = lane; e < nt * W; e += 32)
-      reinterpret_cast<uint32_t*>(dst + L.codes + (e / W) * kStride)[e % W] = cv.codes[row0 * W + e];
-    for (int e = lane; e < nt * G; e += 32)
-      reinterpret_cast<float2*>(dst + L.meta)[e] = reinterpret_cast<const float2*>(cv.meta)[row0 * G + e];
-    for (int e = lane; e < nt * k; e += 32) {
-      dst[L.oidx + e] = cv.oidx[row0 * k + e];
-      reinterpret_cast<T*>(dst + L.oval)[e] = reinterpret_cast<const T*>(cv.oval)[row0 * k + e];
-    }
-    for (int e = lane; e < nt * rm; e += 32) {
-      if (lsz == 4) reinterpret_cast<float*>(dst + L.lf)[e] = reinterpret_cast<const float*>(cv.lfac)[row0 * rm + e];
-      else reinterpret_cast<uint16_t*>(dst + L.lf)[e] = reinterpret_cast<const uint16_t*>(cv.lfac)[row0 * rm + e];
+struct Stager {
+  static constexpr int W = 4 * BITS;           // code words per token (d = 128)
+  static constexpr int kCpr = W / 4;           // 16-byte chunks per code row
+  static constexpr int kStride = (W + 4) * 4;  // padded code row in shared memory
+  static constexpr int lsz = sizeof(T) == 4 ? 4 : 2;
+  const uint8_t* codes;
+  const uint8_t* meta;
+  const uint8_t* oidx;
+  const uint8_t* oval;
+  const uint8_t* lf;
+  int bm, bi, bo, bl;   // bytes per token of meta, oidx, oval, lf
+
+  __device__ __forceinline__ void init(const CacheView& cv, size_t row0, int G, int k, int rm) {
+    bm = G * 8;
+    bi = k;
+    bo = k * (int)sizeof(T);
+    bl = rm * lsz;
+    codes = reinterpret_cast<const uint8_t*>(cv.codes) + row0 * W * 4;
+    meta = reinterpret_cast<const uint8_t*>(cv.meta) + row0 * bm;
+    oidx = cv.oidx + row0 * bi;
+    oval = reinterpret_cast<const uint8_t*>(cv.oval) + row0 * bo;
+    lf = reinterpret_cast<const uint8_t*>(cv.lfac) + row0 * bl;
+  }
+
+  // tokens [dt, dt + nt) of the split into the tile at shared address dst
+  __device__ __forceinline__ void stage(const TileLayout& L, uint8_t* dst, int dt, int nt, bool async,
+                                        int lane) const {
+    if (async) {
+      const uint8_t* sc = codes + (size_t)dt * W * 4;
+#pragma unroll
+      for (int it = 0; it < kCpr; ++it) {
+        const int ci = lane + 32 * it;
+        const int t = ci / kCpr, jj = ci % kCpr;
+        cp_async16(dst + L.codes + t * kStride + jj * 16, sc + ci * 16);
+      }
+      const uint8_t* sm = meta + (size_t)dt * bm;
+      for (int off = lane * 16; off < kDTile * bm; off += 512) cp_async16(dst + L.meta + off, sm + off);
+      const uint8_t* si = oidx + (size_t)dt * bi;
+      for (int off = lane * 16; off < kDTile * bi; off += 512) cp_async16(dst + L.oidx + off, si + off);
+      const uint8_t* so = oval + (size_t)dt * bo;
+      for (int off = lane * 16; off < kDTile * bo; off += 512) cp_async16(dst + L.oval + off, so + off);
+      const uint8_t* sl = lf + (size_t)dt * bl;
+      for (int off = lane * 16; off < kDTile * bl; off += 512) cp_async16(dst + L.lf + off, sl + off);
+    } else {
+      const uint32_t* sc = reinterpret_cast<const uint32_t*>(codes) + (size_t)dt * W;
+      for (int e = lane; e < nt * W; e += 32)
+        reinterpret_cast<uint32_t*>(dst + L.codes + (e / W) * kStride)[e % W] = sc[e];
+      for (int e = lane; e < nt * bm; e += 32) dst[L.meta + e] = meta[(size_t)dt * bm + e];
+      for (int e = lane; e < nt * bi; e += 32) dst[L.oidx + e] = oidx[(size_t)dt * bi + e];
+      for (int e = lane; e < nt * bo; e += 32) dst[L.oval + e] = oval[(size_t)dt * bo + e];
+      for (int e = lane; e < nt * bl; e += 32) dst[L.lf + e] = lf[(size_t)dt * bl + e];
     }
   }
-}
+};
 
 template <typename T>
 __device__ __forceinline__ float stage_l(const uint8_t* tile, const TileLayout& L, int t, int j, int rm) {
@@ -154,11 +163,53 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
+// register-pair moves (no integer arithmetic) for the f32x2 operands
 __device__ __forceinline__ uint64_t pk2(float x, float y) {
-  return (uint64_t)__float_as_uint(x) | ((uint64_t)__float_as_uint(y) << 32);
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
 }
-__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ float lo2(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a;
+}
+__device__ __forceinline__ float hi2(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return b;
+}
+
+// Outlier fix-ups of one token: for up to kFast outliers, the channel and the
+// difference between the exact value and what codes + low rank give there:
+// fix = x_o - (zero_g(c_o) + L_t . Rf[:, c_o]). All loads are issued together.
+constexpr int kFast = 4;
+template <typename T, int RR>
+__device__ __forceinline__ void outlier_fixes(const uint8_t* tile, const TileLayout& L, int t, int k, int G, int rb,
+                                              const float (&lt)[RR], const float* rf, int lg, int (&cix)[kFast],
+                                              float (&fix)[kFast]) {
+  const float2* mt = reinterpret_cast<const float2*>(tile + L.meta) + t * G;
+  float xo[kFast], zr[kFast], rv[kFast][RR];
+#pragma unroll
+  for (int i = 0; i < kFast; ++i) {
+    const bool on = i < k;
+    cix[i] = on ? tile[L.oidx + t * k + i] : 0;
+    xo[i] = on ? (float)reinterpret_cast<const T*>(tile + L.oval)[t * k + i] : 0.0f;
+  }
+#pragma unroll
+  for (int i = 0; i < kFast; ++i) {
+    zr[i] = i < k ? mt[cix[i] >> lg].y : 0.0f;
+#pragma unroll
+    for (int j = 0; j < RR; ++j) rv[i][j] = (i < k && j < rb) ? __ldg(rf + j * 128 + cix[i]) : 0.0f;
+  }
+#pragma unroll
+  for (int i = 0; i < kFast; ++i) {
+    float lr = 0.0f;
+#pragma unroll
+    for (int j = 0; j < RR; ++j) lr = fmaf(lt[j], rv[i][j], lr);
+    fix[i] = i < k ? xo[i] - (zr[i] + lr) : 0.0f;
+  }
+}
 
 // Per-warp shared memory (floats from the warp's base):
 //   q [HQ][128] | qw [HQ][128] (q scaled by the code weights) | u [HQ][16]
@@ -170,7 +221,7 @@ template <typename T, int BITS, int HQ>
 __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t dsm[];
   constexpr int W = 4 * BITS;
-  constexpr int kStride = (W + 4) * 4;
+  constexpr int kStride = Stager<T, BITS>::kStride;
   constexpr int kRReg = 4;   // value low-rank weights kept in registers
   using CF = CodeFloats<BITS>;
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -232,13 +283,16 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
     const float* rfv = nullptr;
     int rb = 0;
     int t0 = c0, it = 0;
+    Stager<T, BITS> sk, sv;
+    sk.init(a.K, (size_t)unit * a.n_max + c0, G, k, rm);
+    sv.init(a.V, (size_t)unit * a.n_max + c0, G, k, rm);
     // tile [t, min(t + 32, c1, end of its block))
     auto next_end = [&](int t, int be) { return min(min(t + kDTile, c1), be); };
     {
       const int t1 = next_end(t0, bend);
       const bool as = (t1 - t0 == kDTile) && (t0 % kDTile == 0);
-      stage_tensor<T, BITS>(a, a.K, stages, unit, t0, t1 - t0, as, lane);
-      stage_tensor<T, BITS>(a, a.V, stages + L.bytes, unit, t0, t1 - t0, as, lane);
+      sk.stage(L, stages, t0 - c0, t1 - t0, as, lane);
+      sv.stage(L, stages + L.bytes, t0 - c0, t1 - t0, as, lane);
       cp_async_commit();
     }
     int cur_blk = -1;
@@ -253,8 +307,8 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
         const int t2 = next_end(t1, be2);
         const bool as = (t2 - t1 == kDTile) && (t1 % kDTile == 0);
         uint8_t* nk = stages + ((it + 1) & 1) * 2 * L.bytes;
-        stage_tensor<T, BITS>(a, a.K, nk, unit, t1, t2 - t1, as, lane);
-        stage_tensor<T, BITS>(a, a.V, nk + L.bytes, unit, t1, t2 - t1, as, lane);
+        sk.stage(L, nk, t1 - c0, t2 - t1, as, lane);
+        sv.stage(L, nk + L.bytes, t1 - c0, t2 - t1, as, lane);
         cp_async_commit();
         cp_async_wait<1>();
       } else {
@@ -373,6 +427,15 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
 #pragma unroll
             for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(lj, u_s[hh * kMaxR + j], s[hh]);
           }
+          if (k <= kFast && rb <= kRReg) {
+            int cix[kFast];
+            float fx[kFast];
+            outlier_fixes<T, kRReg>(tk, L, t, k, G, rb, lt, rfk, lg, cix, fx);
+#pragma unroll
+            for (int i = 0; i < kFast; ++i)
+#pragma unroll
+              for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(q_s[hh * 128 + cix[i]], fx[i], s[hh]);
+          } else
           for (int i = 0; i < k; ++i) {
             const int c = tk[L.oidx + t * k + i];
             float lr = 0.0f;
@@ -436,6 +499,19 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
             for (int hh = 0; hh < HQ; ++hh) alr[hh][j] = fmaf(p[hh], lj, alr[hh][j]);
           }
           // value outliers
+          if (k <= kFast && rb <= kRReg) {
+            float lv[kRReg];
+#pragma unroll
+            for (int j = 0; j < kRReg; ++j) lv[j] = j < rb ? stage_l<T>(tv, L, t, j, rm) : 0.0f;
+            int cix[kFast];
+            float fx[kFast];
+            outlier_fixes<T, kRReg>(tv, L, t, k, G, rb, lv, rfv, lg, cix, fx);
+#pragma unroll
+            for (int i = 0; i < kFast; ++i)
+              if (i < k)
+#pragma unroll
+                for (int hh = 0; hh < HQ; ++hh) atomicAdd(&corr_s[hh * 128 + cix[i]], p[hh] * fx[i]);
+          } else
           for (int i = 0; i < k; ++i) {
             const int c = tv[L.oidx + t * k + i];
             float lr = 0.0f;

@@ -34,11 +34,32 @@
 namespace gear {
 
 // ------------------------------------------------------------------ helpers
+// register-pair moves (no integer arithmetic) for the f32x2 operands
 __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
-  return (uint64_t)__float_as_uint(a) | ((uint64_t)__float_as_uint(b) << 32);
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
 }
-__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ float f2_lo(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a;
+}
+__device__ __forceinline__ float f2_hi(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return b;
+}
+__device__ __forceinline__ uint32_t f2_lo_bits(uint64_t v) {
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
+  return a;
+}
+__device__ __forceinline__ uint32_t f2_hi_bits(uint64_t v) {
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
+  return b;
+}
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
@@ -111,14 +132,20 @@ __device__ __forceinline__ uint32_t pair_max(uint32_t a, uint32_t b) {
 // q0 is within one ulp and a/s is normal). Only rint(q) is used and only
 // q >= 1/4 can round to a non-zero code, where all operands are normal.
 // Otherwise the correctly rounded division intrinsic is used.
-__device__ __forceinline__ uint64_t div_pair(uint64_t a, float s, float y, bool fast) {
-  if (fast) {
-    uint64_t y2 = f2_pack(y, y);
-    uint64_t s2n = f2_pack(-s, -s);
-    uint64_t q0 = f2_mul(a, y2);
-    uint64_t r = f2_fma(q0, s2n, a);
-    return f2_fma(r, y2, q0);
-  }
+// Correctly rounded a / s for the code decision. When 2^-100 <= s <= 2^100
+// (so s and y = RN(1/s) are normal), the quotient is refined from the
+// correctly rounded reciprocal with one exact remainder (Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990: q1 = RN(q0 + r y), r = a - s q0, equals RN(a/s) whenever
+// q0 is within one ulp and a/s is normal). Only rint(q) is used and only
+// q >= 1/4 can round to a non-zero code, where all operands are normal.
+// Otherwise the correctly rounded division intrinsic is used (slow path).
+__device__ __forceinline__ uint64_t div_pair_fast(uint64_t a, uint64_t s2n, uint64_t y2) {
+  const uint64_t q0 = f2_mul(a, y2);
+  const uint64_t r = f2_fma(q0, s2n, a);
+  return f2_fma(r, y2, q0);
+}
+__device__ __forceinline__ uint64_t div_pair_slow(uint64_t a, float s) {
   return f2_pack(__fdiv_rn(f2_lo(a), s), __fdiv_rn(f2_hi(a), s));
 }
 
@@ -208,11 +235,10 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
         uint32_t ab = (e & 1) ? ((p >> 16) & 0x7FFFu) : (p & 0x7FFFu);
         key = (ab << 7) | (tb0 - e);
       }
-      if (!valid) key = 0;
 #pragma unroll
-      for (int i = 0; i < KMAX; ++i) {
-        Key hi = key > top[i] ? key : top[i];
-        key = key > top[i] ? top[i] : key;
+      for (int i = 0; i < KMAX; ++i) {   // one max and one min per level
+        const Key hi = max(key, top[i]);
+        key = min(key, top[i]);
         top[i] = hi;
       }
     }
@@ -225,8 +251,8 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       Key key = other[i];
 #pragma unroll
       for (int m = 0; m < KMAX; ++m) {
-        Key hi = key > top[m] ? key : top[m];
-        key = key > top[m] ? top[m] : key;
+        const Key hi = max(key, top[m]);
+        key = min(key, top[m]);
         top[m] = hi;
       }
     }
@@ -319,8 +345,9 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     mn[sh] = __fadd_rn(mn[sh], 0.0f);                      // -0 -> +0
     mx[sh] = __fadd_rn(mx[sh], 0.0f);
     scale[sh] = __fdiv_rn(__fsub_rn(mx[sh], mn[sh]), levels);
-    fast[sh] = scale[sh] >= 0x1p-100f && scale[sh] <= 0x1p100f;
-    y[sh] = __frcp_rn(scale[sh]);
+    // scale 0: y = 0 makes the fast path return q = 0 exactly (every code 0)
+    fast[sh] = (scale[sh] >= 0x1p-100f && scale[sh] <= 0x1p100f) || scale[sh] == 0.0f;
+    y[sh] = scale[sh] == 0.0f ? 0.0f : __frcp_rn(scale[sh]);
   }
 
   // ---------------- quantize, pack, residual split -------------------------
@@ -328,8 +355,8 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
 #pragma unroll
   for (int w = 0; w < kWordsHalf; ++w) words[w] = 0u;
   uint32_t hi_out[32], lo_out[32];  // packed bf16 pairs of R (hi) and R - hi (lo)
-#pragma unroll
-  for (int p = 0; p < 32; ++p) {
+  // one pair of channels (2p, 2p + 1); DIV is the division of the pair
+  auto qpair = [&](const int p, const uint64_t mnv, const uint64_t sc2, auto div) {
     const int sh = p >> 4;
     float x0, x1;
     if constexpr (sizeof(T) == 4) {
@@ -338,36 +365,50 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     } else {
       uint32_t m2 = Elem16<T>::from_f(mn[sh]);
       m2 |= m2 << 16;
-      float2 f = Elem16<T>::to_f2(pair_max<T>(xr[p], m2));  // NaN -> zero point
+      const float2 f = Elem16<T>::to_f2(pair_max<T>(xr[p], m2));  // NaN -> zero point
       x0 = f.x; x1 = f.y;
     }
-    uint64_t xv = f2_pack(x0, x1);
-    uint64_t mnv = f2_pack(mn[sh], mn[sh]);
-    uint64_t av = f2_sub(xv, mnv);
-    uint64_t q = div_pair(av, scale[sh], y[sh], fast[sh]);
-    if (scale[sh] == 0.0f) q = 0;
-    uint64_t tq = f2_add(q, f2_pack(kRoundMagic, kRoundMagic));
-    uint64_t cf = f2_sub(tq, f2_pack(kRoundMagic, kRoundMagic));
-    uint64_t dh = f2_fma(cf, f2_pack(scale[sh], scale[sh]), mnv);
-    uint64_t rv = f2_sub(xv, dh);
-    if (!valid) rv = 0;
+    const uint64_t xv = f2_pack(x0, x1);
+    const uint64_t av = f2_sub(xv, mnv);
+    const uint64_t q = div(av);
+    const uint64_t tq = f2_add(q, f2_pack(kRoundMagic, kRoundMagic));
+    const uint64_t cf = f2_sub(tq, f2_pack(kRoundMagic, kRoundMagic));
+    const uint64_t dh = f2_fma(cf, sc2, mnv);
+    const uint64_t rv = f2_sub(xv, dh);
     // pack: word += bits(tq) << (b * e); the constant part of bits(tq) is
     // removed once per word below
 #pragma unroll
     for (int e2 = 0; e2 < 2; ++e2) {
       const int e = 2 * p + e2;
-      uint32_t bits = e2 ? (uint32_t)(tq >> 32) : (uint32_t)tq;
+      const uint32_t bits = e2 ? f2_hi_bits(tq) : f2_lo_bits(tq);
       words[e / kCodesPerWord] += bits << (BITS * (e % kCodesPerWord));
     }
     // residual split: hi = bf16(R), lo = bf16(R - hi)
-    float r0 = f2_lo(rv), r1 = f2_hi(rv);
-    __nv_bfloat162 hb = __floats2bfloat162_rn(r0, r1);
-    uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb);
-    uint64_t hv = f2_pack(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u));
-    uint64_t lv = f2_sub(rv, hv);
-    __nv_bfloat162 lb = __floats2bfloat162_rn(f2_lo(lv), f2_hi(lv));
+    const float r0 = f2_lo(rv), r1 = f2_hi(rv);
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(r0, r1);
+    const uint32_t hbits = *reinterpret_cast<const uint32_t*>(&hb);
+    const uint64_t hv = f2_pack(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u));
+    const uint64_t lv = f2_sub(rv, hv);
+    const __nv_bfloat162 lb = __floats2bfloat162_rn(f2_lo(lv), f2_hi(lv));
     hi_out[p] = hbits;
-    lo_out[p] = *reinterpret_cast<uint32_t*>(&lb);
+    lo_out[p] = *reinterpret_cast<const uint32_t*>(&lb);
+  };
+#pragma unroll
+  for (int sh = 0; sh < 2; ++sh) {
+    const uint64_t mnv = f2_pack(mn[sh], mn[sh]);
+    const uint64_t sc2 = f2_pack(scale[sh], scale[sh]);
+    if (fast[sh]) {
+      const uint64_t y2 = f2_pack(y[sh], y[sh]);
+      const uint64_t s2n = f2_pack(-scale[sh], -scale[sh]);
+#pragma unroll
+      for (int pp = 0; pp < 16; ++pp)
+        qpair(16 * sh + pp, mnv, sc2, [&](uint64_t av) { return div_pair_fast(av, s2n, y2); });
+    } else {
+      const float sv = scale[sh];
+#pragma unroll
+      for (int pp = 0; pp < 16; ++pp)
+        qpair(16 * sh + pp, mnv, sc2, [&](uint64_t av) { return div_pair_slow(av, sv); });
+    }
   }
   {
     uint32_t magic_sum = 0;
@@ -378,12 +419,22 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
   }
 
   // ---------------- residual to the R stage (MN-major swizzle-128B) --------
+  // rows past the unit's last token contribute nothing to the Gram
+  if (valid) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    uint8_t* ph = rs + h * 16384 + swz(t, j);
-    *reinterpret_cast<uint4*>(ph) = make_uint4(hi_out[4 * j], hi_out[4 * j + 1], hi_out[4 * j + 2], hi_out[4 * j + 3]);
-    *reinterpret_cast<uint4*>(ph + 32768) =
-        make_uint4(lo_out[4 * j], lo_out[4 * j + 1], lo_out[4 * j + 2], lo_out[4 * j + 3]);
+    for (int j = 0; j < 8; ++j) {
+      uint8_t* ph = rs + h * 16384 + swz(t, j);
+      *reinterpret_cast<uint4*>(ph) = make_uint4(hi_out[4 * j], hi_out[4 * j + 1], hi_out[4 * j + 2], hi_out[4 * j + 3]);
+      *reinterpret_cast<uint4*>(ph + 32768) =
+          make_uint4(lo_out[4 * j], lo_out[4 * j + 1], lo_out[4 * j + 2], lo_out[4 * j + 3]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint8_t* ph = rs + h * 16384 + swz(t, j);
+      *reinterpret_cast<uint4*>(ph) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(ph + 32768) = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 
   // ---------------- cache outputs -------------------------------------------
