@@ -100,7 +100,9 @@ typedef struct gear_params {
  *   oidx   uint8  [U][n_max][k]      outlier channels, ascending.
  *   oval   dtype  [U][n_max][k]      outlier values, bit-exact input copies.
  *   lfac   f16|f32[U][n_max][r_max]  L rows, stored as L * 2^e_blk.
- *   rfac   float  [U][nblk_max][r_max][d]  Rf columns, stored as Rf * 2^-e_blk.
+ *   rfac   float  [U][nblk_max][d][r_pad]  Rf rows (one per channel), stored as
+ *                                    Rf * 2^-e_blk; r_pad = r_max rounded up
+ *                                    to a multiple of 4, the padding zero.
  *   buf    dtype  [U][n_b][d]        streaming buffer (full precision).
  *
  * with U = B*H, k = outliers per token, r_max = max(rank, buffer_rank) and

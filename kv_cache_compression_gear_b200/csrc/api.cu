@@ -51,7 +51,7 @@ static Layout cache_layout(const gear_params* p, int B, int H, int d, int n_max,
   L.oidx = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1));
   L.oval = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1) * esize(dt));
   L.lfac = off;  off = align256(off + U * n_max * rm * (dt == GEAR_F32 ? 4 : 2));
-  L.rfac = off;  off = align256(off + U * nblk_max * rm * (size_t)d * 4);
+  L.rfac = off;  off = align256(off + U * nblk_max * (size_t)rpad_of(rm) * d * 4);
   L.buf = off;   off = align256(off + U * (size_t)p->buffer_len * d * esize(dt));
   L.total = off;
   return L;
@@ -259,6 +259,7 @@ gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const voi
   if (!workspace || ws_bytes < decode_workspace_bytes(a.B, a.Hq, a.nsplit) || !aligned(workspace, 16))
     return GEAR_ERR_WORKSPACE;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.one_bits = 0x3F800000u;
   a.q = q;
   a.out = out;
   a.out_dtype = out_dtype;
@@ -391,6 +392,7 @@ extern "C" gear_status gear_decode_attn_noalloc(const gear_cache* k, const gear_
   float* scratch = noalloc_scratch_for_current_device();
   if (!scratch) return GEAR_ERR_CUDA;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.one_bits = 0x3F800000u;
   a.q = q;
   a.out = out;
   a.out_dtype = out_dtype;

@@ -32,6 +32,17 @@ __device__ __forceinline__ void set_device_error(int32_t code) {
 // Bound of every spin on an mbarrier: 2 seconds of wall time (global timer),
 // checked every 64 probes, plus an absolute cap on the number of probes.
 constexpr uint64_t kSpinNanos = 2000000000ull;
+
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point
+// (null if the driver does not provide it).
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+PFN_encodeTiled tensor_map_encoder();
+
+// Row length of the stored Rf factors: r_max rounded up to a multiple of 4, so
+// that one channel's row is a whole number of 16-byte vectors.
+__host__ __device__ constexpr int rpad_of(int r_max) { return (r_max + 3) & ~3; }
 constexpr uint32_t kSpinLimit = 1u << 26;
 
 __device__ __forceinline__ uint64_t global_timer_ns() {

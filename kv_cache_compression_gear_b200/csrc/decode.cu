@@ -13,11 +13,18 @@
 //
 // Split-K (flash-decoding style): in decode_warp every warp is one split, a
 // run of whole 32-token tiles of one (batch, kv head), for all query heads
-// sharing that kv head. It stages tiles of both tensors in its own shared
-// memory (asynchronous 16-byte copies, double-buffered), scores with one lane
-// per token straight from the packed codes, keeps an online softmax and
-// accumulates values with one lane per 4 channels. One extra split per unit
-// takes the buffer. decode_combine merges the splits by log-sum-exp.
+// sharing that kv head. Its lanes bring the tiles of both tensors into the
+// warp's own shared memory with tensor copies (codes and meta, 16-byte-chunk
+// swizzled so that both the per-token and the per-channel reads are free of
+// bank conflicts) and bulk copies (outlier channels and values, L rows),
+// double-buffered on two mbarriers. It scores with one lane per token
+// straight from the packed codes, keeps an online softmax whose reference
+// moves only when the running maximum passes it by 2^8, and accumulates
+// values with one lane per 8 channels and token parity. The outlier fix-ups
+// of the values are scattered with fire-and-forget float reductions into the
+// split's partial-result row in global memory. One extra split per unit takes
+// the buffer. decode_combine merges the splits by log-sum-exp.
+#include <string.h>
 #include "common.cuh"
 #include "decode.cuh"
 
@@ -26,6 +33,7 @@ namespace gear {
 constexpr int kDThreads = 128;   // 4 warps, each an independent split
 constexpr int kDTile = 32;       // tokens per tile (one per lane)
 constexpr int kMaxR = 16;
+constexpr float kLazy = 8.0f;    // log2 slack of the softmax reference
 
 template <typename T>
 __device__ __forceinline__ float load_elem(const void* p, size_t i) {
@@ -56,12 +64,43 @@ __device__ __forceinline__ int block_end(const DecodeArgs& a, int b) {
   return b == 0 ? a.blk0_len : a.blk0_len + b * a.n_b;
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+// Bulk copy global -> shared, completing on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// 2-D tensor copy global -> shared at column 0, row y (no multicast).
+__device__ __forceinline__ void tensor_copy(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(0), "r"(y)
+      : "memory");
+}
+
+// Accesses of the split's partial-result row that go to the L2 point of
+// coherence, where the value outlier reductions land.
+__device__ __forceinline__ void red_add_gpu(float* p, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+__device__ __forceinline__ float ld_gpu(const float* p) {
+  float v;
+  asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_gpu(float* p, float v) {
+  asm volatile("st.relaxed.gpu.global.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+// The 16-byte-chunk swizzle a tensor copy applies to a tile of R-byte rows
+// (R = 32, 64, 128: the 32-, 64- and 128-byte modes): byte o of row t lands at
+// t*R + (o ^ (swz(t) << 4)), swz(t) = ((t*R) >> 7) & (R/16 - 1). It repeats
+// every 8 rows.
+template <int R>
+__device__ __forceinline__ int swz(int t) {
+  return ((t * R) >> 7) & (R / 16 - 1);
+}
 
 // Codes as floats without integer conversion. Byte b of a code word is moved
 // to mantissa bits 15..22 by one shift; each code of the byte is then masked
@@ -72,8 +111,9 @@ template <int BITS>
 struct CodeFloats {
   static constexpr int kPerByte = 8 / BITS;
   static constexpr int kPerWord = 32 / BITS;
-  // all codes of one 32-bit word, in channel order
-  __device__ static __forceinline__ void word(uint32_t w, float (&f)[kPerWord]) {
+  // all codes of one 32-bit word, in channel order. `one` holds the bits of
+  // 1.0f in a register, so that mask and exponent go into one LOP3 each.
+  __device__ static __forceinline__ void word(uint32_t w, float (&f)[kPerWord], uint32_t one) {
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int sh = 15 - 8 * b;
@@ -81,7 +121,7 @@ struct CodeFloats {
 #pragma unroll
       for (int q = 0; q < kPerByte; ++q) {
         const uint32_t m = ((1u << BITS) - 1u) << (15 + q * BITS);
-        f[b * kPerByte + q] = __uint_as_float((v & m) | 0x3F800000u);
+        f[b * kPerByte + q] = __uint_as_float((v & m) | one);
       }
     }
   }
@@ -91,71 +131,10 @@ struct CodeFloats {
   }
 };
 
-// Stages 32-token tiles of one compressed tensor of one split. The per-token
-// arrays of the split's first token are located once; a tile then only adds
-// its token offset. Whole, 32-aligned tiles use 16-byte asynchronous copies
-// (every region of such a tile is a multiple of 16 bytes and 16-byte
-// aligned); other tiles (block tails) use plain loads.
-template <typename T, int BITS>
-struct Stager {
-  static constexpr int W = 4 * BITS;           // code words per token (d = 128)
-  static constexpr int kCpr = W / 4;           // 16-byte chunks per code row
-  static constexpr int kStride = (W + 4) * 4;  // padded code row in shared memory
-  static constexpr int lsz = sizeof(T) == 4 ? 4 : 2;
-  const uint8_t* codes;
-  const uint8_t* meta;
-  const uint8_t* oidx;
-  const uint8_t* oval;
-  const uint8_t* lf;
-  int bm, bi, bo, bl;   // bytes per token of meta, oidx, oval, lf
-
-  __device__ __forceinline__ void init(const CacheView& cv, size_t row0, int G, int k, int rm) {
-    bm = G * 8;
-    bi = k;
-    bo = k * (int)sizeof(T);
-    bl = rm * lsz;
-    codes = reinterpret_cast<const uint8_t*>(cv.codes) + row0 * W * 4;
-    meta = reinterpret_cast<const uint8_t*>(cv.meta) + row0 * bm;
-    oidx = cv.oidx + row0 * bi;
-    oval = reinterpret_cast<const uint8_t*>(cv.oval) + row0 * bo;
-    lf = reinterpret_cast<const uint8_t*>(cv.lfac) + row0 * bl;
-  }
-
-  // tokens [dt, dt + nt) of the split into the tile at shared address dst
-  __device__ __forceinline__ void stage(const TileLayout& L, uint8_t* dst, int dt, int nt, bool async,
-                                        int lane) const {
-    if (async) {
-      const uint8_t* sc = codes + (size_t)dt * W * 4;
-#pragma unroll
-      for (int it = 0; it < kCpr; ++it) {
-        const int ci = lane + 32 * it;
-        const int t = ci / kCpr, jj = ci % kCpr;
-        cp_async16(dst + L.codes + t * kStride + jj * 16, sc + ci * 16);
-      }
-      const uint8_t* sm = meta + (size_t)dt * bm;
-      for (int off = lane * 16; off < kDTile * bm; off += 512) cp_async16(dst + L.meta + off, sm + off);
-      const uint8_t* si = oidx + (size_t)dt * bi;
-      for (int off = lane * 16; off < kDTile * bi; off += 512) cp_async16(dst + L.oidx + off, si + off);
-      const uint8_t* so = oval + (size_t)dt * bo;
-      for (int off = lane * 16; off < kDTile * bo; off += 512) cp_async16(dst + L.oval + off, so + off);
-      const uint8_t* sl = lf + (size_t)dt * bl;
-      for (int off = lane * 16; off < kDTile * bl; off += 512) cp_async16(dst + L.lf + off, sl + off);
-    } else {
-      const uint32_t* sc = reinterpret_cast<const uint32_t*>(codes) + (size_t)dt * W;
-      for (int e = lane; e < nt * W; e += 32)
-        reinterpret_cast<uint32_t*>(dst + L.codes + (e / W) * kStride)[e % W] = sc[e];
-      for (int e = lane; e < nt * bm; e += 32) dst[L.meta + e] = meta[(size_t)dt * bm + e];
-      for (int e = lane; e < nt * bi; e += 32) dst[L.oidx + e] = oidx[(size_t)dt * bi + e];
-      for (int e = lane; e < nt * bo; e += 32) dst[L.oval + e] = oval[(size_t)dt * bo + e];
-      for (int e = lane; e < nt * bl; e += 32) dst[L.lf + e] = lf[(size_t)dt * bl + e];
-    }
-  }
-};
-
 template <typename T>
-__device__ __forceinline__ float stage_l(const uint8_t* tile, const TileLayout& L, int t, int j, int rm) {
-  if constexpr (sizeof(T) == 4) return reinterpret_cast<const float*>(tile + L.lf)[t * rm + j];
-  else return __half2float(reinterpret_cast<const __half*>(tile + L.lf)[t * rm + j]);
+__device__ __forceinline__ float l_at(const uint8_t* lf, int t, int j, int rm) {
+  if constexpr (sizeof(T) == 4) return reinterpret_cast<const float*>(lf)[t * rm + j];
+  else return __half2float(reinterpret_cast<const __half*>(lf)[t * rm + j]);
 }
 
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
@@ -180,73 +159,120 @@ __device__ __forceinline__ float hi2(uint64_t v) {
   return b;
 }
 
+// One token's meta row in shared memory: (scale, zero) of group gi sits at
+// byte (8*gi) ^ mx of the row, mx the lane's swizzle term (0 unless G = 4).
+__device__ __forceinline__ float2 meta_at(const uint8_t* mrow, int gi, int mx) {
+  return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
+}
+// The whole row, read in 16-byte pieces (conflict-free across the lanes).
+__device__ __forceinline__ void meta_row(const uint8_t* mrow, int G, int mx, float2 (&sz)[4]) {
+  if (G == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(mrow + mx);
+    const float4 b = *reinterpret_cast<const float4*>(mrow + (16 ^ mx));
+    sz[0] = make_float2(a.x, a.y); sz[1] = make_float2(a.z, a.w);
+    sz[2] = make_float2(b.x, b.y); sz[3] = make_float2(b.z, b.w);
+  } else if (G == 2) {
+    const float4 a = *reinterpret_cast<const float4*>(mrow);
+    sz[0] = make_float2(a.x, a.y); sz[1] = make_float2(a.z, a.w);
+    sz[2] = sz[3] = make_float2(0.0f, 0.0f);
+  } else {
+    sz[0] = *reinterpret_cast<const float2*>(mrow);
+    sz[1] = sz[2] = sz[3] = make_float2(0.0f, 0.0f);
+  }
+}
+
 // Outlier fix-ups of one token: for up to kFast outliers, the channel and the
 // difference between the exact value and what codes + low rank give there:
-// fix = x_o - (zero_g(c_o) + L_t . Rf[:, c_o]). All loads are issued together.
+// fix = x_o - (zero_g(c_o) + L_t . Rf[c_o]). Rf rows are 16-byte vectors, so a
+// rank <= 4 block needs one load per outlier. All loads are issued together.
 constexpr int kFast = 4;
-template <typename T, int RR>
-__device__ __forceinline__ void outlier_fixes(const uint8_t* tile, const TileLayout& L, int t, int k, int G, int rb,
-                                              const float (&lt)[RR], const float* rf, int lg, int (&cix)[kFast],
-                                              float (&fix)[kFast]) {
-  const float2* mt = reinterpret_cast<const float2*>(tile + L.meta) + t * G;
-  float xo[kFast], zr[kFast], rv[kFast][RR];
+template <typename T>
+__device__ __forceinline__ void outlier_fixes(const uint8_t* rest, int oval_off, const uint8_t* mrow, int mx, int t,
+                                              int k, int lg, const float (&lt)[4], const float* rf, int rp,
+                                              int (&cix)[kFast], float (&fix)[kFast]) {
+  float xo[kFast], zr[kFast];
+  float4 rv[kFast];
 #pragma unroll
   for (int i = 0; i < kFast; ++i) {
     const bool on = i < k;
-    cix[i] = on ? tile[L.oidx + t * k + i] : 0;
-    xo[i] = on ? (float)reinterpret_cast<const T*>(tile + L.oval)[t * k + i] : 0.0f;
+    cix[i] = on ? rest[t * k + i] : 0;
+    xo[i] = on ? (float)reinterpret_cast<const T*>(rest + oval_off)[t * k + i] : 0.0f;
   }
 #pragma unroll
   for (int i = 0; i < kFast; ++i) {
-    zr[i] = i < k ? mt[cix[i] >> lg].y : 0.0f;
-#pragma unroll
-    for (int j = 0; j < RR; ++j) rv[i][j] = (i < k && j < rb) ? __ldg(rf + j * 128 + cix[i]) : 0.0f;
+    const bool on = i < k;
+    zr[i] = on ? meta_at(mrow, cix[i] >> lg, mx).y : 0.0f;
+    rv[i] = on ? __ldg(reinterpret_cast<const float4*>(rf + cix[i] * rp)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
 #pragma unroll
   for (int i = 0; i < kFast; ++i) {
     float lr = 0.0f;
-#pragma unroll
-    for (int j = 0; j < RR; ++j) lr = fmaf(lt[j], rv[i][j], lr);
+    lr = fmaf(lt[0], rv[i].x, lr);
+    lr = fmaf(lt[1], rv[i].y, lr);
+    lr = fmaf(lt[2], rv[i].z, lr);
+    lr = fmaf(lt[3], rv[i].w, lr);
     fix[i] = i < k ? xo[i] - (zr[i] + lr) : 0.0f;
   }
 }
 
-// Per-warp shared memory (floats from the warp's base):
-//   q [HQ][128] | qw [HQ][128] (q scaled by the code weights) | u [HQ][16]
-//   | alr [HQ][16] | w [32][G][HQ] | corr [HQ][128] | accx [HQ][128]
-//   | stages: 2 x (K, V tile)
-// The [HQ][128] accumulators hold channel c at slot c; loops that touch all
-// of them use slot e*32 + lane so that every lane stays in its own bank.
+// Low-rank value at channel c for any rank: L_t . Rf[c] over rb <= 16 ranks.
+template <typename T>
+__device__ __forceinline__ float lowrank_at(const uint8_t* lf, int t, int rm, int rb, const float* rf, int rp, int c) {
+  float lr = 0.0f;
+  for (int j4 = 0; j4 < rb; j4 += 4) {
+    const float4 r4 = __ldg(reinterpret_cast<const float4*>(rf + c * rp + j4));
+    const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      if (j4 + jj < rb) lr = fmaf(l_at<T>(lf, t, j4 + jj, rm), rr[jj], lr);
+  }
+  return lr;
+}
+
+// Per-warp shared memory (see TileLayout): 4 code tiles | 4 meta tiles |
+// 4 rest tiles | floats | 2 mbarriers. Floats: q [HQ][128] | qw [HQ][128]
+// (q scaled by the code weights) | u [HQ][16] | alr [HQ][16] | w [32][G][HQ]
+// | accx [HQ][128]. The [HQ][128] accumulators hold channel c at slot c;
+// loops that touch all of them use slot e*32 + lane so that every lane stays
+// in its own bank.
 template <typename T, int BITS, int HQ>
-__global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
-  extern __shared__ __align__(16) uint8_t dsm[];
+__global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) decode_warp(const __grid_constant__ DecodeMaps maps,
+                                                         const DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t dsm[];
   constexpr int W = 4 * BITS;
-  constexpr int kStride = Stager<T, BITS>::kStride;
+  constexpr int R = 4 * W;   // code bytes per token
   constexpr int kRReg = 4;   // value low-rank weights kept in registers
   using CF = CodeFloats<BITS>;
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gs = blockIdx.x * 4 + wid;
   if (gs >= a.total_splits) return;
+  const TileLayout& L = a.tl;
   const int G = a.G, rm = a.r_max, k = a.k;
+  const int rp = rpad_of(rm);
+  const uint32_t one = a.one_bits;
   const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
-  float* q_s = reinterpret_cast<float*>(dsm + (size_t)wid * a.warp_bytes);
+  const uint32_t abase = (smem_u32(dsm) + 1023u) & ~1023u;
+  uint8_t* wb = dsm + (abase - smem_u32(dsm)) + (size_t)wid * L.bytes;
+  float* q_s = reinterpret_cast<float*>(wb + L.floats);
   float* qw_s = q_s + HQ * 128;
   float* u_s = qw_s + HQ * 128;
   float* alr_s = u_s + HQ * kMaxR;   // value low-rank weights j >= kRReg
   float* w_s = alr_s + HQ * kMaxR;
-  float* corr_s = w_s + kDTile * G * HQ;
-  float* accx_s = corr_s + HQ * 128;
-  uint8_t* stages = reinterpret_cast<uint8_t*>(accx_s + HQ * 128);
-  const TileLayout& L = a.tl;
+  float* accx_s = w_s + kDTile * G * HQ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wb + L.bars);
 
   const int unit = gs / a.nsplit, sp = gs % a.nsplit;
   const int b = unit / a.H, h = unit % a.H;
+  const bool comp = sp < a.nsplit_comp;
+  // this split's partial row of query head hh: part_row + hh * hstride
+  float* part_row = a.part + (((size_t)b * a.Hq + (size_t)h * HQ) * a.nsplit + sp) * 130;
+  const size_t hstride = (size_t)a.nsplit * 130;
   for (int e = lane; e < HQ * 128; e += 32) {
     const float qv = load_elem<T>(a.q, ((size_t)b * a.Hq + (size_t)h * HQ + (e >> 7)) * 128 + (e & 127));
     q_s[e] = qv;
     qw_s[e] = qv * CF::inv_weight(e & 127);
-    corr_s[e] = 0.0f;
     accx_s[e] = 0.0f;
+    if (comp) st_gpu(part_row + (e >> 7) * hstride + 2 + (e & 127), 0.0f);   // value outlier sums
   }
   for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
   __syncwarp();
@@ -264,7 +290,15 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
     for (int e = 0; e < 4; ++e) { acc[hh][e] = 0; sw[hh][e] = 0.0f; spm[hh][e] = 0.0f; alr[hh][e] = 0.0f; }
   }
 
-  if (sp < a.nsplit_comp) {
+  if (comp) {
+    if (lane == 0) {
+      mbar_init(&bars[0], 1);
+      mbar_init(&bars[1], 1);
+      fence_mbarrier_init();
+    }
+    __threadfence();   // the zeroed outlier sums before any reduction
+    __syncwarp();
+
     // group sums of q and of the weighted q, per 32-channel block
     float qs_blk[HQ][4], qw_blk[HQ][4];
 #pragma unroll
@@ -274,6 +308,100 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
         qs_blk[hh][bk] = warp_sum(q_s[hh * 128 + bk * 32 + lane]);
         qw_blk[hh][bk] = warp_sum(qw_s[hh * 128 + bk * 32 + lane]);
       }
+
+    // ---- copy roles: lanes 0/1 codes (K/V), 2/3 meta by tensor copy (G >= 2),
+    // 4/5 oidx, 6/7 oval, 8/9 L rows, 10/11 meta by bulk copy (G = 1)
+    const bool meta_tma = G >= 2;
+    const int x = lane & 1;
+    const CUtensorMap* my_map = nullptr;
+    const uint8_t* my_src = nullptr;
+    int my_bpr = 0;
+    uint32_t my_dst = 0, my_sst = 0;
+    {
+      const int esz = (int)sizeof(T), lsz = sizeof(T) == 4 ? 4 : 2;
+      const uint32_t wbs = smem_u32(wb);
+      switch (lane >> 1) {
+        case 0:
+          my_map = x ? &maps.vc : &maps.kc;
+          my_dst = wbs + x * L.cb;
+          my_sst = 2 * L.cb;
+          break;
+        case 1:
+          if (meta_tma) {
+            my_map = x ? &maps.vm : &maps.km;
+            my_dst = wbs + L.meta0 + x * L.mb;
+            my_sst = 2 * L.mb;
+          }
+          break;
+        case 2:
+          my_src = x ? a.V.oidx : a.K.oidx;
+          my_bpr = k;
+          my_dst = wbs + L.rest0 + x * L.rb;
+          my_sst = 2 * L.rb;
+          break;
+        case 3:
+          my_src = reinterpret_cast<const uint8_t*>(x ? a.V.oval : a.K.oval);
+          my_bpr = k * esz;
+          my_dst = wbs + L.rest0 + x * L.rb + L.oval;
+          my_sst = 2 * L.rb;
+          break;
+        case 4:
+          my_src = reinterpret_cast<const uint8_t*>(x ? a.V.lfac : a.K.lfac);
+          my_bpr = rm * lsz;
+          my_dst = wbs + L.rest0 + x * L.rb + L.lf;
+          my_sst = 2 * L.rb;
+          break;
+        case 5:
+          if (!meta_tma) {
+            my_src = reinterpret_cast<const uint8_t*>(x ? a.V.meta : a.K.meta);
+            my_bpr = G * 8;
+            my_dst = wbs + L.meta0 + x * L.mb;
+            my_sst = 2 * L.mb;
+          }
+          break;
+        default:
+          break;
+      }
+    }
+    const size_t row0 = (size_t)unit * a.n_max;   // row of the unit's token 0
+    // Brings tokens [t, t + nt) of the unit into stage s. A whole, 32-aligned
+    // tile is all copies; another one (a block boundary or the split's end)
+    // takes codes and meta by tensor copy (rows past nt are read and ignored)
+    // and the rest by plain loads of the lanes.
+    auto issue = [&](int s, int t, int nt) {
+      const bool full = nt == kDTile && (t & (kDTile - 1)) == 0;
+      if (lane == 0) mbar_arrive_expect_tx(&bars[s], (uint32_t)(full ? L.tx_full : L.tx_part));
+      __syncwarp();
+      const uint32_t bar = smem_u32(&bars[s]);
+      const size_t row = row0 + t;
+      if (my_map) {
+        fence_proxy_async_smem();
+        tensor_copy(my_dst + s * my_sst, my_map, bar, (int32_t)row);
+      } else if (full && my_bpr > 0) {
+        fence_proxy_async_smem();
+        bulk_copy(my_dst + s * my_sst, my_src + row * my_bpr, (uint32_t)(kDTile * my_bpr), bar);
+      }
+      if (!full) {
+        const int esz = (int)sizeof(T), lsz = sizeof(T) == 4 ? 4 : 2;
+#pragma unroll
+        for (int xx = 0; xx < 2; ++xx) {
+          const CacheView& cv = xx ? a.V : a.K;
+          uint8_t* rest = wb + L.rest0 + (2 * s + xx) * L.rb;
+          const uint8_t* oi = cv.oidx + row * k;
+          for (int e = lane; e < nt * k; e += 32) rest[e] = oi[e];
+          const uint8_t* ov = reinterpret_cast<const uint8_t*>(cv.oval) + row * k * esz;
+          for (int e = lane; e < nt * k * esz; e += 32) rest[L.oval + e] = ov[e];
+          const uint8_t* lf = reinterpret_cast<const uint8_t*>(cv.lfac) + row * rm * lsz;
+          for (int e = lane; e < nt * rm * lsz; e += 32) rest[L.lf + e] = lf[e];
+          if (!meta_tma) {
+            uint8_t* md = wb + L.meta0 + (2 * s + xx) * L.mb;
+            const uint8_t* ms = reinterpret_cast<const uint8_t*>(cv.meta) + row * G * 8;
+            for (int e = lane; e < nt * G * 8; e += 32) md[e] = ms[e];
+          }
+        }
+      }
+    };
+
     const int c0 = sp * a.chunk;
     const int c1 = min(a.n_comp, c0 + a.chunk);
     // blocks: block 0 = [0, blk0_len), then n_b tokens each; tracked incrementally
@@ -282,78 +410,107 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
     const float* rfk = nullptr;
     const float* rfv = nullptr;
     int rb = 0;
-    int t0 = c0, it = 0;
-    Stager<T, BITS> sk, sv;
-    sk.init(a.K, (size_t)unit * a.n_max + c0, G, k, rm);
-    sv.init(a.V, (size_t)unit * a.n_max + c0, G, k, rm);
-    // tile [t, min(t + 32, c1, end of its block))
     auto next_end = [&](int t, int be) { return min(min(t + kDTile, c1), be); };
+    issue(0, c0, next_end(c0, bend) - c0);
+
+    // lane-constant swizzle terms: key rows (lane = token), meta rows, and the
+    // value reads of token 2*i + par (period 4 in i)
+    const int xs = swz<R>(lane);
+    const int mx = G == 4 ? ((lane >> 2) & 1) << 4 : 0;
+    int voff[4];
     {
-      const int t1 = next_end(t0, bend);
-      const bool as = (t1 - t0 == kDTile) && (t0 % kDTile == 0);
-      sk.stage(L, stages, t0 - c0, t1 - t0, as, lane);
-      sv.stage(L, stages + L.bytes, t0 - c0, t1 - t0, as, lane);
-      cp_async_commit();
+      const int ob = BITS == 4 ? 4 * lq : (BITS == 2 ? 2 * lq : 8 * lq);
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) voff[mm] = ob ^ (swz<R>(2 * mm + par) << 4);
     }
-    int cur_blk = -1;
+
+    // finishes the value low-rank part of the current block: accx += alr Rf_v^T
+    auto finish_block = [&]() {
+#pragma unroll
+      for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+        for (int j = 0; j < kRReg; ++j) alr[hh][j] = warp_sum(alr[hh][j]);
+      __syncwarp();
+#pragma unroll
+      for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = e * 32 + lane;
+          float v = accx_s[hh * 128 + c];
+          const float4 r0 = __ldg(reinterpret_cast<const float4*>(rfv + c * rp));
+          v = fmaf(alr[hh][0], r0.x, v);
+          v = fmaf(alr[hh][1], r0.y, v);
+          v = fmaf(alr[hh][2], r0.z, v);
+          v = fmaf(alr[hh][3], r0.w, v);
+          for (int j4 = kRReg; j4 < rb; j4 += 4) {
+            const float4 r4 = __ldg(reinterpret_cast<const float4*>(rfv + c * rp + j4));
+            v = fmaf(alr_s[hh * kMaxR + j4], r4.x, v);
+            v = fmaf(alr_s[hh * kMaxR + j4 + 1], r4.y, v);
+            v = fmaf(alr_s[hh * kMaxR + j4 + 2], r4.z, v);
+            v = fmaf(alr_s[hh * kMaxR + j4 + 3], r4.w, v);
+          }
+          accx_s[hh * 128 + c] = v;
+        }
+#pragma unroll
+      for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+        for (int j = 0; j < kRReg; ++j) alr[hh][j] = 0.0f;
+      __syncwarp();
+      for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
+    };
+
+    int t0 = c0, it = 0, cur_blk = -1;
     while (t0 < c1) {
       if (t0 >= bend) { ++blk; bend = block_end(a, blk); }
       const int t1 = next_end(t0, bend);
       const int nt = t1 - t0;
-      uint8_t* tk = stages + (it & 1) * 2 * L.bytes;
-      uint8_t* tv = tk + L.bytes;
+      const int s = it & 1;
       if (t1 < c1) {   // prefetch the next tile into the other stage
         const int be2 = t1 >= bend ? block_end(a, blk + 1) : bend;
-        const int t2 = next_end(t1, be2);
-        const bool as = (t2 - t1 == kDTile) && (t1 % kDTile == 0);
-        uint8_t* nk = stages + ((it + 1) & 1) * 2 * L.bytes;
-        sk.stage(L, nk, t1 - c0, t2 - t1, as, lane);
-        sv.stage(L, nk + L.bytes, t1 - c0, t2 - t1, as, lane);
-        cp_async_commit();
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
+        issue(s ^ 1, t1, next_end(t1, be2) - t1);
+      }
+      const bool landed = mbar_wait(&bars[s], (uint32_t)(it >> 1) & 1u);
+      if (!__all_sync(0xFFFFFFFFu, landed)) {
+        // give up on this split; let the other stage's copies land first
+        if (t1 < c1) mbar_wait(&bars[s ^ 1], (uint32_t)((it + 1) >> 1) & 1u);
+        return;
       }
       __syncwarp();
+      const uint8_t* tkc = wb + (2 * s) * L.cb;
+      const uint8_t* tvc = tkc + L.cb;
+      const uint8_t* tkm = wb + L.meta0 + (2 * s) * L.mb;
+      const uint8_t* tvm = tkm + L.mb;
+      const uint8_t* tkr = wb + L.rest0 + (2 * s) * L.rb;
+      const uint8_t* tvr = tkr + L.rb;
 
       if (blk != cur_blk) {
         // finish the previous block's value low-rank part, then switch Rf
-        if (cur_blk >= 0) {
+        if (cur_blk >= 0) finish_block();
+        cur_blk = blk;
+        rb = blk == 0 ? a.blk0_rank : a.buffer_rank;
+        const size_t rf0 = ((size_t)unit * a.nblk_max + blk) * 128 * rp;
+        rfk = a.K.rfac + rf0;
+        rfv = a.V.rfac + rf0;
+        // u = Rf_k^T q for every query head
 #pragma unroll
-          for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-            for (int j = 0; j < kRReg; ++j) alr[hh][j] = warp_sum(alr[hh][j]);
-#pragma unroll
-          for (int hh = 0; hh < HQ; ++hh)
+        for (int hh = 0; hh < HQ; ++hh)
+          for (int j4 = 0; j4 < rb; j4 += 4) {
+            float u4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c = e * 32 + lane;
-              float v = accx_s[hh * 128 + c];
-#pragma unroll
-              for (int j = 0; j < kRReg; ++j) if (j < rb) v = fmaf(alr[hh][j], rfv[j * 128 + c], v);
-              for (int j = kRReg; j < rb; ++j) v = fmaf(alr_s[hh * kMaxR + j], rfv[j * 128 + c], v);
-              accx_s[hh * 128 + c] = v;
+              const float4 r4 = __ldg(reinterpret_cast<const float4*>(rfk + c * rp + j4));
+              const float qv = q_s[hh * 128 + c];
+              u4[0] = fmaf(r4.x, qv, u4[0]);
+              u4[1] = fmaf(r4.y, qv, u4[1]);
+              u4[2] = fmaf(r4.z, qv, u4[2]);
+              u4[3] = fmaf(r4.w, qv, u4[3]);
             }
 #pragma unroll
-          for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-            for (int j = 0; j < kRReg; ++j) alr[hh][j] = 0.0f;
-          __syncwarp();
-          for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
-        }
-        cur_blk = blk;
-        rb = blk == 0 ? a.blk0_rank : a.buffer_rank;
-        const size_t rf0 = ((size_t)unit * a.nblk_max + blk) * rm * 128;
-        rfk = a.K.rfac + rf0;
-        rfv = a.V.rfac + rf0;
-#pragma unroll
-        for (int hh = 0; hh < HQ; ++hh)
-          for (int j = 0; j < rb; ++j) {
-            float part = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) part = fmaf(__ldg(rfk + j * 128 + e * 32 + lane), q_s[hh * 128 + e * 32 + lane], part);
-            part = warp_sum(part);
-            if (lane == 0) u_s[hh * kMaxR + j] = part;
+            for (int jj = 0; jj < 4; ++jj) {
+              const float v = warp_sum(u4[jj]);
+              if (lane == 0) u_s[hh * kMaxR + j4 + jj] = v;
+            }
           }
         __syncwarp();
       }
@@ -361,9 +518,11 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
       // ---------------- scores: lane = token
       const int t = lane;
       const bool live = t < nt;
-      float s[HQ];
+      const uint8_t* kmrow = tkm + t * G * 8;
+      const uint8_t* vmrow = tvm + t * G * 8;
+      float s_[HQ];
       {
-        const uint32_t* crow = reinterpret_cast<const uint32_t*>(tk + L.codes + t * kStride);
+        const uint8_t* crow = tkc + t * R;
         uint64_t sb[HQ][4][2];   // per 32-channel block, two independent chains
 #pragma unroll
         for (int hh = 0; hh < HQ; ++hh)
@@ -371,14 +530,14 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
           for (int bk = 0; bk < 4; ++bk) { sb[hh][bk][0] = 0; sb[hh][bk][1] = 0; }
 #pragma unroll
         for (int j = 0; j < W / 4; ++j) {
-          const uint4 wv = *reinterpret_cast<const uint4*>(crow + 4 * j);
+          const uint4 wv = *reinterpret_cast<const uint4*>(crow + ((j ^ xs) << 4));
           const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
           for (int wi = 0; wi < 4; ++wi) {
             const int cbase = (4 * j + wi) * CF::kPerWord;
             const int bk = cbase >> 5;
             float f[CF::kPerWord];
-            CF::word(wd[wi], f);
+            CF::word(wd[wi], f, one);
 #pragma unroll
             for (int e = 0; e < CF::kPerWord; e += 4) {
               const int ch = ((cbase + e) >> 2) & 1;
@@ -391,7 +550,8 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
             }
           }
         }
-        const float2* mt = reinterpret_cast<const float2*>(tk + L.meta) + t * G;
+        float2 sz[4];
+        meta_row(kmrow, G, mx, sz);
         const int bpg = a.g >> 5;   // 32-channel blocks per group
 #pragma unroll
         for (int hh = 0; hh < HQ; ++hh) {
@@ -407,82 +567,92 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
                 qsw += qw_blk[hh][bk];
                 qss += qs_blk[hh][bk];
               }
-            const float2 sz = mt[gi];
-            v = fmaf(sz.x, f - qsw, v);
-            v = fmaf(sz.y, qss, v);
+            v = fmaf(sz[gi].x, f - qsw, v);
+            v = fmaf(sz[gi].y, qss, v);
           }
-          s[hh] = v;
+          s_[hh] = v;
         }
         if (live) {
           // low-rank part and outlier fix-ups
           float lt[kRReg];
 #pragma unroll
-          for (int j = 0; j < kRReg; ++j) lt[j] = j < rb ? stage_l<T>(tk, L, t, j, rm) : 0.0f;
+          for (int j = 0; j < kRReg; ++j) lt[j] = j < rb ? l_at<T>(tkr + L.lf, t, j, rm) : 0.0f;
 #pragma unroll
           for (int j = 0; j < kRReg; ++j)
 #pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(lt[j], j < rb ? u_s[hh * kMaxR + j] : 0.0f, s[hh]);
+            for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(lt[j], j < rb ? u_s[hh * kMaxR + j] : 0.0f, s_[hh]);
           for (int j = kRReg; j < rb; ++j) {
-            const float lj = stage_l<T>(tk, L, t, j, rm);
+            const float lj = l_at<T>(tkr + L.lf, t, j, rm);
 #pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(lj, u_s[hh * kMaxR + j], s[hh]);
+            for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(lj, u_s[hh * kMaxR + j], s_[hh]);
           }
           if (k <= kFast && rb <= kRReg) {
             int cix[kFast];
             float fx[kFast];
-            outlier_fixes<T, kRReg>(tk, L, t, k, G, rb, lt, rfk, lg, cix, fx);
+            outlier_fixes<T>(tkr, L.oval, kmrow, mx, t, k, lg, lt, rfk, rp, cix, fx);
 #pragma unroll
             for (int i = 0; i < kFast; ++i)
 #pragma unroll
-              for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(q_s[hh * 128 + cix[i]], fx[i], s[hh]);
-          } else
-          for (int i = 0; i < k; ++i) {
-            const int c = tk[L.oidx + t * k + i];
-            float lr = 0.0f;
+              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(q_s[hh * 128 + cix[i]], fx[i], s_[hh]);
+          } else {
+            for (int i = 0; i < k; ++i) {
+              const int c = tkr[t * k + i];
+              const float lr = lowrank_at<T>(tkr + L.lf, t, rm, rb, rfk, rp, c);
+              const float xo = (float)reinterpret_cast<const T*>(tkr + L.oval)[t * k + i];
+              const float fix = xo - (meta_at(kmrow, c >> lg, mx).y + lr);
 #pragma unroll
-            for (int j = 0; j < kRReg; ++j) lr = fmaf(lt[j], j < rb ? __ldg(rfk + j * 128 + c) : 0.0f, lr);
-            for (int j = kRReg; j < rb; ++j) lr = fmaf(stage_l<T>(tk, L, t, j, rm), __ldg(rfk + j * 128 + c), lr);
-            const float xo = (float)reinterpret_cast<const T*>(tk + L.oval)[t * k + i];
-            const float fix = xo - (mt[c >> lg].y + lr);
-#pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(q_s[hh * 128 + c], fix, s[hh]);
+              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(q_s[hh * 128 + c], fix, s_[hh]);
+            }
           }
         }
 #pragma unroll
-        for (int hh = 0; hh < HQ; ++hh) s[hh] = live ? s[hh] * a.scale_log2 : -INFINITY;
+        for (int hh = 0; hh < HQ; ++hh) s_[hh] = live ? s_[hh] * a.scale_log2 : -INFINITY;
       }
 
-      // ---------------- online softmax (rescale only when the max moved)
+      // ---------------- online softmax; the reference m moves only when the
+      // tile's maximum passes it by more than 2^kLazy
       float p[HQ];
 #pragma unroll
       for (int hh = 0; hh < HQ; ++hh) {
-        const float mnew = fmaxf(m[hh], warp_max(s[hh]));
-        p[hh] = live ? exp2f(s[hh] - mnew) : 0.0f;
-        if (mnew != m[hh]) {   // warp-uniform
-          const float al = exp2f(m[hh] - mnew);
-          lsum[hh] *= al;
-          const uint64_t al2 = pk2(al, al);
+        const float mt = warp_max(s_[hh]);
+        if (mt > m[hh] + kLazy) {   // warp-uniform
+          if (m[hh] != -INFINITY) {
+            const float al = exp2f(m[hh] - mt);
+            lsum[hh] *= al;
+            const uint64_t al2 = pk2(al, al);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            acc[hh][e] = fma2(acc[hh][e], al2, 0);
-            sw[hh][e] *= al;
-            spm[hh][e] *= al;
-            alr[hh][e] *= al;
-            corr_s[hh * 128 + e * 32 + lane] *= al;
-            accx_s[hh * 128 + e * 32 + lane] *= al;
+            for (int e = 0; e < 4; ++e) {
+              acc[hh][e] = fma2(acc[hh][e], al2, 0);
+              sw[hh][e] *= al;
+              spm[hh][e] *= al;
+              alr[hh][e] *= al;
+              accx_s[hh * 128 + e * 32 + lane] *= al;
+            }
+            if (rb > kRReg && lane < kMaxR) alr_s[hh * kMaxR + lane] *= al;
+            // the value outlier sums in global memory
+            __threadfence();
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float* pc = part_row + hh * hstride + 2 + e * 32 + lane;
+              st_gpu(pc, ld_gpu(pc) * al);
+            }
+            __threadfence();
+            __syncwarp();
           }
-          if (rb > kRReg && lane < kMaxR) alr_s[hh * kMaxR + lane] *= al;
+          m[hh] = mt;
         }
-        m[hh] = mnew;
+        p[hh] = live ? exp2f(s_[hh] - m[hh]) : 0.0f;
         lsum[hh] += p[hh];
       }
       // value-side per-token weights w = p * scale; zero-point and low-rank sums
       {
-        const float2* mv = reinterpret_cast<const float2*>(tv + L.meta) + t * G;
+        float2 vsz[4];
+        meta_row(vmrow, G, mx, vsz);
 #pragma unroll
         for (int gi = 0; gi < 4; ++gi) {
           if (gi >= G) break;
-          const float2 sz = live ? mv[gi] : make_float2(0.0f, 0.0f);
+          const float2 sz = live ? vsz[gi] : make_float2(0.0f, 0.0f);
 #pragma unroll
           for (int hh = 0; hh < HQ; ++hh) {
             const float wv = p[hh] * sz.x;
@@ -492,79 +662,78 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
           }
         }
         if (live) {
+          float lv[kRReg];
 #pragma unroll
-          for (int j = 0; j < kRReg; ++j) {
-            const float lj = j < rb ? stage_l<T>(tv, L, t, j, rm) : 0.0f;
+          for (int j = 0; j < kRReg; ++j) lv[j] = j < rb ? l_at<T>(tvr + L.lf, t, j, rm) : 0.0f;
 #pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) alr[hh][j] = fmaf(p[hh], lj, alr[hh][j]);
-          }
-          // value outliers
+          for (int j = 0; j < kRReg; ++j)
+#pragma unroll
+            for (int hh = 0; hh < HQ; ++hh) alr[hh][j] = fmaf(p[hh], lv[j], alr[hh][j]);
+          // value outliers: p * fix lands on channel c of the split's row
           if (k <= kFast && rb <= kRReg) {
-            float lv[kRReg];
-#pragma unroll
-            for (int j = 0; j < kRReg; ++j) lv[j] = j < rb ? stage_l<T>(tv, L, t, j, rm) : 0.0f;
             int cix[kFast];
             float fx[kFast];
-            outlier_fixes<T, kRReg>(tv, L, t, k, G, rb, lv, rfv, lg, cix, fx);
+            outlier_fixes<T>(tvr, L.oval, vmrow, mx, t, k, lg, lv, rfv, rp, cix, fx);
 #pragma unroll
             for (int i = 0; i < kFast; ++i)
               if (i < k)
 #pragma unroll
-                for (int hh = 0; hh < HQ; ++hh) atomicAdd(&corr_s[hh * 128 + cix[i]], p[hh] * fx[i]);
-          } else
-          for (int i = 0; i < k; ++i) {
-            const int c = tv[L.oidx + t * k + i];
-            float lr = 0.0f;
+                for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + cix[i], p[hh] * fx[i]);
+          } else {
+            for (int i = 0; i < k; ++i) {
+              const int c = tvr[t * k + i];
+              const float lr = lowrank_at<T>(tvr + L.lf, t, rm, rb, rfv, rp, c);
+              const float xo = (float)reinterpret_cast<const T*>(tvr + L.oval)[t * k + i];
+              const float fix = xo - (meta_at(vmrow, c >> lg, mx).y + lr);
 #pragma unroll
-            for (int j = 0; j < kRReg; ++j)
-              lr = fmaf(j < rb ? stage_l<T>(tv, L, t, j, rm) : 0.0f, j < rb ? __ldg(rfv + j * 128 + c) : 0.0f, lr);
-            for (int j = kRReg; j < rb; ++j) lr = fmaf(stage_l<T>(tv, L, t, j, rm), __ldg(rfv + j * 128 + c), lr);
-            const float xo = (float)reinterpret_cast<const T*>(tv + L.oval)[t * k + i];
-            const float fix = xo - (mv[c >> lg].y + lr);
-#pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) atomicAdd(&corr_s[hh * 128 + c], p[hh] * fix);
+              for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + c, p[hh] * fix);
+            }
           }
         }
       }
       for (int j = kRReg; j < rb; ++j)   // ranks beyond the register slots
 #pragma unroll
         for (int hh = 0; hh < HQ; ++hh) {
-          const float v = warp_sum(live ? p[hh] * stage_l<T>(tv, L, t, j, rm) : 0.0f);
+          const float v = warp_sum(live ? p[hh] * l_at<T>(tvr + L.lf, t, j, rm) : 0.0f);
           if (lane == 0) alr_s[hh * kMaxR + j] += v;
         }
       __syncwarp();
 
-      // ---------------- values: lane = 8 channels, two tokens per step
+      // ---------------- values: lane = 8 channels, tokens 2*i + par. Tokens
+      // past nt have w = 0 (their codes are finite), so every tile runs all 16.
       {
-        const uint8_t* row = tv + L.codes + par * kStride;
+        const uint8_t* vrow = tvc + par * R;
         const float* wrow = w_s + (par * G + my_g) * HQ;
-#pragma unroll 2
-        for (int tt = par; tt < nt; tt += 2) {
-          float f[8];
-          if constexpr (BITS == 4) {
-            CF::word(reinterpret_cast<const uint32_t*>(row)[lq], f);
-          } else if constexpr (BITS == 2) {
-            float ff[16];
-            CF::word(reinterpret_cast<const uint16_t*>(row)[lq], ff);
+#pragma unroll 1
+        for (int i4 = 0; i4 < kDTile / 2; i4 += 4) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = ff[e];
-          } else {
-            const uint2 ww = reinterpret_cast<const uint2*>(row)[lq];
-            float fa[4], fb[4];
-            CF::word(ww.x, fa);
-            CF::word(ww.y, fb);
+          for (int mm = 0; mm < 4; ++mm) {
+            const uint8_t* row = vrow + (i4 + mm) * 2 * R + voff[mm];
+            const float* wr = wrow + (i4 + mm) * 2 * G * HQ;
+            float f[8];
+            if constexpr (BITS == 4) {
+              CF::word(*reinterpret_cast<const uint32_t*>(row), f, one);
+            } else if constexpr (BITS == 2) {
+              float ff[16];
+              CF::word(*reinterpret_cast<const uint16_t*>(row), ff, one);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) { f[e] = fa[e]; f[4 + e] = fb[e]; }
+              for (int e = 0; e < 8; ++e) f[e] = ff[e];
+            } else {
+              const uint2 ww = *reinterpret_cast<const uint2*>(row);
+              float fa[4], fb[4];
+              CF::word(ww.x, fa, one);
+              CF::word(ww.y, fb, one);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) { f[e] = fa[e]; f[4 + e] = fb[e]; }
+            }
+#pragma unroll
+            for (int hh = 0; hh < HQ; ++hh) {
+              const float wv = wr[hh];
+              const uint64_t w2 = pk2(wv, wv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[hh][e] = fma2(w2, pk2(f[2 * e], f[2 * e + 1]), acc[hh][e]);
+            }
           }
-#pragma unroll
-          for (int hh = 0; hh < HQ; ++hh) {
-            const float wv = wrow[hh];
-            const uint64_t w2 = pk2(wv, wv);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[hh][e] = fma2(w2, pk2(f[2 * e], f[2 * e + 1]), acc[hh][e]);
-          }
-          row += 2 * kStride;
-          wrow += 2 * G * HQ;
         }
       }
       __syncwarp();
@@ -572,23 +741,7 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
       ++it;
     }
     // last block's value low-rank part
-    if (cur_blk >= 0) {
-#pragma unroll
-      for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-        for (int j = 0; j < kRReg; ++j) alr[hh][j] = warp_sum(alr[hh][j]);
-#pragma unroll
-      for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = e * 32 + lane;
-          float v = accx_s[hh * 128 + c];
-#pragma unroll
-          for (int j = 0; j < kRReg; ++j) if (j < rb) v = fmaf(alr[hh][j], __ldg(rfv + j * 128 + c), v);
-          for (int j = kRReg; j < rb; ++j) v = fmaf(alr_s[hh * kMaxR + j], __ldg(rfv + j * 128 + c), v);
-          accx_s[hh * 128 + c] = v;
-        }
-    }
+    if (cur_blk >= 0) finish_block();
   } else {
     // ---------------- the streaming buffer: exact tokens, lane = token for keys
     const size_t brow = (size_t)unit * a.n_b;
@@ -632,6 +785,7 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
       __syncwarp();
     }
   }
+  if (comp) __threadfence();   // the value outlier sums, before they are read back
   __syncwarp();
 
   // ---------------- partial result of this split
@@ -651,13 +805,14 @@ __global__ void __launch_bounds__(kDThreads) decode_warp(const DecodeArgs a) {
       v[2 * e] = lo2(acc[hh][e]) + __shfl_xor_sync(0xFFFFFFFFu, lo2(acc[hh][e]), 16);
       v[2 * e + 1] = hi2(acc[hh][e]) + __shfl_xor_sync(0xFFFFFFFFu, hi2(acc[hh][e]), 16);
     }
-    float* dst = a.part + (((size_t)b * a.Hq + (size_t)h * HQ + hh) * a.nsplit + sp) * 130;
+    float* dst = part_row + hh * hstride;
     if (lane == 0) { dst[0] = m[hh]; dst[1] = l_all; }
     if (par == 0) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int c = 8 * lq + e;
-        dst[2 + c] = CF::inv_weight(c) * (v[e] - swg) + spg + accx_s[hh * 128 + c] + corr_s[hh * 128 + c];
+        const float corr = comp ? ld_gpu(dst + 2 + c) : 0.0f;
+        dst[2 + c] = CF::inv_weight(c) * (v[e] - swg) + spg + accx_s[hh * 128 + c] + corr;
       }
     }
   }
@@ -687,19 +842,24 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeArgs a) {
 
 void decode_plan(DecodeArgs& a, int num_sms) {
   const int units = a.B * a.H;
-  // per-tensor tile layout in shared memory (16-byte aligned regions)
   auto r16 = [](int x) { return (x + 15) & ~15; };
-  const int esz = a.dtype == GEAR_F32 ? 4 : 2;
+  const int esz = a.dtype == GEAR_F32 ? 4 : 2;   // oval and L rows share the width
   TileLayout& L = a.tl;
-  L.codes = 0;
-  L.meta = L.codes + kDTile * (a.W + 4) * 4;
-  L.oidx = L.meta + kDTile * a.G * 8;
-  L.oval = L.oidx + r16(kDTile * (a.k > 0 ? a.k : 1));
-  L.lf = L.oval + r16(kDTile * (a.k > 0 ? a.k : 1) * esz);
-  L.bytes = L.lf + r16(kDTile * a.r_max * (a.dtype == GEAR_F32 ? 4 : 2));
+  L.cb = kDTile * a.W * 4;
+  L.mb = kDTile * a.G * 8;
+  L.oval = r16(kDTile * a.k);
+  L.lf = L.oval + r16(kDTile * a.k * esz);
+  L.rb = L.lf + r16(kDTile * a.r_max * esz);
+  L.meta0 = 4 * L.cb;
+  L.rest0 = L.meta0 + 4 * L.mb;
+  L.floats = L.rest0 + 4 * L.rb;
   const int hq = a.hq;
-  const int floats = 2 * hq * 128 + 2 * hq * kMaxR + kDTile * a.G * hq + 2 * hq * 128;
-  a.warp_bytes = r16(floats * 4) + 4 * L.bytes;
+  const int floats = 2 * hq * 128 + 2 * hq * kMaxR + kDTile * a.G * hq + hq * 128;
+  L.bars = L.floats + r16(floats * 4);
+  L.bytes = (L.bars + 16 + 1023) & ~1023;
+  const int meta_tx = a.G >= 2 ? 2 * L.mb : 0;
+  L.tx_part = 2 * L.cb + meta_tx;
+  L.tx_full = L.tx_part + 2 * kDTile * (a.k + a.k * esz + a.r_max * esz) + (a.G >= 2 ? 0 : 2 * L.mb);
   int nsc = 0;
   if (a.n_comp > 0) {
     // about 48 warps per SM over the whole grid, chunks of whole 32-token tiles
@@ -720,8 +880,8 @@ void decode_plan(DecodeArgs& a, int num_sms) {
 size_t decode_workspace_bytes(int B, int Hq, int nsplit) { return (size_t)B * Hq * nsplit * 130 * sizeof(float); }
 
 template <typename T, int BITS, int HQ>
-static cudaError_t launch_warp(const DecodeArgs& a, cudaStream_t st) {
-  const size_t smem = 4 * (size_t)a.warp_bytes;
+static cudaError_t launch_warp(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
+  const size_t smem = 4 * (size_t)a.tl.bytes + 1024;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
     cudaError_t e = cudaFuncSetAttribute(decode_warp<T, BITS, HQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -730,35 +890,66 @@ static cudaError_t launch_warp(const DecodeArgs& a, cudaStream_t st) {
     configured_smem = (int)smem;
   }
   const int grid = (a.total_splits + 3) / 4;
-  decode_warp<T, BITS, HQ><<<grid, kDThreads, smem, st>>>(a);
+  decode_warp<T, BITS, HQ><<<grid, kDThreads, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
 
 template <typename T, int BITS>
-static cudaError_t launch_hq(const DecodeArgs& a, cudaStream_t st) {
+static cudaError_t launch_hq(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
   switch (a.hq) {
-    case 1: return launch_warp<T, BITS, 1>(a, st);
-    case 2: return launch_warp<T, BITS, 2>(a, st);
-    case 4: return launch_warp<T, BITS, 4>(a, st);
-    case 8: return launch_warp<T, BITS, 8>(a, st);
+    case 1: return launch_warp<T, BITS, 1>(maps, a, st);
+    case 2: return launch_warp<T, BITS, 2>(maps, a, st);
+    case 4: return launch_warp<T, BITS, 4>(maps, a, st);
+    case 8: return launch_warp<T, BITS, 8>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }
 
 template <typename T>
-static cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t st) {
+static cudaError_t launch_bits(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
   switch (a.bits) {
-    case 2: return launch_hq<T, 2>(a, st);
-    case 4: return launch_hq<T, 4>(a, st);
-    default: return launch_hq<T, 8>(a, st);
+    case 2: return launch_hq<T, 2>(maps, a, st);
+    case 4: return launch_hq<T, 4>(maps, a, st);
+    default: return launch_hq<T, 8>(maps, a, st);
   }
 }
 
+// 2-D map over rows of `inner` elements of 4 bytes, 32-row boxes.
+static bool row_map(PFN_encodeTiled enc, CUtensorMap* m, const void* base, CUtensorMapDataType dt, int inner,
+                    uint64_t rows) {
+  const int row_bytes = inner * 4;
+  const CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : row_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                  : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)inner, (cuuint32_t)kDTile};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t st) {
-  cudaError_t e;
-  if (a.dtype == GEAR_F16) e = launch_bits<__half>(a, st);
-  else if (a.dtype == GEAR_BF16) e = launch_bits<__nv_bfloat16>(a, st);
-  else e = launch_bits<float>(a, st);
+  cudaError_t e = cudaSuccess;
+  if (a.nsplit_comp > 0 || a.n_buf > 0) {
+    DecodeMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (a.nsplit_comp > 0) {
+      PFN_encodeTiled enc = tensor_map_encoder();
+      if (!enc) return cudaErrorNotSupported;
+      const uint64_t rows = (uint64_t)a.B * a.H * a.n_max;
+      bool ok = row_map(enc, &maps.kc, a.K.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows) &&
+                row_map(enc, &maps.vc, a.V.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows);
+      if (ok && a.G >= 2)
+        ok = row_map(enc, &maps.km, a.K.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows) &&
+             row_map(enc, &maps.vm, a.V.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows);
+      if (!ok) return cudaErrorInvalidValue;
+    }
+    if (a.dtype == GEAR_F16) e = launch_bits<__half>(maps, a, st);
+    else if (a.dtype == GEAR_BF16) e = launch_bits<__nv_bfloat16>(maps, a, st);
+    else e = launch_bits<float>(maps, a, st);
+  }
   if (e != cudaSuccess) return e;
   const int nbj = a.B * a.Hq;
   if (a.out_dtype == GEAR_F32) decode_combine<float><<<nbj, 128, 0, st>>>(a);
@@ -785,8 +976,9 @@ __global__ void __launch_bounds__(128) dense_kernel(const DenseArgs a) {
       const uint32_t code = (a.C.codes[row * a.W + c / kPerWord] >> (BITS * (c % kPerWord))) & ((1u << BITS) - 1u);
       const float2 sz = reinterpret_cast<const float2*>(a.C.meta)[row * a.G + c / a.g];
       v = __fmaf_rn((float)code, sz.x, sz.y);
-      const float* rf = a.C.rfac + ((size_t)u * a.nblk_max + blk) * a.r_max * 128;
-      for (int j = 0; j < rb; ++j) v = fmaf(load_lfac<T>(a.C.lfac, row * a.r_max + j), rf[j * 128 + c], v);
+      const int rp = rpad_of(a.r_max);
+      const float* rf = a.C.rfac + (((size_t)u * a.nblk_max + blk) * 128 + c) * rp;
+      for (int j = 0; j < rb; ++j) v = fmaf(load_lfac<T>(a.C.lfac, row * a.r_max + j), rf[j], v);
       for (int i = 0; i < a.k; ++i)
         if (a.C.oidx[row * a.k + i] == c) v = load_elem<T>(a.C.oval, row * a.k + i);
     } else {

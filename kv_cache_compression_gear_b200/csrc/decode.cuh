@@ -1,6 +1,7 @@
 // decode.cuh -- argument blocks of the GEAR decode-attention kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -17,9 +18,26 @@ struct CacheView {
   const void* buf;
 };
 
-// Byte offsets of one tensor's 32-token tile in shared memory.
+// Per-warp shared memory of decode_warp. Tile idx = 2 * stage + tensor
+// (tensor 0 = keys, 1 = values) has its codes at idx * cb, its meta at
+// meta0 + idx * mb and the rest (oidx | oval | lf) at rest0 + idx * rb, all
+// from the warp's 1024-byte-aligned base.
 struct TileLayout {
-  int32_t codes, meta, oidx, oval, lf, bytes;
+  int32_t cb, mb, rb;      // bytes per tile: codes, meta, rest
+  int32_t oval, lf;        // offsets of oval and lf inside the rest
+  int32_t meta0, rest0;    // offsets of tile 0's meta and rest
+  int32_t floats;          // offset of the float scratch
+  int32_t bars;            // offset of the two stage barriers
+  int32_t bytes;           // bytes per warp, a multiple of 1024
+  int32_t tx_full;         // bytes a stage barrier expects for a whole, aligned tile
+  int32_t tx_part;         // ... for another tile (codes and meta only; the rest is copied by the lanes)
+};
+
+// Tensor maps of the codes and meta arrays of both tensors ([U * n_max] rows).
+// The meta maps are used when G >= 2 (a meta row of one group is 8 bytes,
+// below the 16-byte minimum of a tensor copy).
+struct DecodeMaps {
+  CUtensorMap kc, vc, km, vm;
 };
 
 struct DecodeArgs {
@@ -31,6 +49,7 @@ struct DecodeArgs {
   int32_t n_comp, n_buf;
   int32_t blk0_len, blk0_rank, buffer_rank;
   float scale_log2;       // softmax scale * log2(e)
+  uint32_t one_bits;      // 0x3F800000 (1.0f), passed so that it stays in a register
   const void* q;          // [B][Hq][128] cache dtype
   void* out;              // [B][Hq][128] out dtype
   int32_t out_dtype;
@@ -39,7 +58,6 @@ struct DecodeArgs {
   int32_t nsplit_comp;    // splits over compressed tokens, per unit
   int32_t nsplit;         // + 1 if the buffer is non-empty
   int32_t total_splits;   // units * nsplit: one warp each
-  int32_t warp_bytes;     // shared memory per warp
   TileLayout tl;
 };
 

@@ -830,11 +830,13 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
         float* zrow = a.zbuf + ((int64_t)u * 128 + i) * 16;
 #pragma unroll
         for (int j = 0; j < 16; ++j) zrow[j] = (j < RM && j < r) ? (float)(zq[j < RM ? j : 0] * sL) : 0.0f;
-        for (int j = 0; j < a.r_max; ++j) {
+        const int rp = rpad_of(a.r_max);
+        float* rrow = a.rfac + (((int64_t)u * a.nblk_max + a.blk) * 128 + i) * rp;
+        for (int j = 0; j < rp; ++j) {
           double wv = 0.0;
 #pragma unroll
           for (int jj = 0; jj < RM; ++jj) if (jj == j) wv = wq[jj];
-          a.rfac[(((int64_t)u * a.nblk_max + a.blk) * a.r_max + j) * 128 + i] = j < r ? (float)(wv * sR) : 0.0f;
+          rrow[j] = j < r ? (float)(wv * sR) : 0.0f;
         }
       }
     }
@@ -1000,11 +1002,7 @@ static cudaError_t launch_e3_b(const EncodeArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static PFN_encodeTiled get_encode_tiled() {
+PFN_encodeTiled tensor_map_encoder() {
   static PFN_encodeTiled fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -1032,7 +1030,7 @@ int encode_maxc(int64_t total_tiles, int grid, int tpu) {
 
 cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
   const int esz = a.dtype == GEAR_F32 ? 4 : 2;
-  PFN_encodeTiled enc = get_encode_tiled();
+  PFN_encodeTiled enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap map;
   const cuuint64_t dims[2] = {128, (cuuint64_t)a.U * (cuuint64_t)a.n};

@@ -179,14 +179,14 @@ class Cache:
         n = c.n_max
         ld = torch.float32 if self.dtype == torch.float32 else torch.float16
         k = max(c.k, 1)
+        rp = (c.r_max + 3) // 4 * 4
         return {
             "codes": self._view(c.codes, U * n * c.W, torch.int32).view(U, n, c.W),
             "meta": self._view(c.meta, U * n * c.G * 2, torch.float32).view(U, n, c.G, 2),
             "oidx": self._view(c.oidx, U * n * k, torch.uint8).view(U, n, k),
             "oval": self._view(c.oval, U * n * k, self.dtype).view(U, n, k),
             "lfac": self._view(c.lfac, U * n * c.r_max, ld).view(U, n, c.r_max),
-            "rfac": self._view(c.rfac, U * c.nblk_max * c.r_max * c.d, torch.float32).view(U, c.nblk_max, c.r_max,
-                                                                                          c.d),
+            "rfac": self._view(c.rfac, U * c.nblk_max * c.d * rp, torch.float32).view(U, c.nblk_max, c.d, rp),
             "buf": self._view(c.buf, U * c.p.buffer_len * c.d, self.dtype).view(U, c.p.buffer_len, c.d),
         }
 

@@ -46,7 +46,7 @@ def gpu_block(cache, u: int, t0: int, t1: int, blk: int, rank: int):
         e += 1
     e //= 2
     L = A["lfac"][u, t0:t1, :rank].float().cpu().numpy().astype(np.float64) * 2.0 ** -e
-    Rf = A["rfac"][u, blk, :rank].cpu().numpy().astype(np.float64).T * 2.0 ** e   # [d][r]
+    Rf = A["rfac"][u, blk, :, :rank].cpu().numpy().astype(np.float64) * 2.0 ** e   # [d][r]
     return {
         "codes": A["codes"][u, t0:t1].cpu().numpy(),
         "meta": A["meta"][u, t0:t1].cpu().numpy(),
