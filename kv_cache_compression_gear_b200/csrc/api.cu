@@ -88,6 +88,7 @@ static gear_status encode_block(gear_cache* c, const void* kv, int n, int t_off,
   a.t_off = t_off;
   a.blk = blk;
   a.e_blk = e_of_len(n);
+  a.one_bits = 0x3F800000u;
   a.n_max = c->n_max;
   a.nblk_max = c->nblk_max;
   a.W = c->W;

@@ -40,6 +40,54 @@ typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 PFN_encodeTiled tensor_map_encoder();
 
+// 2-D tensor map over a cache array of rows of `inner` 4-byte elements, boxes
+// of `box_rows` whole rows; rows of 32, 64 or 128 bytes get the matching
+// 16-byte-chunk swizzle (byte o of box row t at t*R + (o ^ (sw(t) << 4)),
+// sw(t) = ((t*R) >> 7) & (R/16 - 1)), others none. Out-of-range rows read 0.
+static inline bool cache_row_map(PFN_encodeTiled enc, CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                                 int inner, uint64_t rows, int box_rows) {
+  const int row_bytes = inner * 4;
+  const CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : row_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                  : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)inner, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Codes as floats without integer conversion. Byte b of a code word is moved
+// to mantissa bits 15..22 by one shift; each code of the byte is then masked
+// into 1.0f: f = 1 + code * 2^(pos*BITS - 8), pos = index of the code inside
+// its byte. The power of two 2^(8 - pos*BITS) is folded into a pre-scaled copy
+// of q (keys) or applied once per channel at the end (values), both exact.
+template <int BITS>
+struct CodeFloats {
+  static constexpr int kPerByte = 8 / BITS;
+  static constexpr int kPerWord = 32 / BITS;
+  // all codes of one 32-bit word, in channel order. `one` holds the bits of
+  // 1.0f in a register, so that mask and exponent go into one LOP3 each.
+  __device__ static __forceinline__ void word(uint32_t w, float (&f)[kPerWord], uint32_t one) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int sh = 15 - 8 * b;
+      const uint32_t v = sh >= 0 ? (w << sh) : (w >> (-sh));
+#pragma unroll
+      for (int q = 0; q < kPerByte; ++q) {
+        const uint32_t m = ((1u << BITS) - 1u) << (15 + q * BITS);
+        f[b * kPerByte + q] = __uint_as_float((v & m) | one);
+      }
+    }
+  }
+  // weight that turns (f - 1) back into the code, for the code at channel c
+  __host__ __device__ static constexpr float inv_weight(int c) {
+    return (float)(1 << (8 - (c % kPerByte) * BITS));
+  }
+};
+
 // Row length of the stored Rf factors: r_max rounded up to a multiple of 4, so
 // that one channel's row is a whole number of 16-byte vectors.
 __host__ __device__ constexpr int rpad_of(int r_max) { return (r_max + 3) & ~3; }

@@ -102,35 +102,6 @@ __device__ __forceinline__ int swz(int t) {
   return ((t * R) >> 7) & (R / 16 - 1);
 }
 
-// Codes as floats without integer conversion. Byte b of a code word is moved
-// to mantissa bits 15..22 by one shift; each code of the byte is then masked
-// into 1.0f: f = 1 + code * 2^(pos*BITS - 8), pos = index of the code inside
-// its byte. The power of two 2^(8 - pos*BITS) is folded into a pre-scaled copy
-// of q (keys) or applied once per channel at the end (values), both exact.
-template <int BITS>
-struct CodeFloats {
-  static constexpr int kPerByte = 8 / BITS;
-  static constexpr int kPerWord = 32 / BITS;
-  // all codes of one 32-bit word, in channel order. `one` holds the bits of
-  // 1.0f in a register, so that mask and exponent go into one LOP3 each.
-  __device__ static __forceinline__ void word(uint32_t w, float (&f)[kPerWord], uint32_t one) {
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int sh = 15 - 8 * b;
-      const uint32_t v = sh >= 0 ? (w << sh) : (w >> (-sh));
-#pragma unroll
-      for (int q = 0; q < kPerByte; ++q) {
-        const uint32_t m = ((1u << BITS) - 1u) << (15 + q * BITS);
-        f[b * kPerByte + q] = __uint_as_float((v & m) | one);
-      }
-    }
-  }
-  // weight that turns (f - 1) back into the code, for the code at channel c
-  __host__ __device__ static constexpr float inv_weight(int c) {
-    return (float)(1 << (8 - (c % kPerByte) * BITS));
-  }
-};
-
 template <typename T>
 __device__ __forceinline__ float l_at(const uint8_t* lf, int t, int j, int rm) {
   if constexpr (sizeof(T) == 4) return reinterpret_cast<const float*>(lf)[t * rm + j];
@@ -914,22 +885,6 @@ static cudaError_t launch_bits(const DecodeMaps& maps, const DecodeArgs& a, cuda
   }
 }
 
-// 2-D map over rows of `inner` elements of 4 bytes, 32-row boxes.
-static bool row_map(PFN_encodeTiled enc, CUtensorMap* m, const void* base, CUtensorMapDataType dt, int inner,
-                    uint64_t rows) {
-  const int row_bytes = inner * 4;
-  const CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                : row_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                                  : CU_TENSOR_MAP_SWIZZLE_NONE;
-  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-  const cuuint32_t box[2] = {(cuuint32_t)inner, (cuuint32_t)kDTile};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t st) {
   cudaError_t e = cudaSuccess;
   if (a.nsplit_comp > 0 || a.n_buf > 0) {
@@ -939,11 +894,11 @@ cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t st) {
       PFN_encodeTiled enc = tensor_map_encoder();
       if (!enc) return cudaErrorNotSupported;
       const uint64_t rows = (uint64_t)a.B * a.H * a.n_max;
-      bool ok = row_map(enc, &maps.kc, a.K.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows) &&
-                row_map(enc, &maps.vc, a.V.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows);
+      bool ok = cache_row_map(enc, &maps.kc, a.K.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kDTile) &&
+                cache_row_map(enc, &maps.vc, a.V.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kDTile);
       if (ok && a.G >= 2)
-        ok = row_map(enc, &maps.km, a.K.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows) &&
-             row_map(enc, &maps.vm, a.V.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows);
+        ok = cache_row_map(enc, &maps.km, a.K.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows, kDTile) &&
+             cache_row_map(enc, &maps.vm, a.V.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows, kDTile);
       if (!ok) return cudaErrorInvalidValue;
     }
     if (a.dtype == GEAR_F16) e = launch_bits<__half>(maps, a, st);

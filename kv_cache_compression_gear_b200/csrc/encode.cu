@@ -27,6 +27,7 @@
 #include <cuda.h>
 
 #include <cfloat>
+#include <cstring>
 
 #include "common.cuh"
 #include "encode.cuh"
@@ -845,110 +846,222 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
 }
 
 // ================================================================ E3 ======
-// L rows: L_t = R_t Z, with R rebuilt from the stored codes and zero points:
-// R = x - fma(code, scale, zero) on every slot, then the outlier slots'
-// contribution (x_o - zero) Z[c_o] is removed again. Each thread takes two
-// tokens (t, t + 64) of a 128-token tile, so every Z entry, duplicated in
-// shared memory, feeds one packed two-token FMA.
-constexpr int kE3Threads = 64;
+// L rows: L_t = R_t Z for every token of the block, with R rebuilt as
+// x - fma(code, scale, zero) on every slot; the outlier slots' contribution
+// (x_o - zero) Z[c_o] is then removed again (their residual is 0).
+// One CTA per 128-token tile of one unit, one thread per token. The tile's
+// input rows (the encoder's tensor map: 128-byte swizzled boxes), code rows
+// (16-byte-chunk swizzle) and, for G >= 2, meta rows arrive by tensor copies
+// on one mbarrier; several CTAs per SM overlap one tile's copies with another
+// tile's arithmetic. A thread accumulates channel pairs in f32x2 registers.
+// Codes become floats by the mantissa trick f = 1 + code * 2^-w (w = 8 - pos
+// * bits for the code at position pos of its byte), so that
+// fma(f - 1, scale * 2^w, zero) is exactly fma(code, scale, zero) as long as
+// scale * 2^8 is finite; a token with a larger scale takes a plain loop.
+constexpr int kE3Threads = 128;
+
+struct E3Maps {
+  CUtensorMap x, codes, meta;   // input rows, cache code rows, cache meta rows (G >= 2)
+};
 
 template <typename T, int BITS, int RMAX>
-__global__ void __launch_bounds__(kE3Threads) encode_lowrank(const EncodeArgs a) {
-  __shared__ __align__(16) float Zd[128][RMAX][2];
-  const int u = blockIdx.y;
-  for (int e = threadIdx.x; e < 128 * RMAX; e += kE3Threads) {
-    const float z = a.zbuf[((int64_t)u * 128 + e / RMAX) * 16 + e % RMAX];
-    Zd[e / RMAX][e % RMAX][0] = z;
-    Zd[e / RMAX][e % RMAX][1] = z;
+struct E3Cfg {
+  static constexpr int kXB = kTile * 128 * (int)sizeof(T);   // input tile
+  static constexpr int kRow = 16 * BITS;                     // code bytes per token
+  static constexpr int kCB = kTile * kRow;                   // code tile
+  static constexpr int kMB = kTile * 32;                     // meta tile (G <= 4)
+  static constexpr int kZOff = kXB + kCB + kMB;              // Z pairs [64][RMAX] float2
+  static constexpr int kBarOff = kZOff + 64 * RMAX * 8;
+  static constexpr int kSmem = kBarOff + 16 + 1024;          // + alignment slack
+};
+
+template <int R>
+__device__ __forceinline__ int swz_rows(int t) {   // chunk swizzle of R-byte rows (R = 32, 64, 128)
+  return ((t * R) >> 7) & (R / 16 - 1);
+}
+
+template <typename T, int BITS, int RMAX>
+__global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_constant__ E3Maps maps, const EncodeArgs a) {
+  using C = E1Cfg<T>;
+  using F = E3Cfg<T, BITS, RMAX>;
+  constexpr int W = 4 * BITS;
+  constexpr int kPerByte = 8 / BITS;
+  extern __shared__ uint8_t e3raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(e3raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xs = sm;
+  uint8_t* cs = sm + F::kXB;
+  uint8_t* ms = cs + F::kCB;
+  float2* Zp = reinterpret_cast<float2*>(sm + F::kZOff);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + F::kBarOff);
+  const int u = blockIdx.y, t0 = blockIdx.x * kTile, t = threadIdx.x;
+  const int G = a.G, k = a.k, r = a.r;
+  const bool meta_tma = G >= 2;
+  const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
+  const int crow = u * a.n_max + a.t_off + t0;   // cache row of the tile's first token
+  if (t == 0) {
+    mbar_init(bar, 1);
+    fence_mbarrier_init();
+    mbar_arrive_expect_tx(bar, (uint32_t)(F::kXB + F::kCB + (meta_tma ? kTile * G * 8 : 0)));
+    for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(xs + b * 16384, &maps.x, bar, b * C::kBoxCols, u * a.n + t0);
+    tma_load_2d(cs, &maps.codes, bar, 0, crow);
+    if (meta_tma) tma_load_2d(ms, &maps.meta, bar, 0, crow);
   }
+  for (int e = t; e < 64 * RMAX; e += kE3Threads) {   // Zp[p][j] = (Z[2p][j], Z[2p + 1][j])
+    const float* zb = a.zbuf + ((int64_t)u * 128 + 2 * (e / RMAX)) * 16 + e % RMAX;
+    Zp[e] = make_float2(zb[0], zb[16]);
+  }
+  const bool valid = t0 + t < a.n;
+  const size_t row = (size_t)crow + t;
+  float2 sz1 = make_float2(0.0f, 0.0f);
+  if (!meta_tma && valid) sz1 = reinterpret_cast<const float2*>(a.meta)[row];
   __syncthreads();
-  constexpr int kCpw = 32 / BITS;
-  const int ta = blockIdx.x * kTile + threadIdx.x;
-  const int tb = ta + 64;
-  const bool va = ta < a.n, vb = tb < a.n;
-  if (!va) return;
-  const int tbx = vb ? tb : ta;   // a missing second token repeats the first
-  const size_t rowa = (size_t)u * a.n_max + (size_t)(a.t_off + ta);
-  const size_t rowb = (size_t)u * a.n_max + (size_t)(a.t_off + tbx);
-  const uint8_t* xa = reinterpret_cast<const uint8_t*>(a.kv) + ((size_t)u * a.n + ta) * 128 * sizeof(T);
-  const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.kv) + ((size_t)u * a.n + tbx) * 128 * sizeof(T);
-  const float2* ma = reinterpret_cast<const float2*>(a.meta) + rowa * a.G;
-  const float2* mb = reinterpret_cast<const float2*>(a.meta) + rowb * a.G;
+  const bool landed = mbar_wait(bar, 0);
+  if (!landed || !valid) return;
+
+  // this token's meta row: group gi at byte (8 gi) ^ mx (32-byte rows swizzled)
+  const uint8_t* mrow = ms + t * G * 8;
+  const int mx = G == 4 ? ((t >> 2) & 1) << 4 : 0;
+  auto group = [&](int gi) -> float2 {
+    return meta_tma ? *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx)) : sz1;
+  };
+  bool big = false;
+  for (int gi = 0; gi < G; ++gi) big |= !(group(gi).x <= 0x1p100f);
+  // the code words of 32 channels [32 q, 32 q + 32): 4*BITS bytes of the row
+  auto codes32 = [&](int q, uint32_t (&cw)[BITS]) {
+    const uint8_t* rowp = cs + t * F::kRow;
+    if constexpr (BITS == 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(rowp + ((((q >> 1) ^ swz_rows<F::kRow>(t)) << 4) | ((q & 1) << 3)));
+      cw[0] = v.x; cw[1] = v.y;
+    } else {
+#pragma unroll
+      for (int h = 0; h < BITS / 4; ++h) {
+        const uint4 v = *reinterpret_cast<const uint4*>(rowp + (((BITS / 4 * q + h) ^ swz_rows<F::kRow>(t)) << 4));
+        cw[4 * h] = v.x; cw[4 * h + 1] = v.y; cw[4 * h + 2] = v.z; cw[4 * h + 3] = v.w;
+      }
+    }
+  };
+
   uint64_t acc[RMAX];
 #pragma unroll
   for (int j = 0; j < RMAX; ++j) acc[j] = 0;
-  const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
-  constexpr int kVec = 16 / sizeof(T);   // elements per 16-byte load
-#pragma unroll 2
-  for (int c0 = 0; c0 < 128; c0 += 8) {
-    // 8 channels of both tokens
-    float xv[2][8];
+  // 8 channels [8 jb, 8 jb + 8) of the input row, as floats
+  auto xblock = [&](int jb, float (&xv)[8]) {
+    if constexpr (sizeof(T) == 4) {
 #pragma unroll
-    for (int q = 0; q < 8 / kVec; ++q) {
-      const uint4 va4 = *reinterpret_cast<const uint4*>(xa + (c0 + q * kVec) * sizeof(T));
-      const uint4 vb4 = *reinterpret_cast<const uint4*>(xb + (c0 + q * kVec) * sizeof(T));
-      const uint32_t wa[4] = {va4.x, va4.y, va4.z, va4.w}, wb[4] = {vb4.x, vb4.y, vb4.z, vb4.w};
+      for (int hq = 0; hq < 2; ++hq) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xs + (jb >> 2) * 16384 + swz(t, 2 * (jb & 3) + hq));
+        xv[4 * hq] = __uint_as_float(v.x); xv[4 * hq + 1] = __uint_as_float(v.y);
+        xv[4 * hq + 2] = __uint_as_float(v.z); xv[4 * hq + 3] = __uint_as_float(v.w);
+      }
+    } else {
+      const uint4 v = *reinterpret_cast<const uint4*>(xs + (jb >> 3) * 16384 + swz(t, jb & 7));
+      const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < kVec; ++e) {
-        if constexpr (sizeof(T) == 4) {
-          xv[0][q * kVec + e] = __uint_as_float(wa[e]);
-          xv[1][q * kVec + e] = __uint_as_float(wb[e]);
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = Elem16<T>::to_f2(pr[q]);
+        xv[2 * q] = f.x; xv[2 * q + 1] = f.y;
+      }
+    }
+  };
+  if (!big) {
+    const uint32_t one = a.one_bits;
+    const uint64_t one2 = f2_pack(1.0f, 1.0f);
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {   // 32 channels per pass, one group (g >= 32)
+      uint32_t cw[BITS];
+      codes32(q, cw);
+      const float2 sz = group((32 * q) >> lg);
+      const uint64_t sc2 = f2_pack(sz.x, sz.x), zr2 = f2_pack(sz.y, sz.y);
+#pragma unroll
+      for (int bq = 0; bq < 4; ++bq) {
+        const int jb = 4 * q + bq;
+        float xv[8];
+        xblock(jb, xv);
+        float f[8];   // the block's 8 codes as 1 + code * 2^-w
+        if constexpr (BITS == 4) {
+          CodeFloats<4>::word(cw[bq], f, one);
+        } else if constexpr (BITS == 2) {
+          float ff[16];
+          CodeFloats<2>::word(cw[bq >> 1] >> (16 * (bq & 1)), ff, one);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = ff[e];
         } else {
-          const uint32_t pa = wa[e >> 1], pb = wb[e >> 1];
-          xv[0][q * kVec + e] = Elem16<T>::lo((e & 1) ? (pa >> 16) : (pa & 0xFFFFu));
-          xv[1][q * kVec + e] = Elem16<T>::lo((e & 1) ? (pb >> 16) : (pb & 0xFFFFu));
+          float fa[4], fb[4];
+          CodeFloats<8>::word(cw[2 * bq], fa, one);
+          CodeFloats<8>::word(cw[2 * bq + 1], fb, one);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) { f[e] = fa[e]; f[4 + e] = fb[e]; }
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const int cl = 2 * p;   // channel inside the block; 8*jb is a whole number of bytes
+          const uint64_t w2 = f2_pack((float)(1 << (8 - (cl % kPerByte) * BITS)),
+                                      (float)(1 << (8 - ((cl + 1) % kPerByte) * BITS)));
+          const uint64_t cf = f2_sub(f2_pack(f[cl], f[cl + 1]), one2);
+          const uint64_t dh = f2_fma(cf, f2_mul(sc2, w2), zr2);
+          const uint64_t rr = f2_sub(f2_pack(xv[cl], xv[cl + 1]), dh);
+          const float4* zq = reinterpret_cast<const float4*>(Zp + (4 * jb + p) * RMAX);
+#pragma unroll
+          for (int j = 0; j < RMAX; j += 2) {
+            const float4 z = zq[j >> 1];
+            acc[j] = f2_fma(rr, f2_pack(z.x, z.y), acc[j]);
+            acc[j + 1] = f2_fma(rr, f2_pack(z.z, z.w), acc[j + 1]);
+          }
         }
       }
     }
-    const float2 sa = ma[c0 >> lg], sb = mb[c0 >> lg];
-    const uint64_t sc2 = f2_pack(sa.x, sb.x), zr2 = f2_pack(sa.y, sb.y);
+  } else {
+    constexpr int kCpw = 32 / BITS;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      uint32_t cw[BITS];
+      codes32(q, cw);
+      const float2 sz = group((32 * q) >> lg);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = c0 + e;
-      const uint32_t wa = a.codes[rowa * a.W + c / kCpw], wb = a.codes[rowb * a.W + c / kCpw];
-      const uint32_t sh = BITS * (c % kCpw), msk = (1u << BITS) - 1u;
-      const uint64_t cf = f2_sub(f2_pack(__uint_as_float(((wa >> sh) & msk) | 0x4B000000u),
-                                         __uint_as_float(((wb >> sh) & msk) | 0x4B000000u)),
-                                 f2_pack(8388608.0f, 8388608.0f));
-      const uint64_t dh = f2_fma(cf, sc2, zr2);
-      const uint64_t rr = f2_sub(f2_pack(xv[0][e], xv[1][e]), dh);
+      for (int bq = 0; bq < 4; ++bq) {
+        const int jb = 4 * q + bq;
+        float xv[8];
+        xblock(jb, xv);
 #pragma unroll
-      for (int j = 0; j < RMAX; j += 2) {
-        const float4 z = *reinterpret_cast<const float4*>(&Zd[c][j][0]);
-        acc[j] = f2_fma(rr, f2_pack(z.x, z.y), acc[j]);
-        acc[j + 1] = f2_fma(rr, f2_pack(z.z, z.w), acc[j + 1]);
+        for (int p = 0; p < 4; ++p) {
+          float rr[2];
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int c = 8 * bq + 2 * p + e2;   // channel inside the 32
+            const float code = (float)((cw[c / kCpw] >> (BITS * (c % kCpw))) & ((1u << BITS) - 1u));
+            rr[e2] = __fsub_rn(xv[2 * p + e2], __fmaf_rn(code, sz.x, sz.y));
+          }
+          const uint64_t rv = f2_pack(rr[0], rr[1]);
+#pragma unroll
+          for (int j = 0; j < RMAX; ++j)
+            acc[j] = f2_fma(rv, *reinterpret_cast<const uint64_t*>(&Zp[(4 * jb + p) * RMAX + j]), acc[j]);
+        }
       }
     }
   }
   // outlier slots: their residual is zero; remove what the loop added
-  const int k = a.k;
-  for (int side = 0; side < 2; ++side) {
-    const size_t row = side ? rowb : rowa;
-    const float2* mt = side ? mb : ma;
-    for (int i = 0; i < k; ++i) {
-      const int c = a.oidx[row * k + i];
-      float x;
-      if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(a.oval)[row * k + i];
-      else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(a.oval)[row * k + i]);
-      const float rr = __fsub_rn(x, __fmaf_rn(0.0f, mt[c >> lg].x, mt[c >> lg].y));
+  for (int i = 0; i < k; ++i) {
+    const int c = a.oidx[row * k + i];
+    float x;
+    if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(a.oval)[row * k + i];
+    else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(a.oval)[row * k + i]);
+    const float2 sz = group(c >> lg);
+    const float rr = __fsub_rn(x, __fmaf_rn(0.0f, sz.x, sz.y));
 #pragma unroll
-      for (int j = 0; j < RMAX; ++j) {
-        const uint64_t mask = side ? f2_pack(0.0f, rr * Zd[c][j][0]) : f2_pack(rr * Zd[c][j][0], 0.0f);
-        acc[j] = f2_sub(acc[j], mask);
-      }
+    for (int j = 0; j < RMAX; ++j) {
+      const float2 z = Zp[(c >> 1) * RMAX + j];
+      const float v = rr * ((c & 1) ? z.y : z.x);
+      acc[j] = f2_sub(acc[j], (c & 1) ? f2_pack(0.0f, v) : f2_pack(v, 0.0f));
     }
   }
-  for (int side = 0; side < (vb ? 2 : 1); ++side) {
-    const size_t row = side ? rowb : rowa;
-    for (int q = 0; q < a.r_max; ++q) {
-      float v = 0.0f;
+  for (int q = 0; q < a.r_max; ++q) {
+    float v = 0.0f;
 #pragma unroll
-      for (int j = 0; j < RMAX; ++j)
-        if (j == q) v = side ? f2_hi(acc[j]) : f2_lo(acc[j]);
-      if (q >= a.r) v = 0.0f;
-      if constexpr (sizeof(T) == 4) reinterpret_cast<float*>(a.lfac)[row * a.r_max + q] = v;
-      else reinterpret_cast<__half*>(a.lfac)[row * a.r_max + q] = __float2half_rn(v);
-    }
+    for (int j = 0; j < RMAX; ++j)
+      if (j == q) v = f2_lo(acc[j]) + f2_hi(acc[j]);
+    if (q >= r) v = 0.0f;
+    if constexpr (sizeof(T) == 4) reinterpret_cast<float*>(a.lfac)[row * a.r_max + q] = v;
+    else reinterpret_cast<__half*>(a.lfac)[row * a.r_max + q] = __float2half_rn(v);
   }
 }
 
@@ -984,22 +1097,35 @@ static cudaError_t launch_e1_b(const CUtensorMap& map, const EncodeArgs& a, int 
   }
 }
 
+template <typename T, int BITS, int RMAX>
+static cudaError_t launch_e3(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
+  auto kern = encode_lowrank<T, BITS, RMAX>;
+  constexpr int smem = E3Cfg<T, BITS, RMAX>::kSmem;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  kern<<<grid, kE3Threads, smem, st>>>(maps, a);
+  return cudaGetLastError();
+}
+
 template <typename T, int BITS>
-static void launch_e3_r(const EncodeArgs& a, dim3 grid, cudaStream_t st) {
-  if (a.r <= 4) encode_lowrank<T, BITS, 4><<<grid, kE3Threads, 0, st>>>(a);
-  else if (a.r <= 8) encode_lowrank<T, BITS, 8><<<grid, kE3Threads, 0, st>>>(a);
-  else encode_lowrank<T, BITS, 16><<<grid, kE3Threads, 0, st>>>(a);
+static cudaError_t launch_e3_r(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
+  if (a.r <= 4) return launch_e3<T, BITS, 4>(maps, a, grid, st);
+  if (a.r <= 8) return launch_e3<T, BITS, 8>(maps, a, grid, st);
+  return launch_e3<T, BITS, 16>(maps, a, grid, st);
 }
 
 template <typename T>
-static cudaError_t launch_e3_b(const EncodeArgs& a, cudaStream_t st) {
+static cudaError_t launch_e3_b(const E3Maps& maps, const EncodeArgs& a, cudaStream_t st) {
   dim3 grid(a.tpu, a.U);
   switch (a.bits) {
-    case 2: launch_e3_r<T, 2>(a, grid, st); break;
-    case 4: launch_e3_r<T, 4>(a, grid, st); break;
-    default: launch_e3_r<T, 8>(a, grid, st); break;
+    case 2: return launch_e3_r<T, 2>(maps, a, grid, st);
+    case 4: return launch_e3_r<T, 4>(maps, a, grid, st);
+    default: return launch_e3_r<T, 8>(maps, a, grid, st);
   }
-  return cudaGetLastError();
 }
 
 PFN_encodeTiled tensor_map_encoder() {
@@ -1068,9 +1194,18 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
-  if (a.dtype == GEAR_F16) return launch_e3_b<__half>(a, st);
-  if (a.dtype == GEAR_BF16) return launch_e3_b<__nv_bfloat16>(a, st);
-  return launch_e3_b<float>(a, st);
+  {
+    E3Maps m3;
+    memset(&m3, 0, sizeof(m3));
+    m3.x = map;
+    const uint64_t rows = (uint64_t)a.U * a.n_max;
+    if (!cache_row_map(enc, &m3.codes, a.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kTile)) return cudaErrorInvalidValue;
+    if (a.G >= 2 && !cache_row_map(enc, &m3.meta, a.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows, kTile))
+      return cudaErrorInvalidValue;
+    if (a.dtype == GEAR_F16) return launch_e3_b<__half>(m3, a, st);
+    if (a.dtype == GEAR_BF16) return launch_e3_b<__nv_bfloat16>(m3, a, st);
+    return launch_e3_b<float>(m3, a, st);
+  }
 }
 
 }  // namespace gear

@@ -16,6 +16,7 @@ struct EncodeArgs {
   uint64_t seed;
   // destination in the cache: tokens [t_off, t_off + n) of block `blk`
   int32_t t_off, blk, e_blk;
+  uint32_t one_bits;     // 0x3F800000 (1.0f), kept in a register by the kernels
   int32_t n_max, nblk_max, W, G, r_max;
   uint32_t* codes;
   float* meta;
