@@ -164,6 +164,22 @@ size_t gear_encode_workspace_bytes(const gear_cache* c, int32_t n);
 gear_status gear_encode(gear_cache* c, const void* kv, int32_t n,
                         void* workspace, size_t ws_bytes, void* stream);
 
+/* Workspace bytes gear_encode_batch needs for `count` caches shaped like
+ * caches[0] (host array), n tokens per unit. */
+size_t gear_encode_batch_workspace_bytes(int32_t count, const gear_cache* const* caches, int32_t n);
+
+/* gear_encode of kv[i] into caches[i] for every i < count, with up to 16
+ * tensors (the K and V of a layer, the layers of a model) sharing each kernel
+ * launch. The pages have no counterpart: it only batches the per-tensor
+ * encode. caches and kv are HOST arrays of `count` pointers; the caches must
+ * be distinct, empty and alike in B, H, dtype, n_max, nblk_max and params.
+ * Codes, meta and outliers are bit-identical to gear_encode's; L and Rf may
+ * differ in the last bits (the Gram partials are grouped by the launch's
+ * tiling). Larger batches run as consecutive launches on the stream.
+ * Errors: INVALID_ARG, CAPACITY, UNSUPPORTED, WORKSPACE, CUDA. */
+gear_status gear_encode_batch(int32_t count, gear_cache* const* caches, const void* const* kv, int32_t n,
+                              void* workspace, size_t ws_bytes, void* stream);
+
 /* Workspace bytes gear_decode_attn needs for these caches and Hq query heads. */
 size_t gear_decode_workspace_bytes(const gear_cache* k, const gear_cache* v, int32_t Hq);
 

@@ -70,13 +70,24 @@ static bool cache_ok(const gear_cache* c) {
   return c && c->codes && c->meta && c->rfac && c->buf && c->d == 128 && c->B > 0 && c->H > 0;
 }
 
-// encode n tokens per unit of `kv` into c as block `blk` at token offset t_off
-static gear_status encode_block(gear_cache* c, const void* kv, int n, int t_off, int blk, int rank, void* ws,
-                                size_t ws_bytes, cudaStream_t st) {
+// True when caches a and b can share one batched encode: same geometry,
+// dtype, codec parameters and counters.
+static bool same_shape(const gear_cache* a, const gear_cache* b) {
+  return a->B == b->B && a->H == b->H && a->d == b->d && a->dtype == b->dtype && a->n_max == b->n_max &&
+         a->nblk_max == b->nblk_max && a->n_comp == b->n_comp && a->n_buf == b->n_buf && a->n_blk == b->n_blk &&
+         memcmp(&a->p, &b->p, sizeof(gear_params)) == 0;
+}
+
+// Encodes n tokens per unit of kvs[i] into cs[i] (i < nt <= kMaxBatch, all of
+// one shape) as block `blk` at token offset t_off, in one launch per kernel.
+static gear_status encode_block(gear_cache* const* cs, const void* const* kvs, int nt, int n, int t_off, int blk,
+                                int rank, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const gear_cache* c = cs[0];
   EncodeArgs a;
   memset(&a, 0, sizeof(a));
-  a.kv = kv;
-  a.U = c->B * c->H;
+  a.nt = nt;
+  a.Uper = c->B * c->H;
+  a.U = nt * a.Uper;
   a.n = n;
   a.dtype = c->dtype;
   a.bits = c->p.bits;
@@ -94,12 +105,8 @@ static gear_status encode_block(gear_cache* c, const void* kv, int n, int t_off,
   a.W = c->W;
   a.G = c->G;
   a.r_max = c->r_max;
-  a.codes = c->codes;
-  a.meta = c->meta;
-  a.oidx = c->oidx;
-  a.oval = c->oval;
-  a.lfac = c->lfac;
-  a.rfac = c->rfac;
+  for (int i = 0; i < nt; ++i)
+    a.ten[i] = EncodeTensor{kvs[i], cs[i]->codes, cs[i]->meta, cs[i]->oidx, cs[i]->oval, cs[i]->lfac, cs[i]->rfac};
   a.tpu = (n + 127) / 128;
   a.total_tiles = (int64_t)a.U * a.tpu;
   const int sms = current_sm_count();
@@ -113,11 +120,12 @@ static gear_status encode_block(gear_cache* c, const void* kv, int n, int t_off,
   return cuda_status(encode_launch(a, sms, st));
 }
 
-static size_t encode_ws_bytes(const gear_cache* c, int n) {
-  if (!c || n <= 0) return 0;
+// workspace of one batched encode of nt tensors shaped like c, n tokens per unit
+static size_t encode_ws_bytes(const gear_cache* c, int nt, int n) {
+  if (!c || n <= 0 || nt <= 0) return 0;
   EncodeArgs a;
   memset(&a, 0, sizeof(a));
-  a.U = c->B * c->H;
+  a.U = nt * c->B * c->H;
   a.tpu = (n + 127) / 128;
   a.total_tiles = (int64_t)a.U * a.tpu;
   const int grid = encode_grid(a, current_sm_count());
@@ -203,7 +211,7 @@ gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int3
   return GEAR_OK;
 }
 
-size_t gear_encode_workspace_bytes(const gear_cache* c, int32_t n) { return encode_ws_bytes(c, n); }
+size_t gear_encode_workspace_bytes(const gear_cache* c, int32_t n) { return encode_ws_bytes(c, 1, n); }
 
 gear_status gear_encode(gear_cache* c, const void* kv, int32_t n, void* workspace, size_t ws_bytes, void* stream) {
   if (!cache_ok(c) || !kv) return GEAR_ERR_INVALID_ARG;
@@ -213,12 +221,48 @@ gear_status gear_encode(gear_cache* c, const void* kv, int32_t n, void* workspac
   if (c->p.rank > n) return GEAR_ERR_INVALID_ARG;
   if (n > c->n_max || c->nblk_max < 1) return GEAR_ERR_CAPACITY;
   if ((int64_t)c->B * c->H * n >= ((int64_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
-  gear_status s = encode_block(c, kv, n, 0, 0, c->p.rank, workspace, ws_bytes, (cudaStream_t)stream);
+  gear_status s = encode_block(&c, &kv, 1, n, 0, 0, c->p.rank, workspace, ws_bytes, (cudaStream_t)stream);
   if (s != GEAR_OK) return s;
   c->n_comp = n;
   c->n_blk = 1;
   c->blk0_len = n;
   c->blk0_rank = c->p.rank;
+  return GEAR_OK;
+}
+
+size_t gear_encode_batch_workspace_bytes(int32_t count, const gear_cache* const* caches, int32_t n) {
+  if (count < 1 || !caches || !caches[0]) return 0;
+  return encode_ws_bytes(caches[0], count < kMaxBatch ? count : kMaxBatch, n);
+}
+
+gear_status gear_encode_batch(int32_t count, gear_cache* const* caches, const void* const* kv, int32_t n,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (count < 1 || !caches || !kv || n < 1) return GEAR_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    gear_cache* c = caches[i];
+    if (!cache_ok(c) || !kv[i] || !aligned(kv[i], 16)) return GEAR_ERR_INVALID_ARG;
+    if (!same_shape(caches[0], c)) return GEAR_ERR_INVALID_ARG;
+    for (int j = 0; j < i; ++j)
+      if (caches[j] == c || caches[j]->codes == c->codes) return GEAR_ERR_INVALID_ARG;
+  }
+  gear_cache* c = caches[0];
+  if (c->n_comp != 0 || c->n_buf != 0 || c->n_blk != 0) return GEAR_ERR_INVALID_ARG;
+  if (c->p.rank > n) return GEAR_ERR_INVALID_ARG;
+  if (n > c->n_max || c->nblk_max < 1) return GEAR_ERR_CAPACITY;
+  if ((int64_t)c->B * c->H * n >= ((int64_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
+  for (int i0 = 0; i0 < count; i0 += kMaxBatch) {
+    const int nt = count - i0 < kMaxBatch ? count - i0 : kMaxBatch;
+    gear_status s = encode_block(caches + i0, kv + i0, nt, n, 0, 0, c->p.rank, workspace, ws_bytes,
+                                 (cudaStream_t)stream);
+    if (s != GEAR_OK) return s;
+  }
+  for (int i = 0; i < count; ++i) {
+    gear_cache* ci = caches[i];
+    ci->n_comp = n;
+    ci->n_blk = 1;
+    ci->blk0_len = n;
+    ci->blk0_rank = ci->p.rank;
+  }
   return GEAR_OK;
 }
 
@@ -270,7 +314,7 @@ gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const voi
 
 size_t gear_append_workspace_bytes(const gear_cache* k) {
   if (!cache_ok(k)) return 0;
-  return encode_ws_bytes(k, k->p.buffer_len);
+  return encode_ws_bytes(k, 2, k->p.buffer_len);
 }
 
 gear_status gear_append_buffer(gear_cache* k, gear_cache* v, const void* k_new, const void* v_new, void* workspace,
@@ -284,11 +328,19 @@ gear_status gear_append_buffer(gear_cache* k, gear_cache* v, const void* k_new, 
   const bool flush = k->n_buf == n_b;
   if (flush) {
     if (k->n_comp + n_b > k->n_max || k->n_blk + 1 > k->nblk_max) return GEAR_ERR_CAPACITY;
-    if (ws_bytes < encode_ws_bytes(k, n_b)) return GEAR_ERR_WORKSPACE;
     gear_cache* cs[2] = {k, v};
-    for (gear_cache* c : cs) {
-      gear_status s = encode_block(c, c->buf, n_b, c->n_comp, c->n_blk, c->p.buffer_rank, workspace, ws_bytes, st);
+    const void* bufs[2] = {k->buf, v->buf};
+    if (same_shape(k, v)) {   // both tensors in one pass
+      if (ws_bytes < encode_ws_bytes(k, 2, n_b)) return GEAR_ERR_WORKSPACE;
+      gear_status s = encode_block(cs, bufs, 2, n_b, k->n_comp, k->n_blk, k->p.buffer_rank, workspace, ws_bytes, st);
       if (s != GEAR_OK) return s;
+    } else {
+      if (ws_bytes < encode_ws_bytes(k, 1, n_b)) return GEAR_ERR_WORKSPACE;
+      for (int i = 0; i < 2; ++i) {
+        gear_status s = encode_block(&cs[i], &bufs[i], 1, n_b, cs[i]->n_comp, cs[i]->n_blk, cs[i]->p.buffer_rank,
+                                     workspace, ws_bytes, st);
+        if (s != GEAR_OK) return s;
+      }
     }
     for (gear_cache* c : cs) {
       if (c->n_blk == 0) { c->blk0_len = n_b; c->blk0_rank = c->p.buffer_rank; }

@@ -172,6 +172,10 @@ struct E1Cfg {
   static constexpr uint32_t kSmem = kBarOff + 256 + 1024;     // + alignment slack
 };
 
+struct XMaps {
+  CUtensorMap x[kMaxBatch];   // input rows of each tensor, 128-byte swizzled boxes of 128 rows
+};
+
 struct E1Bars {
   uint64_t x_full[2], x_empty[2], r_full[kNR], r_empty[kNR], acc_full, acc_empty;
   uint32_t tmem_slot;
@@ -440,13 +444,14 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
 
   // ---------------- cache outputs -------------------------------------------
   if (valid) {
-    const size_t row = (size_t)u * a.n_max + (size_t)(a.t_off + tok);
-    uint32_t* cw = a.codes + row * a.W + h * kWordsHalf;
+    const EncodeTensor& ten = a.ten[u / a.Uper];
+    const size_t row = (size_t)(u % a.Uper) * a.n_max + (size_t)(a.t_off + tok);
+    uint32_t* cw = ten.codes + row * a.W + h * kWordsHalf;
 #pragma unroll
     for (int w = 0; w < kWordsHalf; w += 4)
       *reinterpret_cast<uint4*>(cw + w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
     // meta: (scale, zero) per group; this thread owns groups in its half
-    float2* meta = reinterpret_cast<float2*>(a.meta) + row * a.G;
+    float2* meta = reinterpret_cast<float2*>(ten.meta) + row * a.G;
     const int gsz = a.g;
     if (gsz == 32) {
       meta[2 * h] = make_float2(scale[0], mn[0]);
@@ -459,7 +464,7 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     if constexpr (KMAX > 0) {
       if (h == 0 && k > 0) {
         // ascending channel order: selection by rank among the k channels
-        uint8_t* oi = a.oidx + row * k;
+        uint8_t* oi = ten.oidx + row * k;
 #pragma unroll
         for (int i = 0; i < KMAX; ++i) {
           if (i < k) {
@@ -468,9 +473,9 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
             for (int m = 0; m < KMAX; ++m) rank += (m < k && cidx[m] < cidx[i]) ? 1 : 0;
             oi[rank] = (uint8_t)cidx[i];
             if constexpr (sizeof(T) == 4)
-              reinterpret_cast<uint32_t*>(a.oval)[row * k + rank] = oval_bits[i];
+              reinterpret_cast<uint32_t*>(ten.oval)[row * k + rank] = oval_bits[i];
             else
-              reinterpret_cast<uint16_t*>(a.oval)[row * k + rank] = (uint16_t)oval_bits[i];
+              reinterpret_cast<uint16_t*>(ten.oval)[row * k + rank] = (uint16_t)oval_bits[i];
           }
         }
       }
@@ -480,7 +485,7 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
 
 template <typename T, int BITS, int KMAX>
 __global__ void __launch_bounds__(kE1Threads, 1)
-    encode_quant_gram(const __grid_constant__ CUtensorMap tmap, const EncodeArgs a) {
+    encode_quant_gram(const __grid_constant__ XMaps maps, const EncodeArgs a) {
   using C = E1Cfg<T>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -517,17 +522,17 @@ __global__ void __launch_bounds__(kE1Threads, 1)
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       int last_it[2] = {-1, -1};
-      prefetch_tensormap(&tmap);
       for (int it = 0; it < ntiles; ++it) {
         const int s = it % C::kNX;
         if (!mbar_wait(&bars->x_empty[s], ((it / C::kNX) & 1) ^ 1)) { bars->abort_flag = 1; break; }
         const int64_t tile = t_begin + it;
         const int u = (int)(tile / a.tpu);
         const int t0 = (int)(tile % a.tpu) * kTile;
-        const int32_t row0 = u * a.n + t0;
+        const int32_t row0 = (u % a.Uper) * a.n + t0;
+        const CUtensorMap* xm = &maps.x[u / a.Uper];
         mbar_arrive_expect_tx(&bars->x_full[s], C::kXBytes);
         for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_2d(xst + s * C::kXBytes + b * 16384, &tmap, &bars->x_full[s], b * C::kBoxCols, row0);
+          tma_load_2d(xst + s * C::kXBytes + b * 16384, xm, &bars->x_full[s], b * C::kBoxCols, row0);
         last_it[s] = it;
       }
       // every issued load must have landed before the CTA may exit
@@ -832,7 +837,7 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
 #pragma unroll
         for (int j = 0; j < 16; ++j) zrow[j] = (j < RM && j < r) ? (float)(zq[j < RM ? j : 0] * sL) : 0.0f;
         const int rp = rpad_of(a.r_max);
-        float* rrow = a.rfac + (((int64_t)u * a.nblk_max + a.blk) * 128 + i) * rp;
+        float* rrow = a.ten[u / a.Uper].rfac + (((int64_t)(u % a.Uper) * a.nblk_max + a.blk) * 128 + i) * rp;
         for (int j = 0; j < rp; ++j) {
           double wv = 0.0;
 #pragma unroll
@@ -861,7 +866,8 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
 constexpr int kE3Threads = 128;
 
 struct E3Maps {
-  CUtensorMap x, codes, meta;   // input rows, cache code rows, cache meta rows (G >= 2)
+  // per tensor: input rows, cache code rows, cache meta rows (G >= 2)
+  CUtensorMap x[kMaxBatch], codes[kMaxBatch], meta[kMaxBatch];
 };
 
 template <typename T, int BITS, int RMAX>
@@ -897,14 +903,16 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   const int G = a.G, k = a.k, r = a.r;
   const bool meta_tma = G >= 2;
   const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
-  const int crow = u * a.n_max + a.t_off + t0;   // cache row of the tile's first token
+  const int tn = u / a.Uper, ul = u % a.Uper;
+  const EncodeTensor& ten = a.ten[tn];
+  const int crow = ul * a.n_max + a.t_off + t0;   // cache row of the tile's first token
   if (t == 0) {
     mbar_init(bar, 1);
     fence_mbarrier_init();
     mbar_arrive_expect_tx(bar, (uint32_t)(F::kXB + F::kCB + (meta_tma ? kTile * G * 8 : 0)));
-    for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(xs + b * 16384, &maps.x, bar, b * C::kBoxCols, u * a.n + t0);
-    tma_load_2d(cs, &maps.codes, bar, 0, crow);
-    if (meta_tma) tma_load_2d(ms, &maps.meta, bar, 0, crow);
+    for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(xs + b * 16384, &maps.x[tn], bar, b * C::kBoxCols, ul * a.n + t0);
+    tma_load_2d(cs, &maps.codes[tn], bar, 0, crow);
+    if (meta_tma) tma_load_2d(ms, &maps.meta[tn], bar, 0, crow);
   }
   for (int e = t; e < 64 * RMAX; e += kE3Threads) {   // Zp[p][j] = (Z[2p][j], Z[2p + 1][j])
     const float* zb = a.zbuf + ((int64_t)u * 128 + 2 * (e / RMAX)) * 16 + e % RMAX;
@@ -913,7 +921,7 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   const bool valid = t0 + t < a.n;
   const size_t row = (size_t)crow + t;
   float2 sz1 = make_float2(0.0f, 0.0f);
-  if (!meta_tma && valid) sz1 = reinterpret_cast<const float2*>(a.meta)[row];
+  if (!meta_tma && valid) sz1 = reinterpret_cast<const float2*>(ten.meta)[row];
   __syncthreads();
   const bool landed = mbar_wait(bar, 0);
   if (!landed || !valid) return;
@@ -1041,10 +1049,10 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   }
   // outlier slots: their residual is zero; remove what the loop added
   for (int i = 0; i < k; ++i) {
-    const int c = a.oidx[row * k + i];
+    const int c = ten.oidx[row * k + i];
     float x;
-    if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(a.oval)[row * k + i];
-    else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(a.oval)[row * k + i]);
+    if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(ten.oval)[row * k + i];
+    else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]);
     const float2 sz = group(c >> lg);
     const float rr = __fsub_rn(x, __fmaf_rn(0.0f, sz.x, sz.y));
 #pragma unroll
@@ -1060,14 +1068,14 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
     for (int j = 0; j < RMAX; ++j)
       if (j == q) v = f2_lo(acc[j]) + f2_hi(acc[j]);
     if (q >= r) v = 0.0f;
-    if constexpr (sizeof(T) == 4) reinterpret_cast<float*>(a.lfac)[row * a.r_max + q] = v;
-    else reinterpret_cast<__half*>(a.lfac)[row * a.r_max + q] = __float2half_rn(v);
+    if constexpr (sizeof(T) == 4) reinterpret_cast<float*>(ten.lfac)[row * a.r_max + q] = v;
+    else reinterpret_cast<__half*>(ten.lfac)[row * a.r_max + q] = __float2half_rn(v);
   }
 }
 
 // ================================================================ host =====
 template <typename T, int BITS, int KMAX>
-static cudaError_t launch_e1(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
+static cudaError_t launch_e1(const XMaps& map, const EncodeArgs& a, int grid, cudaStream_t st) {
   auto kern = encode_quant_gram<T, BITS, KMAX>;
   static bool configured = false;   // the attribute persists for the process
   if (!configured) {
@@ -1080,7 +1088,7 @@ static cudaError_t launch_e1(const CUtensorMap& map, const EncodeArgs& a, int gr
 }
 
 template <typename T, int BITS>
-static cudaError_t launch_e1_k(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
+static cudaError_t launch_e1_k(const XMaps& map, const EncodeArgs& a, int grid, cudaStream_t st) {
   if (a.k == 0) return launch_e1<T, BITS, 0>(map, a, grid, st);
   if (a.k == 3) return launch_e1<T, BITS, 3>(map, a, grid, st);
   if (a.k <= 4) return launch_e1<T, BITS, 4>(map, a, grid, st);
@@ -1089,7 +1097,7 @@ static cudaError_t launch_e1_k(const CUtensorMap& map, const EncodeArgs& a, int 
 }
 
 template <typename T>
-static cudaError_t launch_e1_b(const CUtensorMap& map, const EncodeArgs& a, int grid, cudaStream_t st) {
+static cudaError_t launch_e1_b(const XMaps& map, const EncodeArgs& a, int grid, cudaStream_t st) {
   switch (a.bits) {
     case 2: return launch_e1_k<T, 2>(map, a, grid, st);
     case 4: return launch_e1_k<T, 4>(map, a, grid, st);
@@ -1158,24 +1166,36 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
   const int esz = a.dtype == GEAR_F32 ? 4 : 2;
   PFN_encodeTiled enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {128, (cuuint64_t)a.U * (cuuint64_t)a.n};
-  const cuuint64_t strides[1] = {(cuuint64_t)128 * esz};
-  const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)kTile};
-  const cuuint32_t estr[2] = {1, 1};
-  CUtensorMapDataType dt = a.dtype == GEAR_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                           : a.dtype == GEAR_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUresult cr = enc(&map, dt, 2, const_cast<void*>(a.kv), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // x: [Uper * n rows][128], boxes of 128 bytes x 128 rows, 128-byte swizzle
+  E3Maps m3;
+  memset(&m3, 0, sizeof(m3));
+  const CUtensorMapDataType dt = a.dtype == GEAR_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : a.dtype == GEAR_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const uint64_t crows = (uint64_t)a.Uper * a.n_max;
+  for (int tn = 0; tn < a.nt; ++tn) {
+    const cuuint64_t dims[2] = {128, (cuuint64_t)a.Uper * (cuuint64_t)a.n};
+    const cuuint64_t strides[1] = {(cuuint64_t)128 * esz};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)kTile};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult cr = enc(&m3.x[tn], dt, 2, const_cast<void*>(a.ten[tn].kv), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (!cache_row_map(enc, &m3.codes[tn], a.ten[tn].codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, crows, kTile))
+      return cudaErrorInvalidValue;
+    if (a.G >= 2 &&
+        !cache_row_map(enc, &m3.meta[tn], a.ten[tn].meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, crows, kTile))
+      return cudaErrorInvalidValue;
+  }
+  XMaps xm;
+  memcpy(xm.x, m3.x, sizeof(xm.x));
 
   const int grid = a.grid_e1;
   cudaError_t e;
-  if (a.dtype == GEAR_F16) e = launch_e1_b<__half>(map, a, grid, st);
-  else if (a.dtype == GEAR_BF16) e = launch_e1_b<__nv_bfloat16>(map, a, grid, st);
-  else e = launch_e1_b<float>(map, a, grid, st);
+  if (a.dtype == GEAR_F16) e = launch_e1_b<__half>(xm, a, grid, st);
+  else if (a.dtype == GEAR_BF16) e = launch_e1_b<__nv_bfloat16>(xm, a, grid, st);
+  else e = launch_e1_b<float>(xm, a, grid, st);
   if (e != cudaSuccess) return e;
   if (a.r == 0) return cudaSuccess;
 
@@ -1194,18 +1214,9 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
-  {
-    E3Maps m3;
-    memset(&m3, 0, sizeof(m3));
-    m3.x = map;
-    const uint64_t rows = (uint64_t)a.U * a.n_max;
-    if (!cache_row_map(enc, &m3.codes, a.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kTile)) return cudaErrorInvalidValue;
-    if (a.G >= 2 && !cache_row_map(enc, &m3.meta, a.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows, kTile))
-      return cudaErrorInvalidValue;
-    if (a.dtype == GEAR_F16) return launch_e3_b<__half>(m3, a, st);
-    if (a.dtype == GEAR_BF16) return launch_e3_b<__nv_bfloat16>(m3, a, st);
-    return launch_e3_b<float>(m3, a, st);
-  }
+  if (a.dtype == GEAR_F16) return launch_e3_b<__half>(m3, a, st);
+  if (a.dtype == GEAR_BF16) return launch_e3_b<__nv_bfloat16>(m3, a, st);
+  return launch_e3_b<float>(m3, a, st);
 }
 
 }  // namespace gear

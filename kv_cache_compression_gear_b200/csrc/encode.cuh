@@ -6,24 +6,32 @@
 
 namespace gear {
 
-struct EncodeArgs {
-  // input block: U units of n tokens, row-major [U][n][128], cache dtype
-  const void* kv;
-  int32_t U, n;
-  int32_t dtype;     // gear_dtype
-  // codec
-  int32_t bits, g, k, r, T;
-  uint64_t seed;
-  // destination in the cache: tokens [t_off, t_off + n) of block `blk`
-  int32_t t_off, blk, e_blk;
-  uint32_t one_bits;     // 0x3F800000 (1.0f), kept in a register by the kernels
-  int32_t n_max, nblk_max, W, G, r_max;
-  uint32_t* codes;
+// Up to kMaxBatch same-shaped tensors (for example the K and V of a layer)
+// are encoded by one launch of each kernel. Unit u of the batch is unit
+// u % Uper of tensor u / Uper.
+constexpr int kMaxBatch = 16;
+
+struct EncodeTensor {
+  const void* kv;    // input rows [Uper][n][128], cache dtype
+  uint32_t* codes;   // the tensor's cache arrays
   float* meta;
   uint8_t* oidx;
   void* oval;
   void* lfac;
   float* rfac;
+};
+
+struct EncodeArgs {
+  int32_t nt, Uper;  // tensors, units per tensor
+  int32_t U, n;      // U = nt * Uper units of n tokens each
+  int32_t dtype;     // gear_dtype
+  // codec
+  int32_t bits, g, k, r, T;
+  uint64_t seed;
+  // destination in the caches: tokens [t_off, t_off + n) of block `blk`
+  int32_t t_off, blk, e_blk;
+  uint32_t one_bits;     // 0x3F800000 (1.0f), kept in a register by the kernels
+  int32_t n_max, nblk_max, W, G, r_max;
   // workspace: partial Grams [U][maxc][128][128] and Z [U][128][16]
   float* gram;
   float* zbuf;
@@ -32,6 +40,7 @@ struct EncodeArgs {
   int64_t total_tiles;   // U * tpu
   int32_t grid_e1;       // persistent CTAs of E1
   int32_t maxc;          // partial-Gram slots per unit
+  EncodeTensor ten[kMaxBatch];
 };
 
 int encode_grid(const EncodeArgs& a, int num_sms);

@@ -62,6 +62,8 @@ def _load():
         "gear_cache_init": (i32, [pc, pp, i32, i32, i32, i32, i32, i32, P, S]),
         "gear_encode_workspace_bytes": (S, [pc, i32]),
         "gear_encode": (i32, [pc, P, i32, P, S, P]),
+        "gear_encode_batch_workspace_bytes": (S, [i32, P, i32]),
+        "gear_encode_batch": (i32, [i32, P, P, i32, P, S, P]),
         "gear_decode_workspace_bytes": (S, [pc, pc, i32]),
         "gear_decode_attn": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P, S, P]),
         "gear_decode_attn_noalloc": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P]),
@@ -189,6 +191,21 @@ class Cache:
             "rfac": self._view(c.rfac, U * c.nblk_max * c.d * rp, torch.float32).view(U, c.nblk_max, c.d, rp),
             "buf": self._view(c.buf, U * c.p.buffer_len * c.d, self.dtype).view(U, c.p.buffer_len, c.d),
         }
+
+
+def encode_batch(caches, kvs, stream=None):
+    """gear_encode_batch: encodes kvs[i] [B][H][n][d] into caches[i] in shared launches."""
+    assert len(caches) == len(kvs) and len(caches) > 0
+    for c, kv in zip(caches, kvs):
+        assert kv.is_cuda and kv.dtype == c.dtype and kv.is_contiguous()
+    n = kvs[0].shape[2]
+    cnt = len(caches)
+    cptrs = (ctypes.c_void_p * cnt)(*[ctypes.addressof(c.c) for c in caches])
+    xptrs = (ctypes.c_void_p * cnt)(*[kv.data_ptr() for kv in kvs])
+    nbytes = lib.gear_encode_batch_workspace_bytes(cnt, cptrs, n)
+    wp, wn = _ws.get(nbytes, kvs[0].device)
+    _check(lib.gear_encode_batch(cnt, cptrs, xptrs, n, ctypes.c_void_p(wp), wn, _stream_ptr(stream)),
+           "gear_encode_batch")
 
 
 def decode_attn(kc: Cache, vc: Cache, q: torch.Tensor, softmax_scale: float, out_dtype=None, out=None,

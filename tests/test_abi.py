@@ -111,3 +111,29 @@ def test_cache_layout_and_host_errors(gear):
     assert L.gear_decode_dense(ctypes.byref(c), None, None) == E.GEAR_ERR_INVALID_ARG
     assert L.gear_status_string(6) == b"workspace missing or too small"
     assert L.gear_version() == b"0.1.0"
+
+
+def test_encode_batch_host_errors(gear):
+    """gear_encode_batch rejects bad batches before touching the device."""
+    L, E = gear.lib, gear.gear
+    p = gear.make_params()
+    p2 = gear.make_params(bits=2, group_size=32)
+    caches = []
+    for i, pp in enumerate([p, p, p2]):
+        nbytes = L.gear_cache_bytes(ctypes.byref(pp), 1, 4, 128, 1024, 1, 0)
+        c = gear.GearCacheStruct()
+        assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(pp), 1, 4, 128, 1024, 1, 0,
+                                 ctypes.c_void_p((1 << 40) * (i + 1)), nbytes) == 0
+        caches.append(c)
+    ptrs = lambda cs: (ctypes.c_void_p * len(cs))(*[ctypes.addressof(c) for c in cs])  # noqa: E731
+    xs = lambda m: (ctypes.c_void_p * m)(*[4096 * (j + 1) for j in range(m)])  # noqa: E731
+    assert L.gear_encode_batch(0, ptrs(caches[:1]), xs(1), 10, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_encode_batch(2, ptrs(caches[:2]), xs(2), 0, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    # different parameters, the same cache twice, a misaligned input
+    assert L.gear_encode_batch(2, ptrs([caches[0], caches[2]]), xs(2), 10, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_encode_batch(2, ptrs([caches[0], caches[0]]), xs(2), 10, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    bad = (ctypes.c_void_p * 2)(4096, 4096 + 8)
+    assert L.gear_encode_batch(2, ptrs(caches[:2]), bad, 10, None, 0, None) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_encode_batch(2, ptrs(caches[:2]), xs(2), 2000, None, 0, None) == E.GEAR_ERR_CAPACITY
+    assert L.gear_encode_batch(2, ptrs(caches[:2]), xs(2), 2, None, 0, None) == E.GEAR_ERR_INVALID_ARG  # rank 4 > n
+    assert all(c.n_comp == 0 for c in caches)

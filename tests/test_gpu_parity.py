@@ -167,6 +167,39 @@ def test_decode_and_append_match_oracle(dtype, B, H, Hq, n0, nappend, bits, g, s
     assert gear.device_status() == 0
 
 
+# ------------------------------------------------------------ batched encode
+BATCH_CASES = [
+    # dtype, count, B, H, n, bits, g, s, r, T
+    ("f16", 2, 2, 2, 300, 4, 64, 0.02, 4, 3),
+    ("bf16", 3, 1, 3, 129, 2, 32, 0.05, 8, 2),
+    ("f32", 2, 1, 2, 200, 8, 128, 0.02, 3, 3),
+    ("f16", 17, 1, 1, 65, 4, 64, 0.02, 2, 3),   # more than one launch
+]
+
+
+@pytest.mark.parametrize("dtype,count,B,H,n,bits,g,s,r,T", BATCH_CASES)
+def test_encode_batch_matches_single_and_oracle(dtype, count, B, H, n, bits, g, s, r, T):
+    p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, power_iters=T, seed=99 + n)
+    op = oracle_params(p)
+    xs = [seeded_kv(300 + i, 1, (B, H, n, 128), dtype, channel_scale=True) for i in range(count)]
+    caches = [gear.Cache(p, B, H, n + 32, 2, TORCH_DT[dtype]) for _ in range(count)]
+    gear.encode_batch(caches, [to_dev(x, dtype) for x in xs])
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    for i in sorted({0, count // 2, count - 1}):
+        single = gear.Cache(p, B, H, n + 32, 2, TORCH_DT[dtype])
+        single.encode(to_dev(xs[i], dtype))
+        A, S = caches[i].arrays(), single.arrays()
+        for name in ["codes", "meta", "oidx", "oval"]:
+            assert torch.equal(A[name][:, :n], S[name][:, :n]), (i, name)
+        assert caches[i].c.n_comp == n and caches[i].c.n_blk == 1
+        dense = caches[i].dense().cpu().numpy()
+        for u in range(B * H):
+            o = oracle.encode_unit(xs[i][u // H, u % H], op)
+            compare_unit(gpu_block(caches[i], u, 0, n, 0, r), o, p, f"tensor {i} unit {u}")
+            compare_dense(dense[u // H, u % H], oracle.reconstruct_unit(o, op), o.scale, g, f"tensor {i} unit {u}")
+
+
 # ------------------------------------------------------ full-size workloads
 def _workload_encode_check(w: wl.Workload, units_to_check, layer=0):
     p = gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
@@ -191,6 +224,23 @@ def _workload_encode_check(w: wl.Workload, units_to_check, layer=0):
 def test_full_llama7b_layer_encode():
     w = wl.WORKLOADS["llama7b_layer_encode"]
     _workload_encode_check(w, [(0, 0), (0, 13), (0, 31)])
+
+
+def test_full_llama7b_layer_encode_batch():
+    """The K and V of the layer in one batched encode, as the benchmark runs it."""
+    w = wl.WORKLOADS["llama7b_layer_encode"]
+    p = gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
+                         buffer_len=w.buffer_len, buffer_rank=w.buffer_rank, seed=w.seed)
+    op = oracle_params(p)
+    xs = [wl.kv_tensor_torch(w, which, 0, "cuda") for which in ["k", "v"]]
+    cs = [gear.Cache(p, w.B, w.H, w.n, 1, TORCH_DT[w.dtype]) for _ in range(2)]
+    gear.encode_batch(cs, xs)
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    for c, which in zip(cs, ["k", "v"]):
+        for (b, h) in [(0, 1), (0, 30)]:
+            o = oracle.encode_unit(wl.kv_unit_np(w, which, 0, b, h), op)
+            compare_unit(gpu_block(c, b * w.H + h, 0, w.n, 0, w.rank), o, p, f"batch {which} ({b},{h})")
 
 
 def test_full_twobit_b64_encode_and_decode():
