@@ -156,15 +156,23 @@ __device__ __forceinline__ uint64_t div_pair_slow(uint64_t a, float s) {
 //   R stages  kNR x 64 KiB    residual hi (32 KiB) then lo (32 KiB), each two
 //                             64-channel blocks of [128 tokens][128 B], swz-128B
 //   barriers, tensor-memory slot, abort flag
+// For 16-bit inputs two groups of 8 quantizer warps take alternate tiles
+// (tile it goes to group it % 2, X stage it % 2 and R stage it % 2), so that
+// 16 warps hide each other's latency; fp32 tiles are twice as large and use
+// one group. A group hands its X stage back as soon as it has read it, so the
+// next tile loads while it quantizes. Every quantizer warp drains every
+// segment's accumulator (its share of the columns), so each one waits on
+// every phase of the accumulator barriers in order.
 constexpr int kTile = 128;       // tokens per tile
-constexpr int kQThreads = 256;   // quantizer threads (2 per token)
-constexpr int kE1Threads = 64 + kQThreads;
+constexpr int kQThreads = 256;   // quantizer threads per group (2 per token)
 constexpr int kNR = 2;
 constexpr uint32_t kRBytes = 65536;
 
 template <typename T>
 struct E1Cfg {
-  static constexpr int kNX = sizeof(T) == 4 ? 1 : 2;
+  static constexpr int kGroups = sizeof(T) == 4 ? 1 : 2;
+  static constexpr int kThreads = 64 + kGroups * kQThreads;
+  static constexpr int kNX = kGroups;   // X stage g belongs to group g
   static constexpr uint32_t kXBytes = kTile * 128 * sizeof(T);
   static constexpr int kBoxCols = 128 / sizeof(T);            // 128-byte rows
   static constexpr int kBoxes = 128 / kBoxCols;
@@ -177,7 +185,7 @@ struct XMaps {
 };
 
 struct E1Bars {
-  uint64_t x_full[2], x_empty[2], r_full[kNR], r_empty[kNR], acc_full, acc_empty;
+  uint64_t x_full[2], x_empty[2], r_full[kNR], r_empty[kNR], acc_full, acc_empty, mma_done;
   uint32_t tmem_slot;
   int32_t abort_flag;
 };
@@ -194,7 +202,7 @@ __device__ __forceinline__ int64_t seg_first_cta(int64_t tile, int64_t grid, int
 // into the R stage. `valid` is false for tile rows past the unit's last token.
 template <typename T, int BITS, int KMAX>
 __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, uint8_t* rs, int t, int h,
-                                              bool valid, int u, int tok) {
+                                              bool valid, int u, int tok, uint64_t* x_release) {
   constexpr int kCodesPerWord = 32 / BITS;
   constexpr int kWordsHalf = 64 * BITS / 32;
   const float levels = (float)((1 << BITS) - 1);
@@ -302,6 +310,9 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       xr[4 * j + 0] = v.x; xr[4 * j + 1] = v.y; xr[4 * j + 2] = v.z; xr[4 * j + 3] = v.w;
     }
   }
+  // the X stage is not read again: hand it back to the producer
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(x_release);
 
   // ---------------- group min / max over non-outliers ----------------------
   // Two 32-channel sub-halves; combined for g >= 64, and with the partner for
@@ -359,9 +370,9 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
   uint32_t words[kWordsHalf];
 #pragma unroll
   for (int w = 0; w < kWordsHalf; ++w) words[w] = 0u;
-  uint32_t hi_out[32], lo_out[32];  // packed bf16 pairs of R (hi) and R - hi (lo)
-  // one pair of channels (2p, 2p + 1); DIV is the division of the pair
-  auto qpair = [&](const int p, const uint64_t mnv, const uint64_t sc2, auto div) {
+  // one pair of channels (2p, 2p + 1); DIV is the division of the pair. The
+  // residual split (hi = bf16(R), lo = bf16(R - hi)) comes back packed in ho, lo.
+  auto qpair = [&](const int p, const uint64_t mnv, const uint64_t sc2, auto div, uint32_t& ho, uint32_t& lo) {
     const int sh = p >> 4;
     float x0, x1;
     if constexpr (sizeof(T) == 4) {
@@ -388,15 +399,26 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       const uint32_t bits = e2 ? f2_hi_bits(tq) : f2_lo_bits(tq);
       words[e / kCodesPerWord] += bits << (BITS * (e % kCodesPerWord));
     }
-    // residual split: hi = bf16(R), lo = bf16(R - hi)
-    const float r0 = f2_lo(rv), r1 = f2_hi(rv);
-    const __nv_bfloat162 hb = __floats2bfloat162_rn(r0, r1);
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(f2_lo(rv), f2_hi(rv));
     const uint32_t hbits = *reinterpret_cast<const uint32_t*>(&hb);
     const uint64_t hv = f2_pack(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u));
     const uint64_t lv = f2_sub(rv, hv);
     const __nv_bfloat162 lb = __floats2bfloat162_rn(f2_lo(lv), f2_hi(lv));
-    hi_out[p] = hbits;
-    lo_out[p] = *reinterpret_cast<const uint32_t*>(&lb);
+    ho = hbits;
+    lo = *reinterpret_cast<const uint32_t*>(&lb);
+  };
+  // 8 channels (one 16-byte chunk j of the half row) at a time; their residual
+  // goes straight to the R stage (MN-major swizzle-128B). Rows past the
+  // unit's last token contribute nothing to the Gram.
+  auto chunk_out = [&](int j, const uint32_t (&h4)[4], const uint32_t (&l4)[4]) {
+    uint8_t* ph = rs + h * 16384 + swz(t, j);
+    if (valid) {
+      *reinterpret_cast<uint4*>(ph) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+      *reinterpret_cast<uint4*>(ph + 32768) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    } else {
+      *reinterpret_cast<uint4*>(ph) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(ph + 32768) = make_uint4(0u, 0u, 0u, 0u);
+    }
   };
 #pragma unroll
   for (int sh = 0; sh < 2; ++sh) {
@@ -406,13 +428,24 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       const uint64_t y2 = f2_pack(y[sh], y[sh]);
       const uint64_t s2n = f2_pack(-scale[sh], -scale[sh]);
 #pragma unroll
-      for (int pp = 0; pp < 16; ++pp)
-        qpair(16 * sh + pp, mnv, sc2, [&](uint64_t av) { return div_pair_fast(av, s2n, y2); });
+      for (int jj = 0; jj < 4; ++jj) {
+        uint32_t h4[4], l4[4];
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp)
+          qpair(16 * sh + 4 * jj + pp, mnv, sc2, [&](uint64_t av) { return div_pair_fast(av, s2n, y2); }, h4[pp],
+                l4[pp]);
+        chunk_out(4 * sh + jj, h4, l4);
+      }
     } else {
       const float sv = scale[sh];
 #pragma unroll
-      for (int pp = 0; pp < 16; ++pp)
-        qpair(16 * sh + pp, mnv, sc2, [&](uint64_t av) { return div_pair_slow(av, sv); });
+      for (int jj = 0; jj < 4; ++jj) {
+        uint32_t h4[4], l4[4];
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp)
+          qpair(16 * sh + 4 * jj + pp, mnv, sc2, [&](uint64_t av) { return div_pair_slow(av, sv); }, h4[pp], l4[pp]);
+        chunk_out(4 * sh + jj, h4, l4);
+      }
     }
   }
   {
@@ -421,25 +454,6 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     for (int e = 0; e < kCodesPerWord; ++e) magic_sum += kRoundMagicBits << (BITS * e);
 #pragma unroll
     for (int w = 0; w < kWordsHalf; ++w) words[w] -= magic_sum;
-  }
-
-  // ---------------- residual to the R stage (MN-major swizzle-128B) --------
-  // rows past the unit's last token contribute nothing to the Gram
-  if (valid) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint8_t* ph = rs + h * 16384 + swz(t, j);
-      *reinterpret_cast<uint4*>(ph) = make_uint4(hi_out[4 * j], hi_out[4 * j + 1], hi_out[4 * j + 2], hi_out[4 * j + 3]);
-      *reinterpret_cast<uint4*>(ph + 32768) =
-          make_uint4(lo_out[4 * j], lo_out[4 * j + 1], lo_out[4 * j + 2], lo_out[4 * j + 3]);
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint8_t* ph = rs + h * 16384 + swz(t, j);
-      *reinterpret_cast<uint4*>(ph) = make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(ph + 32768) = make_uint4(0u, 0u, 0u, 0u);
-    }
   }
 
   // ---------------- cache outputs -------------------------------------------
@@ -484,11 +498,11 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
 }
 
 template <typename T, int BITS, int KMAX>
-__global__ void __launch_bounds__(kE1Threads, 1)
+__global__ void __launch_bounds__(E1Cfg<T>::kThreads, 1)
     encode_quant_gram(const __grid_constant__ XMaps maps, const EncodeArgs a) {
   using C = E1Cfg<T>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint8_t* xst = smem;
   uint8_t* rst = smem + C::kNX * C::kXBytes;
   E1Bars* bars = reinterpret_cast<E1Bars*>(smem + C::kBarOff);
@@ -505,7 +519,8 @@ __global__ void __launch_bounds__(kE1Threads, 1)
     for (int s = 0; s < C::kNX; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 8); }
     for (int s = 0; s < kNR; ++s) { mbar_init(&bars->r_full[s], 8); mbar_init(&bars->r_empty[s], 1); }
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, 8);
+    mbar_init(&bars->acc_empty, C::kGroups * 8);
+    mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -562,38 +577,38 @@ __global__ void __launch_bounds__(kE1Threads, 1)
         tc_commit(&bars->r_empty[sr]);
         if (is_seg_end(tile)) { tc_commit(&bars->acc_full); ++seg; }
       }
+      // every MMA this thread issued has completed before tensor memory is freed
+      tc_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0);
     }
   } else {
     // ------------------------------------------------ quantizer warps
-    const int qid = threadIdx.x - 64;
+    const int group = (warp - 2) >> 3;
+    const int qid = (threadIdx.x - 64) & (kQThreads - 1);
     const int t = qid >> 1, h = qid & 1;
-    const int qw = warp - 2;
-    int seg = 0;
-    for (int it = 0; it < ntiles; ++it) {
-      const int64_t tile = t_begin + it;
-      const int u = (int)(tile / a.tpu);
-      const int t0 = (int)(tile % a.tpu) * kTile;
-      const int s = it % C::kNX, sr = it % kNR;
-      bool ok = mbar_wait(&bars->x_full[s], (it / C::kNX) & 1);
-      ok = ok && mbar_wait(&bars->r_empty[sr], ((it / kNR) & 1) ^ 1);
-      if (!ok || bars->abort_flag) { bars->abort_flag = 1; break; }
-      quantize_half<T, BITS, KMAX>(a, xst + s * C::kXBytes, rst + sr * kRBytes, t, h, t0 + t < a.n, u, t0 + t);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) { mbar_arrive(&bars->r_full[sr]); mbar_arrive(&bars->x_empty[s]); }
-      if (is_seg_end(tile)) {
-        // ---------------- epilogue: partial Gram of this (CTA, unit) segment
-        if (!mbar_wait(&bars->acc_full, seg & 1)) { bars->abort_flag = 1; break; }
+    // drain share: TMEM lanes of quarter warp & 3, output columns [col0, col0 + ncol)
+    constexpr int kNcol = 128 / (2 * C::kGroups);
+    const int quarter = warp & 3;
+    const int col0 = ((warp - 2) >> 2) * kNcol;
+    // segments of this CTA: S = 0 .. nseg-1, one per unit its tiles touch
+    const int64_t u_first = t_begin / a.tpu;
+    const int nseg = ntiles > 0 ? (int)((t_end - 1) / a.tpu - u_first + 1) : 0;
+    int drained = 0;   // segments drained by this warp
+    // drains, in order, every segment that ended at tile index <= upto
+    auto drain = [&](int upto) -> bool {
+      while (drained < nseg) {
+        const int64_t end_tile = min(t_end, (u_first + drained + 1) * (int64_t)a.tpu) - 1;
+        if (end_tile > t_begin + upto) return true;
+        if (!mbar_wait(&bars->acc_full, drained & 1)) return false;
         tc_fence_after();
-        const int quarter = warp & 3;
+        const int ue = (int)(end_tile / a.tpu);
         const int ch = quarter * 32 + lane;
-        const int col0 = (qw < 4) ? 0 : 64;
-        const int64_t slot = (int64_t)blockIdx.x - seg_first_cta((int64_t)u * a.tpu, grid, total);
-        float* dst = a.gram + (((int64_t)u * a.maxc + slot) * 128 + ch) * 128;
+        const int64_t slot = (int64_t)blockIdx.x - seg_first_cta((int64_t)ue * a.tpu, grid, total);
+        float* dst = a.gram + (((int64_t)ue * a.maxc + slot) * 128 + ch) * 128;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 32) {
+        for (int cc = 0; cc < kNcol; cc += 32) {
           uint32_t d1[32], d2[32];
-          const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
           tmem_ld_32x32b_x32(lane_addr + col0 + cc, d1);
           tmem_ld_32x32b_x32(lane_addr + 128 + col0 + cc, d2);
           tmem_ld_wait();
@@ -610,9 +625,29 @@ __global__ void __launch_bounds__(kE1Threads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->acc_empty);
-        ++seg;
+        ++drained;
       }
+      return true;
+    };
+    bool ok = true;
+    for (int it = 0; it < ntiles && ok; ++it) {
+      const int64_t tile = t_begin + it;
+      if (it % C::kGroups != group) continue;
+      const int u = (int)(tile / a.tpu);
+      const int t0 = (int)(tile % a.tpu) * kTile;
+      const int s = it % C::kNX, sr = it % kNR;
+      ok = mbar_wait(&bars->x_full[s], (it / C::kNX) & 1);
+      ok = ok && mbar_wait(&bars->r_empty[sr], ((it / kNR) & 1) ^ 1);
+      if (!ok || bars->abort_flag) { ok = false; break; }
+      quantize_half<T, BITS, KMAX>(a, xst + s * C::kXBytes, rst + sr * kRBytes, t, h, t0 + t < a.n, u, t0 + t,
+                                   &bars->x_empty[s]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->r_full[sr]);
+      ok = drain(it);
     }
+    if (ok) ok = drain(ntiles - 1);
+    if (!ok) bars->abort_flag = 1;
   }
 
   tc_fence_before();
@@ -703,11 +738,12 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
     ok = mbar_wait(&S.bar[b], (sg >> 1) & 1) && ok;
     for (int e4 = tid; e4 < 4096; e4 += kE2Threads) {
       const float4 v = reinterpret_cast<const float4*>(S.u.stage[b])[e4];
-      float* dst = &S.M[(e4 >> 5) * kMStride + ((e4 & 31) << 2)];
+      float4* dst = reinterpret_cast<float4*>(&S.M[(e4 >> 5) * kMStride + ((e4 & 31) << 2)]);   // 16-byte aligned rows
       if (sg == 0) {
-        dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+        *dst = v;
       } else {
-        dst[0] += v.x; dst[1] += v.y; dst[2] += v.z; dst[3] += v.w;
+        const float4 o = *dst;
+        *dst = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
       }
     }
     __syncthreads();
@@ -893,7 +929,7 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   constexpr int W = 4 * BITS;
   constexpr int kPerByte = 8 / BITS;
   extern __shared__ uint8_t e3raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(e3raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = align_smem_1024(e3raw);
   uint8_t* xs = sm;
   uint8_t* cs = sm + F::kXB;
   uint8_t* ms = cs + F::kCB;
@@ -1083,7 +1119,7 @@ static cudaError_t launch_e1(const XMaps& map, const EncodeArgs& a, int grid, cu
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<grid, kE1Threads, E1Cfg<T>::kSmem, st>>>(map, a);
+  kern<<<grid, E1Cfg<T>::kThreads, E1Cfg<T>::kSmem, st>>>(map, a);
   return cudaGetLastError();
 }
 
