@@ -44,6 +44,12 @@ def peaks():
         return 6650.0, "fallback"
 
 
+# DRAM bytes of one decode_warp launch on the decode workload, measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum of one launch); set to None
+# whenever the kernel changes, until it is captured again.
+DECODE_TRAFFIC_BYTES = 824346112 + 6866432
+
+
 def per_token_bytes(w) -> int:
     """Compressed bytes per token of one tensor: codes + (scale, zero) per group
     + outlier index and value + L row."""
@@ -311,7 +317,8 @@ def run_gpu(args, rank: int, world: int):
     roof = {"bound": "hbm", "kernel": "gear_decode_attn" if dominant == "decode" else "gear_encode",
             "achieved": round(dec_gbs if dominant == "decode" else enc_gbs, 2), "peak": hbm,
             "unit": "GB/s", "frac": round((dec_gbs if dominant == "decode" else enc_gbs) / hbm, 4),
-            "peak_kind": peak_kind, "traffic": None}
+            "peak_kind": peak_kind,
+            "traffic": DECODE_TRAFFIC_BYTES if dominant == "decode" else None}
     other = {"kernel": "gear_encode" if dominant == "decode" else "gear_decode_attn",
              "achieved": round(enc_gbs if dominant == "decode" else dec_gbs, 2),
              "frac": round((enc_gbs if dominant == "decode" else dec_gbs) / hbm, 4)}
