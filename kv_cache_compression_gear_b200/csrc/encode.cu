@@ -665,7 +665,8 @@ __global__ void __launch_bounds__(E1Cfg<T>::kThreads, 1)
 // The partials arrive by 64 KiB bulk asynchronous copies, two in flight, and
 // are summed in a fixed order (deterministic); M is kept in fp32 (the
 // partials carry about 17 significant bits), products accumulate in fp64.
-constexpr int kE2Threads = 256;
+constexpr int kE2Threads = 512;
+constexpr int kE2Parts = kE2Threads / 128;   // threads per row of W = M Q
 constexpr int kMStride = 132;  // padded fp32 row of M
 
 __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t i) {
@@ -692,7 +693,7 @@ struct E2Smem {
   union {
     float stage[2][16384];   // partial Grams in flight (phase 1)
     struct {                 // power-iteration scratch (phase 2)
-      double Wp[2 * 128 * RM];
+      double Wp[kE2Parts * 128 * RM];
       double red[4 * RM * RM];
       double Xi[RM * RM];
     } it;
@@ -763,21 +764,21 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
   }
   __syncthreads();
 
-  const int i = tid & 127, half = tid >> 7;
+  const int i = tid & 127, wpart = tid >> 7;
   for (int step = 0; step < a.T; ++step) {
-    // W = M Q: two threads per row, each over 64 of the 128 channels
+    // W = M Q: kE2Parts threads per row, each over 128 / kE2Parts channels
     {
       double w[RM];
 #pragma unroll
       for (int j = 0; j < RM; ++j) w[j] = 0.0;
 #pragma unroll 8
-      for (int c = half * 64; c < half * 64 + 64; ++c) {
+      for (int c = wpart * (128 / kE2Parts); c < (wpart + 1) * (128 / kE2Parts); ++c) {
         const double mv = (double)S.M[c * kMStride + i];
 #pragma unroll
         for (int j = 0; j < RM; ++j) w[j] = fma(mv, S.Q[c * RM + j], w[j]);
       }
 #pragma unroll
-      for (int j = 0; j < RM; ++j) S.u.it.Wp[(half * 128 + i) * RM + j] = w[j];
+      for (int j = 0; j < RM; ++j) S.u.it.Wp[(wpart * 128 + i) * RM + j] = w[j];
     }
     __syncthreads();
     // G = Q^T W (upper triangle), reduced by warp then across warps
@@ -785,7 +786,10 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
       double w[RM], qv[RM];
 #pragma unroll
       for (int j = 0; j < RM; ++j) {
-        w[j] = S.u.it.Wp[i * RM + j] + S.u.it.Wp[(128 + i) * RM + j];
+        double v = S.u.it.Wp[i * RM + j];
+#pragma unroll
+        for (int pp = 1; pp < kE2Parts; ++pp) v += S.u.it.Wp[(pp * 128 + i) * RM + j];
+        w[j] = v;
         qv[j] = S.Q[i * RM + j];
       }
 #pragma unroll
@@ -958,6 +962,17 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   const size_t row = (size_t)crow + t;
   float2 sz1 = make_float2(0.0f, 0.0f);
   if (!meta_tma && valid) sz1 = reinterpret_cast<const float2*>(ten.meta)[row];
+  // the token's first outliers, fetched while the tile is in flight
+  constexpr int kOF = 4;
+  int oc[kOF];
+  float ox[kOF];
+#pragma unroll
+  for (int i = 0; i < kOF; ++i) {
+    const bool on = valid && i < k;
+    oc[i] = on ? ten.oidx[row * k + i] : 0;
+    if constexpr (sizeof(T) == 4) ox[i] = on ? reinterpret_cast<const float*>(ten.oval)[row * k + i] : 0.0f;
+    else ox[i] = on ? Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]) : 0.0f;
+  }
   __syncthreads();
   const bool landed = mbar_wait(bar, 0);
   if (!landed || !valid) return;
@@ -1085,10 +1100,17 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   }
   // outlier slots: their residual is zero; remove what the loop added
   for (int i = 0; i < k; ++i) {
-    const int c = ten.oidx[row * k + i];
+    int c;
     float x;
-    if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(ten.oval)[row * k + i];
-    else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]);
+    if (i < kOF) {
+#pragma unroll
+      for (int i2 = 0; i2 < kOF; ++i2)
+        if (i2 == i) { c = oc[i2]; x = ox[i2]; }
+    } else {
+      c = ten.oidx[row * k + i];
+      if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(ten.oval)[row * k + i];
+      else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]);
+    }
     const float2 sz = group(c >> lg);
     const float rr = __fsub_rn(x, __fmaf_rn(0.0f, sz.x, sz.y));
 #pragma unroll
