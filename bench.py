@@ -20,6 +20,7 @@ over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -344,10 +345,77 @@ def run_gpu(args, rank: int, world: int):
         "clocks": clk,
     }
     if world == 1:
+        line["gear_l"] = gear_l_measure(gear, wl, we, wd, dev, max(3, K // 2), hbm)
         v, cores, sample = oracle_encode_gbps()
         line["cpu_baseline"] = {"value": round(v, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     print(json.dumps(line), flush=True)
+
+
+def gear_l_measure(gear, wl, we, wd, dev, reps, hbm):
+    """The same two workloads with s = 0 (the pages' GEAR-L: group-wise quantization
+    plus low rank, no outliers), timed like the main stages (CUDA events, L2 flushed
+    before each timed launch sequence). Reported beside GEAR; not the headline."""
+    import torch
+    w0e = dataclasses.replace(we, s=0.0)
+    w0d = dataclasses.replace(wd, s=0.0)
+
+    def params(w):
+        return gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=0.0, rank=w.rank,
+                                power_iters=w.iters, buffer_len=w.buffer_len, buffer_rank=w.buffer_rank,
+                                seed=w.seed)
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    # encode: K and V of the layer in one batched encode
+    xs = [wl.kv_tensor_torch(w0e, which, 0, dev) for which in ("k", "v")]
+    pe = params(w0e)
+    cs = [gear.Cache(pe, w0e.B, w0e.H, w0e.n, 1, torch.float16, dev) for _ in range(2)]
+    enc = []
+    for it in range(reps + 3):
+        for c in cs:
+            c.c.n_comp = c.c.n_buf = c.c.n_blk = c.c.blk0_len = c.c.blk0_rank = 0
+        flush.fill_(it & 0xFF)
+        a, b = ev(), ev()
+        a.record()
+        gear.encode_batch(cs, xs)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= 3:
+            enc.append(a.elapsed_time(b))
+    del xs, cs
+    # decode: compressed context + full buffer
+    pd = params(w0d)
+    dk = gear.Cache(pd, w0d.B, w0d.H, w0d.n + w0d.buffer_len, 2, torch.float16, dev)
+    dv = gear.Cache(pd, w0d.B, w0d.H, w0d.n + w0d.buffer_len, 2, torch.float16, dev)
+    for c, which in ((dk, "k"), (dv, "v")):
+        t = wl.kv_tensor_torch(w0d, which, 0, dev)
+        c.encode(t)
+        del t
+    for i in range(w0d.buffer_fill):
+        gear.append_buffer(dk, dv, wl.rows_torch(w0d, wl.S_KBUF, 0, i, w0d.H, dev),
+                           wl.rows_torch(w0d, wl.S_VBUF, 0, i, w0d.H, dev))
+    q = wl.rows_torch(w0d, wl.S_Q, 0, 0, w0d.Hq, dev)
+    out = torch.empty((w0d.B, w0d.Hq, 128), dtype=torch.float16, device=dev)
+    dec = []
+    for it in range(reps + 3):
+        flush.fill_(it & 0xFF)
+        a, b = ev(), ev()
+        a.record()
+        gear.decode_attn(dk, dv, q, 1.0 / math.sqrt(128), out=out)
+        b.record()
+        torch.cuda.synchronize()
+        if it >= 3:
+            dec.append(a.elapsed_time(b))
+    assert gear.device_status() == 0, "device-side error word set"
+    enc_ms, dec_ms = statistics.median(enc), statistics.median(dec)
+    enc_in = 2 * w0e.B * w0e.H * w0e.n * w0e.d * 2
+    dec_alg = (2 * w0d.B * w0d.H * w0d.n * per_token_bytes(w0d) + 2 * w0d.B * w0d.H * w0d.rank * 128 * 4
+               + 2 * w0d.B * w0d.H * w0d.buffer_fill * 128 * 2 + 2 * w0d.B * w0d.Hq * 128 * 2)
+    return {"s": 0.0, "encode_ms": round(enc_ms, 4), "encode_gbs": round(enc_in / enc_ms / 1e6, 3),
+            "decode_ms": round(dec_ms, 4), "decode_tokens_per_s": round(w0d.B / dec_ms * 1e3, 1),
+            "decode_hbm_frac": round(dec_alg / dec_ms / 1e6 / hbm, 4),
+            "bytes_per_token": per_token_bytes(w0d)}
 
 
 def main():

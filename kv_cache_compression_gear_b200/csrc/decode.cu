@@ -23,7 +23,9 @@
 // values with one lane per 8 channels and token parity. The outlier fix-ups
 // of the values are scattered with fire-and-forget float reductions into the
 // split's partial-result row in global memory. One extra split per unit takes
-// the buffer. decode_combine merges the splits by log-sum-exp.
+// the buffer. decode_combine merges the splits by log-sum-exp. Caches without
+// outliers (s = 0, the pages' GEAR-L variant: quantization plus low rank) run an
+// instantiation with the outlier code compiled out (OUT = false).
 #include <string.h>
 #include "common.cuh"
 #include "decode.cuh"
@@ -206,7 +208,7 @@ __device__ __forceinline__ float lowrank_at(const uint8_t* lf, int t, int rm, in
 // | accx [HQ][128]. The [HQ][128] accumulators hold channel c at slot c;
 // loops that touch all of them use slot e*32 + lane so that every lane stays
 // in its own bank.
-template <typename T, int BITS, int HQ>
+template <typename T, int BITS, int HQ, bool OUT>
 __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) decode_warp(const __grid_constant__ DecodeMaps maps,
                                                          const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
     q_s[e] = qv;
     qw_s[e] = qv * CF::inv_weight(e & 127);
     accx_s[e] = 0.0f;
-    if (comp) st_gpu(part_row + (e >> 7) * hstride + 2 + (e & 127), 0.0f);   // value outlier sums
+    if (OUT && comp) st_gpu(part_row + (e >> 7) * hstride + 2 + (e & 127), 0.0f);   // value outlier sums
   }
   for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
   __syncwarp();
@@ -557,7 +559,8 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
 #pragma unroll
             for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(lj, u_s[hh * kMaxR + j], s_[hh]);
           }
-          if (k <= kFast && rb <= kRReg) {
+          if constexpr (!OUT) {
+          } else if (k <= kFast && rb <= kRReg) {
             int cix[kFast];
             float fx[kFast];
             outlier_fixes<T>(tkr, L.oval, kmrow, mx, t, k, lg, lt, rfk, rp, cix, fx);
@@ -600,16 +603,17 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
               accx_s[hh * 128 + e * 32 + lane] *= al;
             }
             if (rb > kRReg && lane < kMaxR) alr_s[hh * kMaxR + lane] *= al;
-            // the value outlier sums in global memory
-            __threadfence();
-            __syncwarp();
+            if constexpr (OUT) {   // the value outlier sums in global memory
+              __threadfence();
+              __syncwarp();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float* pc = part_row + hh * hstride + 2 + e * 32 + lane;
-              st_gpu(pc, ld_gpu(pc) * al);
+              for (int e = 0; e < 4; ++e) {
+                float* pc = part_row + hh * hstride + 2 + e * 32 + lane;
+                st_gpu(pc, ld_gpu(pc) * al);
+              }
+              __threadfence();
+              __syncwarp();
             }
-            __threadfence();
-            __syncwarp();
           }
           m[hh] = mt;
         }
@@ -641,7 +645,8 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
 #pragma unroll
             for (int hh = 0; hh < HQ; ++hh) alr[hh][j] = fmaf(p[hh], lv[j], alr[hh][j]);
           // value outliers: p * fix lands on channel c of the split's row
-          if (k <= kFast && rb <= kRReg) {
+          if constexpr (!OUT) {
+          } else if (k <= kFast && rb <= kRReg) {
             int cix[kFast];
             float fx[kFast];
             outlier_fixes<T>(tvr, L.oval, vmrow, mx, t, k, lg, lv, rfv, rp, cix, fx);
@@ -756,7 +761,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
       __syncwarp();
     }
   }
-  if (comp) __threadfence();   // the value outlier sums, before they are read back
+  if (OUT && comp) __threadfence();   // the value outlier sums, before they are read back
   __syncwarp();
 
   // ---------------- partial result of this split
@@ -782,7 +787,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int c = 8 * lq + e;
-        const float corr = comp ? ld_gpu(dst + 2 + c) : 0.0f;
+        const float corr = (OUT && comp) ? ld_gpu(dst + 2 + c) : 0.0f;
         dst[2 + c] = CF::inv_weight(c) * (v[e] - swg) + spg + accx_s[hh * 128 + c] + corr;
       }
     }
@@ -850,28 +855,28 @@ void decode_plan(DecodeArgs& a, int num_sms) {
 
 size_t decode_workspace_bytes(int B, int Hq, int nsplit) { return (size_t)B * Hq * nsplit * 130 * sizeof(float); }
 
-template <typename T, int BITS, int HQ>
+template <typename T, int BITS, int HQ, bool OUT>
 static cudaError_t launch_warp(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = 4 * (size_t)a.tl.bytes + 1024;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(decode_warp<T, BITS, HQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_warp<T, BITS, HQ, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     configured_smem = (int)smem;
   }
   const int grid = (a.total_splits + 3) / 4;
-  decode_warp<T, BITS, HQ><<<grid, kDThreads, smem, st>>>(maps, a);
+  decode_warp<T, BITS, HQ, OUT><<<grid, kDThreads, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
 
 template <typename T, int BITS>
 static cudaError_t launch_hq(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
   switch (a.hq) {
-    case 1: return launch_warp<T, BITS, 1>(maps, a, st);
-    case 2: return launch_warp<T, BITS, 2>(maps, a, st);
-    case 4: return launch_warp<T, BITS, 4>(maps, a, st);
-    case 8: return launch_warp<T, BITS, 8>(maps, a, st);
+    case 1: return a.k > 0 ? launch_warp<T, BITS, 1, true>(maps, a, st) : launch_warp<T, BITS, 1, false>(maps, a, st);
+    case 2: return a.k > 0 ? launch_warp<T, BITS, 2, true>(maps, a, st) : launch_warp<T, BITS, 2, false>(maps, a, st);
+    case 4: return a.k > 0 ? launch_warp<T, BITS, 4, true>(maps, a, st) : launch_warp<T, BITS, 4, false>(maps, a, st);
+    case 8: return a.k > 0 ? launch_warp<T, BITS, 8, true>(maps, a, st) : launch_warp<T, BITS, 8, false>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -48,6 +48,7 @@ ENC_CASES = [
     ("f16", 2, 2, 300, 4, 32, 0.02, 8, 3),
     ("f16", 1, 3, 1000, 4, 128, 0.02, 4, 3),
     ("f16", 1, 2, 257, 4, 64, 0.0, 0, 1),
+    ("f16", 2, 2, 300, 4, 64, 0.0, 4, 3),    # GEAR-L: no outliers, low rank
     ("f16", 1, 2, 257, 4, 64, 0.1, 16, 2),
     ("bf16", 1, 2, 300, 4, 64, 0.02, 4, 3),
     ("bf16", 2, 2, 77, 2, 64, 0.05, 2, 1),
@@ -136,6 +137,8 @@ DEC_CASES = [
     ("f16", 2, 1, 4, 130, 45, 2, 32, 0.05, 8, 20, 2),
     ("f16", 1, 2, 2, 0, 7, 4, 64, 0.02, 4, 3, 1),
     ("f16", 1, 2, 2, 1000, 21, 4, 128, 0.0, 0, 20, 0),
+    ("f16", 2, 2, 8, 300, 25, 4, 64, 0.0, 4, 20, 2),    # GEAR-L
+    ("bf16", 1, 2, 2, 200, 3, 2, 32, 0.0, 8, 20, 2),    # GEAR-L
     ("bf16", 1, 2, 8, 257, 20, 4, 64, 0.02, 4, 20, 2),
     ("f32", 1, 1, 1, 256, 0, 4, 64, 0.02, 4, 20, 2),
     ("f32", 1, 2, 4, 64, 9, 8, 32, 0.05, 2, 4, 2),
