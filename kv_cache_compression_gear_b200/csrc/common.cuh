@@ -86,6 +86,10 @@ struct CodeFloats {
   __host__ __device__ static constexpr float inv_weight(int c) {
     return (float)(1 << (8 - (c % kPerByte) * BITS));
   }
+  // its inverse 2^(pos*BITS - 8), exactly (a power of two built from its bits)
+  __device__ static __forceinline__ float weight(int c) {
+    return __int_as_float((127 + (c % kPerByte) * BITS - 8) << 23);
+  }
 };
 
 // Row length of the stored Rf factors: r_max rounded up to a multiple of 4, so

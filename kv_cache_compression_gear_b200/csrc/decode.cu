@@ -202,14 +202,14 @@ __device__ __forceinline__ float lowrank_at(const uint8_t* lf, int t, int rm, in
   return lr;
 }
 
-// Per-warp shared memory (see TileLayout): 4 code tiles | 4 meta tiles |
-// 4 rest tiles | floats | 2 mbarriers. Floats: q [HQ][128] | qw [HQ][128]
-// (q scaled by the code weights) | u [HQ][16] | alr [HQ][16] | w [32][G][HQ]
-// | accx [HQ][128]. The [HQ][128] accumulators hold channel c at slot c;
-// loops that touch all of them use slot e*32 + lane so that every lane stays
-// in its own bank.
+// Shared memory (see TileLayout): the warps' code tiles, then per warp 4 meta
+// tiles | 4 rest tiles | floats | 2 mbarriers. Floats: qw [HQ][128] (q scaled
+// by the code weights; q itself is qw * CF::weight, exactly) | u [HQ][16] |
+// alr [HQ][16] | w [32][G][HQ] | accx [HQ][128]. The [HQ][128] arrays hold
+// channel c at slot c; loops that touch all of them use slot e*32 + lane so
+// that every lane stays in its own bank.
 template <typename T, int BITS, int HQ, bool OUT>
-__global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) decode_warp(const __grid_constant__ DecodeMaps maps,
+__global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) decode_warp(const __grid_constant__ DecodeMaps maps,
                                                          const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
   constexpr int W = 4 * BITS;
@@ -224,10 +224,10 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
   const int rp = rpad_of(rm);
   const uint32_t one = a.one_bits;
   const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
-  const uint32_t abase = (smem_u32(dsm) + 1023u) & ~1023u;
-  uint8_t* wb = dsm + (abase - smem_u32(dsm)) + (size_t)wid * L.bytes;
-  float* q_s = reinterpret_cast<float*>(wb + L.floats);
-  float* qw_s = q_s + HQ * 128;
+  uint8_t* cta = align_smem_1024(dsm);
+  uint8_t* cb = cta + (size_t)wid * 4 * L.cb;                          // this warp's 4 code tiles
+  uint8_t* wb = cta + (size_t)16 * L.cb + (size_t)wid * L.bytes;     // its other regions
+  float* qw_s = reinterpret_cast<float*>(wb + L.floats);
   float* u_s = qw_s + HQ * 128;
   float* alr_s = u_s + HQ * kMaxR;   // value low-rank weights j >= kRReg
   float* w_s = alr_s + HQ * kMaxR;
@@ -242,7 +242,6 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
   const size_t hstride = (size_t)a.nsplit * 130;
   for (int e = lane; e < HQ * 128; e += 32) {
     const float qv = load_elem<T>(a.q, ((size_t)b * a.Hq + (size_t)h * HQ + (e >> 7)) * 128 + (e & 127));
-    q_s[e] = qv;
     qw_s[e] = qv * CF::inv_weight(e & 127);
     accx_s[e] = 0.0f;
     if (OUT && comp) st_gpu(part_row + (e >> 7) * hstride + 2 + (e & 127), 0.0f);   // value outlier sums
@@ -278,7 +277,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
     for (int hh = 0; hh < HQ; ++hh)
 #pragma unroll
       for (int bk = 0; bk < 4; ++bk) {
-        qs_blk[hh][bk] = warp_sum(q_s[hh * 128 + bk * 32 + lane]);
+        qs_blk[hh][bk] = warp_sum(qw_s[hh * 128 + bk * 32 + lane] * CF::weight(bk * 32 + lane));
         qw_blk[hh][bk] = warp_sum(qw_s[hh * 128 + bk * 32 + lane]);
       }
 
@@ -296,7 +295,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
       switch (lane >> 1) {
         case 0:
           my_map = x ? &maps.vc : &maps.kc;
-          my_dst = wbs + x * L.cb;
+          my_dst = smem_u32(cb) + x * L.cb;
           my_sst = 2 * L.cb;
           break;
         case 1:
@@ -449,7 +448,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
         return;
       }
       __syncwarp();
-      const uint8_t* tkc = wb + (2 * s) * L.cb;
+      const uint8_t* tkc = cb + (2 * s) * L.cb;
       const uint8_t* tvc = tkc + L.cb;
       const uint8_t* tkm = wb + L.meta0 + (2 * s) * L.mb;
       const uint8_t* tvm = tkm + L.mb;
@@ -473,7 +472,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
             for (int e = 0; e < 4; ++e) {
               const int c = e * 32 + lane;
               const float4 r4 = __ldg(reinterpret_cast<const float4*>(rfk + c * rp + j4));
-              const float qv = q_s[hh * 128 + c];
+              const float qv = qw_s[hh * 128 + c] * CF::weight(c);
               u4[0] = fmaf(r4.x, qv, u4[0]);
               u4[1] = fmaf(r4.y, qv, u4[1]);
               u4[2] = fmaf(r4.z, qv, u4[2]);
@@ -567,7 +566,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
 #pragma unroll
             for (int i = 0; i < kFast; ++i)
 #pragma unroll
-              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(q_s[hh * 128 + cix[i]], fx[i], s_[hh]);
+              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + cix[i]] * CF::weight(cix[i]), fx[i], s_[hh]);
           } else {
             for (int i = 0; i < k; ++i) {
               const int c = tkr[t * k + i];
@@ -575,7 +574,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
               const float xo = (float)reinterpret_cast<const T*>(tkr + L.oval)[t * k + i];
               const float fix = xo - (meta_at(kmrow, c >> lg, mx).y + lr);
 #pragma unroll
-              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(q_s[hh * 128 + c], fix, s_[hh]);
+              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + c] * CF::weight(c), fix, s_[hh]);
             }
           }
         }
@@ -731,7 +730,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 3 : (HQ == 4 ? 2 : 1)) de
         for (int c = 0; c < 128; ++c) {
           const float x = load_elem<T>(a.K.buf, (brow + t0 + lane) * 128 + c);
 #pragma unroll
-          for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(x, q_s[hh * 128 + c], s[hh]);
+          for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(x, qw_s[hh * 128 + c] * CF::weight(c), s[hh]);
         }
       }
       float p[HQ];
@@ -826,13 +825,13 @@ void decode_plan(DecodeArgs& a, int num_sms) {
   L.oval = r16(kDTile * a.k);
   L.lf = L.oval + r16(kDTile * a.k * esz);
   L.rb = L.lf + r16(kDTile * a.r_max * esz);
-  L.meta0 = 4 * L.cb;
+  L.meta0 = 0;
   L.rest0 = L.meta0 + 4 * L.mb;
   L.floats = L.rest0 + 4 * L.rb;
   const int hq = a.hq;
-  const int floats = 2 * hq * 128 + 2 * hq * kMaxR + kDTile * a.G * hq + hq * 128;
+  const int floats = hq * 128 + 2 * hq * kMaxR + kDTile * a.G * hq + hq * 128;   // qw, u, alr, w, accx
   L.bars = L.floats + r16(floats * 4);
-  L.bytes = (L.bars + 16 + 1023) & ~1023;
+  L.bytes = (L.bars + 16 + 255) & ~255;   // meta tiles stay 256-byte aligned
   const int meta_tx = a.G >= 2 ? 2 * L.mb : 0;
   L.tx_part = 2 * L.cb + meta_tx;
   L.tx_full = L.tx_part + 2 * kDTile * (a.k + a.k * esz + a.r_max * esz) + (a.G >= 2 ? 0 : 2 * L.mb);
@@ -857,7 +856,7 @@ size_t decode_workspace_bytes(int B, int Hq, int nsplit) { return (size_t)B * Hq
 
 template <typename T, int BITS, int HQ, bool OUT>
 static cudaError_t launch_warp(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
-  const size_t smem = 4 * (size_t)a.tl.bytes + 1024;
+  const size_t smem = 1024 + 16 * (size_t)a.tl.cb + 4 * (size_t)a.tl.bytes;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
     cudaError_t e = cudaFuncSetAttribute(decode_warp<T, BITS, HQ, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -18,17 +18,18 @@ struct CacheView {
   const void* buf;
 };
 
-// Per-warp shared memory of decode_warp. Tile idx = 2 * stage + tensor
-// (tensor 0 = keys, 1 = values) has its codes at idx * cb, its meta at
-// meta0 + idx * mb and the rest (oidx | oval | lf) at rest0 + idx * rb, all
-// from the warp's 1024-byte-aligned base.
+// Shared memory of a decode_warp CTA (4 warps), from a 1024-byte-aligned base:
+// first the code tiles of all warps (warp w, tile idx at (4w + idx) * cb), then
+// one region of `bytes` per warp holding its meta tiles (meta0 + idx * mb), its
+// rest tiles (oidx | oval | lf at rest0 + idx * rb), the float scratch and the
+// two stage barriers. Tile idx = 2 * stage + tensor (0 = keys, 1 = values).
 struct TileLayout {
   int32_t cb, mb, rb;      // bytes per tile: codes, meta, rest
   int32_t oval, lf;        // offsets of oval and lf inside the rest
-  int32_t meta0, rest0;    // offsets of tile 0's meta and rest
+  int32_t meta0, rest0;    // offsets of tile 0's meta and rest in the warp's region
   int32_t floats;          // offset of the float scratch
   int32_t bars;            // offset of the two stage barriers
-  int32_t bytes;           // bytes per warp, a multiple of 1024
+  int32_t bytes;           // bytes of the warp's region, a multiple of 256
   int32_t tx_full;         // bytes a stage barrier expects for a whole, aligned tile
   int32_t tx_part;         // ... for another tile (codes and meta only; the rest is copied by the lanes)
 };
