@@ -799,20 +799,14 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeArgs a) {
   const int c = threadIdx.x;
   const float* p = a.part + (size_t)bj * a.nsplit * 130;
   float M = -INFINITY;
-#pragma unroll 8
   for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, p[s * 130]);
   float den = 0.0f, num = 0.0f;
-  // eight splits' loads in flight at a time; the sums keep split order
-#pragma unroll 8
   for (int s = 0; s < a.nsplit; ++s) {
     const float m = p[s * 130];
-    const float l = p[s * 130 + 1];
-    const float v = p[s * 130 + 2 + c];
-    if (m != -INFINITY) {   // a split without a finite score contributes nothing
-      const float w = exp2f(m - M);
-      den = fmaf(l, w, den);
-      num = fmaf(v, w, num);
-    }
+    if (m == -INFINITY) continue;   // a split without a finite score contributes nothing
+    const float w = exp2f(m - M);
+    den = fmaf(p[s * 130 + 1], w, den);
+    num = fmaf(p[s * 130 + 2 + c], w, num);
   }
   const float o = num / den;
   TO* out = reinterpret_cast<TO*>(a.out) + (size_t)bj * 128 + c;
