@@ -808,7 +808,7 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
       // Cholesky G = C^T C (upper C) with column dropping, then X = C^-1 so
       // that P~ X has orthonormal (or zero) columns. All indices are
       // compile-time, so C and X stay in registers.
-      double C[RM][RM], X[RM][RM];
+      double C[RM][RM], X[RM][RM], rinv[RM];
       bool nz[RM];
 #pragma unroll
       for (int p = 0; p < RM; ++p)
@@ -828,17 +828,20 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
           double v = C[m2][j];
 #pragma unroll
           for (int i2 = 0; i2 < m2; ++i2) v -= C[i2][m2] * C[i2][j];
-          C[m2][j] = nz[m2] ? v / C[m2][m2] : 0.0;
+          C[m2][j] = v * rinv[m2];   // 0 for a dropped column
         }
         double piv = gjj;
 #pragma unroll
         for (int m2 = 0; m2 < j; ++m2) piv -= C[m2][j] * C[m2][j];
         nz[j] = j < r && gjj > 0.0 && piv > 1e-10 * gjj;
-        C[j][j] = nz[j] ? sqrt(piv) : 1.0;
+        // one reciprocal square root per column gives both C_jj and 1 / C_jj
+        const double rs = nz[j] ? rsqrt(piv) : 0.0;
+        C[j][j] = nz[j] ? piv * rs : 1.0;
+        rinv[j] = rs;
       }
 #pragma unroll
       for (int j = 0; j < RM; ++j) {
-        const double inv = nz[j] ? 1.0 / C[j][j] : 0.0;
+        const double inv = rinv[j];
 #pragma unroll
         for (int i2 = 0; i2 <= j; ++i2) {
           double v = (i2 == j) ? 1.0 : 0.0;
@@ -873,9 +876,10 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
         for (int j = 0; j < RM; ++j) S.Q[i * RM + j] = wq[j];
       } else {
         const double sL = ldexp(1.0, a.e_blk), sR = ldexp(1.0, -a.e_blk);
-        float* zrow = a.zbuf + ((int64_t)u * 128 + i) * 16;
+        // Z rows in channel pairs: zbuf[u][i / 2][j][i % 2], the layout E3 copies in one piece
+        float* zrow = a.zbuf + (((int64_t)u * 64 + (i >> 1)) * 16) * 2 + (i & 1);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) zrow[j] = (j < RM && j < r) ? (float)(zq[j < RM ? j : 0] * sL) : 0.0f;
+        for (int j = 0; j < 16; ++j) zrow[2 * j] = (j < RM && j < r) ? (float)(zq[j < RM ? j : 0] * sL) : 0.0f;
         const int rp = rpad_of(a.r_max);
         float* rrow = a.ten[u / a.Uper].rfac + (((int64_t)(u % a.Uper) * a.nblk_max + a.blk) * 128 + i) * rp;
         for (int j = 0; j < rp; ++j) {
@@ -916,8 +920,9 @@ struct E3Cfg {
   static constexpr int kRow = 16 * BITS;                     // code bytes per token
   static constexpr int kCB = kTile * kRow;                   // code tile
   static constexpr int kMB = kTile * 32;                     // meta tile (G <= 4)
-  static constexpr int kZOff = kXB + kCB + kMB;              // Z pairs [64][RMAX] float2
-  static constexpr int kBarOff = kZOff + 64 * RMAX * 8;
+  static constexpr int kZOff = kXB + kCB + kMB;              // Z pairs [64][16] float2
+  static constexpr int kZBytes = 64 * 16 * 8;
+  static constexpr int kBarOff = kZOff + kZBytes;
   static constexpr int kSmem = kBarOff + 16 + 1024;          // + alignment slack
 };
 
@@ -949,15 +954,16 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   if (t == 0) {
     mbar_init(bar, 1);
     fence_mbarrier_init();
-    mbar_arrive_expect_tx(bar, (uint32_t)(F::kXB + F::kCB + (meta_tma ? kTile * G * 8 : 0)));
+    mbar_arrive_expect_tx(bar, (uint32_t)(F::kXB + F::kCB + F::kZBytes + (meta_tma ? kTile * G * 8 : 0)));
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(Zp)),
+                 "l"(a.zbuf + (int64_t)u * (F::kZBytes / 4)), "r"((uint32_t)F::kZBytes), "r"(smem_u32(bar))
+                 : "memory");
     for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(xs + b * 16384, &maps.x[tn], bar, b * C::kBoxCols, ul * a.n + t0);
     tma_load_2d(cs, &maps.codes[tn], bar, 0, crow);
     if (meta_tma) tma_load_2d(ms, &maps.meta[tn], bar, 0, crow);
   }
-  for (int e = t; e < 64 * RMAX; e += kE3Threads) {   // Zp[p][j] = (Z[2p][j], Z[2p + 1][j])
-    const float* zb = a.zbuf + ((int64_t)u * 128 + 2 * (e / RMAX)) * 16 + e % RMAX;
-    Zp[e] = make_float2(zb[0], zb[16]);
-  }
+  // Zp[p][j] = (Z[2p][j], Z[2p + 1][j]) arrives with the tile (E2 writes it in this layout)
   const bool valid = t0 + t < a.n;
   const size_t row = (size_t)crow + t;
   float2 sz1 = make_float2(0.0f, 0.0f);
@@ -1059,7 +1065,7 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
           const uint64_t cf = f2_sub(f2_pack(f[cl], f[cl + 1]), one2);
           const uint64_t dh = f2_fma(cf, f2_mul(sc2, w2), zr2);
           const uint64_t rr = f2_sub(f2_pack(xv[cl], xv[cl + 1]), dh);
-          const float4* zq = reinterpret_cast<const float4*>(Zp + (4 * jb + p) * RMAX);
+          const float4* zq = reinterpret_cast<const float4*>(Zp + (4 * jb + p) * 16);
 #pragma unroll
           for (int j = 0; j < RMAX; j += 2) {
             const float4 z = zq[j >> 1];
@@ -1093,7 +1099,7 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
           const uint64_t rv = f2_pack(rr[0], rr[1]);
 #pragma unroll
           for (int j = 0; j < RMAX; ++j)
-            acc[j] = f2_fma(rv, *reinterpret_cast<const uint64_t*>(&Zp[(4 * jb + p) * RMAX + j]), acc[j]);
+            acc[j] = f2_fma(rv, *reinterpret_cast<const uint64_t*>(&Zp[(4 * jb + p) * 16 + j]), acc[j]);
         }
       }
     }
@@ -1115,7 +1121,7 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
     const float rr = __fsub_rn(x, __fmaf_rn(0.0f, sz.x, sz.y));
 #pragma unroll
     for (int j = 0; j < RMAX; ++j) {
-      const float2 z = Zp[(c >> 1) * RMAX + j];
+      const float2 z = Zp[(c >> 1) * 16 + j];
       const float v = rr * ((c & 1) ? z.y : z.x);
       acc[j] = f2_sub(acc[j], (c & 1) ? f2_pack(0.0f, v) : f2_pack(v, 0.0f));
     }

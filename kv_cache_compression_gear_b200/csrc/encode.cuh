@@ -32,7 +32,7 @@ struct EncodeArgs {
   int32_t t_off, blk, e_blk;
   uint32_t one_bits;     // 0x3F800000 (1.0f), kept in a register by the kernels
   int32_t n_max, nblk_max, W, G, r_max;
-  // workspace: partial Grams [U][maxc][128][128] and Z [U][128][16]
+  // workspace: partial Grams [U][maxc][128][128] and Z [U][64][16][2] (channel pairs)
   float* gram;
   float* zbuf;
   // tiling of E1
