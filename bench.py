@@ -144,6 +144,28 @@ def oracle_encode_gbps(seconds_budget: float = 12.0, units_cap: int = 64):
     return nbytes / dt / 1e9, cores, f"{done} of {2 * w.H} (head, K/V) units of {ENC}, {w.n} tokens each"
 
 
+def bench_config(world: int) -> dict:
+    """The workload both arms report (the reference arm times its encode part)."""
+    import workloads as wl
+    we, wd = wl.WORKLOADS[ENC], wl.WORKLOADS[DEC]
+    return {"workload": f"{ENC} + {DEC}",
+            "encode": {"batch": we.B, "heads": we.H, "tokens": we.n, "head_dim": we.d, "bits": we.bits,
+                       "group": we.group, "s": we.s, "rank": we.rank, "iters": we.iters},
+            "decode": {"batch": wd.B, "heads": wd.H, "context": wd.n, "buffer": wd.buffer_len},
+            "l2": "flushed (512 MiB write) before every timed stage", "parallelism": f"replicas x{world}"}
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest of every rank's value (the slowest rank's time). All ranks call
+    it in the same order; one all-reduce of a scalar, nothing on the data path."""
+    if world == 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
@@ -151,15 +173,18 @@ def run_reference(args, rank: int, world: int):
     cores, sample = None, None
     for _ in range(args.warmup):
         oracle_encode_gbps(seconds_budget=3.0, units_cap=8)
+    step_ms = []
     for _ in range(args.steps):
+        t0 = time.perf_counter()
         v, cores, sample = oracle_encode_gbps(seconds_budget=6.0, units_cap=16)
+        step_ms.append((time.perf_counter() - t0) * 1e3)
         vals.append(v)
     v = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(statistics.median(step_ms), 3),
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64 (oracle)", "data": "synthetic",
-            "config": {"workload": ENC, "global_batch": 1, "seq_len": 4096, "heads": 32, "head_dim": 128,
-                       "parallelism": "host threads"},
+            "config": bench_config(world),
             "cpu_baseline": {"value": round(v, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -288,11 +313,7 @@ def run_gpu(args, rank: int, world: int):
         e2e_dec.append(c.elapsed_time(d))
 
     def maxrank(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(v, world, dev)
 
     enc_t = maxrank(sum(enc_ms) / 1e3)
     dec_t = maxrank(sum(dec_ms) / 1e3)
@@ -328,11 +349,7 @@ def run_gpu(args, rank: int, world: int):
         "warmup": args.warmup, "ms_per_step": round((enc_t + dec_t + app_t) / K * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded, workloads/)",
-        "config": {"workload": f"{ENC} + {DEC}", "encode": {"batch": we.B, "heads": we.H, "tokens": we.n,
-                                                             "head_dim": we.d, "bits": we.bits, "group": we.group,
-                                                             "s": we.s, "rank": we.rank, "iters": we.iters},
-                   "decode": {"batch": wd.B, "heads": wd.H, "context": wd.n, "buffer": wd.buffer_len},
-                   "l2": "flushed (512 MiB write) before every timed stage", "parallelism": f"replicas x{world}"},
+        "config": bench_config(world),
         "decode_tokens_per_s": round(dec_tps, 1),
         "stage_ms": {"encode": round(enc_t / K * 1e3, 4), "decode": round(dec_t / K * 1e3, 4),
                      "append": round(app_t / K * 1e3, 4), "appends_with_flush": nflush},

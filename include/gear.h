@@ -239,6 +239,15 @@ gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream)
  * kernels set instead of trapping (GEAR_ERR_* value, 0 if none). */
 gear_status gear_get_device_status(int32_t* status);
 
+/* Failure-detection self-test (no counterpart in the paper): launches one warp
+ * that waits on an mbarrier nothing ever completes, bounded by limit_us
+ * microseconds (1 .. 1000000) of wall time. The bound runs out, the kernel
+ * records GEAR_ERR_TIMEOUT in the device error word and returns; nothing
+ * traps, and the context stays usable. Asynchronous on `stream`; read the
+ * result with gear_get_device_status after synchronizing.
+ * Errors: INVALID_ARG (limit out of range), CUDA. */
+gear_status gear_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 /* Static description of a status code. */
 const char* gear_status_string(gear_status s);
 

@@ -134,6 +134,19 @@ static size_t encode_ws_bytes(const gear_cache* c, int nt, int n) {
 }
 
 // ------------------------------------------------------------------ append
+// One warp waits on an mbarrier that nothing arrives on; the bounded wait gives
+// up after limit_ns and records GEAR_ERR_TIMEOUT (the failure-detection path
+// every kernel's waits take).
+__global__ void selftest_wait(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncwarp();
+  mbar_wait_for(&bar, 0, limit_ns);
+}
+
 template <typename T>
 __global__ void append_rows(T* __restrict__ kbuf, T* __restrict__ vbuf, const T* __restrict__ kn,
                             const T* __restrict__ vn, int U, int n_b, int slot) {
@@ -385,6 +398,12 @@ gear_status gear_get_device_status(int32_t* status) {
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return GEAR_ERR_CUDA;
   *status = v;
   return GEAR_OK;
+}
+
+gear_status gear_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return GEAR_ERR_INVALID_ARG;
+  selftest_wait<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull);
+  return cuda_status(cudaGetLastError());
 }
 
 const char* gear_status_string(gear_status s) {

@@ -161,16 +161,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Waits for the phase with the given parity to complete, sleeping between
 // probes. Returns false (and records GEAR_ERR_TIMEOUT) if the barrier does not
-// complete within the bound.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// complete within `limit_ns` of wall time.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint32_t every = limit_ns < kSpinNanos ? 1u : 64u;   // short bounds: check the clock each probe
   for (uint32_t i = 1; i < kSpinLimit; ++i) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if ((i & 63) == 0 && global_timer_ns() - t0 > kSpinNanos) break;
+    if ((i % every) == 0 && global_timer_ns() - t0 > limit_ns) break;
   }
   set_device_error(GEAR_ERR_TIMEOUT);
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kSpinNanos);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -71,6 +71,7 @@ def _load():
         "gear_append_buffer": (i32, [pc, pc, P, P, P, S, P]),
         "gear_decode_dense": (i32, [pc, P, P]),
         "gear_get_device_status": (i32, [ctypes.POINTER(i32)]),
+        "gear_selftest_wait_timeout": (i32, [ctypes.c_uint32, P]),
         "gear_status_string": (ctypes.c_char_p, [i32]),
         "gear_version": (ctypes.c_char_p, []),
     }
