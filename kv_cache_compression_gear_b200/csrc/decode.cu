@@ -11,21 +11,24 @@
 // and the value side accumulates p_t * (scale*code + zero) per channel, the
 // block's low-rank part as (sum_t p_t L_t) Rf_b^T, and the outlier fix-ups.
 //
-// Split-K (flash-decoding style): in decode_warp every warp is one split, a
-// run of whole 32-token tiles of one (batch, kv head), for all query heads
-// sharing that kv head. Its lanes bring the tiles of both tensors into the
-// warp's own shared memory with tensor copies (codes and meta, 16-byte-chunk
-// swizzled so that both the per-token and the per-channel reads are free of
-// bank conflicts) and bulk copies (outlier channels and values, L rows),
-// double-buffered on two mbarriers. It scores with one lane per token
-// straight from the packed codes, keeps an online softmax whose reference
-// moves only when the running maximum passes it by 2^8, and accumulates
-// values with one lane per 8 channels and token parity. The outlier fix-ups
-// of the values are scattered with fire-and-forget float reductions into the
-// split's partial-result row in global memory. One extra split per unit takes
-// the buffer. decode_combine merges the splits by log-sum-exp. Caches without
-// outliers (s = 0, the pages' GEAR-L variant: quantization plus low rank) run an
-// instantiation with the outlier code compiled out (OUT = false).
+// Split-K (flash-decoding style), stream-K scheduled: the grid is one wave of
+// resident warps, and warp w takes compressed tokens [w*T, (w+1)*T) of all
+// (batch, kv head) units laid end to end, for all query heads sharing the kv
+// head. A unit boundary inside that run starts a new segment with its own
+// partial result; the warp that ends a unit also folds in the unit's buffer.
+// The warp brings the tiles of both tensors into its own shared memory with
+// tensor copies (codes and meta, 16-byte-chunk swizzled so that both the
+// per-token and the per-channel reads are free of bank conflicts) and bulk
+// copies (outlier channels and values, L rows), double-buffered on two
+// mbarriers. It scores with one lane per token straight from the packed
+// codes, keeps an online softmax whose reference moves only when the running
+// maximum passes it by 2^8, and accumulates values with one lane per 8
+// channels and token parity. The value outlier fix-ups are scattered with
+// fire-and-forget float reductions into the segment's partial-result row in
+// global memory. decode_combine merges a unit's segments by log-sum-exp.
+// Caches without outliers (s = 0, the pages' GEAR-L variant: quantization plus
+// low rank) run an instantiation with the outlier code compiled out
+// (OUT = false).
 #include <string.h>
 #include "common.cuh"
 #include "decode.cuh"
@@ -234,375 +237,67 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
   float* accx_s = w_s + kDTile * G * HQ;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wb + L.bars);
 
-  const int unit = gs / a.nsplit, sp = gs % a.nsplit;
-  const int b = unit / a.H, h = unit % a.H;
-  const bool comp = sp < a.nsplit_comp;
-  // this split's partial row of query head hh: part_row + hh * hstride
-  float* part_row = a.part + (((size_t)b * a.Hq + (size_t)h * HQ) * a.nsplit + sp) * 130;
-  const size_t hstride = (size_t)a.nsplit * 130;
-  for (int e = lane; e < HQ * 128; e += 32) {
-    const float qv = load_elem<T>(a.q, ((size_t)b * a.Hq + (size_t)h * HQ + (e >> 7)) * 128 + (e & 127));
-    qw_s[e] = qv * CF::inv_weight(e & 127);
-    accx_s[e] = 0.0f;
-    if (OUT && comp) st_gpu(part_row + (e >> 7) * hstride + 2 + (e & 127), 0.0f);   // value outlier sums
-  }
-  for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
-  __syncwarp();
-
   // value side: lane owns channels 8*(lane & 15) .. +7 and tokens of parity lane >> 4
   const int lq = lane & 15, par = lane >> 4;
   const int my_g = (8 * lq) >> lg;
-  float m[HQ], lsum[HQ], sw[HQ][4], spm[HQ][4], alr[HQ][kRReg];
-  uint64_t acc[HQ][4];   // channel pairs (8 channels)
-#pragma unroll
-  for (int hh = 0; hh < HQ; ++hh) {
-    m[hh] = -INFINITY;
-    lsum[hh] = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) { acc[hh][e] = 0; sw[hh][e] = 0.0f; spm[hh][e] = 0.0f; alr[hh][e] = 0.0f; }
+  if (lane == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbarrier_init();
   }
+  __syncwarp();
+  int it = 0;   // tiles staged so far; the stage parities run on across segments
 
-  if (comp) {
-    if (lane == 0) {
-      mbar_init(&bars[0], 1);
-      mbar_init(&bars[1], 1);
-      fence_mbarrier_init();
+  // One segment: compressed tokens [c0, c1) of `unit` (maybe none), then the
+  // unit's buffer if with_buf, into partial row sp of the unit. Returns false if
+  // a bounded wait gave up (the error word is set; nothing is written).
+  auto segment = [&](const int unit, const int c0, const int c1, const int sp, const bool with_buf) -> bool {
+    const int b = unit / a.H, h = unit % a.H;
+    const bool comp = c1 > c0;
+    // this split's partial row of query head hh: part_row + hh * hstride
+    float* part_row = a.part + (((size_t)b * a.Hq + (size_t)h * HQ) * a.nsplit + sp) * 130;
+    const size_t hstride = (size_t)a.nsplit * 130;
+    for (int e = lane; e < HQ * 128; e += 32) {
+      const float qv = load_elem<T>(a.q, ((size_t)b * a.Hq + (size_t)h * HQ + (e >> 7)) * 128 + (e & 127));
+      qw_s[e] = qv * CF::inv_weight(e & 127);
+      accx_s[e] = 0.0f;
+      if (OUT && comp) st_gpu(part_row + (e >> 7) * hstride + 2 + (e & 127), 0.0f);   // value outlier sums
     }
-    __threadfence();   // the zeroed outlier sums before any reduction
+    for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
     __syncwarp();
 
-    // group sums of q and of the weighted q, per 32-channel block
-    float qs_blk[HQ][4], qw_blk[HQ][4];
+    float m[HQ], lsum[HQ], sw[HQ][4], spm[HQ][4], alr[HQ][kRReg];
+    uint64_t acc[HQ][4];   // channel pairs (8 channels)
 #pragma unroll
-    for (int hh = 0; hh < HQ; ++hh)
+    for (int hh = 0; hh < HQ; ++hh) {
+      m[hh] = -INFINITY;
+      lsum[hh] = 0.0f;
 #pragma unroll
-      for (int bk = 0; bk < 4; ++bk) {
-        qs_blk[hh][bk] = warp_sum(qw_s[hh * 128 + bk * 32 + lane] * CF::weight(bk * 32 + lane));
-        qw_blk[hh][bk] = warp_sum(qw_s[hh * 128 + bk * 32 + lane]);
-      }
-
-    // ---- copy roles: lanes 0/1 codes (K/V), 2/3 meta by tensor copy (G >= 2),
-    // 4/5 oidx, 6/7 oval, 8/9 L rows, 10/11 meta by bulk copy (G = 1)
-    const bool meta_tma = G >= 2;
-    const int x = lane & 1;
-    const CUtensorMap* my_map = nullptr;
-    const uint8_t* my_src = nullptr;
-    int my_bpr = 0;
-    uint32_t my_dst = 0, my_sst = 0;
-    {
-      const int esz = (int)sizeof(T), lsz = sizeof(T) == 4 ? 4 : 2;
-      const uint32_t wbs = smem_u32(wb);
-      switch (lane >> 1) {
-        case 0:
-          my_map = x ? &maps.vc : &maps.kc;
-          my_dst = smem_u32(cb) + x * L.cb;
-          my_sst = 2 * L.cb;
-          break;
-        case 1:
-          if (meta_tma) {
-            my_map = x ? &maps.vm : &maps.km;
-            my_dst = wbs + L.meta0 + x * L.mb;
-            my_sst = 2 * L.mb;
-          }
-          break;
-        case 2:
-          my_src = x ? a.V.oidx : a.K.oidx;
-          my_bpr = k;
-          my_dst = wbs + L.rest0 + x * L.rb;
-          my_sst = 2 * L.rb;
-          break;
-        case 3:
-          my_src = reinterpret_cast<const uint8_t*>(x ? a.V.oval : a.K.oval);
-          my_bpr = k * esz;
-          my_dst = wbs + L.rest0 + x * L.rb + L.oval;
-          my_sst = 2 * L.rb;
-          break;
-        case 4:
-          my_src = reinterpret_cast<const uint8_t*>(x ? a.V.lfac : a.K.lfac);
-          my_bpr = rm * lsz;
-          my_dst = wbs + L.rest0 + x * L.rb + L.lf;
-          my_sst = 2 * L.rb;
-          break;
-        case 5:
-          if (!meta_tma) {
-            my_src = reinterpret_cast<const uint8_t*>(x ? a.V.meta : a.K.meta);
-            my_bpr = G * 8;
-            my_dst = wbs + L.meta0 + x * L.mb;
-            my_sst = 2 * L.mb;
-          }
-          break;
-        default:
-          break;
-      }
-    }
-    const size_t row0 = (size_t)unit * a.n_max;   // row of the unit's token 0
-    // Brings tokens [t, t + nt) of the unit into stage s. A whole, 32-aligned
-    // tile is all copies; another one (a block boundary or the split's end)
-    // takes codes and meta by tensor copy (rows past nt are read and ignored)
-    // and the rest by plain loads of the lanes.
-    auto issue = [&](int s, int t, int nt) {
-      const bool full = nt == kDTile && (t & (kDTile - 1)) == 0;
-      if (lane == 0) mbar_arrive_expect_tx(&bars[s], (uint32_t)(full ? L.tx_full : L.tx_part));
-      __syncwarp();
-      const uint32_t bar = smem_u32(&bars[s]);
-      const size_t row = row0 + t;
-      if (my_map) {
-        fence_proxy_async_smem();
-        tensor_copy(my_dst + s * my_sst, my_map, bar, (int32_t)row);
-      } else if (full && my_bpr > 0) {
-        fence_proxy_async_smem();
-        bulk_copy(my_dst + s * my_sst, my_src + row * my_bpr, (uint32_t)(kDTile * my_bpr), bar);
-      }
-      if (!full) {
-        const int esz = (int)sizeof(T), lsz = sizeof(T) == 4 ? 4 : 2;
-#pragma unroll
-        for (int xx = 0; xx < 2; ++xx) {
-          const CacheView& cv = xx ? a.V : a.K;
-          uint8_t* rest = wb + L.rest0 + (2 * s + xx) * L.rb;
-          const uint8_t* oi = cv.oidx + row * k;
-          for (int e = lane; e < nt * k; e += 32) rest[e] = oi[e];
-          const uint8_t* ov = reinterpret_cast<const uint8_t*>(cv.oval) + row * k * esz;
-          for (int e = lane; e < nt * k * esz; e += 32) rest[L.oval + e] = ov[e];
-          const uint8_t* lf = reinterpret_cast<const uint8_t*>(cv.lfac) + row * rm * lsz;
-          for (int e = lane; e < nt * rm * lsz; e += 32) rest[L.lf + e] = lf[e];
-          if (!meta_tma) {
-            uint8_t* md = wb + L.meta0 + (2 * s + xx) * L.mb;
-            const uint8_t* ms = reinterpret_cast<const uint8_t*>(cv.meta) + row * G * 8;
-            for (int e = lane; e < nt * G * 8; e += 32) md[e] = ms[e];
-          }
-        }
-      }
-    };
-
-    const int c0 = sp * a.chunk;
-    const int c1 = min(a.n_comp, c0 + a.chunk);
-    // blocks: block 0 = [0, blk0_len), then n_b tokens each; tracked incrementally
-    int blk = block_of(a, c0);
-    int bend = block_end(a, blk);
-    const float* rfk = nullptr;
-    const float* rfv = nullptr;
-    int rb = 0;
-    auto next_end = [&](int t, int be) { return min(min(t + kDTile, c1), be); };
-    issue(0, c0, next_end(c0, bend) - c0);
-
-    // lane-constant swizzle terms: key rows (lane = token), meta rows, and the
-    // value reads of token 2*i + par (period 4 in i)
-    const int xs = swz<R>(lane);
-    const int mx = G == 4 ? ((lane >> 2) & 1) << 4 : 0;
-    int voff[4];
-    {
-      const int ob = BITS == 4 ? 4 * lq : (BITS == 2 ? 2 * lq : 8 * lq);
-#pragma unroll
-      for (int mm = 0; mm < 4; ++mm) voff[mm] = ob ^ (swz<R>(2 * mm + par) << 4);
+      for (int e = 0; e < 4; ++e) { acc[hh][e] = 0; sw[hh][e] = 0.0f; spm[hh][e] = 0.0f; alr[hh][e] = 0.0f; }
     }
 
-    // finishes the value low-rank part of the current block: accx += alr Rf_v^T
-    auto finish_block = [&]() {
-#pragma unroll
-      for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-        for (int j = 0; j < kRReg; ++j) alr[hh][j] = warp_sum(alr[hh][j]);
-      __syncwarp();
-#pragma unroll
-      for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = e * 32 + lane;
-          float v = accx_s[hh * 128 + c];
-          const float4 r0 = __ldg(reinterpret_cast<const float4*>(rfv + c * rp));
-          v = fmaf(alr[hh][0], r0.x, v);
-          v = fmaf(alr[hh][1], r0.y, v);
-          v = fmaf(alr[hh][2], r0.z, v);
-          v = fmaf(alr[hh][3], r0.w, v);
-          for (int j4 = kRReg; j4 < rb; j4 += 4) {
-            const float4 r4 = __ldg(reinterpret_cast<const float4*>(rfv + c * rp + j4));
-            v = fmaf(alr_s[hh * kMaxR + j4], r4.x, v);
-            v = fmaf(alr_s[hh * kMaxR + j4 + 1], r4.y, v);
-            v = fmaf(alr_s[hh * kMaxR + j4 + 2], r4.z, v);
-            v = fmaf(alr_s[hh * kMaxR + j4 + 3], r4.w, v);
-          }
-          accx_s[hh * 128 + c] = v;
-        }
-#pragma unroll
-      for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-        for (int j = 0; j < kRReg; ++j) alr[hh][j] = 0.0f;
-      __syncwarp();
-      for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
-    };
+    int rb = 0;   // rank of the current block
 
-    int t0 = c0, it = 0, cur_blk = -1;
-    while (t0 < c1) {
-      if (t0 >= bend) { ++blk; bend = block_end(a, blk); }
-      const int t1 = next_end(t0, bend);
-      const int nt = t1 - t0;
-      const int s = it & 1;
-      if (t1 < c1) {   // prefetch the next tile into the other stage
-        const int be2 = t1 >= bend ? block_end(a, blk + 1) : bend;
-        issue(s ^ 1, t1, next_end(t1, be2) - t1);
-      }
-      const bool landed = mbar_wait(&bars[s], (uint32_t)(it >> 1) & 1u);
-      if (!__all_sync(0xFFFFFFFFu, landed)) {
-        // give up on this split; let the other stage's copies land first
-        if (t1 < c1) mbar_wait(&bars[s ^ 1], (uint32_t)((it + 1) >> 1) & 1u);
-        return;
-      }
-      __syncwarp();
-      const uint8_t* tkc = cb + (2 * s) * L.cb;
-      const uint8_t* tvc = tkc + L.cb;
-      const uint8_t* tkm = wb + L.meta0 + (2 * s) * L.mb;
-      const uint8_t* tvm = tkm + L.mb;
-      const uint8_t* tkr = wb + L.rest0 + (2 * s) * L.rb;
-      const uint8_t* tvr = tkr + L.rb;
-
-      if (blk != cur_blk) {
-        // finish the previous block's value low-rank part, then switch Rf
-        if (cur_blk >= 0) finish_block();
-        cur_blk = blk;
-        rb = blk == 0 ? a.blk0_rank : a.buffer_rank;
-        const size_t rf0 = ((size_t)unit * a.nblk_max + blk) * 128 * rp;
-        rfk = a.K.rfac + rf0;
-        rfv = a.V.rfac + rf0;
-        // u = Rf_k^T q for every query head
+    // Moves the softmax reference of head hh to mt if mt passes it by more than
+    // 2^kLazy, rescaling every accumulator (registers, shared memory and the
+    // value outlier sums in global memory).
+    auto move_ref = [&](const int hh, const float mt) {
+      if (mt > m[hh] + kLazy) {   // warp-uniform
+        if (m[hh] != -INFINITY) {
+          const float al = exp2f(m[hh] - mt);
+          lsum[hh] *= al;
+          const uint64_t al2 = pk2(al, al);
 #pragma unroll
-        for (int hh = 0; hh < HQ; ++hh)
-          for (int j4 = 0; j4 < rb; j4 += 4) {
-            float u4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = e * 32 + lane;
-              const float4 r4 = __ldg(reinterpret_cast<const float4*>(rfk + c * rp + j4));
-              const float qv = qw_s[hh * 128 + c] * CF::weight(c);
-              u4[0] = fmaf(r4.x, qv, u4[0]);
-              u4[1] = fmaf(r4.y, qv, u4[1]);
-              u4[2] = fmaf(r4.z, qv, u4[2]);
-              u4[3] = fmaf(r4.w, qv, u4[3]);
-            }
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const float v = warp_sum(u4[jj]);
-              if (lane == 0) u_s[hh * kMaxR + j4 + jj] = v;
-            }
+          for (int e = 0; e < 4; ++e) {
+            acc[hh][e] = fma2(acc[hh][e], al2, 0);
+            sw[hh][e] *= al;
+            spm[hh][e] *= al;
+            alr[hh][e] *= al;
+            accx_s[hh * 128 + e * 32 + lane] *= al;
           }
-        __syncwarp();
-      }
-
-      // ---------------- scores: lane = token
-      const int t = lane;
-      const bool live = t < nt;
-      const uint8_t* kmrow = tkm + t * G * 8;
-      const uint8_t* vmrow = tvm + t * G * 8;
-      float s_[HQ];
-      {
-        const uint8_t* crow = tkc + t * R;
-        uint64_t sb[HQ][4][2];   // per 32-channel block, two independent chains
-#pragma unroll
-        for (int hh = 0; hh < HQ; ++hh)
-#pragma unroll
-          for (int bk = 0; bk < 4; ++bk) { sb[hh][bk][0] = 0; sb[hh][bk][1] = 0; }
-#pragma unroll
-        for (int j = 0; j < W / 4; ++j) {
-          const uint4 wv = *reinterpret_cast<const uint4*>(crow + ((j ^ xs) << 4));
-          const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            const int cbase = (4 * j + wi) * CF::kPerWord;
-            const int bk = cbase >> 5;
-            float f[CF::kPerWord];
-            CF::word(wd[wi], f, one);
-#pragma unroll
-            for (int e = 0; e < CF::kPerWord; e += 4) {
-              const int ch = ((cbase + e) >> 2) & 1;
-#pragma unroll
-              for (int hh = 0; hh < HQ; ++hh) {
-                const float4 qv = *reinterpret_cast<const float4*>(qw_s + hh * 128 + cbase + e);
-                sb[hh][bk][ch] = fma2(pk2(f[e], f[e + 1]), pk2(qv.x, qv.y), sb[hh][bk][ch]);
-                sb[hh][bk][ch] = fma2(pk2(f[e + 2], f[e + 3]), pk2(qv.z, qv.w), sb[hh][bk][ch]);
-              }
-            }
-          }
-        }
-        float2 sz[4];
-        meta_row(kmrow, G, mx, sz);
-        const int bpg = a.g >> 5;   // 32-channel blocks per group
-#pragma unroll
-        for (int hh = 0; hh < HQ; ++hh) {
-          float v = 0.0f;
-#pragma unroll
-          for (int gi = 0; gi < 4; ++gi) {
-            if (gi >= G) break;
-            float f = 0.0f, qsw = 0.0f, qss = 0.0f;
-#pragma unroll
-            for (int bk = 0; bk < 4; ++bk)
-              if ((bk / bpg) == gi) {
-                f += (lo2(sb[hh][bk][0]) + hi2(sb[hh][bk][0])) + (lo2(sb[hh][bk][1]) + hi2(sb[hh][bk][1]));
-                qsw += qw_blk[hh][bk];
-                qss += qs_blk[hh][bk];
-              }
-            v = fmaf(sz[gi].x, f - qsw, v);
-            v = fmaf(sz[gi].y, qss, v);
-          }
-          s_[hh] = v;
-        }
-        if (live) {
-          // low-rank part and outlier fix-ups
-          float lt[kRReg];
-#pragma unroll
-          for (int j = 0; j < kRReg; ++j) lt[j] = j < rb ? l_at<T>(tkr + L.lf, t, j, rm) : 0.0f;
-#pragma unroll
-          for (int j = 0; j < kRReg; ++j)
-#pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(lt[j], j < rb ? u_s[hh * kMaxR + j] : 0.0f, s_[hh]);
-          for (int j = kRReg; j < rb; ++j) {
-            const float lj = l_at<T>(tkr + L.lf, t, j, rm);
-#pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(lj, u_s[hh * kMaxR + j], s_[hh]);
-          }
-          if constexpr (!OUT) {
-          } else if (k <= kFast && rb <= kRReg) {
-            int cix[kFast];
-            float fx[kFast];
-            outlier_fixes<T>(tkr, L.oval, kmrow, mx, t, k, lg, lt, rfk, rp, cix, fx);
-#pragma unroll
-            for (int i = 0; i < kFast; ++i)
-#pragma unroll
-              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + cix[i]] * CF::weight(cix[i]), fx[i], s_[hh]);
-          } else {
-            for (int i = 0; i < k; ++i) {
-              const int c = tkr[t * k + i];
-              const float lr = lowrank_at<T>(tkr + L.lf, t, rm, rb, rfk, rp, c);
-              const float xo = (float)reinterpret_cast<const T*>(tkr + L.oval)[t * k + i];
-              const float fix = xo - (meta_at(kmrow, c >> lg, mx).y + lr);
-#pragma unroll
-              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + c] * CF::weight(c), fix, s_[hh]);
-            }
-          }
-        }
-#pragma unroll
-        for (int hh = 0; hh < HQ; ++hh) s_[hh] = live ? s_[hh] * a.scale_log2 : -INFINITY;
-      }
-
-      // ---------------- online softmax; the reference m moves only when the
-      // tile's maximum passes it by more than 2^kLazy
-      float p[HQ];
-#pragma unroll
-      for (int hh = 0; hh < HQ; ++hh) {
-        const float mt = warp_max(s_[hh]);
-        if (mt > m[hh] + kLazy) {   // warp-uniform
-          if (m[hh] != -INFINITY) {
-            const float al = exp2f(m[hh] - mt);
-            lsum[hh] *= al;
-            const uint64_t al2 = pk2(al, al);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              acc[hh][e] = fma2(acc[hh][e], al2, 0);
-              sw[hh][e] *= al;
-              spm[hh][e] *= al;
-              alr[hh][e] *= al;
-              accx_s[hh * 128 + e * 32 + lane] *= al;
-            }
-            if (rb > kRReg && lane < kMaxR) alr_s[hh * kMaxR + lane] *= al;
-            if constexpr (OUT) {   // the value outlier sums in global memory
+          if (rb > kRReg && lane < kMaxR) alr_s[hh * kMaxR + lane] *= al;
+          if constexpr (OUT) {
+            if (comp) {
               __threadfence();
               __syncwarp();
 #pragma unroll
@@ -614,182 +309,526 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
               __syncwarp();
             }
           }
-          m[hh] = mt;
         }
-        p[hh] = live ? exp2f(s_[hh] - m[hh]) : 0.0f;
-        lsum[hh] += p[hh];
+        m[hh] = mt;
       }
-      // value-side per-token weights w = p * scale; zero-point and low-rank sums
-      {
-        float2 vsz[4];
-        meta_row(vmrow, G, mx, vsz);
+    };
+
+    if (comp) {
+      __threadfence();   // the zeroed outlier sums before any reduction
+      __syncwarp();
+
+      // group sums of q and of the weighted q, per 32-channel block
+      float qs_blk[HQ][4], qw_blk[HQ][4];
 #pragma unroll
-        for (int gi = 0; gi < 4; ++gi) {
-          if (gi >= G) break;
-          const float2 sz = live ? vsz[gi] : make_float2(0.0f, 0.0f);
+      for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+        for (int bk = 0; bk < 4; ++bk) {
+          qs_blk[hh][bk] = warp_sum(qw_s[hh * 128 + bk * 32 + lane] * CF::weight(bk * 32 + lane));
+          qw_blk[hh][bk] = warp_sum(qw_s[hh * 128 + bk * 32 + lane]);
+        }
+
+      // ---- copy roles: lanes 0/1 codes (K/V), 2/3 meta by tensor copy (G >= 2),
+      // 4/5 oidx, 6/7 oval, 8/9 L rows, 10/11 meta by bulk copy (G = 1)
+      const bool meta_tma = G >= 2;
+      const int x = lane & 1;
+      const CUtensorMap* my_map = nullptr;
+      const uint8_t* my_src = nullptr;
+      int my_bpr = 0;
+      uint32_t my_dst = 0, my_sst = 0;
+      {
+        const int esz = (int)sizeof(T), lsz = sizeof(T) == 4 ? 4 : 2;
+        const uint32_t wbs = smem_u32(wb);
+        switch (lane >> 1) {
+          case 0:
+            my_map = x ? &maps.vc : &maps.kc;
+            my_dst = smem_u32(cb) + x * L.cb;
+            my_sst = 2 * L.cb;
+            break;
+          case 1:
+            if (meta_tma) {
+              my_map = x ? &maps.vm : &maps.km;
+              my_dst = wbs + L.meta0 + x * L.mb;
+              my_sst = 2 * L.mb;
+            }
+            break;
+          case 2:
+            my_src = x ? a.V.oidx : a.K.oidx;
+            my_bpr = k;
+            my_dst = wbs + L.rest0 + x * L.rb;
+            my_sst = 2 * L.rb;
+            break;
+          case 3:
+            my_src = reinterpret_cast<const uint8_t*>(x ? a.V.oval : a.K.oval);
+            my_bpr = k * esz;
+            my_dst = wbs + L.rest0 + x * L.rb + L.oval;
+            my_sst = 2 * L.rb;
+            break;
+          case 4:
+            my_src = reinterpret_cast<const uint8_t*>(x ? a.V.lfac : a.K.lfac);
+            my_bpr = rm * lsz;
+            my_dst = wbs + L.rest0 + x * L.rb + L.lf;
+            my_sst = 2 * L.rb;
+            break;
+          case 5:
+            if (!meta_tma) {
+              my_src = reinterpret_cast<const uint8_t*>(x ? a.V.meta : a.K.meta);
+              my_bpr = G * 8;
+              my_dst = wbs + L.meta0 + x * L.mb;
+              my_sst = 2 * L.mb;
+            }
+            break;
+          default:
+            break;
+        }
+      }
+      const size_t row0 = (size_t)unit * a.n_max;   // row of the unit's token 0
+      // Brings tokens [t, t + nt) of the unit into stage s. A whole, 32-aligned
+      // tile is all copies; another one (a block boundary or the split's end)
+      // takes codes and meta by tensor copy (rows past nt are read and ignored)
+      // and the rest by plain loads of the lanes.
+      auto issue = [&](int s, int t, int nt) {
+        const bool full = nt == kDTile && (t & (kDTile - 1)) == 0;
+        if (lane == 0) mbar_arrive_expect_tx(&bars[s], (uint32_t)(full ? L.tx_full : L.tx_part));
+        __syncwarp();
+        const uint32_t bar = smem_u32(&bars[s]);
+        const size_t row = row0 + t;
+        if (my_map) {
+          fence_proxy_async_smem();
+          tensor_copy(my_dst + s * my_sst, my_map, bar, (int32_t)row);
+        } else if (full && my_bpr > 0) {
+          fence_proxy_async_smem();
+          bulk_copy(my_dst + s * my_sst, my_src + row * my_bpr, (uint32_t)(kDTile * my_bpr), bar);
+        }
+        if (!full) {
+          const int esz = (int)sizeof(T), lsz = sizeof(T) == 4 ? 4 : 2;
+#pragma unroll
+          for (int xx = 0; xx < 2; ++xx) {
+            const CacheView& cv = xx ? a.V : a.K;
+            uint8_t* rest = wb + L.rest0 + (2 * s + xx) * L.rb;
+            const uint8_t* oi = cv.oidx + row * k;
+            for (int e = lane; e < nt * k; e += 32) rest[e] = oi[e];
+            const uint8_t* ov = reinterpret_cast<const uint8_t*>(cv.oval) + row * k * esz;
+            for (int e = lane; e < nt * k * esz; e += 32) rest[L.oval + e] = ov[e];
+            const uint8_t* lf = reinterpret_cast<const uint8_t*>(cv.lfac) + row * rm * lsz;
+            for (int e = lane; e < nt * rm * lsz; e += 32) rest[L.lf + e] = lf[e];
+            if (!meta_tma) {
+              uint8_t* md = wb + L.meta0 + (2 * s + xx) * L.mb;
+              const uint8_t* ms = reinterpret_cast<const uint8_t*>(cv.meta) + row * G * 8;
+              for (int e = lane; e < nt * G * 8; e += 32) md[e] = ms[e];
+            }
+          }
+        }
+      };
+
+      // blocks: block 0 = [0, blk0_len), then n_b tokens each; tracked incrementally
+      int blk = block_of(a, c0);
+      int bend = block_end(a, blk);
+      const float* rfk = nullptr;
+      const float* rfv = nullptr;
+      // tiles follow the unit's 32-token grid: [t, next multiple of 32), clipped
+      auto next_end = [&](int t, int be) { return min(min((t & ~(kDTile - 1)) + kDTile, c1), be); };
+      issue(it & 1, c0, next_end(c0, bend) - c0);
+
+      // lane-constant swizzle terms: key rows (lane = token), meta rows, and the
+      // value reads of token 2*i + par (period 4 in i)
+      const int xs = swz<R>(lane);
+      const int mx = G == 4 ? ((lane >> 2) & 1) << 4 : 0;
+      int voff[4];
+      {
+        const int ob = BITS == 4 ? 4 * lq : (BITS == 2 ? 2 * lq : 8 * lq);
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) voff[mm] = ob ^ (swz<R>(2 * mm + par) << 4);
+      }
+
+      // finishes the value low-rank part of the current block: accx += alr Rf_v^T
+      auto finish_block = [&]() {
+#pragma unroll
+        for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+          for (int j = 0; j < kRReg; ++j) alr[hh][j] = warp_sum(alr[hh][j]);
+        __syncwarp();
+#pragma unroll
+        for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = e * 32 + lane;
+            float v = accx_s[hh * 128 + c];
+            const float4 r0 = __ldg(reinterpret_cast<const float4*>(rfv + c * rp));
+            v = fmaf(alr[hh][0], r0.x, v);
+            v = fmaf(alr[hh][1], r0.y, v);
+            v = fmaf(alr[hh][2], r0.z, v);
+            v = fmaf(alr[hh][3], r0.w, v);
+            for (int j4 = kRReg; j4 < rb; j4 += 4) {
+              const float4 r4 = __ldg(reinterpret_cast<const float4*>(rfv + c * rp + j4));
+              v = fmaf(alr_s[hh * kMaxR + j4], r4.x, v);
+              v = fmaf(alr_s[hh * kMaxR + j4 + 1], r4.y, v);
+              v = fmaf(alr_s[hh * kMaxR + j4 + 2], r4.z, v);
+              v = fmaf(alr_s[hh * kMaxR + j4 + 3], r4.w, v);
+            }
+            accx_s[hh * 128 + c] = v;
+          }
+#pragma unroll
+        for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+          for (int j = 0; j < kRReg; ++j) alr[hh][j] = 0.0f;
+        __syncwarp();
+        for (int e = lane; e < HQ * kMaxR; e += 32) alr_s[e] = 0.0f;
+      };
+
+      int t0 = c0, cur_blk = -1;
+      while (t0 < c1) {
+        if (t0 >= bend) { ++blk; bend = block_end(a, blk); }
+        const int t1 = next_end(t0, bend);
+        const int nt = t1 - t0;
+        const int s = it & 1;
+        if (t1 < c1) {   // prefetch the next tile into the other stage
+          const int be2 = t1 >= bend ? block_end(a, blk + 1) : bend;
+          issue(s ^ 1, t1, next_end(t1, be2) - t1);
+        }
+        const bool landed = mbar_wait(&bars[s], (uint32_t)(it >> 1) & 1u);
+        if (!__all_sync(0xFFFFFFFFu, landed)) {
+          // give up on this split; let the other stage's copies land first
+          if (t1 < c1) mbar_wait(&bars[s ^ 1], (uint32_t)((it + 1) >> 1) & 1u);
+          return false;
+        }
+        __syncwarp();
+        const uint8_t* tkc = cb + (2 * s) * L.cb;
+        const uint8_t* tvc = tkc + L.cb;
+        const uint8_t* tkm = wb + L.meta0 + (2 * s) * L.mb;
+        const uint8_t* tvm = tkm + L.mb;
+        const uint8_t* tkr = wb + L.rest0 + (2 * s) * L.rb;
+        const uint8_t* tvr = tkr + L.rb;
+
+        if (blk != cur_blk) {
+          // finish the previous block's value low-rank part, then switch Rf
+          if (cur_blk >= 0) finish_block();
+          cur_blk = blk;
+          rb = blk == 0 ? a.blk0_rank : a.buffer_rank;
+          const size_t rf0 = ((size_t)unit * a.nblk_max + blk) * 128 * rp;
+          rfk = a.K.rfac + rf0;
+          rfv = a.V.rfac + rf0;
+          // u = Rf_k^T q for every query head
+#pragma unroll
+          for (int hh = 0; hh < HQ; ++hh)
+            for (int j4 = 0; j4 < rb; j4 += 4) {
+              float u4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = e * 32 + lane;
+                const float4 r4 = __ldg(reinterpret_cast<const float4*>(rfk + c * rp + j4));
+                const float qv = qw_s[hh * 128 + c] * CF::weight(c);
+                u4[0] = fmaf(r4.x, qv, u4[0]);
+                u4[1] = fmaf(r4.y, qv, u4[1]);
+                u4[2] = fmaf(r4.z, qv, u4[2]);
+                u4[3] = fmaf(r4.w, qv, u4[3]);
+              }
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                const float v = warp_sum(u4[jj]);
+                if (lane == 0) u_s[hh * kMaxR + j4 + jj] = v;
+              }
+            }
+          __syncwarp();
+        }
+
+        // ---------------- scores: lane = token
+        const int t = lane;
+        const bool live = t < nt;
+        const uint8_t* kmrow = tkm + t * G * 8;
+        const uint8_t* vmrow = tvm + t * G * 8;
+        float s_[HQ];
+        {
+          const uint8_t* crow = tkc + t * R;
+          uint64_t sb[HQ][4][2];   // per 32-channel block, two independent chains
+#pragma unroll
+          for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+            for (int bk = 0; bk < 4; ++bk) { sb[hh][bk][0] = 0; sb[hh][bk][1] = 0; }
+#pragma unroll
+          for (int j = 0; j < W / 4; ++j) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(crow + ((j ^ xs) << 4));
+            const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {
+              const int cbase = (4 * j + wi) * CF::kPerWord;
+              const int bk = cbase >> 5;
+              float f[CF::kPerWord];
+              CF::word(wd[wi], f, one);
+#pragma unroll
+              for (int e = 0; e < CF::kPerWord; e += 4) {
+                const int ch = ((cbase + e) >> 2) & 1;
+#pragma unroll
+                for (int hh = 0; hh < HQ; ++hh) {
+                  const float4 qv = *reinterpret_cast<const float4*>(qw_s + hh * 128 + cbase + e);
+                  sb[hh][bk][ch] = fma2(pk2(f[e], f[e + 1]), pk2(qv.x, qv.y), sb[hh][bk][ch]);
+                  sb[hh][bk][ch] = fma2(pk2(f[e + 2], f[e + 3]), pk2(qv.z, qv.w), sb[hh][bk][ch]);
+                }
+              }
+            }
+          }
+          float2 sz[4];
+          meta_row(kmrow, G, mx, sz);
+          const int bpg = a.g >> 5;   // 32-channel blocks per group
 #pragma unroll
           for (int hh = 0; hh < HQ; ++hh) {
-            const float wv = p[hh] * sz.x;
-            w_s[(t * G + gi) * HQ + hh] = wv;
-            sw[hh][gi] += wv;
-            spm[hh][gi] = fmaf(p[hh], sz.y, spm[hh][gi]);
+            float v = 0.0f;
+#pragma unroll
+            for (int gi = 0; gi < 4; ++gi) {
+              if (gi >= G) break;
+              float f = 0.0f, qsw = 0.0f, qss = 0.0f;
+#pragma unroll
+              for (int bk = 0; bk < 4; ++bk)
+                if ((bk / bpg) == gi) {
+                  f += (lo2(sb[hh][bk][0]) + hi2(sb[hh][bk][0])) + (lo2(sb[hh][bk][1]) + hi2(sb[hh][bk][1]));
+                  qsw += qw_blk[hh][bk];
+                  qss += qs_blk[hh][bk];
+                }
+              v = fmaf(sz[gi].x, f - qsw, v);
+              v = fmaf(sz[gi].y, qss, v);
+            }
+            s_[hh] = v;
           }
-        }
-        if (live) {
-          float lv[kRReg];
+          if (live) {
+            // low-rank part and outlier fix-ups
+            float lt[kRReg];
 #pragma unroll
-          for (int j = 0; j < kRReg; ++j) lv[j] = j < rb ? l_at<T>(tvr + L.lf, t, j, rm) : 0.0f;
+            for (int j = 0; j < kRReg; ++j) lt[j] = j < rb ? l_at<T>(tkr + L.lf, t, j, rm) : 0.0f;
 #pragma unroll
-          for (int j = 0; j < kRReg; ++j)
+            for (int j = 0; j < kRReg; ++j)
 #pragma unroll
-            for (int hh = 0; hh < HQ; ++hh) alr[hh][j] = fmaf(p[hh], lv[j], alr[hh][j]);
-          // value outliers: p * fix lands on channel c of the split's row
-          if constexpr (!OUT) {
-          } else if (k <= kFast && rb <= kRReg) {
-            int cix[kFast];
-            float fx[kFast];
-            outlier_fixes<T>(tvr, L.oval, vmrow, mx, t, k, lg, lv, rfv, rp, cix, fx);
+              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(lt[j], j < rb ? u_s[hh * kMaxR + j] : 0.0f, s_[hh]);
+            for (int j = kRReg; j < rb; ++j) {
+              const float lj = l_at<T>(tkr + L.lf, t, j, rm);
 #pragma unroll
-            for (int i = 0; i < kFast; ++i)
-              if (i < k)
+              for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(lj, u_s[hh * kMaxR + j], s_[hh]);
+            }
+            if constexpr (!OUT) {
+            } else if (k <= kFast && rb <= kRReg) {
+              int cix[kFast];
+              float fx[kFast];
+              outlier_fixes<T>(tkr, L.oval, kmrow, mx, t, k, lg, lt, rfk, rp, cix, fx);
 #pragma unroll
-                for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + cix[i], p[hh] * fx[i]);
-          } else {
-            for (int i = 0; i < k; ++i) {
-              const int c = tvr[t * k + i];
-              const float lr = lowrank_at<T>(tvr + L.lf, t, rm, rb, rfv, rp, c);
-              const float xo = (float)reinterpret_cast<const T*>(tvr + L.oval)[t * k + i];
-              const float fix = xo - (meta_at(vmrow, c >> lg, mx).y + lr);
+              for (int i = 0; i < kFast; ++i)
 #pragma unroll
-              for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + c, p[hh] * fix);
+                for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + cix[i]] * CF::weight(cix[i]), fx[i], s_[hh]);
+            } else {
+              for (int i = 0; i < k; ++i) {
+                const int c = tkr[t * k + i];
+                const float lr = lowrank_at<T>(tkr + L.lf, t, rm, rb, rfk, rp, c);
+                const float xo = (float)reinterpret_cast<const T*>(tkr + L.oval)[t * k + i];
+                const float fix = xo - (meta_at(kmrow, c >> lg, mx).y + lr);
+#pragma unroll
+                for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + c] * CF::weight(c), fix, s_[hh]);
+              }
             }
           }
+#pragma unroll
+          for (int hh = 0; hh < HQ; ++hh) s_[hh] = live ? s_[hh] * a.scale_log2 : -INFINITY;
         }
-      }
-      for (int j = kRReg; j < rb; ++j)   // ranks beyond the register slots
+
+        // ---------------- online softmax; the reference m moves only when the
+        // tile's maximum passes it by more than 2^kLazy
+        float p[HQ];
 #pragma unroll
         for (int hh = 0; hh < HQ; ++hh) {
-          const float v = warp_sum(live ? p[hh] * l_at<T>(tvr + L.lf, t, j, rm) : 0.0f);
-          if (lane == 0) alr_s[hh * kMaxR + j] += v;
+          move_ref(hh, warp_max(s_[hh]));
+          p[hh] = live ? exp2f(s_[hh] - m[hh]) : 0.0f;
+          lsum[hh] += p[hh];
         }
-      __syncwarp();
-
-      // ---------------- values: lane = 8 channels, tokens 2*i + par. Tokens
-      // past nt have w = 0 (their codes are finite), so every tile runs all 16.
-      {
-        const uint8_t* vrow = tvc + par * R;
-        const float* wrow = w_s + (par * G + my_g) * HQ;
-#pragma unroll 1
-        for (int i4 = 0; i4 < kDTile / 2; i4 += 4) {
+        // value-side per-token weights w = p * scale; zero-point and low-rank sums
+        {
+          float2 vsz[4];
+          meta_row(vmrow, G, mx, vsz);
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
-            const uint8_t* row = vrow + (i4 + mm) * 2 * R + voff[mm];
-            const float* wr = wrow + (i4 + mm) * 2 * G * HQ;
-            float f[8];
-            if constexpr (BITS == 4) {
-              CF::word(*reinterpret_cast<const uint32_t*>(row), f, one);
-            } else if constexpr (BITS == 2) {
-              float ff[16];
-              CF::word(*reinterpret_cast<const uint16_t*>(row), ff, one);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = ff[e];
-            } else {
-              const uint2 ww = *reinterpret_cast<const uint2*>(row);
-              float fa[4], fb[4];
-              CF::word(ww.x, fa, one);
-              CF::word(ww.y, fb, one);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) { f[e] = fa[e]; f[4 + e] = fb[e]; }
-            }
+          for (int gi = 0; gi < 4; ++gi) {
+            if (gi >= G) break;
+            const float2 sz = live ? vsz[gi] : make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int hh = 0; hh < HQ; ++hh) {
-              const float wv = wr[hh];
-              const uint64_t w2 = pk2(wv, wv);
+              const float wv = p[hh] * sz.x;
+              w_s[(t * G + gi) * HQ + hh] = wv;
+              sw[hh][gi] += wv;
+              spm[hh][gi] = fmaf(p[hh], sz.y, spm[hh][gi]);
+            }
+          }
+          if (live) {
+            float lv[kRReg];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) acc[hh][e] = fma2(w2, pk2(f[2 * e], f[2 * e + 1]), acc[hh][e]);
+            for (int j = 0; j < kRReg; ++j) lv[j] = j < rb ? l_at<T>(tvr + L.lf, t, j, rm) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < kRReg; ++j)
+#pragma unroll
+              for (int hh = 0; hh < HQ; ++hh) alr[hh][j] = fmaf(p[hh], lv[j], alr[hh][j]);
+            // value outliers: p * fix lands on channel c of the split's row
+            if constexpr (!OUT) {
+            } else if (k <= kFast && rb <= kRReg) {
+              int cix[kFast];
+              float fx[kFast];
+              outlier_fixes<T>(tvr, L.oval, vmrow, mx, t, k, lg, lv, rfv, rp, cix, fx);
+#pragma unroll
+              for (int i = 0; i < kFast; ++i)
+                if (i < k)
+#pragma unroll
+                  for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + cix[i], p[hh] * fx[i]);
+            } else {
+              for (int i = 0; i < k; ++i) {
+                const int c = tvr[t * k + i];
+                const float lr = lowrank_at<T>(tvr + L.lf, t, rm, rb, rfv, rp, c);
+                const float xo = (float)reinterpret_cast<const T*>(tvr + L.oval)[t * k + i];
+                const float fix = xo - (meta_at(vmrow, c >> lg, mx).y + lr);
+#pragma unroll
+                for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + c, p[hh] * fix);
+              }
             }
           }
         }
-      }
-      __syncwarp();
-      t0 = t1;
-      ++it;
-    }
-    // last block's value low-rank part
-    if (cur_blk >= 0) finish_block();
-  } else {
-    // ---------------- the streaming buffer: exact tokens, lane = token for keys
-    const size_t brow = (size_t)unit * a.n_b;
-    for (int t0 = 0; t0 < a.n_buf; t0 += kDTile) {
-      const int nt = min(kDTile, a.n_buf - t0);
-      const bool live = lane < nt;
-      float s[HQ];
+        for (int j = kRReg; j < rb; ++j)   // ranks beyond the register slots
 #pragma unroll
-      for (int hh = 0; hh < HQ; ++hh) s[hh] = 0.0f;
-      if (live) {
-        for (int c = 0; c < 128; ++c) {
-          const float x = load_elem<T>(a.K.buf, (brow + t0 + lane) * 128 + c);
+          for (int hh = 0; hh < HQ; ++hh) {
+            const float v = warp_sum(live ? p[hh] * l_at<T>(tvr + L.lf, t, j, rm) : 0.0f);
+            if (lane == 0) alr_s[hh * kMaxR + j] += v;
+          }
+        __syncwarp();
+
+        // ---------------- values: lane = 8 channels, tokens 2*i + par. Tokens
+        // past nt have w = 0 (their codes are finite), so every tile runs all 16.
+        {
+          const uint8_t* vrow = tvc + par * R;
+          const float* wrow = w_s + (par * G + my_g) * HQ;
+#pragma unroll 1
+          for (int i4 = 0; i4 < kDTile / 2; i4 += 4) {
 #pragma unroll
-          for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(x, qw_s[hh * 128 + c] * CF::weight(c), s[hh]);
+            for (int mm = 0; mm < 4; ++mm) {
+              const uint8_t* row = vrow + (i4 + mm) * 2 * R + voff[mm];
+              const float* wr = wrow + (i4 + mm) * 2 * G * HQ;
+              float f[8];
+              if constexpr (BITS == 4) {
+                CF::word(*reinterpret_cast<const uint32_t*>(row), f, one);
+              } else if constexpr (BITS == 2) {
+                float ff[16];
+                CF::word(*reinterpret_cast<const uint16_t*>(row), ff, one);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = ff[e];
+              } else {
+                const uint2 ww = *reinterpret_cast<const uint2*>(row);
+                float fa[4], fb[4];
+                CF::word(ww.x, fa, one);
+                CF::word(ww.y, fb, one);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) { f[e] = fa[e]; f[4 + e] = fb[e]; }
+              }
+#pragma unroll
+              for (int hh = 0; hh < HQ; ++hh) {
+                const float wv = wr[hh];
+                const uint64_t w2 = pk2(wv, wv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[hh][e] = fma2(w2, pk2(f[2 * e], f[2 * e + 1]), acc[hh][e]);
+              }
+            }
+          }
         }
+        __syncwarp();
+        t0 = t1;
+        ++it;
       }
-      float p[HQ];
+      // last block's value low-rank part
+      if (cur_blk >= 0) finish_block();
+    }
+    if (with_buf) {
+      // ---------------- the streaming buffer: exact tokens, lane = token for keys
+      const size_t brow = (size_t)unit * a.n_b;
+      for (int t0 = 0; t0 < a.n_buf; t0 += kDTile) {
+        const int nt = min(kDTile, a.n_buf - t0);
+        const bool live = lane < nt;
+        float s[HQ];
 #pragma unroll
-      for (int hh = 0; hh < HQ; ++hh) {
-        const float sv = live ? s[hh] * a.scale_log2 : -INFINITY;
-        const float mnew = fmaxf(m[hh], warp_max(sv));
-        const float al = exp2f(m[hh] - mnew);
-        m[hh] = mnew;
-        p[hh] = live ? exp2f(sv - mnew) : 0.0f;
-        lsum[hh] = fmaf(lsum[hh], al, p[hh]);
+        for (int hh = 0; hh < HQ; ++hh) s[hh] = 0.0f;
+        if (live) {
+          for (int c = 0; c < 128; ++c) {
+            const float x = load_elem<T>(a.K.buf, (brow + t0 + lane) * 128 + c);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) accx_s[hh * 128 + e * 32 + lane] *= al;
-      }
-      __syncwarp();
-      for (int tt = 0; tt < nt; ++tt) {
-        float xv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) xv[e] = load_elem<T>(a.V.buf, (brow + t0 + tt) * 128 + e * 32 + lane);
+            for (int hh = 0; hh < HQ; ++hh) s[hh] = fmaf(x, qw_s[hh * 128 + c] * CF::weight(c), s[hh]);
+          }
+        }
+        float p[HQ];
 #pragma unroll
         for (int hh = 0; hh < HQ; ++hh) {
-          const float pt = __shfl_sync(0xFFFFFFFFu, p[hh], tt);
+          const float sv = live ? s[hh] * a.scale_log2 : -INFINITY;
+          move_ref(hh, warp_max(sv));
+          p[hh] = live ? exp2f(sv - m[hh]) : 0.0f;
+          lsum[hh] += p[hh];
+        }
+        __syncwarp();
+        for (int tt = 0; tt < nt; ++tt) {
+          float xv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) accx_s[hh * 128 + e * 32 + lane] += pt * xv[e];
+          for (int e = 0; e < 4; ++e) xv[e] = load_elem<T>(a.V.buf, (brow + t0 + tt) * 128 + e * 32 + lane);
+#pragma unroll
+          for (int hh = 0; hh < HQ; ++hh) {
+            const float pt = __shfl_sync(0xFFFFFFFFu, p[hh], tt);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) accx_s[hh * 128 + e * 32 + lane] += pt * xv[e];
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (OUT && comp) __threadfence();   // the value outlier sums, before they are read back
+    __syncwarp();
+
+    // ---------------- partial result of this split
+#pragma unroll
+    for (int hh = 0; hh < HQ; ++hh) {
+      const float l_all = warp_sum(lsum[hh]);
+      float swg = 0.0f, spg = 0.0f;
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) {
+        const float a1 = warp_sum(sw[hh][gi]), a2 = warp_sum(spm[hh][gi]);
+        if (gi == my_g) { swg = a1; spg = a2; }
+      }
+      // the two token parities hold the same channels: add them up
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = lo2(acc[hh][e]) + __shfl_xor_sync(0xFFFFFFFFu, lo2(acc[hh][e]), 16);
+        v[2 * e + 1] = hi2(acc[hh][e]) + __shfl_xor_sync(0xFFFFFFFFu, hi2(acc[hh][e]), 16);
+      }
+      float* dst = part_row + hh * hstride;
+      if (lane == 0) { dst[0] = m[hh]; dst[1] = l_all; }
+      if (par == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = 8 * lq + e;
+          const float corr = (OUT && comp) ? ld_gpu(dst + 2 + c) : 0.0f;
+          dst[2 + c] = CF::inv_weight(c) * (v[e] - swg) + spg + accx_s[hh * 128 + c] + corr;
         }
       }
-      __syncwarp();
     }
-  }
-  if (OUT && comp) __threadfence();   // the value outlier sums, before they are read back
-  __syncwarp();
+    return true;
+  };
 
-  // ---------------- partial result of this split
-#pragma unroll
-  for (int hh = 0; hh < HQ; ++hh) {
-    const float l_all = warp_sum(lsum[hh]);
-    float swg = 0.0f, spg = 0.0f;
-#pragma unroll
-    for (int gi = 0; gi < 4; ++gi) {
-      const float a1 = warp_sum(sw[hh][gi]), a2 = warp_sum(spm[hh][gi]);
-      if (gi == my_g) { swg = a1; spg = a2; }
+  // stream-K: this warp's run [gs * seg_tokens, (gs + 1) * seg_tokens) of the
+  // units' compressed tokens, cut at unit boundaries; the warp that ends a unit
+  // also takes its buffer. Without compressed tokens, warp gs takes unit gs's
+  // buffer.
+  const int64_t n = a.n_comp;
+  int64_t gpos = n > 0 ? (int64_t)gs * a.seg_tokens : 0;
+  const int64_t gend = n > 0 ? min(gpos + (int64_t)a.seg_tokens, (int64_t)a.B * a.H * n) : 1;
+  while (gpos < gend) {
+    int unit, c0, c1, sp;
+    if (n > 0) {
+      unit = (int)(gpos / n);
+      c0 = (int)(gpos - unit * n);
+      c1 = (int)min(n, gend - unit * n);
+      sp = gs - (int)((unit * n) / a.seg_tokens);
+      gpos = unit * n + c1;
+    } else {
+      unit = gs;
+      c0 = c1 = sp = 0;
+      gpos = gend;
     }
-    // the two token parities hold the same channels: add them up
-    float v[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[2 * e] = lo2(acc[hh][e]) + __shfl_xor_sync(0xFFFFFFFFu, lo2(acc[hh][e]), 16);
-      v[2 * e + 1] = hi2(acc[hh][e]) + __shfl_xor_sync(0xFFFFFFFFu, hi2(acc[hh][e]), 16);
-    }
-    float* dst = part_row + hh * hstride;
-    if (lane == 0) { dst[0] = m[hh]; dst[1] = l_all; }
-    if (par == 0) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int c = 8 * lq + e;
-        const float corr = (OUT && comp) ? ld_gpu(dst + 2 + c) : 0.0f;
-        dst[2 + c] = CF::inv_weight(c) * (v[e] - swg) + spg + accx_s[hh * 128 + c] + corr;
-      }
-    }
+    if (!segment(unit, c0, c1, sp, c1 == (int)n && a.n_buf > 0)) return;
   }
 }
 
@@ -798,10 +837,16 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeArgs a) {
   const int bj = blockIdx.x;  // b * Hq + j
   const int c = threadIdx.x;
   const float* p = a.part + (size_t)bj * a.nsplit * 130;
+  // the warps that met this query head's unit wrote partial rows 0 .. nseg-1
+  int nseg = 1;
+  if (a.n_comp > 0) {
+    const int64_t u = (int64_t)(bj / a.Hq) * a.H + (bj % a.Hq) / a.hq, n = a.n_comp;
+    nseg = (int)(((u + 1) * n - 1) / a.seg_tokens - (u * n) / a.seg_tokens + 1);
+  }
   float M = -INFINITY;
-  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, p[s * 130]);
+  for (int s = 0; s < nseg; ++s) M = fmaxf(M, p[s * 130]);
   float den = 0.0f, num = 0.0f;
-  for (int s = 0; s < a.nsplit; ++s) {
+  for (int s = 0; s < nseg; ++s) {
     const float m = p[s * 130];
     if (m == -INFINITY) continue;   // a split without a finite score contributes nothing
     const float w = exp2f(m - M);
@@ -835,21 +880,24 @@ void decode_plan(DecodeArgs& a, int num_sms) {
   const int meta_tx = a.G >= 2 ? 2 * L.mb : 0;
   L.tx_part = 2 * L.cb + meta_tx;
   L.tx_full = L.tx_part + 2 * kDTile * (a.k + a.k * esz + a.r_max * esz) + (a.G >= 2 ? 0 : 2 * L.mb);
-  int nsc = 0;
+  // stream-K over the units' compressed tokens: one wave of resident warps,
+  // each taking an equal run of tokens (a multiple of 32)
+  const int smem_cta = 1024 + 16 * L.cb + 4 * L.bytes;
+  const int by_smem = 233472 / (smem_cta + 1024);   // 228 KiB per SM, 1 KiB reserved per CTA
+  const int by_regs = hq <= 2 ? 4 : (hq == 4 ? 2 : 1);
+  const long long resident = (long long)num_sms * (by_smem < by_regs ? (by_smem > 0 ? by_smem : 1) : by_regs) * 4;
   if (a.n_comp > 0) {
-    // about 48 warps per SM over the whole grid, chunks of whole 32-token tiles
-    const long long target = (long long)num_sms * 48;
-    long long chunk = ((long long)a.n_comp * units + target - 1) / target;
-    chunk = (chunk + kDTile - 1) / kDTile * kDTile;
-    if (chunk < 256) chunk = 256;
-    a.chunk = (int)chunk;
-    nsc = (a.n_comp + a.chunk - 1) / a.chunk;
+    const long long tot = (long long)a.n_comp * units;
+    long long seg = (tot + resident - 1) / resident;
+    seg = (seg + kDTile - 1) / kDTile * kDTile;
+    a.seg_tokens = (int)seg;
+    a.total_splits = (int)((tot + seg - 1) / seg);
+    a.nsplit = (int)((a.n_comp + seg - 1) / seg) + 1;
   } else {
-    a.chunk = kDTile;
+    a.seg_tokens = 0;
+    a.total_splits = units;
+    a.nsplit = 1;
   }
-  a.nsplit_comp = nsc;
-  a.nsplit = nsc + (a.n_buf > 0 ? 1 : 0);
-  a.total_splits = units * a.nsplit;
 }
 
 size_t decode_workspace_bytes(int B, int Hq, int nsplit) { return (size_t)B * Hq * nsplit * 130 * sizeof(float); }
@@ -891,10 +939,10 @@ static cudaError_t launch_bits(const DecodeMaps& maps, const DecodeArgs& a, cuda
 
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t st) {
   cudaError_t e = cudaSuccess;
-  if (a.nsplit_comp > 0 || a.n_buf > 0) {
+  if (a.n_comp > 0 || a.n_buf > 0) {
     DecodeMaps maps;
     memset(&maps, 0, sizeof(maps));
-    if (a.nsplit_comp > 0) {
+    if (a.n_comp > 0) {
       PFN_encodeTiled enc = tensor_map_encoder();
       if (!enc) return cudaErrorNotSupported;
       const uint64_t rows = (uint64_t)a.B * a.H * a.n_max;

@@ -54,11 +54,10 @@ struct DecodeArgs {
   const void* q;          // [B][Hq][128] cache dtype
   void* out;              // [B][Hq][128] out dtype
   int32_t out_dtype;
-  float* part;            // [B][Hq][nsplit][130] partial (m, l, acc[128])
-  int32_t chunk;          // compressed tokens per split (whole 32-token tiles)
-  int32_t nsplit_comp;    // splits over compressed tokens, per unit
-  int32_t nsplit;         // + 1 if the buffer is non-empty
-  int32_t total_splits;   // units * nsplit: one warp each
+  float* part;            // [B][Hq][nsplit][130] partial (m, l, acc[128]) per warp that meets the unit
+  int32_t seg_tokens;     // compressed tokens per warp (a multiple of 32); 0 without any
+  int32_t nsplit;         // partial rows per unit: at most ceil(n_comp / seg_tokens) + 1 warps meet a unit
+  int32_t total_splits;   // warps: ceil(units * n_comp / seg_tokens), or units without compressed tokens
   TileLayout tl;
 };
 
