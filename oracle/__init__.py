@@ -49,12 +49,12 @@ def lib():
         L.oracle_num_outliers.argtypes = [ctypes.c_float, i32]
         L.oracle_num_outliers.restype = i32
         L.oracle_select_outliers.argtypes = [P, i32, i32, P]
-        L.oracle_quantize_token.argtypes = [P, i32, i32, i32, P, i32, P, P, P, P, P]
+        L.oracle_quantize_token.argtypes = [P, i32, i32, i32, P, i32, i32, P, P, P, P, P]
         L.oracle_splitmix64_next.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
         L.oracle_splitmix64_next.restype = ctypes.c_uint64
         L.oracle_start_matrix.argtypes = [ctypes.c_uint64, i32, i32, P]
         L.oracle_power_iteration.argtypes = [P, i32, i32, i32, i32, P, P, P]
-        L.oracle_encode_unit.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, ctypes.c_uint64,
+        L.oracle_encode_unit.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.c_uint64,
                                          P, P, P, P, P, P, P, P]
         L.oracle_reconstruct_unit.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
         L.oracle_attention.argtypes = [P, P, P, i32, i32, ctypes.c_double, P]
@@ -80,6 +80,7 @@ class Params:
     buffer_len: int = 20
     buffer_rank: int = 2
     seed: int = 0
+    meta_f16: bool = False   # scale and zero stored as binary16 (byte-lean metadata)
 
 
 def num_outliers(s: float, d: int) -> int:
@@ -93,7 +94,7 @@ def select_outliers(x: np.ndarray, k: int) -> np.ndarray:
     return idx
 
 
-def quantize_token(x: np.ndarray, bits: int, g: int, oidx: np.ndarray):
+def quantize_token(x: np.ndarray, bits: int, g: int, oidx: np.ndarray, meta_f16: bool = False):
     """One token: returns (codes u32[W], scale f32[G], zero f32[G], dhat f32[d], resid f32[d])."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     d = x.shape[0]
@@ -103,7 +104,7 @@ def quantize_token(x: np.ndarray, bits: int, g: int, oidx: np.ndarray):
     zero = np.zeros(d // g, dtype=np.float32)
     dhat = np.zeros(d, dtype=np.float32)
     resid = np.zeros(d, dtype=np.float32)
-    lib().oracle_quantize_token(_p(x), d, bits, g, _p(oidx), oidx.shape[0], _p(codes), _p(scale),
+    lib().oracle_quantize_token(_p(x), d, bits, g, _p(oidx), oidx.shape[0], int(meta_f16), _p(codes), _p(scale),
                                 _p(zero), _p(dhat), _p(resid))
     return codes, scale, zero, dhat, resid
 
@@ -155,7 +156,7 @@ def encode_unit(X: np.ndarray, p: Params, rank: int | None = None) -> Unit:
              zero=np.zeros((n, G), np.float32), oidx=np.zeros((n, k), np.int32),
              oval=np.zeros((n, k), np.float32), resid=np.zeros((n, d), np.float32),
              L=np.zeros((n, r), np.float64), Rf=np.zeros((d, r), np.float64), rank=r)
-    lib().oracle_encode_unit(_p(X), n, d, p.bits, p.group_size, k, r, p.power_iters,
+    lib().oracle_encode_unit(_p(X), n, d, p.bits, p.group_size, k, int(p.meta_f16), r, p.power_iters,
                              ctypes.c_uint64(p.seed), _p(u.codes), _p(u.scale), _p(u.zero),
                              _p(u.oidx), _p(u.oval), _p(u.resid), _p(u.L), _p(u.Rf))
     return u

@@ -76,7 +76,7 @@ void oracle_select_outliers(const float* x, int32_t d, int32_t k, int32_t* idx_o
 /* Step 3: residual r = x - dhat at non-outlier slots, 0 at outlier slots.    */
 /* ------------------------------------------------------------------------ */
 void oracle_quantize_token(const float* x, int32_t d, int32_t bits, int32_t g,
-                           const int32_t* oidx, int32_t k,
+                           const int32_t* oidx, int32_t k, int32_t meta_f16,
                            uint32_t* codes, float* scale_out, float* zero_out,
                            float* dhat_out, float* resid_out) {
   const int32_t levels = (1 << bits) - 1;
@@ -101,6 +101,13 @@ void oracle_quantize_token(const float* x, int32_t d, int32_t bits, int32_t g,
     mn = mn + 0.0f;
     mx = mx + 0.0f;
     float scale = (mx - mn) / (float)levels;
+    if (meta_f16) {
+      /* Reading (byte-lean metadata): scale and zero point are stored as
+         binary16, rounded to nearest even from the binary32 values, and the
+         codes below are decided against the stored values. */
+      scale = (float)(_Float16)scale;
+      mn = (float)(_Float16)mn + 0.0f;
+    }
     scale_out[grp] = scale;
     zero_out[grp] = mn;
     for (int32_t c = c0; c < c0 + g; ++c) {
@@ -211,7 +218,7 @@ void oracle_power_iteration(const float* R, int32_t n, int32_t d, int32_t r, int
 /*   oval [n][k], resid [n][d], L [n][r], Rf [d][r].                          */
 /* ------------------------------------------------------------------------ */
 void oracle_encode_unit(const float* X, int32_t n, int32_t d, int32_t bits, int32_t g,
-                        int32_t k, int32_t r, int32_t T, uint64_t seed,
+                        int32_t k, int32_t meta_f16, int32_t r, int32_t T, uint64_t seed,
                         uint32_t* codes, float* scale, float* zero, int32_t* oidx,
                         float* oval, float* resid, double* L, double* Rf) {
   const int32_t words = d * bits / 32;
@@ -221,7 +228,7 @@ void oracle_encode_unit(const float* X, int32_t n, int32_t d, int32_t bits, int3
     const float* x = X + (size_t)t * d;
     oracle_select_outliers(x, d, k, oidx + (size_t)t * k);
     for (int32_t i = 0; i < k; ++i) oval[(size_t)t * k + i] = x[oidx[(size_t)t * k + i]];
-    oracle_quantize_token(x, d, bits, g, oidx + (size_t)t * k, k, codes + (size_t)t * words,
+    oracle_quantize_token(x, d, bits, g, oidx + (size_t)t * k, k, meta_f16, codes + (size_t)t * words,
                           scale + (size_t)t * G, zero + (size_t)t * G, dhat,
                           resid + (size_t)t * d);
   }

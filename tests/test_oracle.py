@@ -301,3 +301,55 @@ def test_append_flush_protocol():
         got = kc.blocks[1][u]
         assert np.array_equal(got.codes, alone.codes) and np.array_equal(got.oidx, alone.oidx)
         assert np.array_equal(got.L, alone.L) and got.rank == 2
+
+
+# ------------------------------------------------ byte-lean (binary16) metadata
+@pytest.mark.parametrize("bits,g", [(4, 64), (2, 32), (8, 128)])
+def test_f16_metadata_is_textbook_quantization_against_rounded_metadata(bits, g):
+    """With scale and zero stored as binary16, s = r = 0 is the textbook quantizer
+    run against the rounded metadata (numpy's float16 rounding, independent of
+    the C compiler's)."""
+    x = (RNG.standard_normal((48, 128)) * RNG.uniform(0.05, 30, size=(48, 1))).astype(np.float16).astype(np.float32)
+    x[2, :g] = 0.5             # constant group: scale 0
+    p = Params(bits=bits, group_size=g, outlier_frac=0.0, rank=0, meta_f16=True)
+    u = oracle.encode_unit(x, p)
+    L = 2 ** bits - 1
+    xg = x.reshape(48, -1, g)
+    mn = xg.min(axis=2, keepdims=True)
+    mx = xg.max(axis=2, keepdims=True)
+    scale = ((mx - mn) / np.float32(L)).astype(np.float32).astype(np.float16).astype(np.float32)
+    zero = mn.astype(np.float16).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(scale > 0, np.rint((xg - zero) / scale), 0).astype(np.float32)
+    codes = np.clip(q, 0, L).reshape(48, 128).astype(np.uint32)
+    assert np.array_equal(unpack_codes(u.codes, 128, bits), codes)
+    assert np.array_equal(u.scale, scale[..., 0])
+    assert np.array_equal(u.zero, zero[..., 0])
+    # binary16 inputs: the zero point (a group minimum) is stored exactly
+    assert np.array_equal(u.zero, mn[..., 0])
+
+
+@pytest.mark.parametrize("bits,g,s", [(4, 64, 0.02), (2, 32, 0.05)])
+def test_f16_metadata_error_bound(bits, g, s):
+    """Half a step of the stored scale, plus what rounding the scale moves the
+    top of the range by (the code there is clamped)."""
+    n, d = 200, 128
+    x = (RNG.standard_normal((n, d)) * np.exp(RNG.uniform(np.log(0.5), np.log(8), size=(1, d))))
+    x = x.astype(np.float16).astype(np.float32)
+    p = Params(bits=bits, group_size=g, outlier_frac=s, rank=0, meta_f16=True)
+    u = oracle.encode_unit(x, p)
+    L = 2 ** bits - 1
+    out_mask = np.zeros((n, d), bool)
+    np.put_along_axis(out_mask, u.oidx.astype(np.int64), True, axis=1)
+    G = d // g
+    xg = np.where(out_mask, np.nan, x).reshape(n, G, g).astype(np.float64)
+    exact = (np.nanmax(xg, axis=2) - np.nanmin(xg, axis=2)) / L
+    sc = u.scale.astype(np.float64)
+    # binary16 rounding (half an ulp, 2^-11 relative; 2^-25 absolute below the normal range) of a binary32 value
+    assert np.all(np.abs(sc - exact) <= exact * (2.0 ** -11 + 2.0 ** -22) + 2.0 ** -25)
+    dh = oracle.reconstruct_unit(u, p).astype(np.float32).astype(np.float64)
+    err = np.abs(x.astype(np.float64) - dh)
+    bound = np.repeat(sc * (0.5 + L * 2.0 ** -22) + L * np.abs(sc - exact), g, axis=1) \
+        + 0.5 * np.spacing(np.abs(dh.astype(np.float32))).astype(np.float64)
+    assert np.all(err[~out_mask] <= bound[~out_mask])
+    assert np.array_equal(dh[out_mask], x[out_mask].astype(np.float64))
