@@ -51,12 +51,13 @@ def peaks():
 DECODE_TRAFFIC_BYTES = 829486336 + 6881536
 
 
-def per_token_bytes(w) -> int:
+def per_token_bytes(w, meta_f16: bool = False) -> int:
     """Compressed bytes per token of one tensor: codes + (scale, zero) per group
-    + outlier index and value + L row."""
+    (binary32 pairs, or binary16 pairs with meta_f16) + outlier index and value + L row."""
     k = math.ceil(w.s * w.d - 1e-9)
     esz = 4 if w.dtype == "f32" else 2
-    return w.d * w.bits // 8 + (w.d // w.group) * 8 + k * (1 + esz) + w.rank * (4 if w.dtype == "f32" else 2)
+    return (w.d * w.bits // 8 + (w.d // w.group) * (4 if meta_f16 else 8) + k * (1 + esz)
+            + w.rank * (4 if w.dtype == "f32" else 2))
 
 
 # ---------------------------------------------------------------- clocks
@@ -362,25 +363,27 @@ def run_gpu(args, rank: int, world: int):
         "clocks": clk,
     }
     if world == 1:
-        line["gear_l"] = gear_l_measure(gear, wl, we, wd, dev, max(3, K // 2), hbm)
+        line["gear_l"] = variant_measure(gear, wl, we, wd, dev, max(3, K // 2), hbm, s=0.0)
+        line["meta_f16"] = variant_measure(gear, wl, we, wd, dev, max(3, K // 2), hbm, s=we.s, meta_f16=True)
         v, cores, sample = oracle_encode_gbps()
         line["cpu_baseline"] = {"value": round(v, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     print(json.dumps(line), flush=True)
 
 
-def gear_l_measure(gear, wl, we, wd, dev, reps, hbm):
-    """The same two workloads with s = 0 (the pages' GEAR-L: group-wise quantization
-    plus low rank, no outliers), timed like the main stages (CUDA events, L2 flushed
-    before each timed launch sequence). Reported beside GEAR; not the headline."""
+def variant_measure(gear, wl, we, wd, dev, reps, hbm, s, meta_f16=False):
+    """The same two workloads with another outlier fraction s (s = 0 is the pages'
+    GEAR-L: group-wise quantization plus low rank, no outliers) or with binary16
+    metadata, timed like the main stages (CUDA events, L2 flushed before each timed
+    launch sequence). Reported beside GEAR; not the headline."""
     import torch
-    w0e = dataclasses.replace(we, s=0.0)
-    w0d = dataclasses.replace(wd, s=0.0)
+    w0e = dataclasses.replace(we, s=s)
+    w0d = dataclasses.replace(wd, s=s)
 
     def params(w):
-        return gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=0.0, rank=w.rank,
+        return gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank,
                                 power_iters=w.iters, buffer_len=w.buffer_len, buffer_rank=w.buffer_rank,
-                                seed=w.seed)
+                                seed=w.seed, meta_f16=meta_f16)
 
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -427,12 +430,14 @@ def gear_l_measure(gear, wl, we, wd, dev, reps, hbm):
     assert gear.device_status() == 0, "device-side error word set"
     enc_ms, dec_ms = statistics.median(enc), statistics.median(dec)
     enc_in = 2 * w0e.B * w0e.H * w0e.n * w0e.d * 2
-    dec_alg = (2 * w0d.B * w0d.H * w0d.n * per_token_bytes(w0d) + 2 * w0d.B * w0d.H * w0d.rank * 128 * 4
+    ptb = per_token_bytes(w0d, meta_f16)
+    dec_alg = (2 * w0d.B * w0d.H * w0d.n * ptb + 2 * w0d.B * w0d.H * w0d.rank * 128 * 4
                + 2 * w0d.B * w0d.H * w0d.buffer_fill * 128 * 2 + 2 * w0d.B * w0d.Hq * 128 * 2)
-    return {"s": 0.0, "encode_ms": round(enc_ms, 4), "encode_gbs": round(enc_in / enc_ms / 1e6, 3),
+    return {"s": s, "meta_f16": bool(meta_f16), "encode_ms": round(enc_ms, 4),
+            "encode_gbs": round(enc_in / enc_ms / 1e6, 3),
             "decode_ms": round(dec_ms, 4), "decode_tokens_per_s": round(w0d.B / dec_ms * 1e3, 1),
             "decode_hbm_frac": round(dec_alg / dec_ms / 1e6 / hbm, 4),
-            "bytes_per_token": per_token_bytes(w0d)}
+            "bytes_per_token": ptb}
 
 
 def main():

@@ -69,6 +69,10 @@ typedef enum { GEAR_F16 = 0, GEAR_BF16 = 1, GEAR_F32 = 2 } gear_dtype;
  *  buffer_rank  r_buf in [0, 16], r_buf <= min(n_b, d): rank of each flushed
  *               buffer block (ZeroQuant entry: the paper gives every group of
  *               n_b decoded tokens rank 2).
+ *  meta_f16     0: scale and zero point stored as fp32 (default); 1: stored as
+ *               binary16, rounded to nearest even, with the codes decided
+ *               against the stored values (a byte-lean layout: 4 instead of
+ *               8 bytes per group; fp16 caches only, else UNSUPPORTED).
  *  seed         seeds the power-iteration start matrix Q0 (d x r): entry
  *               (i, j) is the (i*r + j)-th output of the splitmix64 stream
  *               whose state starts at `seed` (Steele, Lea & Flood, OOPSLA
@@ -81,7 +85,7 @@ typedef struct gear_params {
   int32_t power_iters;
   int32_t buffer_len;
   int32_t buffer_rank;
-  int32_t reserved0;
+  int32_t meta_f16;
   uint64_t seed;
 } gear_params;
 
@@ -96,7 +100,8 @@ typedef struct gear_params {
  *   codes  uint32 [U][n_max][W]      W = d*b/32. Channel c of a token is bits
  *                                    [(c*b)%32, (c*b)%32 + b) of word c*b/32.
  *   meta   float  [U][n_max][G][2]   G = d/g; (scale, zero) of each group,
- *                                    zero = group minimum over non-outliers.
+ *                                    zero = group minimum over non-outliers
+ *                                    (binary16 [U][n_max][G][2] if meta_f16).
  *   oidx   uint8  [U][n_max][k]      outlier channels, ascending.
  *   oval   dtype  [U][n_max][k]      outlier values, bit-exact input copies.
  *   lfac   f16|f32[U][n_max][r_max]  L rows, stored as L * 2^e_blk.

@@ -47,7 +47,7 @@ static Layout cache_layout(const gear_params* p, int B, int H, int d, int n_max,
   const int rm = rmax > 0 ? rmax : 1;
   size_t off = 0;
   L.codes = off; off = align256(off + U * n_max * W * 4);
-  L.meta = off;  off = align256(off + U * n_max * G * 8);
+  L.meta = off;  off = align256(off + U * n_max * G * (size_t)meta_row_bytes(1, p->meta_f16));
   L.oidx = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1));
   L.oval = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1) * esize(dt));
   L.lfac = off;  off = align256(off + U * n_max * rm * (dt == GEAR_F32 ? 4 : 2));
@@ -105,6 +105,7 @@ static gear_status encode_block(gear_cache* const* cs, const void* const* kvs, i
   a.W = c->W;
   a.G = c->G;
   a.r_max = c->r_max;
+  a.meta_f16 = c->p.meta_f16;
   for (int i = 0; i < nt; ++i)
     a.ten[i] = EncodeTensor{kvs[i], cs[i]->codes, cs[i]->meta, cs[i]->oidx, cs[i]->oval, cs[i]->lfac, cs[i]->rfac};
   a.tpu = (n + 127) / 128;
@@ -181,6 +182,7 @@ gear_status gear_validate_params(const gear_params* p, int32_t d) {
     return GEAR_ERR_INVALID_ARG;
   if ((p->rank > 0 || p->buffer_rank > 0) && p->power_iters < 1) return GEAR_ERR_INVALID_ARG;
   if (p->power_iters < 0) return GEAR_ERR_INVALID_ARG;
+  if (p->meta_f16 != 0 && p->meta_f16 != 1) return GEAR_ERR_INVALID_ARG;
   if (d != 128) return GEAR_ERR_UNSUPPORTED;
   if (p->group_size < 32) return GEAR_ERR_UNSUPPORTED;
   if (gear_num_outliers(p->outlier_frac, d) > 16) return GEAR_ERR_UNSUPPORTED;
@@ -191,6 +193,7 @@ size_t gear_cache_bytes(const gear_params* p, int32_t B, int32_t H, int32_t d, i
                         gear_dtype dtype) {
   if (gear_validate_params(p, d) != GEAR_OK) return 0;
   if (B <= 0 || H <= 0 || n_max <= 0 || nblk_max <= 0 || dtype < GEAR_F16 || dtype > GEAR_F32) return 0;
+  if (p->meta_f16 && dtype != GEAR_F16) return 0;
   return cache_layout(p, B, H, d, n_max, nblk_max, dtype).total;
 }
 
@@ -202,6 +205,7 @@ gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int3
   if (B <= 0 || H <= 0 || n_max <= 0 || nblk_max <= 0 || dtype < GEAR_F16 || dtype > GEAR_F32)
     return GEAR_ERR_INVALID_ARG;
   if (!aligned(dev, 256)) return GEAR_ERR_INVALID_ARG;
+  if (p->meta_f16 && dtype != GEAR_F16) return GEAR_ERR_UNSUPPORTED;   // binary16 metadata of fp16 input only
   if ((size_t)B * H * round_nmax(n_max) >= ((size_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
   Layout L = cache_layout(p, B, H, d, n_max, nblk_max, dtype);
   if (bytes < L.total) return GEAR_ERR_CAPACITY;
@@ -293,6 +297,7 @@ static gear_status decode_args(const gear_cache* k, const gear_cache* v, int32_t
   a.dtype = k->dtype;
   a.B = k->B; a.H = k->H; a.Hq = Hq; a.hq = Hq / k->H;
   a.bits = k->p.bits; a.g = k->p.group_size; a.G = k->G; a.W = k->W; a.k = k->k; a.r_max = k->r_max;
+  a.meta_f16 = k->p.meta_f16;
   a.n_max = k->n_max; a.nblk_max = k->nblk_max; a.n_b = k->p.buffer_len;
   a.n_comp = k->n_comp; a.n_buf = k->n_buf;
   a.blk0_len = k->blk0_len; a.blk0_rank = k->blk0_rank; a.buffer_rank = k->p.buffer_rank;
@@ -384,6 +389,7 @@ gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream)
   a.dtype = c->dtype;
   a.U = c->B * c->H;
   a.bits = c->p.bits; a.g = c->p.group_size; a.G = c->G; a.W = c->W; a.k = c->k; a.r_max = c->r_max;
+  a.meta_f16 = c->p.meta_f16;
   a.n_max = c->n_max; a.nblk_max = c->nblk_max; a.n_b = c->p.buffer_len;
   a.n_comp = c->n_comp; a.n_buf = c->n_buf;
   a.blk0_len = c->blk0_len; a.blk0_rank = c->blk0_rank; a.buffer_rank = c->p.buffer_rank;

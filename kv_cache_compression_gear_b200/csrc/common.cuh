@@ -92,6 +92,9 @@ struct CodeFloats {
   }
 };
 
+// Bytes of G groups' (scale, zero) pairs: fp32 pairs, or binary16 pairs.
+__host__ __device__ constexpr int meta_row_bytes(int G, int meta_f16) { return G * (meta_f16 ? 4 : 8); }
+
 // Row length of the stored Rf factors: r_max rounded up to a multiple of 4, so
 // that one channel's row is a whole number of 16-byte vectors.
 __host__ __device__ constexpr int rpad_of(int r_max) { return (r_max + 3) & ~3; }

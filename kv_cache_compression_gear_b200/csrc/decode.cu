@@ -135,13 +135,36 @@ __device__ __forceinline__ float hi2(uint64_t v) {
   return b;
 }
 
-// One token's meta row in shared memory: (scale, zero) of group gi sits at
-// byte (8*gi) ^ mx of the row, mx the lane's swizzle term (0 unless G = 4).
+// One token's meta row in shared memory. With binary32 metadata (MF false),
+// (scale, zero) of group gi sits at byte (8*gi) ^ mx of the row, mx the lane's
+// swizzle term (0 unless G = 4, the only 32-byte row); with binary16 metadata
+// the pair is a half2 at byte 4*gi of a row of at most 16 bytes (no swizzle).
+template <bool MF>
 __device__ __forceinline__ float2 meta_at(const uint8_t* mrow, int gi, int mx) {
-  return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
+  if constexpr (MF) return __half22float2(*reinterpret_cast<const __half2*>(mrow + 4 * gi));
+  else return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
 }
-// The whole row, read in 16-byte pieces (conflict-free across the lanes).
+// The whole row, read in pieces of up to 16 bytes (conflict-free across the lanes).
+template <bool MF>
 __device__ __forceinline__ void meta_row(const uint8_t* mrow, int G, int mx, float2 (&sz)[4]) {
+  if constexpr (MF) {
+    if (G == 4) {
+      const uint4 a = *reinterpret_cast<const uint4*>(mrow);
+      sz[0] = __half22float2(*reinterpret_cast<const __half2*>(&a.x));
+      sz[1] = __half22float2(*reinterpret_cast<const __half2*>(&a.y));
+      sz[2] = __half22float2(*reinterpret_cast<const __half2*>(&a.z));
+      sz[3] = __half22float2(*reinterpret_cast<const __half2*>(&a.w));
+    } else if (G == 2) {
+      const uint2 a = *reinterpret_cast<const uint2*>(mrow);
+      sz[0] = __half22float2(*reinterpret_cast<const __half2*>(&a.x));
+      sz[1] = __half22float2(*reinterpret_cast<const __half2*>(&a.y));
+      sz[2] = sz[3] = make_float2(0.0f, 0.0f);
+    } else {
+      sz[0] = __half22float2(*reinterpret_cast<const __half2*>(mrow));
+      sz[1] = sz[2] = sz[3] = make_float2(0.0f, 0.0f);
+    }
+    return;
+  }
   if (G == 4) {
     const float4 a = *reinterpret_cast<const float4*>(mrow + mx);
     const float4 b = *reinterpret_cast<const float4*>(mrow + (16 ^ mx));
@@ -162,7 +185,7 @@ __device__ __forceinline__ void meta_row(const uint8_t* mrow, int G, int mx, flo
 // fix = x_o - (zero_g(c_o) + L_t . Rf[c_o]). Rf rows are 16-byte vectors, so a
 // rank <= 4 block needs one load per outlier. All loads are issued together.
 constexpr int kFast = 4;
-template <typename T>
+template <typename T, bool MF>
 __device__ __forceinline__ void outlier_fixes(const uint8_t* rest, int oval_off, const uint8_t* mrow, int mx, int t,
                                               int k, int lg, const float (&lt)[4], const float* rf, int rp,
                                               int (&cix)[kFast], float (&fix)[kFast]) {
@@ -177,7 +200,7 @@ __device__ __forceinline__ void outlier_fixes(const uint8_t* rest, int oval_off,
 #pragma unroll
   for (int i = 0; i < kFast; ++i) {
     const bool on = i < k;
-    zr[i] = on ? meta_at(mrow, cix[i] >> lg, mx).y : 0.0f;
+    zr[i] = on ? meta_at<MF>(mrow, cix[i] >> lg, mx).y : 0.0f;
     rv[i] = on ? __ldg(reinterpret_cast<const float4*>(rf + cix[i] * rp)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
 #pragma unroll
@@ -211,7 +234,7 @@ __device__ __forceinline__ float lowrank_at(const uint8_t* lf, int t, int rm, in
 // alr [HQ][16] | w [32][G][HQ] | accx [HQ][128]. The [HQ][128] arrays hold
 // channel c at slot c; loops that touch all of them use slot e*32 + lane so
 // that every lane stays in its own bank.
-template <typename T, int BITS, int HQ, bool OUT>
+template <typename T, int BITS, int HQ, bool OUT, bool MF>
 __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) decode_warp(const __grid_constant__ DecodeMaps maps,
                                                          const DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm[];
@@ -329,8 +352,9 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         }
 
       // ---- copy roles: lanes 0/1 codes (K/V), 2/3 meta by tensor copy (G >= 2),
-      // 4/5 oidx, 6/7 oval, 8/9 L rows, 10/11 meta by bulk copy (G = 1)
-      const bool meta_tma = G >= 2;
+      // 4/5 oidx, 6/7 oval, 8/9 L rows, 10/11 meta by bulk copy (rows under 16 bytes)
+      const int mrb = MF ? 4 * G : 8 * G;   // meta bytes per token
+      const bool meta_tma = mrb >= 16;
       const int x = lane & 1;
       const CUtensorMap* my_map = nullptr;
       const uint8_t* my_src = nullptr;
@@ -373,7 +397,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
           case 5:
             if (!meta_tma) {
               my_src = reinterpret_cast<const uint8_t*>(x ? a.V.meta : a.K.meta);
-              my_bpr = G * 8;
+              my_bpr = mrb;
               my_dst = wbs + L.meta0 + x * L.mb;
               my_sst = 2 * L.mb;
             }
@@ -414,8 +438,8 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
             for (int e = lane; e < nt * rm * lsz; e += 32) rest[L.lf + e] = lf[e];
             if (!meta_tma) {
               uint8_t* md = wb + L.meta0 + (2 * s + xx) * L.mb;
-              const uint8_t* ms = reinterpret_cast<const uint8_t*>(cv.meta) + row * G * 8;
-              for (int e = lane; e < nt * G * 8; e += 32) md[e] = ms[e];
+              const uint8_t* ms = reinterpret_cast<const uint8_t*>(cv.meta) + row * mrb;
+              for (int e = lane; e < nt * mrb; e += 32) md[e] = ms[e];
             }
           }
         }
@@ -433,7 +457,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
       // lane-constant swizzle terms: key rows (lane = token), meta rows, and the
       // value reads of token 2*i + par (period 4 in i)
       const int xs = swz<R>(lane);
-      const int mx = G == 4 ? ((lane >> 2) & 1) << 4 : 0;
+      const int mx = mrb == 32 ? ((lane >> 2) & 1) << 4 : 0;
       int voff[4];
       {
         const int ob = BITS == 4 ? 4 * lq : (BITS == 2 ? 2 * lq : 8 * lq);
@@ -535,8 +559,8 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         // ---------------- scores: lane = token
         const int t = lane;
         const bool live = t < nt;
-        const uint8_t* kmrow = tkm + t * G * 8;
-        const uint8_t* vmrow = tvm + t * G * 8;
+        const uint8_t* kmrow = tkm + t * mrb;
+        const uint8_t* vmrow = tvm + t * mrb;
         float s_[HQ];
         {
           const uint8_t* crow = tkc + t * R;
@@ -568,7 +592,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
             }
           }
           float2 sz[4];
-          meta_row(kmrow, G, mx, sz);
+          meta_row<MF>(kmrow, G, mx, sz);
           const int bpg = a.g >> 5;   // 32-channel blocks per group
 #pragma unroll
           for (int hh = 0; hh < HQ; ++hh) {
@@ -607,7 +631,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
             } else if (k <= kFast && rb <= kRReg) {
               int cix[kFast];
               float fx[kFast];
-              outlier_fixes<T>(tkr, L.oval, kmrow, mx, t, k, lg, lt, rfk, rp, cix, fx);
+              outlier_fixes<T, MF>(tkr, L.oval, kmrow, mx, t, k, lg, lt, rfk, rp, cix, fx);
 #pragma unroll
               for (int i = 0; i < kFast; ++i)
 #pragma unroll
@@ -617,7 +641,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
                 const int c = tkr[t * k + i];
                 const float lr = lowrank_at<T>(tkr + L.lf, t, rm, rb, rfk, rp, c);
                 const float xo = (float)reinterpret_cast<const T*>(tkr + L.oval)[t * k + i];
-                const float fix = xo - (meta_at(kmrow, c >> lg, mx).y + lr);
+                const float fix = xo - (meta_at<MF>(kmrow, c >> lg, mx).y + lr);
 #pragma unroll
                 for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + c] * CF::weight(c), fix, s_[hh]);
               }
@@ -639,7 +663,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         // value-side per-token weights w = p * scale; zero-point and low-rank sums
         {
           float2 vsz[4];
-          meta_row(vmrow, G, mx, vsz);
+          meta_row<MF>(vmrow, G, mx, vsz);
 #pragma unroll
           for (int gi = 0; gi < 4; ++gi) {
             if (gi >= G) break;
@@ -665,7 +689,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
             } else if (k <= kFast && rb <= kRReg) {
               int cix[kFast];
               float fx[kFast];
-              outlier_fixes<T>(tvr, L.oval, vmrow, mx, t, k, lg, lv, rfv, rp, cix, fx);
+              outlier_fixes<T, MF>(tvr, L.oval, vmrow, mx, t, k, lg, lv, rfv, rp, cix, fx);
 #pragma unroll
               for (int i = 0; i < kFast; ++i)
                 if (i < k)
@@ -676,7 +700,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
                 const int c = tvr[t * k + i];
                 const float lr = lowrank_at<T>(tvr + L.lf, t, rm, rb, rfv, rp, c);
                 const float xo = (float)reinterpret_cast<const T*>(tvr + L.oval)[t * k + i];
-                const float fix = xo - (meta_at(vmrow, c >> lg, mx).y + lr);
+                const float fix = xo - (meta_at<MF>(vmrow, c >> lg, mx).y + lr);
 #pragma unroll
                 for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + c, p[hh] * fix);
               }
@@ -866,7 +890,8 @@ void decode_plan(DecodeArgs& a, int num_sms) {
   const int esz = a.dtype == GEAR_F32 ? 4 : 2;   // oval and L rows share the width
   TileLayout& L = a.tl;
   L.cb = kDTile * a.W * 4;
-  L.mb = kDTile * a.G * 8;
+  const int mrb = meta_row_bytes(a.G, a.meta_f16);
+  L.mb = kDTile * mrb;
   L.oval = r16(kDTile * a.k);
   L.lf = L.oval + r16(kDTile * a.k * esz);
   L.rb = L.lf + r16(kDTile * a.r_max * esz);
@@ -877,9 +902,9 @@ void decode_plan(DecodeArgs& a, int num_sms) {
   const int floats = hq * 128 + 2 * hq * kMaxR + kDTile * a.G * hq + hq * 128;   // qw, u, alr, w, accx
   L.bars = L.floats + r16(floats * 4);
   L.bytes = (L.bars + 16 + 255) & ~255;   // meta tiles stay 256-byte aligned
-  const int meta_tx = a.G >= 2 ? 2 * L.mb : 0;
+  const int meta_tx = mrb >= 16 ? 2 * L.mb : 0;
   L.tx_part = 2 * L.cb + meta_tx;
-  L.tx_full = L.tx_part + 2 * kDTile * (a.k + a.k * esz + a.r_max * esz) + (a.G >= 2 ? 0 : 2 * L.mb);
+  L.tx_full = L.tx_part + 2 * kDTile * (a.k + a.k * esz + a.r_max * esz) + (mrb >= 16 ? 0 : 2 * L.mb);
   // stream-K over the units' compressed tokens: one wave of resident warps,
   // each taking an equal run of tokens (a multiple of 32)
   const int smem_cta = 1024 + 16 * L.cb + 4 * L.bytes;
@@ -902,38 +927,47 @@ void decode_plan(DecodeArgs& a, int num_sms) {
 
 size_t decode_workspace_bytes(int B, int Hq, int nsplit) { return (size_t)B * Hq * nsplit * 130 * sizeof(float); }
 
-template <typename T, int BITS, int HQ, bool OUT>
+template <typename T, int BITS, int HQ, bool OUT, bool MF>
 static cudaError_t launch_warp(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = 1024 + 16 * (size_t)a.tl.cb + 4 * (size_t)a.tl.bytes;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(decode_warp<T, BITS, HQ, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_warp<T, BITS, HQ, OUT, MF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     configured_smem = (int)smem;
   }
   const int grid = (a.total_splits + 3) / 4;
-  decode_warp<T, BITS, HQ, OUT><<<grid, kDThreads, smem, st>>>(maps, a);
+  decode_warp<T, BITS, HQ, OUT, MF><<<grid, kDThreads, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
 
-template <typename T, int BITS>
+template <typename T, int BITS, bool MF>
 static cudaError_t launch_hq(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
   switch (a.hq) {
-    case 1: return a.k > 0 ? launch_warp<T, BITS, 1, true>(maps, a, st) : launch_warp<T, BITS, 1, false>(maps, a, st);
-    case 2: return a.k > 0 ? launch_warp<T, BITS, 2, true>(maps, a, st) : launch_warp<T, BITS, 2, false>(maps, a, st);
-    case 4: return a.k > 0 ? launch_warp<T, BITS, 4, true>(maps, a, st) : launch_warp<T, BITS, 4, false>(maps, a, st);
-    case 8: return a.k > 0 ? launch_warp<T, BITS, 8, true>(maps, a, st) : launch_warp<T, BITS, 8, false>(maps, a, st);
+    case 1: return a.k > 0 ? launch_warp<T, BITS, 1, true, MF>(maps, a, st) : launch_warp<T, BITS, 1, false, MF>(maps, a, st);
+    case 2: return a.k > 0 ? launch_warp<T, BITS, 2, true, MF>(maps, a, st) : launch_warp<T, BITS, 2, false, MF>(maps, a, st);
+    case 4: return a.k > 0 ? launch_warp<T, BITS, 4, true, MF>(maps, a, st) : launch_warp<T, BITS, 4, false, MF>(maps, a, st);
+    case 8: return a.k > 0 ? launch_warp<T, BITS, 8, true, MF>(maps, a, st) : launch_warp<T, BITS, 8, false, MF>(maps, a, st);
   }
   return cudaErrorInvalidValue;
 }
 
+// binary16 metadata exists for fp16 caches only (the validation rejects it elsewhere)
 template <typename T>
 static cudaError_t launch_bits(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
+  constexpr bool kHalf = std::is_same<T, __half>::value;
+  if (kHalf && a.meta_f16) {
+    switch (a.bits) {
+      case 2: return launch_hq<T, 2, kHalf>(maps, a, st);
+      case 4: return launch_hq<T, 4, kHalf>(maps, a, st);
+      default: return launch_hq<T, 8, kHalf>(maps, a, st);
+    }
+  }
   switch (a.bits) {
-    case 2: return launch_hq<T, 2>(maps, a, st);
-    case 4: return launch_hq<T, 4>(maps, a, st);
-    default: return launch_hq<T, 8>(maps, a, st);
+    case 2: return launch_hq<T, 2, false>(maps, a, st);
+    case 4: return launch_hq<T, 4, false>(maps, a, st);
+    default: return launch_hq<T, 8, false>(maps, a, st);
   }
 }
 
@@ -948,9 +982,11 @@ cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t st) {
       const uint64_t rows = (uint64_t)a.B * a.H * a.n_max;
       bool ok = cache_row_map(enc, &maps.kc, a.K.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kDTile) &&
                 cache_row_map(enc, &maps.vc, a.V.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kDTile);
-      if (ok && a.G >= 2)
-        ok = cache_row_map(enc, &maps.km, a.K.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows, kDTile) &&
-             cache_row_map(enc, &maps.vm, a.V.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, rows, kDTile);
+      // meta rows of 16 bytes or more come by tensor copy, as 32-bit words
+      const int mrb = meta_row_bytes(a.G, a.meta_f16);
+      if (ok && mrb >= 16)
+        ok = cache_row_map(enc, &maps.km, a.K.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, mrb / 4, rows, kDTile) &&
+             cache_row_map(enc, &maps.vm, a.V.meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, mrb / 4, rows, kDTile);
       if (!ok) return cudaErrorInvalidValue;
     }
     if (a.dtype == GEAR_F16) e = launch_bits<__half>(maps, a, st);
@@ -981,7 +1017,8 @@ __global__ void __launch_bounds__(128) dense_kernel(const DenseArgs a) {
       const int blk = t < a.blk0_len ? 0 : 1 + (t - a.blk0_len) / a.n_b;
       const int rb = blk == 0 ? a.blk0_rank : a.buffer_rank;
       const uint32_t code = (a.C.codes[row * a.W + c / kPerWord] >> (BITS * (c % kPerWord))) & ((1u << BITS) - 1u);
-      const float2 sz = reinterpret_cast<const float2*>(a.C.meta)[row * a.G + c / a.g];
+      const float2 sz = a.meta_f16 ? __half22float2(reinterpret_cast<const __half2*>(a.C.meta)[row * a.G + c / a.g])
+                                   : reinterpret_cast<const float2*>(a.C.meta)[row * a.G + c / a.g];
       v = __fmaf_rn((float)code, sz.x, sz.y);
       const int rp = rpad_of(a.r_max);
       const float* rf = a.C.rfac + (((size_t)u * a.nblk_max + blk) * 128 + c) * rp;

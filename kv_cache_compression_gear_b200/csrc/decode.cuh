@@ -46,6 +46,7 @@ struct DecodeArgs {
   int32_t dtype;          // cache dtype
   int32_t B, H, Hq, hq;   // hq = Hq / H query heads per kv head
   int32_t bits, g, G, W, k, r_max;
+  int32_t meta_f16;       // (scale, zero) pairs stored as binary16
   int32_t n_max, nblk_max, n_b;
   int32_t n_comp, n_buf;
   int32_t blk0_len, blk0_rank, buffer_rank;
@@ -65,6 +66,7 @@ struct DenseArgs {
   CacheView C;
   int32_t dtype;
   int32_t U, bits, g, G, W, k, r_max, n_max, nblk_max, n_b;
+  int32_t meta_f16;
   int32_t n_comp, n_buf, blk0_len, blk0_rank, buffer_rank;
   float* out;             // [U][n_comp + n_buf][128]
 };

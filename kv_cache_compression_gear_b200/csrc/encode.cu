@@ -361,6 +361,10 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     mn[sh] = __fadd_rn(mn[sh], 0.0f);                      // -0 -> +0
     mx[sh] = __fadd_rn(mx[sh], 0.0f);
     scale[sh] = __fdiv_rn(__fsub_rn(mx[sh], mn[sh]), levels);
+    if (a.meta_f16) {   // stored as binary16; the codes are decided against the stored values
+      scale[sh] = __half2float(__float2half_rn(scale[sh]));
+      mn[sh] = __fadd_rn(__half2float(__float2half_rn(mn[sh])), 0.0f);
+    }
     // scale 0: y = 0 makes the fast path return q = 0 exactly (every code 0)
     fast[sh] = (scale[sh] >= 0x1p-100f && scale[sh] <= 0x1p100f) || scale[sh] == 0.0f;
     y[sh] = scale[sh] == 0.0f ? 0.0f : __frcp_rn(scale[sh]);
@@ -465,15 +469,18 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     for (int w = 0; w < kWordsHalf; w += 4)
       *reinterpret_cast<uint4*>(cw + w) = make_uint4(words[w], words[w + 1], words[w + 2], words[w + 3]);
     // meta: (scale, zero) per group; this thread owns groups in its half
-    float2* meta = reinterpret_cast<float2*>(ten.meta) + row * a.G;
     const int gsz = a.g;
+    auto put_meta = [&](int gi, float sc, float z) {
+      if (a.meta_f16) reinterpret_cast<__half2*>(ten.meta)[row * a.G + gi] = __floats2half2_rn(sc, z);   // exact
+      else reinterpret_cast<float2*>(ten.meta)[row * a.G + gi] = make_float2(sc, z);
+    };
     if (gsz == 32) {
-      meta[2 * h] = make_float2(scale[0], mn[0]);
-      meta[2 * h + 1] = make_float2(scale[1], mn[1]);
+      put_meta(2 * h, scale[0], mn[0]);
+      put_meta(2 * h + 1, scale[1], mn[1]);
     } else if (gsz == 64) {
-      meta[h] = make_float2(scale[0], mn[0]);
+      put_meta(h, scale[0], mn[0]);
     } else if (h == 0) {
-      meta[0] = make_float2(scale[0], mn[0]);
+      put_meta(0, scale[0], mn[0]);
     }
     if constexpr (KMAX > 0) {
       if (h == 0 && k > 0) {
@@ -946,7 +953,8 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + F::kBarOff);
   const int u = blockIdx.y, t0 = blockIdx.x * kTile, t = threadIdx.x;
   const int G = a.G, k = a.k, r = a.r;
-  const bool meta_tma = G >= 2;
+  const int mrb = meta_row_bytes(G, a.meta_f16);   // meta bytes per token
+  const bool meta_tma = mrb >= 16;
   const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
   const int tn = u / a.Uper, ul = u % a.Uper;
   const EncodeTensor& ten = a.ten[tn];
@@ -954,7 +962,7 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   if (t == 0) {
     mbar_init(bar, 1);
     fence_mbarrier_init();
-    mbar_arrive_expect_tx(bar, (uint32_t)(F::kXB + F::kCB + F::kZBytes + (meta_tma ? kTile * G * 8 : 0)));
+    mbar_arrive_expect_tx(bar, (uint32_t)(F::kXB + F::kCB + F::kZBytes + (meta_tma ? kTile * mrb : 0)));
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                      smem_u32(Zp)),
                  "l"(a.zbuf + (int64_t)u * (F::kZBytes / 4)), "r"((uint32_t)F::kZBytes), "r"(smem_u32(bar))
@@ -966,8 +974,17 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   // Zp[p][j] = (Z[2p][j], Z[2p + 1][j]) arrives with the tile (E2 writes it in this layout)
   const bool valid = t0 + t < a.n;
   const size_t row = (size_t)crow + t;
-  float2 sz1 = make_float2(0.0f, 0.0f);
-  if (!meta_tma && valid) sz1 = reinterpret_cast<const float2*>(ten.meta)[row];
+  // short meta rows (under 16 bytes) come straight from global memory
+  float2 szr[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+  if (!meta_tma && valid) {
+    if (a.meta_f16) {
+      const __half2* mh = reinterpret_cast<const __half2*>(ten.meta) + row * G;
+      szr[0] = __half22float2(mh[0]);
+      if (G == 2) szr[1] = __half22float2(mh[1]);
+    } else {
+      szr[0] = reinterpret_cast<const float2*>(ten.meta)[row];
+    }
+  }
   // the token's first outliers, fetched while the tile is in flight
   constexpr int kOF = 4;
   int oc[kOF];
@@ -983,11 +1000,14 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
   const bool landed = mbar_wait(bar, 0);
   if (!landed || !valid) return;
 
-  // this token's meta row: group gi at byte (8 gi) ^ mx (32-byte rows swizzled)
-  const uint8_t* mrow = ms + t * G * 8;
-  const int mx = G == 4 ? ((t >> 2) & 1) << 4 : 0;
+  // this token's meta row: fp32 group gi at byte (8 gi) ^ mx (32-byte rows
+  // swizzled), binary16 group gi at byte 4 gi
+  const uint8_t* mrow = ms + t * mrb;
+  const int mx = mrb == 32 ? ((t >> 2) & 1) << 4 : 0;
   auto group = [&](int gi) -> float2 {
-    return meta_tma ? *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx)) : sz1;
+    if (!meta_tma) return gi == 0 ? szr[0] : szr[1];
+    if (a.meta_f16) return __half22float2(*reinterpret_cast<const __half2*>(mrow + 4 * gi));
+    return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
   };
   bool big = false;
   for (int gi = 0; gi < G; ++gi) big |= !(group(gi).x <= 0x1p100f);
@@ -1248,8 +1268,9 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
     if (!cache_row_map(enc, &m3.codes[tn], a.ten[tn].codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, crows, kTile))
       return cudaErrorInvalidValue;
-    if (a.G >= 2 &&
-        !cache_row_map(enc, &m3.meta[tn], a.ten[tn].meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2 * a.G, crows, kTile))
+    const int mrb = meta_row_bytes(a.G, a.meta_f16);
+    if (mrb >= 16 &&
+        !cache_row_map(enc, &m3.meta[tn], a.ten[tn].meta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, mrb / 4, crows, kTile))
       return cudaErrorInvalidValue;
   }
   XMaps xm;

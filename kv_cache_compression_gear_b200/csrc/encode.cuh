@@ -32,6 +32,7 @@ struct EncodeArgs {
   int32_t t_off, blk, e_blk;
   uint32_t one_bits;     // 0x3F800000 (1.0f), kept in a register by the kernels
   int32_t n_max, nblk_max, W, G, r_max;
+  int32_t meta_f16;      // scale and zero stored as binary16
   // workspace: partial Grams [U][maxc][128][128] and Z [U][64][16][2] (channel pairs)
   float* gram;
   float* zbuf;

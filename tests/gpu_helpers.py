@@ -13,7 +13,8 @@ TORCH_DT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
 
 def oracle_params(p) -> oracle.Params:
     return oracle.Params(bits=p.bits, group_size=p.group_size, outlier_frac=p.outlier_frac, rank=p.rank,
-                         power_iters=p.power_iters, buffer_len=p.buffer_len, buffer_rank=p.buffer_rank, seed=p.seed)
+                         power_iters=p.power_iters, buffer_len=p.buffer_len, buffer_rank=p.buffer_rank, seed=p.seed,
+                         meta_f16=bool(p.meta_f16))
 
 
 def seeded_kv(seed: int, stream: int, shape, dtype: str, channel_scale: bool = False) -> np.ndarray:
@@ -58,11 +59,13 @@ def gpu_block(cache, u: int, t0: int, t1: int, blk: int, rank: int):
 
 
 def compare_unit(g: dict, o: oracle.Unit, p, what: str = ""):
-    """Bit-exact codes / scale / zero / outliers; tolerance on L Rf^T."""
+    """Bit-exact codes / scale / zero / outliers; tolerance on L Rf^T. Binary16
+    metadata widens exactly to the oracle's binary32 copy of the stored values."""
     k = o.oidx.shape[1]
+    meta = g["meta"].astype(np.float32)
     assert np.array_equal(g["codes"].view(np.uint32), o.codes), f"{what}: codes differ"
-    assert np.array_equal(g["meta"][..., 0].view(np.uint32), o.scale.view(np.uint32)), f"{what}: scale differs"
-    assert np.array_equal(g["meta"][..., 1].view(np.uint32), o.zero.view(np.uint32)), f"{what}: zero differs"
+    assert np.array_equal(meta[..., 0].view(np.uint32), o.scale.view(np.uint32)), f"{what}: scale differs"
+    assert np.array_equal(meta[..., 1].view(np.uint32), o.zero.view(np.uint32)), f"{what}: zero differs"
     if k:
         assert np.array_equal(g["oidx"][:, :k].astype(np.int32), o.oidx), f"{what}: outlier index differs"
         assert np.array_equal(g["oval"][:, :k].view(np.uint32), o.oval.view(np.uint32)), f"{what}: outlier value"

@@ -114,6 +114,28 @@ def test_cache_layout_and_host_errors(gear):
     assert L.gear_version() == b"0.1.0"
 
 
+def test_f16_metadata_layout_and_errors(gear):
+    L, E = gear.lib, gear.gear
+    p16 = gear.make_params(meta_f16=True)
+    p32 = gear.make_params()
+    b16 = L.gear_cache_bytes(ctypes.byref(p16), 1, 32, 128, 4096, 1, 0)
+    b32 = L.gear_cache_bytes(ctypes.byref(p32), 1, 32, 128, 4096, 1, 0)
+    # two binary16 pairs per token instead of two binary32 pairs: 8 bytes less
+    assert b32 - b16 == 8 * 32 * 4096
+    assert L.gear_cache_bytes(ctypes.byref(p16), 1, 32, 128, 4096, 1, 1) == 0   # bf16 input
+    assert L.gear_cache_bytes(ctypes.byref(p16), 1, 32, 128, 4096, 1, 2) == 0   # f32 input
+    c = gear.GearCacheStruct()
+    fake = ctypes.c_void_p(1 << 40)
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(p16), 1, 32, 128, 4096, 1, 1, fake, 1 << 30) == \
+        E.GEAR_ERR_UNSUPPORTED
+    bad = gear.make_params()
+    bad.meta_f16 = 2
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(bad), 1, 32, 128, 4096, 1, 0, fake, 1 << 30) == \
+        E.GEAR_ERR_INVALID_ARG
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(p16), 1, 32, 128, 4096, 1, 0, fake, b16) == 0
+    assert c.p.meta_f16 == 1 and c.oidx - c.meta >= 32 * 4096 * 8
+
+
 def test_encode_batch_host_errors(gear):
     """gear_encode_batch rejects bad batches before touching the device."""
     L, E = gear.lib, gear.gear

@@ -57,9 +57,30 @@ ENC_CASES = [
 ]
 
 
+# binary16 metadata (fp16 caches): 16-, 8- and 4-byte meta rows, GEAR-L
+F16_META_ENC_CASES = [
+    # B, H, n, bits, g, s, r, T
+    (1, 2, 300, 4, 32, 0.02, 4, 3),
+    (2, 2, 129, 4, 64, 0.02, 4, 3),
+    (1, 3, 257, 2, 128, 0.05, 2, 2),
+    (1, 2, 200, 8, 64, 0.0, 4, 3),
+    (1, 2, 33, 4, 64, 0.1, 16, 2),
+]
+
+
 @pytest.mark.parametrize("dtype,B,H,n,bits,g,s,r,T", ENC_CASES)
 def test_encode_matches_oracle(dtype, B, H, n, bits, g, s, r, T):
-    p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, power_iters=T, seed=1234 + n)
+    _encode_case(dtype, B, H, n, bits, g, s, r, T, meta_f16=False)
+
+
+@pytest.mark.parametrize("B,H,n,bits,g,s,r,T", F16_META_ENC_CASES)
+def test_encode_f16_metadata_matches_oracle(B, H, n, bits, g, s, r, T):
+    _encode_case("f16", B, H, n, bits, g, s, r, T, meta_f16=True)
+
+
+def _encode_case(dtype, B, H, n, bits, g, s, r, T, meta_f16):
+    p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, power_iters=T, seed=1234 + n,
+                         meta_f16=meta_f16)
     x = seeded_kv(7 + n + bits, 1, (B, H, n, 128), dtype, channel_scale=True)
     kc, units, op = _encode_both(x, dtype, p)
     dense = kc.dense().cpu().numpy()
@@ -145,10 +166,28 @@ DEC_CASES = [
 ]
 
 
+F16_META_DEC_CASES = [
+    # B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf
+    (2, 2, 2, 300, 25, 4, 32, 0.02, 4, 20, 2),
+    (1, 2, 8, 257, 20, 4, 64, 0.02, 4, 20, 2),
+    (1, 2, 4, 130, 45, 2, 128, 0.05, 8, 20, 2),
+    (2, 2, 2, 300, 0, 8, 64, 0.0, 4, 20, 2),
+]
+
+
 @pytest.mark.parametrize("dtype,B,H,Hq,n0,nappend,bits,g,s,r,n_b,r_buf", DEC_CASES)
 def test_decode_and_append_match_oracle(dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf):
+    _decode_case(dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf, meta_f16=False)
+
+
+@pytest.mark.parametrize("B,H,Hq,n0,nappend,bits,g,s,r,n_b,r_buf", F16_META_DEC_CASES)
+def test_decode_f16_metadata_match_oracle(B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf):
+    _decode_case("f16", B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf, meta_f16=True)
+
+
+def _decode_case(dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf, meta_f16):
     p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, buffer_len=n_b, buffer_rank=r_buf,
-                         power_iters=3, seed=77)
+                         power_iters=3, seed=77, meta_f16=meta_f16)
     kc, vc, ok, ov = _build_caches(dtype, B, H, n0, p, nappend, seed=11 + n0)
     assert kc.n_comp == ok.n_comp and kc.n_buf == len(ok.buffer) and kc.n_blk == len(ok.blocks)
     q = seeded_kv(99 + n0, 5, (B, Hq, 128), dtype)
