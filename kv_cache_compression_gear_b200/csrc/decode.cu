@@ -37,6 +37,9 @@ namespace gear {
 
 constexpr int kDThreads = 128;   // 4 warps, each an independent split
 constexpr int kDTile = 32;       // tokens per tile (one per lane)
+// token stride of one group's value weights in shared memory: the two
+// tokens and G groups a value-loop step reads fall in distinct banks
+constexpr int kWStride = kDTile + 2;
 constexpr int kMaxR = 16;
 constexpr float kLazy = 8.0f;    // log2 slack of the softmax reference
 
@@ -257,7 +260,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
   float* u_s = qw_s + HQ * 128;
   float* alr_s = u_s + HQ * kMaxR;   // value low-rank weights j >= kRReg
   float* w_s = alr_s + HQ * kMaxR;
-  float* accx_s = w_s + kDTile * G * HQ;
+  float* accx_s = w_s + kWStride * G * HQ;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wb + L.bars);
 
   // value side: lane owns channels 8*(lane & 15) .. +7 and tokens of parity lane >> 4
@@ -671,7 +674,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
 #pragma unroll
             for (int hh = 0; hh < HQ; ++hh) {
               const float wv = p[hh] * sz.x;
-              w_s[(t * G + gi) * HQ + hh] = wv;
+              w_s[(gi * kWStride + t) * HQ + hh] = wv;   // group-major: token stride HQ
               sw[hh][gi] += wv;
               spm[hh][gi] = fmaf(p[hh], sz.y, spm[hh][gi]);
             }
@@ -718,14 +721,17 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         // ---------------- values: lane = 8 channels, tokens 2*i + par. Tokens
         // past nt have w = 0 (their codes are finite), so every tile runs all 16.
         {
-          const uint8_t* vrow = tvc + par * R;
-          const float* wrow = w_s + (par * G + my_g) * HQ;
-#pragma unroll 1
+          // per-lane bases; every further offset is a compile-time constant
+          const uint8_t* vb[4];
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm) vb[mm] = tvc + par * R + voff[mm];
+          const float* wrow = w_s + (my_g * kWStride + par) * HQ;
+#pragma unroll
           for (int i4 = 0; i4 < kDTile / 2; i4 += 4) {
 #pragma unroll
             for (int mm = 0; mm < 4; ++mm) {
-              const uint8_t* row = vrow + (i4 + mm) * 2 * R + voff[mm];
-              const float* wr = wrow + (i4 + mm) * 2 * G * HQ;
+              const uint8_t* row = vb[mm] + (i4 + mm) * 2 * R;
+              const float* wr = wrow + (i4 + mm) * 2 * HQ;
               float f[8];
               if constexpr (BITS == 4) {
                 CF::word(*reinterpret_cast<const uint32_t*>(row), f, one);
@@ -899,7 +905,7 @@ void decode_plan(DecodeArgs& a, int num_sms) {
   L.rest0 = L.meta0 + 4 * L.mb;
   L.floats = L.rest0 + 4 * L.rb;
   const int hq = a.hq;
-  const int floats = hq * 128 + 2 * hq * kMaxR + kDTile * a.G * hq + hq * 128;   // qw, u, alr, w, accx
+  const int floats = hq * 128 + 2 * hq * kMaxR + kWStride * a.G * hq + hq * 128;   // qw, u, alr, w, accx
   L.bars = L.floats + r16(floats * 4);
   L.bytes = (L.bars + 16 + 255) & ~255;   // meta tiles stay 256-byte aligned
   const int meta_tx = mrb >= 16 ? 2 * L.mb : 0;
