@@ -201,6 +201,21 @@ gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const voi
                              int32_t Hq, float softmax_scale, void* out, gear_dtype out_dtype,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* Decode attention over a batch whose prefills were right-padded to one length
+ * (serving with sequences of different prompt lengths; no counterpart in the
+ * paper, which decodes one batch of equal lengths). Same computation, layouts
+ * and errors as gear_decode_attn, except that for batch row b the block-0
+ * tokens [prefill_len[b], blk0_len) are padding and take no part in the
+ * softmax; every later token (flushed blocks and buffer) is real.
+ *   prefill_len  [B] int32 in DEVICE memory, read by the kernel; values are
+ *                clamped to [0, blk0_len]. Block 0 is the block gear_encode wrote.
+ * A row of q whose every token is padding gets an output of 0.
+ * Errors: INVALID_ARG (also for a null or unaligned prefill_len), WORKSPACE, CUDA. */
+gear_status gear_decode_attn_ragged(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq,
+                                    float softmax_scale, void* out, gear_dtype out_dtype,
+                                    const int32_t* prefill_len, void* workspace, size_t ws_bytes,
+                                    void* stream);
+
 /* Decode attention that allocates nothing. The GEAR paper has no counterpart
  * of this entry point: it exists for callers that cannot call cudaMalloc or
  * hand the library a workspace -- for example a plugin inside a host framework

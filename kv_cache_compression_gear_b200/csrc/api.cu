@@ -311,11 +311,13 @@ size_t gear_decode_workspace_bytes(const gear_cache* k, const gear_cache* v, int
   return decode_workspace_bytes(a.B, a.Hq, a.nsplit);
 }
 
-gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq, float softmax_scale,
-                             void* out, gear_dtype out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+static gear_status decode_attn(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq,
+                               float softmax_scale, void* out, gear_dtype out_dtype, const int32_t* prefill_len,
+                               void* workspace, size_t ws_bytes, void* stream) {
   DecodeArgs a;
   gear_status s = decode_args(k, v, Hq, a);
   if (s != GEAR_OK) return s;
+  a.plen = prefill_len;
   if (!q || !out) return GEAR_ERR_INVALID_ARG;
   if (out_dtype != k->dtype && out_dtype != GEAR_F32) return GEAR_ERR_INVALID_ARG;
   if (!isfinite(softmax_scale)) return GEAR_ERR_INVALID_ARG;
@@ -328,6 +330,18 @@ gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const voi
   a.out_dtype = out_dtype;
   a.part = reinterpret_cast<float*>(workspace);
   return cuda_status(decode_launch(a, (cudaStream_t)stream));
+}
+
+gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq, float softmax_scale,
+                             void* out, gear_dtype out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_attn(k, v, q, Hq, softmax_scale, out, out_dtype, nullptr, workspace, ws_bytes, stream);
+}
+
+gear_status gear_decode_attn_ragged(const gear_cache* k, const gear_cache* v, const void* q, int32_t Hq,
+                                    float softmax_scale, void* out, gear_dtype out_dtype, const int32_t* prefill_len,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  if (!prefill_len || !aligned(prefill_len, 4)) return GEAR_ERR_INVALID_ARG;
+  return decode_attn(k, v, q, Hq, softmax_scale, out, out_dtype, prefill_len, workspace, ws_bytes, stream);
 }
 
 size_t gear_append_workspace_bytes(const gear_cache* k) {

@@ -280,6 +280,9 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
   auto segment = [&](const int unit, const int c0, const int c1, const int sp, const bool with_buf) -> bool {
     const int b = unit / a.H, h = unit % a.H;
     const bool comp = c1 > c0;
+    // right-padded prefill: block-0 tokens [pl, blk0_len) of this batch row are
+    // padding and take no part in the softmax
+    const int pl = a.plen ? min(max(__ldg(a.plen + b), 0), a.blk0_len) : a.blk0_len;
     // this split's partial row of query head hh: part_row + hh * hstride
     float* part_row = a.part + (((size_t)b * a.Hq + (size_t)h * HQ) * a.nsplit + sp) * 130;
     const size_t hstride = (size_t)a.nsplit * 130;
@@ -561,7 +564,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
 
         // ---------------- scores: lane = token
         const int t = lane;
-        const bool live = t < nt;
+        const bool live = t < nt && (t0 + t < pl || t0 + t >= a.blk0_len);
         const uint8_t* kmrow = tkm + t * mrb;
         const uint8_t* vmrow = tvm + t * mrb;
         float s_[HQ];
@@ -883,7 +886,7 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeArgs a) {
     den = fmaf(p[s * 130 + 1], w, den);
     num = fmaf(p[s * 130 + 2 + c], w, num);
   }
-  const float o = num / den;
+  const float o = den > 0.0f ? num / den : 0.0f;   // a row whose every token is padding gives 0
   TO* out = reinterpret_cast<TO*>(a.out) + (size_t)bj * 128 + c;
   if constexpr (sizeof(TO) == 4) *out = o;
   else if constexpr (std::is_same<TO, __half>::value) *out = __float2half_rn(o);

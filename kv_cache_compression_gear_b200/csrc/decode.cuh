@@ -56,6 +56,7 @@ struct DecodeArgs {
   void* out;              // [B][Hq][128] out dtype
   int32_t out_dtype;
   float* part;            // [B][Hq][nsplit][130] partial (m, l, acc[128]) per warp that meets the unit
+  const int32_t* plen;    // [B] device: real tokens at the head of block 0 per batch row, or null (all)
   int32_t seg_tokens;     // compressed tokens per warp (a multiple of 32); 0 without any
   int32_t nsplit;         // partial rows per unit: at most ceil(n_comp / seg_tokens) + 1 warps meet a unit
   int32_t total_splits;   // warps: ceil(units * n_comp / seg_tokens), or units without compressed tokens

@@ -66,6 +66,7 @@ def _load():
         "gear_encode_batch": (i32, [i32, P, P, i32, P, S, P]),
         "gear_decode_workspace_bytes": (S, [pc, pc, i32]),
         "gear_decode_attn": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P, S, P]),
+        "gear_decode_attn_ragged": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P, P, S, P]),
         "gear_decode_attn_noalloc": (i32, [pc, pc, P, i32, ctypes.c_float, P, i32, P]),
         "gear_append_workspace_bytes": (S, [pc]),
         "gear_append_buffer": (i32, [pc, pc, P, P, P, S, P]),
@@ -211,7 +212,9 @@ def encode_batch(caches, kvs, stream=None):
 
 
 def decode_attn(kc: Cache, vc: Cache, q: torch.Tensor, softmax_scale: float, out_dtype=None, out=None,
-                stream=None) -> torch.Tensor:
+                stream=None, prefill_len: torch.Tensor | None = None) -> torch.Tensor:
+    """gear_decode_attn, or gear_decode_attn_ragged when prefill_len (int32 [B] on the
+    device: real tokens at the head of each batch row's prefill) is given."""
     assert q.is_cuda and q.dtype == kc.dtype and q.is_contiguous()
     B, Hq, d = q.shape
     od = out_dtype or kc.dtype
@@ -221,6 +224,14 @@ def decode_attn(kc: Cache, vc: Cache, q: torch.Tensor, softmax_scale: float, out
     if nbytes == 0:
         raise GearError(GEAR_ERR_INVALID_ARG, "gear_decode_workspace_bytes")
     wp, wn = _ws.get(nbytes, q.device)
+    if prefill_len is not None:
+        assert prefill_len.is_cuda and prefill_len.dtype == torch.int32 and prefill_len.is_contiguous()
+        assert prefill_len.numel() == B
+        _check(lib.gear_decode_attn_ragged(ctypes.byref(kc.c), ctypes.byref(vc.c), ctypes.c_void_p(q.data_ptr()),
+                                           Hq, ctypes.c_float(softmax_scale), ctypes.c_void_p(out.data_ptr()),
+                                           _DT[od], ctypes.c_void_p(prefill_len.data_ptr()), ctypes.c_void_p(wp),
+                                           wn, _stream_ptr(stream)), "gear_decode_attn_ragged")
+        return out
     _check(lib.gear_decode_attn(ctypes.byref(kc.c), ctypes.byref(vc.c), ctypes.c_void_p(q.data_ptr()), Hq,
                                 ctypes.c_float(softmax_scale), ctypes.c_void_p(out.data_ptr()), _DT[od],
                                 ctypes.c_void_p(wp), wn, _stream_ptr(stream)), "gear_decode_attn")

@@ -239,15 +239,29 @@ class Cache:
         return out
 
 
-def decode_attn(kc: Cache, vc: Cache, q: np.ndarray, scale: float) -> np.ndarray:
+def decode_attn(kc: Cache, vc: Cache, q: np.ndarray, scale: float, prefill_len=None) -> np.ndarray:
     """Attention of q [B][Hq][d] over the reconstructed caches; float64 [B][Hq][d].
-    Query head j reads kv-head j // (Hq // H)."""
+    Query head j reads kv-head j // (Hq // H).
+
+    prefill_len (optional, B ints): batch row b's prefill was right-padded, so only
+    the first prefill_len[b] tokens of block 0 are real (clamped to [0, block-0
+    length]); the padding takes no part in the softmax, every later token does.
+    A row with no real token gives 0. (Serving with prompts of different lengths;
+    the paper decodes equal lengths, so this is a reading, not a passage.)"""
     B, Hq, d = q.shape
     H = kc.H
     Kd, Vd = kc.dense(), vc.dense()
+    n = Kd.shape[2]
+    n0 = kc.blocks[0][0].codes.shape[0] if kc.blocks else 0
     out = np.zeros((B, Hq, d), dtype=np.float64)
     for b in range(B):
+        rows = np.arange(n)
+        if prefill_len is not None:
+            pl = min(max(int(prefill_len[b]), 0), n0)
+            rows = rows[(rows < pl) | (rows >= n0)]
+        if rows.size == 0:
+            continue
         for j in range(Hq):
             h = j // (Hq // H)
-            out[b, j] = attention(q[b, j], Kd[b, h], Vd[b, h], scale)
+            out[b, j] = attention(q[b, j], Kd[b, h][rows], Vd[b, h][rows], scale)
     return out

@@ -108,6 +108,9 @@ def test_cache_layout_and_host_errors(gear):
     assert L.gear_encode(ctypes.byref(c), ctypes.c_void_p(4096), 2, None, 0, None) == E.GEAR_ERR_INVALID_ARG
     assert L.gear_decode_attn(ctypes.byref(c), ctypes.byref(c), ctypes.c_void_p(4096), 32, ctypes.c_float(0.1),
                               ctypes.c_void_p(4096), 0, None, 0, None) == E.GEAR_ERR_INVALID_ARG  # empty cache
+    assert L.gear_decode_attn_ragged(ctypes.byref(c), ctypes.byref(c), ctypes.c_void_p(4096), 32, ctypes.c_float(0.1),
+                                     ctypes.c_void_p(4096), 0, None, ctypes.c_void_p(4096), 1 << 20,
+                                     None) == E.GEAR_ERR_INVALID_ARG   # no prefill lengths
     assert L.gear_decode_dense(ctypes.byref(c), None, None) == E.GEAR_ERR_INVALID_ARG
     assert L.gear_selftest_wait_timeout(0, None) == E.GEAR_ERR_INVALID_ARG   # rejected before any launch
     assert L.gear_status_string(6) == b"workspace missing or too small"

@@ -209,6 +209,34 @@ def _decode_case(dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf, meta_f
     assert gear.device_status() == 0
 
 
+RAGGED_CASES = [
+    # dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf, prefill lengths
+    ("f16", 4, 2, 4, 300, 25, 4, 64, 0.02, 4, 20, 2, [0, 1, 157, 300]),
+    ("bf16", 3, 2, 2, 257, 0, 4, 32, 0.05, 4, 20, 2, [0, 100, 400]),   # row 0: nothing real, output 0
+    ("f32", 2, 1, 1, 64, 9, 8, 64, 0.02, 2, 4, 1, [33, 5]),
+    ("f16", 2, 2, 8, 130, 21, 2, 128, 0.0, 4, 20, 2, [129, 31]),         # GEAR-L, GQA
+]
+
+
+@pytest.mark.parametrize("dtype,B,H,Hq,n0,nappend,bits,g,s,r,n_b,r_buf,plen", RAGGED_CASES)
+def test_ragged_prefill_decode_matches_oracle(dtype, B, H, Hq, n0, nappend, bits, g, s, r, n_b, r_buf, plen):
+    p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, buffer_len=n_b, buffer_rank=r_buf,
+                         power_iters=3, seed=41)
+    kc, vc, ok, ov = _build_caches(dtype, B, H, n0, p, nappend, seed=5 + n0)
+    q = seeded_kv(77 + n0, 5, (B, Hq, 128), dtype)
+    tau = 1.0 / math.sqrt(128)
+    od = oracle.decode_attn(ok, ov, q, tau, prefill_len=plen)
+    vmax = np.abs(ov.dense()).max()
+    pl = torch.tensor(plen, dtype=torch.int32, device="cuda")
+    out = gear.decode_attn(kc, vc, to_dev(q, dtype), tau, out_dtype=torch.float32, prefill_len=pl).cpu().numpy()
+    err = np.abs(out - od).max()
+    assert err <= _tol_out(dtype) * vmax, f"attention error {err:.3e} vs {_tol_out(dtype) * vmax:.3e}"
+    for b, n in enumerate(plen):
+        if n <= 0 and nappend == 0:
+            assert not out[b].any()
+    assert gear.device_status() == 0
+
+
 # ------------------------------------------------------------ batched encode
 BATCH_CASES = [
     # dtype, count, B, H, n, bits, g, s, r, T

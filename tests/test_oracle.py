@@ -353,3 +353,59 @@ def test_f16_metadata_error_bound(bits, g, s):
         + 0.5 * np.spacing(np.abs(dh.astype(np.float32))).astype(np.float64)
     assert np.all(err[~out_mask] <= bound[~out_mask])
     assert np.array_equal(dh[out_mask], x[out_mask].astype(np.float64))
+
+
+def test_ragged_prefill_equals_unpadded_cache():
+    """With r = 0 every token's reconstruction depends on that token alone, so
+    attention over a right-padded prefill with the padding masked must equal
+    attention over a cache built from the real tokens only (same appends). This
+    ties the masked path to an independently built cache, not to itself."""
+    rng = np.random.default_rng(17)
+    B, H, Hq, n0, d, nb = 3, 2, 4, 40, 128, 5
+    p = Params(bits=4, group_size=64, outlier_frac=0.05, rank=0, power_iters=1, buffer_len=nb, buffer_rank=0,
+               seed=3)
+    xk = rng.standard_normal((B, H, n0, d)).astype(np.float32)
+    xv = rng.standard_normal((B, H, n0, d)).astype(np.float32)
+    rows_k = [rng.standard_normal((B, H, d)).astype(np.float32) for _ in range(7)]
+    rows_v = [rng.standard_normal((B, H, d)).astype(np.float32) for _ in range(7)]
+    q = rng.standard_normal((B, Hq, d))
+    plen = [17, 40, 1]
+    pk, pv = oracle.Cache(p, B, H, d), oracle.Cache(p, B, H, d)
+    pk.encode(xk)
+    pv.encode(xv)
+    for rk, rv in zip(rows_k, rows_v):
+        pk.append(rk)
+        pv.append(rv)
+    got = oracle.decode_attn(pk, pv, q, 0.09, prefill_len=plen)
+    for b in range(B):
+        sk, sv = oracle.Cache(p, 1, H, d), oracle.Cache(p, 1, H, d)
+        sk.encode(xk[b:b + 1, :, :plen[b]])
+        sv.encode(xv[b:b + 1, :, :plen[b]])
+        for rk, rv in zip(rows_k, rows_v):
+            sk.append(rk[b:b + 1])
+            sv.append(rv[b:b + 1])
+        want = oracle.decode_attn(sk, sv, q[b:b + 1], 0.09)
+        assert np.array_equal(got[b], want[0]), b
+    # a full-length prefill is the plain decode
+    np.testing.assert_array_equal(oracle.decode_attn(pk, pv, q, 0.09, prefill_len=[n0] * B),
+                                  oracle.decode_attn(pk, pv, q, 0.09))
+
+
+def test_ragged_prefill_all_padding():
+    """Prefill length 0: only appended tokens count; with none, the output is 0."""
+    rng = np.random.default_rng(5)
+    B, H, d = 2, 1, 128
+    p = Params(bits=4, group_size=64, outlier_frac=0.02, rank=2, power_iters=2, buffer_len=4, buffer_rank=1, seed=1)
+    x = rng.standard_normal((B, H, 30, d)).astype(np.float32)
+    q = rng.standard_normal((B, H, d))
+    kc, vc = oracle.Cache(p, B, H, d), oracle.Cache(p, B, H, d)
+    kc.encode(x)
+    vc.encode(-x)
+    out = oracle.decode_attn(kc, vc, q, 0.1, prefill_len=[0, 30])
+    assert not out[0].any()
+    np.testing.assert_array_equal(out[1], oracle.decode_attn(kc, vc, q, 0.1)[1])
+    row = rng.standard_normal((B, H, d)).astype(np.float32)
+    kc.append(row)
+    vc.append(2 * row)
+    out = oracle.decode_attn(kc, vc, q, 0.1, prefill_len=[0, 0])
+    np.testing.assert_allclose(out[:, 0], 2 * row[:, 0], rtol=0, atol=1e-12)   # one real token: its value
