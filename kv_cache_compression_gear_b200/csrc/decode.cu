@@ -187,7 +187,8 @@ __device__ __forceinline__ void meta_row(const uint8_t* mrow, int G, int mx, flo
 // difference between the exact value and what codes + low rank give there:
 // fix = x_o - (zero_g(c_o) + L_t . Rf[c_o]). Rf rows are 16-byte vectors, so a
 // rank <= 4 block needs one load per outlier. All loads are issued together.
-constexpr int kFast = 4;
+// Three slots cover s <= 2 % of 128 channels; more outliers take the general loop.
+constexpr int kFast = 3;
 template <typename T, bool MF>
 __device__ __forceinline__ void outlier_fixes(const uint8_t* rest, int oval_off, const uint8_t* mrow, int mx, int t,
                                               int k, int lg, const float (&lt)[4], const float* rf, int rp,
@@ -724,17 +725,18 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         // ---------------- values: lane = 8 channels, tokens 2*i + par. Tokens
         // past nt have w = 0 (their codes are finite), so every tile runs all 16.
         {
-          // per-lane bases; every further offset is a compile-time constant
+          // per-lane bases advanced by constants; offsets inside a step are
+          // compile-time constants (the loop stays rolled to keep the code small)
           const uint8_t* vb[4];
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) vb[mm] = tvc + par * R + voff[mm];
           const float* wrow = w_s + (my_g * kWStride + par) * HQ;
-#pragma unroll
+#pragma unroll 1
           for (int i4 = 0; i4 < kDTile / 2; i4 += 4) {
 #pragma unroll
             for (int mm = 0; mm < 4; ++mm) {
-              const uint8_t* row = vb[mm] + (i4 + mm) * 2 * R;
-              const float* wr = wrow + (i4 + mm) * 2 * HQ;
+              const uint8_t* row = vb[mm] + mm * 2 * R;
+              const float* wr = wrow + mm * 2 * HQ;
               float f[8];
               if constexpr (BITS == 4) {
                 CF::word(*reinterpret_cast<const uint32_t*>(row), f, one);
@@ -759,6 +761,9 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
                 for (int e = 0; e < 4; ++e) acc[hh][e] = fma2(w2, pk2(f[2 * e], f[2 * e + 1]), acc[hh][e]);
               }
             }
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) vb[mm] += 8 * R;
+            wrow += 8 * HQ;
           }
         }
         __syncwarp();
