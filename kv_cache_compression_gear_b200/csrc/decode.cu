@@ -726,12 +726,13 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         // past nt have w = 0 (their codes are finite), so every tile runs all 16.
         {
           // per-lane bases advanced by constants; offsets inside a step are
-          // compile-time constants (the loop stays rolled to keep the code small)
+          // compile-time constants. With the outlier code compiled in, the loop
+          // stays rolled to keep the kernel inside the instruction cache.
           const uint8_t* vb[4];
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) vb[mm] = tvc + par * R + voff[mm];
           const float* wrow = w_s + (my_g * kWStride + par) * HQ;
-#pragma unroll 1
+#pragma unroll (OUT ? 1 : 4)
           for (int i4 = 0; i4 < kDTile / 2; i4 += 4) {
 #pragma unroll
             for (int mm = 0; mm < 4; ++mm) {
