@@ -48,7 +48,7 @@ def peaks():
 # DRAM bytes of one decode_warp launch on the decode workload, measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum of one launch); set to None
 # whenever the kernel changes, until it is captured again.
-DECODE_TRAFFIC_BYTES = 829613312 + 4008960
+DECODE_TRAFFIC_BYTES = 830936064 + 7828224
 
 
 def per_token_bytes(w, meta_f16: bool = False) -> int:

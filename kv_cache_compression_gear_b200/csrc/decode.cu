@@ -571,15 +571,25 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         float s_[HQ];
         {
           const uint8_t* crow = tkc + t * R;
-          uint64_t sb[HQ][4][2];   // per 32-channel block, two independent chains
+          // per 32-channel block: four independent f32x2 chains while the block's
+          // 16 bytes are read (one block per 16-byte load for 4-bit codes, then
+          // summed into fb), or two chains per block kept to the end otherwise
+          constexpr bool kOneBlk = CF::kPerWord * 4 == 32;
+          uint64_t sb[HQ][4][2];
+          float fb[HQ][4];
 #pragma unroll
           for (int hh = 0; hh < HQ; ++hh)
 #pragma unroll
-            for (int bk = 0; bk < 4; ++bk) { sb[hh][bk][0] = 0; sb[hh][bk][1] = 0; }
+            for (int bk = 0; bk < 4; ++bk) { sb[hh][bk][0] = 0; sb[hh][bk][1] = 0; fb[hh][bk] = 0.0f; }
 #pragma unroll
           for (int j = 0; j < W / 4; ++j) {
             const uint4 wv = *reinterpret_cast<const uint4*>(crow + ((j ^ xs) << 4));
             const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+            uint64_t c4[HQ][4];
+#pragma unroll
+            for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) c4[hh][e] = 0;
 #pragma unroll
             for (int wi = 0; wi < 4; ++wi) {
               const int cbase = (4 * j + wi) * CF::kPerWord;
@@ -592,11 +602,29 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
 #pragma unroll
                 for (int hh = 0; hh < HQ; ++hh) {
                   const float4 qv = *reinterpret_cast<const float4*>(qw_s + hh * 128 + cbase + e);
-                  sb[hh][bk][ch] = fma2(pk2(f[e], f[e + 1]), pk2(qv.x, qv.y), sb[hh][bk][ch]);
-                  sb[hh][bk][ch] = fma2(pk2(f[e + 2], f[e + 3]), pk2(qv.z, qv.w), sb[hh][bk][ch]);
+                  if constexpr (kOneBlk) {
+                    c4[hh][2 * ch] = fma2(pk2(f[e], f[e + 1]), pk2(qv.x, qv.y), c4[hh][2 * ch]);
+                    c4[hh][2 * ch + 1] = fma2(pk2(f[e + 2], f[e + 3]), pk2(qv.z, qv.w), c4[hh][2 * ch + 1]);
+                  } else {
+                    sb[hh][bk][ch] = fma2(pk2(f[e], f[e + 1]), pk2(qv.x, qv.y), sb[hh][bk][ch]);
+                    sb[hh][bk][ch] = fma2(pk2(f[e + 2], f[e + 3]), pk2(qv.z, qv.w), sb[hh][bk][ch]);
+                  }
                 }
               }
             }
+            if constexpr (kOneBlk) {
+#pragma unroll
+              for (int hh = 0; hh < HQ; ++hh)
+                fb[hh][j] = ((lo2(c4[hh][0]) + hi2(c4[hh][0])) + (lo2(c4[hh][1]) + hi2(c4[hh][1]))) +
+                            ((lo2(c4[hh][2]) + hi2(c4[hh][2])) + (lo2(c4[hh][3]) + hi2(c4[hh][3])));
+            }
+          }
+          if constexpr (!kOneBlk) {
+#pragma unroll
+            for (int hh = 0; hh < HQ; ++hh)
+#pragma unroll
+              for (int bk = 0; bk < 4; ++bk)
+                fb[hh][bk] = (lo2(sb[hh][bk][0]) + hi2(sb[hh][bk][0])) + (lo2(sb[hh][bk][1]) + hi2(sb[hh][bk][1]));
           }
           float2 sz[4];
           meta_row<MF>(kmrow, G, mx, sz);
@@ -611,7 +639,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
 #pragma unroll
               for (int bk = 0; bk < 4; ++bk)
                 if ((bk / bpg) == gi) {
-                  f += (lo2(sb[hh][bk][0]) + hi2(sb[hh][bk][0])) + (lo2(sb[hh][bk][1]) + hi2(sb[hh][bk][1]));
+                  f += fb[hh][bk];
                   qsw += qw_blk[hh][bk];
                   qss += qs_blk[hh][bk];
                 }
