@@ -1,21 +1,26 @@
 """Benchmark of the GEAR KV codec hot path on B200.
 
-One step = one pass over every stage of the path:
-  1. encode K and V of a LLaMA-7B-shaped layer (batch 1, 32 heads, 4096
-     tokens, d = 128, fp16; 4-bit, group 64, s = 2%, r = 4, T = 3),
-  2. one decode-attention step over a compressed cache of batch 16, 32 heads,
-     8192 tokens plus the full-precision buffer (fp16, softmax scale 1/sqrt(128)),
-  3. appending the new token to that cache (compressing the buffer whenever it
-     is full, i.e. every 20th step).
-`value` is the encode throughput in GB/s of fp16 KV input; the decode-attention
-throughput (tokens/s = sequences per second) is reported beside it. All inputs
-are synthetic and seeded (workloads/), resident in HBM before the timed region.
-L2 is flushed (a 512 MiB write) before every stage of every timed step.
+One step = one pass over every stage of the path on one workload:
+  1. encode the K and V tensors (outliers, group-wise quantization, power
+     iteration of the residual; every layer of the workload, batched),
+  2. one decode-attention step over the compressed caches plus their
+     full-precision buffers (softmax scale 1/sqrt(128)),
+  3. append one new token per layer (compressing a full buffer first).
+The headline workload is the 2-bit codec at high batch (batch 64, 32 heads,
+8192 tokens, fp16; 2-bit, group 32, s = 5%, r = 8, T = 3), the largest fp16
+configuration: `value` is its encode throughput in GB/s of fp16 KV input, and
+its decode-attention throughput (tokens/s = sequences per second) is reported
+beside it. The same fields follow under "configs" for the Llama-3-8B-shaped GQA
+cache (32 layers, bf16, 32768 tokens, 20-token buffer) and for the Llama-7B
+layer encode with the batch-16, 8192-token decode. All inputs are synthetic
+and seeded (workloads/), resident in HBM before the timed region. L2 is flushed
+(a 512 MiB write) before every stage of every timed step.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 For N > 1 launch under torch.distributed.run: every rank runs the same step on
 its own data (replicas, no collective on the data path); times are the max
-over ranks.
+over ranks. --batch-override B runs only the headline workload at batch B, the
+small case that counter captures use (its line is not a benchmark value).
 """
 from __future__ import annotations
 
@@ -43,12 +48,6 @@ def peaks():
         return float(j["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
-
-
-# DRAM bytes of one decode_warp launch on the decode workload, measured by ncu
-# (dram__bytes_read.sum + dram__bytes_write.sum of one launch); set to None
-# whenever the kernel changes, until it is captured again.
-DECODE_TRAFFIC_BYTES = 830936064 + 7828224
 
 
 def per_token_bytes(w, meta_f16: bool = False) -> int:
@@ -119,19 +118,83 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+# ---------------------------------------------------------------- scenarios
+@dataclasses.dataclass(frozen=True)
+class Scenario:
+    """One benchmark line: the encode workload, the decode workload (the same one
+    when the step decodes the cache it has just encoded) and its name."""
+    name: str
+    enc: str
+    dec: str
+
+    @property
+    def same(self) -> bool:
+        return self.enc == self.dec
+
+
+HEADLINE = Scenario("twobit_b64_ctx8192", "twobit_b64_ctx8192", "twobit_b64_ctx8192")
+BESIDE = [Scenario("llama3_8b_gqa", "llama3_8b_gqa", "llama3_8b_gqa"),
+          Scenario(f"{ENC} + {DEC}", ENC, DEC)]
+
+
+def scenario_config(sc: Scenario, world: int, batch_override: int | None = None) -> dict:
+    import workloads as wl
+    we, wd = wl.WORKLOADS[sc.enc], wl.WORKLOADS[sc.dec]
+
+    def desc(w, enc):
+        d = {"layers": w.layers, "batch": batch_override or w.B, "kv_heads": w.H, "q_heads": w.Hq,
+             "tokens" if enc else "context": w.n, "head_dim": w.d, "dtype": w.dtype, "bits": w.bits,
+             "group": w.group, "s": w.s, "rank": w.rank, "iters": w.iters}
+        if not enc:
+            d["buffer"] = w.buffer_fill
+        return d
+
+    cfg = {"workload": sc.name, "encode": desc(we, True), "decode": desc(wd, False),
+           "l2": "flushed (512 MiB write) before every timed stage; inputs of the two large configs exceed L2",
+           "parallelism": f"replicas x{world}"}
+    if batch_override:
+        cfg["batch_override"] = batch_override
+    return cfg
+
+
+def bench_config(world: int) -> dict:
+    """The headline workload both arms report."""
+    return scenario_config(HEADLINE, world)
+
+
 # ---------------------------------------------------------------- oracle arm
-def oracle_encode_gbps(seconds_budget: float = 12.0, units_cap: int = 64):
-    """The C oracle encoding units of the LLaMA-7B layer workload on all host
-    cores; returns (GB/s of fp16 input, cores, sample description)."""
+def _oparams(w):
+    import oracle
+    return oracle.Params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
+                         buffer_len=w.buffer_len, buffer_rank=w.buffer_rank, seed=w.seed)
+
+
+def _sample_units(w, count):
+    """(which, layer, b, h) of `count` units spread over the workload, K and V alternating."""
+    total = w.layers * w.B * w.H
+    out = []
+    for i in range(count):
+        u = (i * 7919) % total
+        layer, rem = divmod(u, w.B * w.H)
+        out.append(("k" if i % 2 == 0 else "v", layer, rem // w.H, rem % w.H))
+    return out
+
+
+def oracle_encode_gbps(wname: str, seconds_budget: float = 8.0, units_cap: int = 32, threads: int | None = None):
+    """The C oracle encoding a bounded sample of units of a workload on `threads`
+    host threads (all cores by default); returns (GB/s of KV input, threads, sample
+    description). The sample's throughput stands for the whole workload's (all units
+    cost the same)."""
     import oracle
     import workloads as wl
     from concurrent.futures import ThreadPoolExecutor
-    w = wl.WORKLOADS[ENC]
-    p = oracle.Params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
-                      buffer_len=w.buffer_len, buffer_rank=w.buffer_rank, seed=w.seed)
-    cores = os.cpu_count() or 1
-    jobs = [(which, h) for h in range(w.H) for which in ("k", "v")][:units_cap]
-    inputs = [wl.kv_unit_np(w, which, 0, 0, h) for which, h in jobs]
+    w = wl.WORKLOADS[wname]
+    p = _oparams(w)
+    cores = threads or os.cpu_count() or 1
+    jobs = _sample_units(w, units_cap)
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        inputs = list(ex.map(lambda j: wl.kv_unit_np(w, *j), jobs))
+    esz = 4 if w.dtype == "f32" else 2
     t0 = time.perf_counter()
     done = 0
     with ThreadPoolExecutor(max_workers=cores) as ex:
@@ -141,19 +204,65 @@ def oracle_encode_gbps(seconds_budget: float = 12.0, units_cap: int = 64):
             if time.perf_counter() - t0 > seconds_budget:
                 break
     dt = time.perf_counter() - t0
-    nbytes = done * w.n * w.d * 2
-    return nbytes / dt / 1e9, cores, f"{done} of {2 * w.H} (head, K/V) units of {ENC}, {w.n} tokens each"
+    nbytes = done * w.n * w.d * esz
+    return nbytes / dt / 1e9, cores, f"{done} units of {wname} ({w.n} tokens each), extrapolated"
 
 
-def bench_config(world: int) -> dict:
-    """The workload both arms report (the reference arm times its encode part)."""
+def oracle_decode_tps(wname: str, seconds_budget: float = 4.0, units_cap: int = 16, threads: int | None = None):
+    """The C oracle's decode attention (reconstruct K and V of a unit from its
+    encoding, then softmax attention for every query head of the unit) on a bounded
+    sample of units, scaled to a whole decode step of the workload (all layers,
+    batches and kv heads); returns (tokens/s = sequences per second, threads, sample)."""
+    import numpy as np
+    import oracle
     import workloads as wl
-    we, wd = wl.WORKLOADS[ENC], wl.WORKLOADS[DEC]
-    return {"workload": f"{ENC} + {DEC}",
-            "encode": {"batch": we.B, "heads": we.H, "tokens": we.n, "head_dim": we.d, "bits": we.bits,
-                       "group": we.group, "s": we.s, "rank": we.rank, "iters": we.iters},
-            "decode": {"batch": wd.B, "heads": wd.H, "context": wd.n, "buffer": wd.buffer_len},
-            "l2": "flushed (512 MiB write) before every timed stage", "parallelism": f"replicas x{world}"}
+    from concurrent.futures import ThreadPoolExecutor
+    w = wl.WORKLOADS[wname]
+    p = _oparams(w)
+    cores = threads or os.cpu_count() or 1
+    hq = w.Hq // w.H
+    jobs = [(layer, b, h) for (_, layer, b, h) in _sample_units(w, units_cap)]
+
+    def prep(j):
+        layer, b, h = j
+        return (oracle.encode_unit(wl.kv_unit_np(w, "k", layer, b, h), p),
+                oracle.encode_unit(wl.kv_unit_np(w, "v", layer, b, h), p),
+                wl.rows_np(w, wl.S_Q, layer, 0, w.Hq)[b, h * hq:(h + 1) * hq])
+
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        enc = list(ex.map(prep, jobs))
+    tau = 1.0 / math.sqrt(w.d)
+
+    def dec(e):
+        ku, vu, q = e
+        K = oracle.reconstruct_unit(ku, p)
+        V = oracle.reconstruct_unit(vu, p)
+        return [oracle.attention(q[j], K, V, tau) for j in range(q.shape[0])]
+
+    t0 = time.perf_counter()
+    done = 0
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        for i in range(0, len(enc), cores):
+            list(ex.map(dec, enc[i:i + cores]))
+            done += len(enc[i:i + cores])
+            if time.perf_counter() - t0 > seconds_budget:
+                break
+    dt = time.perf_counter() - t0
+    units_per_step = w.layers * w.B * w.H
+    step_s = dt / done * units_per_step
+    np.asarray(0)
+    return w.B / step_s, cores, f"{done} units of {wname} (K and V reconstructed, {hq} query heads each), scaled to {units_per_step} units per step"
+
+
+def cpu_baseline(sc: Scenario) -> dict:
+    enc_all, cores, enc_sample = oracle_encode_gbps(sc.enc)
+    enc_one, _, enc_sample1 = oracle_encode_gbps(sc.enc, seconds_budget=2.0, units_cap=2, threads=1)
+    dec_all, _, dec_sample = oracle_decode_tps(sc.dec)
+    dec_one, _, _ = oracle_decode_tps(sc.dec, seconds_budget=1.0, units_cap=2, threads=1)
+    return {"value": round(enc_all, 6), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": enc_sample,
+            "single_thread": {"value": round(enc_one, 6), "unit": "GB/s", "cores": 1, "sample": enc_sample1},
+            "decode": {"value": round(dec_all, 3), "unit": "tokens/s", "cores": cores, "sample": dec_sample,
+                       "single_thread": round(dec_one, 3)}}
 
 
 def max_over_ranks(v: float, world: int, device) -> float:
@@ -173,11 +282,11 @@ def run_reference(args, rank: int, world: int):
     vals = []
     cores, sample = None, None
     for _ in range(args.warmup):
-        oracle_encode_gbps(seconds_budget=3.0, units_cap=8)
+        oracle_encode_gbps(HEADLINE.enc, seconds_budget=2.0, units_cap=4)
     step_ms = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        v, cores, sample = oracle_encode_gbps(seconds_budget=6.0, units_cap=16)
+        v, cores, sample = oracle_encode_gbps(HEADLINE.enc, seconds_budget=4.0, units_cap=16)
         step_ms.append((time.perf_counter() - t0) * 1e3)
         vals.append(v)
     v = statistics.median(vals)
@@ -193,82 +302,206 @@ def run_reference(args, rank: int, world: int):
 
 
 # ---------------------------------------------------------------- GPU arm
-def run_gpu(args, rank: int, world: int):
-    import torch
-    import kv_cache_compression_gear_b200 as gear
-    import workloads as wl
+def _gparams(gear, w, meta_f16=False):
+    return gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
+                            buffer_len=w.buffer_len, buffer_rank=w.buffer_rank, seed=w.seed, meta_f16=meta_f16)
 
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    we, wd = wl.WORKLOADS[ENC], wl.WORKLOADS[DEC]
 
-    def params(w):
-        return gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank,
-                                power_iters=w.iters, buffer_len=w.buffer_len, buffer_rank=w.buffer_rank,
-                                seed=w.seed)
+def enc_alg_bytes(w, n_tensors: int) -> int:
+    """Algorithmic bytes of encoding n_tensors tensors shaped like w: the input
+    read once, the compressed tokens and the Rf rows written once."""
+    esz = 4 if w.dtype == "f32" else 2
+    units = w.B * w.H
+    return n_tensors * units * (w.n * (w.d * esz + per_token_bytes(w)) + w.d * ((w.rank + 3) // 4 * 4) * 4)
 
-    # ---- encode workload (per-rank layer index so ranks hold different data)
-    pe = params(we)
-    xk = wl.kv_tensor_torch(we, "k", rank, dev)
-    xv = wl.kv_tensor_torch(we, "v", rank, dev)
-    enc_k = gear.Cache(pe, we.B, we.H, we.n, 1, torch.float16, dev)
-    enc_v = gear.Cache(pe, we.B, we.H, we.n, 1, torch.float16, dev)
-    # ---- decode workload: compressed context + full buffer, room for the appends
-    pd = params(wd)
-    n_steps_total = args.warmup + args.steps + 1
-    n_max = wd.n + wd.buffer_len * (2 + n_steps_total // wd.buffer_len)
-    nblk = 2 + n_steps_total // wd.buffer_len
-    dk = gear.Cache(pd, wd.B, wd.H, n_max, nblk, torch.float16, dev)
-    dv = gear.Cache(pd, wd.B, wd.H, n_max, nblk, torch.float16, dev)
-    t = wl.kv_tensor_torch(wd, "k", rank, dev)
-    dk.encode(t)
-    del t
-    t = wl.kv_tensor_torch(wd, "v", rank, dev)
-    dv.encode(t)
-    del t
-    for i in range(wd.buffer_fill):
-        gear.append_buffer(dk, dv, wl.rows_torch(wd, wl.S_KBUF, rank, i, wd.H, dev),
-                           wl.rows_torch(wd, wl.S_VBUF, rank, i, wd.H, dev))
-    q = wl.rows_torch(wd, wl.S_Q, rank, 0, wd.Hq, dev)
-    new_k = [wl.rows_torch(wd, wl.S_KNEW, rank, i, wd.H, dev) for i in range(n_steps_total)]
-    new_v = [wl.rows_torch(wd, wl.S_VNEW, rank, i, wd.H, dev) for i in range(n_steps_total)]
-    tau = 1.0 / math.sqrt(128)
-    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    out = torch.empty((wd.B, wd.Hq, 128), dtype=torch.float16, device=dev)
-    torch.cuda.synchronize()
 
-    def reset_encode_caches():
-        for c in (enc_k, enc_v):
-            c.c.n_comp = c.c.n_buf = c.c.n_blk = c.c.blk0_len = c.c.blk0_rank = 0
+def dec_alg_bytes(w, n_comp: int, n_blk: int, n_buf: int, layers: int) -> int:
+    """Algorithmic bytes of one decode step: K and V compressed tokens, their Rf
+    rows and buffers read once, q read and the output written once."""
+    esz = 4 if w.dtype == "f32" else 2
+    units = w.B * w.H
+    rp = (max(w.rank, w.buffer_rank) + 3) // 4 * 4
+    per_layer = (2 * units * n_comp * per_token_bytes(w) + 2 * units * n_blk * rp * 128 * 4
+                 + 2 * units * n_buf * 128 * esz + 2 * w.B * w.Hq * 128 * esz)
+    return layers * per_layer
 
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    step_idx = [0]
 
-    def one_step(record):
-        s = step_idx[0]
-        step_idx[0] += 1
-        reset_encode_caches()
-        flush_buf.fill_(s & 0xFF)
+class Runner:
+    """Holds the device state of one scenario and runs its steps."""
+
+    def __init__(self, gear, wl, sc: Scenario, dev, rank: int, n_steps_total: int, batch_override=None):
+        import torch
+        self.gear, self.wl, self.sc, self.dev = gear, wl, sc, dev
+        we, wd = wl.WORKLOADS[sc.enc], wl.WORKLOADS[sc.dec]
+        if batch_override:
+            we = dataclasses.replace(we, B=batch_override)
+            wd = dataclasses.replace(wd, B=batch_override) if not sc.same else we
+        self.we, self.wd = we, wd
+        dt = wl.torch_dtype(we.dtype)
+        # ---- encode inputs and caches (per layer: K and V); rank r selects the data
+        pe = _gparams(gear, we)
+        L = we.layers
+        if sc.same:
+            n_max, nblk = we.n + 2 * we.buffer_len, 2
+        else:
+            n_max, nblk = we.n, 1
+        self.x, self.enc = [], []
+        for layer in range(L):
+            for which in ("k", "v"):
+                self.x.append(wl.kv_tensor_torch(we, which, rank * L + layer, dev))
+                self.enc.append(gear.Cache(pe, we.B, we.H, n_max, nblk, dt, dev))
+        if sc.same:
+            self.dk, self.dv = self.enc[0::2], self.enc[1::2]
+        else:
+            # persistent decode caches: compressed context + full buffer, room for the appends
+            pd = _gparams(gear, wd)
+            n_max = wd.n + wd.buffer_len * (2 + n_steps_total // wd.buffer_len)
+            nblk = 2 + n_steps_total // wd.buffer_len
+            self.dk, self.dv = [], []
+            for layer in range(wd.layers):
+                kc = gear.Cache(pd, wd.B, wd.H, n_max, nblk, dt, dev)
+                vc = gear.Cache(pd, wd.B, wd.H, n_max, nblk, dt, dev)
+                for c, which in ((kc, "k"), (vc, "v")):
+                    t = wl.kv_tensor_torch(wd, which, rank * wd.layers + layer, dev)
+                    c.encode(t)
+                    del t
+                self.dk.append(kc)
+                self.dv.append(vc)
+                self.fill_buffer(layer, rank)
+        self.q = [wl.rows_torch(wd, wl.S_Q, rank * wd.layers + layer, 0, wd.Hq, dev) for layer in range(wd.layers)]
+        self.new_k = [[wl.rows_torch(wd, wl.S_KNEW, rank * wd.layers + layer, i, wd.H, dev)
+                       for i in range(n_steps_total)] for layer in range(wd.layers)]
+        self.new_v = [[wl.rows_torch(wd, wl.S_VNEW, rank * wd.layers + layer, i, wd.H, dev)
+                       for i in range(n_steps_total)] for layer in range(wd.layers)]
+        self.out = [torch.empty((wd.B, wd.Hq, 128), dtype=dt, device=dev) for _ in range(wd.layers)]
+        self.flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.tau = 1.0 / math.sqrt(128)
+        self.rank = rank
+        self.step_idx = 0
+        torch.cuda.synchronize()
+
+    def fill_buffer(self, layer, rank):
+        wl, wd = self.wl, self.wd
+        for i in range(wd.buffer_fill):
+            self.gear.append_buffer(self.dk[layer], self.dv[layer],
+                                    wl.rows_torch(wd, wl.S_KBUF, rank * wd.layers + layer, i, wd.H, self.dev),
+                                    wl.rows_torch(wd, wl.S_VBUF, rank * wd.layers + layer, i, wd.H, self.dev))
+
+    def encode(self, xs=None):
+        for c in self.enc:
+            c.reset()
+        self.gear.encode_batch(self.enc, xs or self.x)
+
+    def decode(self, qs=None):
+        for layer in range(self.wd.layers):
+            self.gear.decode_attn(self.dk[layer], self.dv[layer], (qs or self.q)[layer], self.tau,
+                                  out=self.out[layer])
+
+    def step(self, record):
+        """encode, (buffer fill, untimed), decode, append; CUDA events around each stage."""
+        import torch
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        s = self.step_idx
+        self.step_idx += 1
+        self.flush.fill_(s & 0xFF)
         e0, e1 = ev(), ev()
         e0.record()
-        gear.encode_batch([enc_k, enc_v], [xk, xv])
+        self.encode()
         e1.record()
-        flush_buf.fill_((s + 1) & 0xFF)
+        if self.sc.same:
+            for layer in range(self.wd.layers):
+                self.fill_buffer(layer, self.rank)
+        self.flush.fill_((s + 1) & 0xFF)
         d0, d1 = ev(), ev()
         d0.record()
-        gear.decode_attn(dk, dv, q, tau, out=out)
+        self.decode()
         d1.record()
-        flush_buf.fill_((s + 2) & 0xFF)
+        self.flush.fill_((s + 2) & 0xFF)
+        flushed = self.dk[0].n_buf == self.wd.buffer_len
         a0, a1 = ev(), ev()
-        flushed = dk.n_buf == wd.buffer_len
         a0.record()
-        gear.append_buffer(dk, dv, new_k[s], new_v[s])
+        for layer in range(self.wd.layers):
+            self.gear.append_buffer(self.dk[layer], self.dv[layer], self.new_k[layer][s], self.new_v[layer][s])
         a1.record()
         if record is not None:
             record.append((e0, e1, d0, d1, a0, a1, flushed))
 
-    for _ in range(args.warmup):
-        one_step(None)
+    def launches_per_step(self, flushed: bool) -> int:
+        n_enc = len(self.enc)
+        enc = 3 * ((n_enc + 15) // 16)
+        dec = 2 * self.wd.layers
+        app = self.wd.layers * (1 + (3 if flushed else 0))
+        return enc + dec + app
+
+    def e2e(self, reps: int):
+        """Encode and decode through the public API with the inputs in pinned host
+        memory: host-to-device copies inside the timed region, the attention output
+        read back to the host. Returns (encode s, decode s, h2d bytes, d2h bytes) or
+        None when the host cannot hold a pinned copy of the inputs."""
+        import torch
+        in_bytes = sum(x.numel() * x.element_size() for x in self.x)
+        try:
+            import psutil
+            avail = psutil.virtual_memory().available
+        except Exception:
+            avail = 0
+        if avail < 2 * in_bytes + (16 << 30):
+            return None
+        hx = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in self.x]
+        for h, x in zip(hx, self.x):
+            h.copy_(x)
+        hq = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for q in self.q]
+        for h, q in zip(hq, self.q):
+            h.copy_(q)
+        hout = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in self.out]
+        dx = [torch.empty_like(x) for x in self.x]
+        dq = [torch.empty_like(q) for q in self.q]
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        te, td = [], []
+        for it in range(reps + 1):
+            self.flush.fill_(7)
+            a, b, c, d = ev(), ev(), ev(), ev()
+            a.record()
+            for h, x in zip(hx, dx):
+                x.copy_(h, non_blocking=True)
+            self.encode(dx)
+            b.record()
+            if self.sc.same:
+                for layer in range(self.wd.layers):
+                    self.fill_buffer(layer, self.rank)
+            c.record()
+            for h, q in zip(hq, dq):
+                q.copy_(h, non_blocking=True)
+            self.decode(dq)
+            for h, o in zip(hout, self.out):
+                h.copy_(o, non_blocking=True)
+            d.record()
+            torch.cuda.synchronize()
+            if it > 0:
+                te.append(a.elapsed_time(b) / 1e3)
+                td.append(c.elapsed_time(d) / 1e3)
+        del dx, hx
+        h2d = in_bytes + sum(q.numel() * q.element_size() for q in self.q)
+        d2h = sum(o.numel() * o.element_size() for o in self.out)
+        return statistics.median(te), statistics.median(td), h2d, d2h
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a
+# stage's dominant kernel, from one ncu capture each (profiles/), keyed by
+# (scenario, stage); an entry is removed whenever its kernel changes, until it is
+# captured again.
+TRAFFIC_BYTES = {
+    (f"{ENC} + {DEC}", "decode"): 830936064 + 7828224,
+}
+
+
+def measure(gear, wl, sc: Scenario, dev, rank, world, steps, warmup, hbm, peak_kind, batch_override=None,
+            with_e2e=True):
+    import torch
+    runner = Runner(gear, wl, sc, dev, rank, warmup + steps + 1, batch_override)
+    we, wd = runner.we, runner.wd
+    for _ in range(warmup):
+        runner.step(None)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -276,98 +509,105 @@ def run_gpu(args, rank: int, world: int):
     clocks.start()
     recs = []
     torch.cuda.synchronize()
-    for _ in range(args.steps):
-        one_step(recs)
+    for _ in range(steps):
+        runner.step(recs)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    enc_ms = [r[0].elapsed_time(r[1]) for r in recs]
-    dec_ms = [r[2].elapsed_time(r[3]) for r in recs]
-    app_ms = [r[4].elapsed_time(r[5]) for r in recs]
-    nflush = sum(1 for r in recs if r[6])
     assert gear.device_status() == 0, "device-side error word set"
+    enc_t = max_over_ranks(sum(r[0].elapsed_time(r[1]) for r in recs) / 1e3, world, dev)
+    dec_t = max_over_ranks(sum(r[2].elapsed_time(r[3]) for r in recs) / 1e3, world, dev)
+    app_t = max_over_ranks(sum(r[4].elapsed_time(r[5]) for r in recs) / 1e3, world, dev)
+    nflush = sum(1 for r in recs if r[6])
+    launches = sum(runner.launches_per_step(r[6]) for r in recs)
+    n_comp, n_blk, n_buf = runner.dk[0].n_comp, runner.dk[0].n_blk, runner.dk[0].n_buf
+    ee = runner.e2e(max(3, steps // 4)) if with_e2e else None
+    if ee is not None:
+        ee = tuple(max_over_ranks(v, world, dev) for v in ee[:2]) + ee[2:]
+    del runner
+    torch.cuda.empty_cache()
 
-    # ---- end to end through the public API with host buffers
-    hk = xk.cpu().pin_memory()
-    hv = xv.cpu().pin_memory()
-    hq = q.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dxk, dxv, dq = torch.empty_like(xk), torch.empty_like(xv), torch.empty_like(q)
-    e2e_enc, e2e_dec = [], []
-    for _ in range(max(3, args.steps // 2)):
-        reset_encode_caches()
-        flush_buf.fill_(7)
-        a, b, c, d = ev(), ev(), ev(), ev()
-        a.record()
-        dxk.copy_(hk, non_blocking=True)
-        dxv.copy_(hv, non_blocking=True)
-        gear.encode_batch([enc_k, enc_v], [dxk, dxv])
-        b.record()
-        c.record()
-        dq.copy_(hq, non_blocking=True)
-        gear.decode_attn(dk, dv, dq, tau, out=out)
-        hout.copy_(out, non_blocking=True)
-        d.record()
-        torch.cuda.synchronize()
-        e2e_enc.append(a.elapsed_time(b))
-        e2e_dec.append(c.elapsed_time(d))
-
-    def maxrank(v):
-        return max_over_ranks(v, world, dev)
-
-    enc_t = maxrank(sum(enc_ms) / 1e3)
-    dec_t = maxrank(sum(dec_ms) / 1e3)
-    app_t = maxrank(sum(app_ms) / 1e3)
-    e2e_enc_t = maxrank(statistics.median(e2e_enc) / 1e3)
-    e2e_dec_t = maxrank(statistics.median(e2e_dec) / 1e3)
-    if rank != 0:
-        return
-
-    K = args.steps
-    enc_in_bytes = 2 * we.B * we.H * we.n * we.d * 2                  # K and V, fp16
-    value = world * K * enc_in_bytes / enc_t / 1e9
-    dec_tps = world * K * wd.B / dec_t
-    hbm, peak_kind = peaks()
-    # algorithmic bytes: encode reads the input once and writes the compressed form once
-    enc_alg = 2 * (we.B * we.H * we.n * (we.d * 2 + per_token_bytes(we)) + we.B * we.H * we.d * we.rank * 4)
-    n_comp = dk.n_comp
-    dec_alg = (2 * wd.B * wd.H * n_comp * per_token_bytes(wd) + 2 * wd.B * wd.H * dk.n_blk * wd.rank * 128 * 4
-               + 2 * wd.B * wd.H * wd.buffer_fill * 128 * 2 + 2 * wd.B * wd.Hq * 128 * 2)
+    K = steps
+    esz = 4 if we.dtype == "f32" else 2
+    n_enc_tensors = 2 * we.layers
+    enc_in = n_enc_tensors * we.B * we.H * we.n * we.d * esz
+    # algorithmic bytes as the decode stage saw them: before the step's append
+    # (the step's own append always follows its decode)
+    if sc.same:
+        dec_alg = dec_alg_bytes(wd, wd.n, 1, wd.buffer_fill, wd.layers)
+    else:
+        dec_alg = dec_alg_bytes(wd, n_comp, n_blk, n_buf, wd.layers)
+    enc_alg = enc_alg_bytes(we, n_enc_tensors)
     enc_gbs = enc_alg / (enc_t / K) / 1e9
     dec_gbs = dec_alg / (dec_t / K) / 1e9
-    dominant = "decode" if dec_t >= enc_t else "encode"
-    roof = {"bound": "hbm", "kernel": "gear_decode_attn" if dominant == "decode" else "gear_encode",
-            "achieved": round(dec_gbs if dominant == "decode" else enc_gbs, 2), "peak": hbm,
-            "unit": "GB/s", "frac": round((dec_gbs if dominant == "decode" else enc_gbs) / hbm, 4),
-            "peak_kind": peak_kind,
-            "traffic": DECODE_TRAFFIC_BYTES if dominant == "decode" else None}
-    other = {"kernel": "gear_encode" if dominant == "decode" else "gear_decode_attn",
-             "achieved": round(enc_gbs if dominant == "decode" else dec_gbs, 2),
-             "frac": round((enc_gbs if dominant == "decode" else dec_gbs) / hbm, 4)}
-    line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round((enc_t + dec_t + app_t) / K * 1e3, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-        "data": "synthetic (seeded, workloads/)",
-        "config": bench_config(world),
-        "decode_tokens_per_s": round(dec_tps, 1),
+    stages = {"encode": (enc_t, enc_gbs, "gear_encode"), "decode": (dec_t, dec_gbs, "gear_decode_attn")}
+    dom = "decode" if dec_t >= enc_t else "encode"
+    oth = "encode" if dom == "decode" else "decode"
+    roof = {"bound": "hbm", "kernel": stages[dom][2], "achieved": round(stages[dom][1], 2), "peak": hbm,
+            "unit": "GB/s", "frac": round(stages[dom][1] / hbm, 4), "peak_kind": peak_kind,
+            "traffic": TRAFFIC_BYTES.get((sc.name, dom)),
+            "algorithmic_bytes": enc_alg if dom == "encode" else dec_alg}
+    other = {"kernel": stages[oth][2], "achieved": round(stages[oth][1], 2), "frac": round(stages[oth][1] / hbm, 4),
+             "traffic": TRAFFIC_BYTES.get((sc.name, oth)),
+             "algorithmic_bytes": enc_alg if oth == "encode" else dec_alg}
+    res = {
+        "value": round(world * K * enc_in / enc_t / 1e9, 3), "unit": "GB/s",
+        "ms_per_step": round((enc_t + dec_t + app_t) / K * 1e3, 4),
+        "decode_tokens_per_s": round(world * K * wd.B / dec_t, 1),
         "stage_ms": {"encode": round(enc_t / K * 1e3, 4), "decode": round(dec_t / K * 1e3, 4),
                      "append": round(app_t / K * 1e3, 4), "appends_with_flush": nflush},
         "roofline": roof, "roofline_other": other,
-        "e2e": {"value": round(world * enc_in_bytes / e2e_enc_t / 1e9, 3), "unit": "GB/s",
-                "h2d_bytes_per_step": enc_in_bytes + wd.B * wd.Hq * 128 * 2,
-                "d2h_bytes_per_step": wd.B * wd.Hq * 128 * 2,
-                "decode_tokens_per_s": round(world * wd.B / e2e_dec_t, 1)},
-        "gpu_launches": K * (3 + 2 + 1) + nflush * 3,
-        "clocks": clk,
+        "gpu_launches": launches, "clocks": clk,
+    }
+    if ee is not None:
+        te, td, h2d, d2h = ee
+        res["e2e"] = {"value": round(world * enc_in / te / 1e9, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "decode_tokens_per_s": round(world * wd.B / td, 1)}
+    else:
+        res["e2e"] = {"value": None, "unit": "GB/s", "skipped": "host memory cannot hold a pinned copy of the inputs"}
+    return res
+
+
+def run_gpu(args, rank: int, world: int):
+    import torch
+    import kv_cache_compression_gear_b200 as gear
+    import workloads as wl
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    hbm, peak_kind = peaks()
+    if args.batch_override:
+        # a smaller batch of the headline workload, for counter captures only (not a bench value)
+        res = measure(gear, wl, HEADLINE, dev, rank, world, args.steps, args.warmup, hbm, peak_kind,
+                      batch_override=args.batch_override, with_e2e=False)
+        if rank == 0:
+            print(json.dumps({"profile_case": scenario_config(HEADLINE, world, args.batch_override), **res}),
+                  flush=True)
+        return
+    head = measure(gear, wl, HEADLINE, dev, rank, world, args.steps, args.warmup, hbm, peak_kind)
+    beside = {}
+    for sc in BESIDE:
+        beside[sc.name] = measure(gear, wl, sc, dev, rank, world, max(3, args.steps // 2), 3, hbm, peak_kind)
+        beside[sc.name]["config"] = scenario_config(sc, world)
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded, workloads/)",
+        "config": bench_config(world),
+        **{k: v for k, v in head.items() if k not in ("value", "unit", "ms_per_step")},
+        "configs": beside,
     }
     if world == 1:
-        line["gear_l"] = variant_measure(gear, wl, we, wd, dev, max(3, K // 2), hbm, s=0.0)
-        line["meta_f16"] = variant_measure(gear, wl, we, wd, dev, max(3, K // 2), hbm, s=we.s, meta_f16=True)
-        v, cores, sample = oracle_encode_gbps()
-        line["cpu_baseline"] = {"value": round(v, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        we, wd = wl.WORKLOADS[ENC], wl.WORKLOADS[DEC]
+        line["gear_l"] = variant_measure(gear, wl, we, wd, dev, max(3, args.steps // 2), hbm, s=0.0)
+        line["meta_f16"] = variant_measure(gear, wl, we, wd, dev, max(3, args.steps // 2), hbm, s=we.s,
+                                           meta_f16=True)
+        line["cpu_baseline"] = cpu_baseline(HEADLINE)
+        for sc in BESIDE:
+            line["configs"][sc.name]["cpu_baseline"] = cpu_baseline(sc)
     print(json.dumps(line), flush=True)
 
 
@@ -446,6 +686,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="gear", choices=["gear", "reference"])
+    ap.add_argument("--batch-override", type=int, default=None,
+                    help="run only the headline workload at this batch (a small case for counter captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

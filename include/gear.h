@@ -157,6 +157,13 @@ gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int3
                             int32_t d, int32_t n_max, int32_t nblk_max, gear_dtype dtype,
                             void* dev, size_t bytes);
 
+/* Empties a cache for reuse with the same geometry and parameters: sets the
+ * counters (n_comp, n_buf, n_blk, blk0_len, blk0_rank) to zero, so that the
+ * next gear_encode writes block 0 again. Host bookkeeping only: writes no device
+ * memory and enqueues nothing (the old contents are simply overwritten by the
+ * next encode and appends). Errors: INVALID_ARG (null). */
+gear_status gear_cache_reset(gear_cache* c);
+
 /* Workspace bytes gear_encode needs to encode n tokens per unit of c. */
 size_t gear_encode_workspace_bytes(const gear_cache* c, int32_t n);
 
@@ -227,7 +234,11 @@ gear_status gear_decode_attn_ragged(const gear_cache* k, const gear_cache* v, co
  * holds until the process exits. The caller still passes q and out.
  * Limit: returns GEAR_ERR_WORKSPACE, enqueuing nothing, when the partials would
  * not fit, i.e. when gear_decode_workspace_bytes(k, v, Hq) > 4 MiB (each of the
- * B * Hq query rows needs 520 bytes per split).
+ * B * Hq query rows needs 520 bytes per split). The number of splits follows
+ * from the device's SM count (the split-K grid is one wave of resident warps),
+ * so whether a problem fits depends on the device: a caller that must know in
+ * advance checks gear_decode_workspace_bytes(k, v, Hq) <= 4 MiB with the target
+ * device current.
  * Set-up: the first call on a device looks up the array's device address with
  * cudaGetSymbolAddress and caches it; make that first call before any stream
  * capture. All calls share the one array and it keeps the last call's contents:

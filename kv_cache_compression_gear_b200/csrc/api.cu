@@ -14,13 +14,16 @@
 namespace gear {
 __device__ int32_t g_device_status = 0;
 
+// SM count of the current device, cached per device (host threads may fill a
+// slot concurrently with the same value).
 static int current_sm_count() {
-  static int cached[256];
+  static std::atomic<int> cached[kMaxDevices];
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 256 && cached[dev] > 0) return cached[dev];
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  if (dev >= 0 && dev < 256) cached[dev] = n;
+  if (slot) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -225,6 +228,12 @@ gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int3
   c->lfac = base + L.lfac;
   c->rfac = reinterpret_cast<float*>(base + L.rfac);
   c->buf = base + L.buf;
+  return GEAR_OK;
+}
+
+gear_status gear_cache_reset(gear_cache* c) {
+  if (!c) return GEAR_ERR_INVALID_ARG;
+  c->n_comp = c->n_buf = c->n_blk = c->blk0_len = c->blk0_rank = 0;
   return GEAR_OK;
 }
 

@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/gear.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -275,6 +277,32 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16, bool a_mn, bool b_mn) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((a_mn ? 1u : 0u) << 15) |
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- launch set-up
+// cudaFuncSetAttribute acts on the CURRENT device only, so a kernel's dynamic
+// shared-memory limit has to be raised once on every device that launches it.
+// Each launch site keeps one slot per device (devices 0 .. kMaxDevices-1)
+// holding the largest size already set there. Host threads may race to set the
+// same attribute, which is harmless; the slots are atomics so that the race is
+// well defined. Devices beyond the table are set on every launch.
+constexpr int kMaxDevices = 64;
+
+template <typename Kern>
+inline cudaError_t ensure_smem_limit(Kern kern, int bytes, std::atomic<int> (&slots)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && slots[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (cached) {
+    int cur = slots[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !slots[dev].compare_exchange_weak(cur, bytes, std::memory_order_release)) {
+    }
+  }
+  return cudaSuccess;
 }
 
 // ---------------------------------------------------------------- misc

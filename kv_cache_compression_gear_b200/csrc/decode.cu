@@ -973,13 +973,9 @@ size_t decode_workspace_bytes(int B, int Hq, int nsplit) { return (size_t)B * Hq
 template <typename T, int BITS, int HQ, bool OUT, bool MF>
 static cudaError_t launch_warp(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = 1024 + 16 * (size_t)a.tl.cb + 4 * (size_t)a.tl.bytes;
-  static int configured_smem = 0;
-  if ((int)smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(decode_warp<T, BITS, HQ, OUT, MF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    configured_smem = (int)smem;
-  }
+  static std::atomic<int> smem_set[kMaxDevices];   // per device: the limit is a per-device setting
+  cudaError_t e = ensure_smem_limit(decode_warp<T, BITS, HQ, OUT, MF>, (int)smem, smem_set);
+  if (e != cudaSuccess) return e;
   const int grid = (a.total_splits + 3) / 4;
   decode_warp<T, BITS, HQ, OUT, MF><<<grid, kDThreads, smem, st>>>(maps, a);
   return cudaGetLastError();

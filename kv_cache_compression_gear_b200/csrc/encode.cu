@@ -132,14 +132,6 @@ __device__ __forceinline__ uint32_t pair_max(uint32_t a, uint32_t b) {
 // Dev. 34(1), 1990: q1 = RN(q0 + r y), r = a - s q0, equals RN(a/s) whenever
 // q0 is within one ulp and a/s is normal). Only rint(q) is used and only
 // q >= 1/4 can round to a non-zero code, where all operands are normal.
-// Otherwise the correctly rounded division intrinsic is used.
-// Correctly rounded a / s for the code decision. When 2^-100 <= s <= 2^100
-// (so s and y = RN(1/s) are normal), the quotient is refined from the
-// correctly rounded reciprocal with one exact remainder (Markstein, "Computation
-// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
-// Dev. 34(1), 1990: q1 = RN(q0 + r y), r = a - s q0, equals RN(a/s) whenever
-// q0 is within one ulp and a/s is normal). Only rint(q) is used and only
-// q >= 1/4 can round to a non-zero code, where all operands are normal.
 // Otherwise the correctly rounded division intrinsic is used (slow path).
 __device__ __forceinline__ uint64_t div_pair_fast(uint64_t a, uint64_t s2n, uint64_t y2) {
   const uint64_t q0 = f2_mul(a, y2);
@@ -740,10 +732,16 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
     S.Q[e] = v;
   }
   __syncthreads();
-  bool ok = true;
   for (int sg = 0; sg < nseg; ++sg) {
     const int b = sg & 1;
-    ok = mbar_wait(&S.bar[b], (sg >> 1) & 1) && ok;
+    // a wait that gives up (error word set) ends the unit: no factors are
+    // computed from an incomplete Gram; the other stage's copy, if one was
+    // issued, is given its own bounded wait so that nothing lands after exit
+    if (!__syncthreads_and(mbar_wait(&S.bar[b], (sg >> 1) & 1))) {
+      if (tid == 0 && sg + 1 < nseg) mbar_wait(&S.bar[b ^ 1], ((sg + 1) >> 1) & 1);
+      __syncthreads();
+      return;
+    }
     for (int e4 = tid; e4 < 4096; e4 += kE2Threads) {
       const float4 v = reinterpret_cast<const float4*>(S.u.stage[b])[e4];
       float4* dst = reinterpret_cast<float4*>(&S.M[(e4 >> 5) * kMStride + ((e4 & 31) << 2)]);   // 16-byte aligned rows
@@ -760,7 +758,6 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
       bulk_load(S.u.stage[b], part + (int64_t)(sg + 2) * 16384, 65536, &S.bar[b]);
     }
   }
-  (void)ok;
   for (int e = tid; e < 128 * 128; e += kE2Threads) {
     const int i = e >> 7, j = e & 127;
     if (i < j) {
@@ -1161,12 +1158,9 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
 template <typename T, int BITS, int KMAX>
 static cudaError_t launch_e1(const XMaps& map, const EncodeArgs& a, int grid, cudaStream_t st) {
   auto kern = encode_quant_gram<T, BITS, KMAX>;
-  static bool configured = false;   // the attribute persists for the process
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, E1Cfg<T>::kSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<int> smem_set[kMaxDevices];   // per device: the limit is a per-device setting
+  cudaError_t e = ensure_smem_limit(kern, E1Cfg<T>::kSmem, smem_set);
+  if (e != cudaSuccess) return e;
   kern<<<grid, E1Cfg<T>::kThreads, E1Cfg<T>::kSmem, st>>>(map, a);
   return cudaGetLastError();
 }
@@ -1193,12 +1187,9 @@ template <typename T, int BITS, int RMAX>
 static cudaError_t launch_e3(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
   auto kern = encode_lowrank<T, BITS, RMAX>;
   constexpr int smem = E3Cfg<T, BITS, RMAX>::kSmem;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<int> smem_set[kMaxDevices];
+  cudaError_t e = ensure_smem_limit(kern, smem, smem_set);
+  if (e != cudaSuccess) return e;
   kern<<<grid, kE3Threads, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
@@ -1288,13 +1279,9 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
     const int RM = a.r <= 4 ? 4 : (a.r <= 8 ? 8 : 16);
     const size_t sm2 = RM == 4 ? sizeof(E2Smem<4>) : (RM == 8 ? sizeof(E2Smem<8>) : sizeof(E2Smem<16>));
     auto kern = RM == 4 ? encode_power<4> : (RM == 8 ? encode_power<8> : encode_power<16>);
-    static bool configured[3] = {false, false, false};
-    const int ci = RM == 4 ? 0 : (RM == 8 ? 1 : 2);
-    if (!configured[ci]) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-      if (e != cudaSuccess) return e;
-      configured[ci] = true;
-    }
+    static std::atomic<int> smem_set[3][kMaxDevices];
+    e = ensure_smem_limit(kern, (int)sm2, smem_set[RM == 4 ? 0 : (RM == 8 ? 1 : 2)]);
+    if (e != cudaSuccess) return e;
     kern<<<a.U, kE2Threads, sm2, st>>>(a);
     e = cudaGetLastError();
   }

@@ -60,6 +60,7 @@ def _load():
         "gear_validate_params": (i32, [pp, i32]),
         "gear_cache_bytes": (S, [pp, i32, i32, i32, i32, i32, i32]),
         "gear_cache_init": (i32, [pc, pp, i32, i32, i32, i32, i32, i32, P, S]),
+        "gear_cache_reset": (i32, [pc]),
         "gear_encode_workspace_bytes": (S, [pc, i32]),
         "gear_encode": (i32, [pc, P, i32, P, S, P]),
         "gear_encode_batch_workspace_bytes": (S, [i32, P, i32]),
@@ -155,6 +156,10 @@ class Cache:
     @property
     def n_blk(self) -> int:
         return self.c.n_blk
+
+    def reset(self):
+        """gear_cache_reset: empty the cache (host counters only) for a new encode."""
+        _check(lib.gear_cache_reset(ctypes.byref(self.c)), "gear_cache_reset")
 
     def encode(self, kv: torch.Tensor, stream=None):
         assert kv.is_cuda and kv.dtype == self.dtype and kv.is_contiguous()

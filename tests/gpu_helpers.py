@@ -17,10 +17,16 @@ def oracle_params(p) -> oracle.Params:
                          meta_f16=bool(p.meta_f16))
 
 
-def seeded_kv(seed: int, stream: int, shape, dtype: str, channel_scale: bool = False) -> np.ndarray:
-    """float32 array of exact dtype-rounded values from the shared generator."""
+def seeded_kv(seed: int, stream: int, shape, dtype: str, channel_scale: bool = False,
+              dist: str = "irwin_hall") -> np.ndarray:
+    """float32 array of exact dtype-rounded values from the shared generator, or
+    (dist = "t3") heavy-tailed Student-t draws with 3 degrees of freedom from
+    numpy's seeded generator, whose large entries exercise the outlier path."""
     n = int(np.prod(shape))
-    x = wl.normal_np(seed, stream, np.arange(n, dtype=np.int64)).reshape(shape)
+    if dist == "t3":
+        x = np.random.default_rng([seed, stream]).standard_t(3, size=n).astype(np.float32).reshape(shape)
+    else:
+        x = wl.normal_np(seed, stream, np.arange(n, dtype=np.int64)).reshape(shape)
     if channel_scale:
         u = wl.uniform_u32_np(seed, 999, np.arange(shape[-1], dtype=np.int64))
         sig = np.exp(np.log(0.5) + (u / 4294967296.0) * (np.log(8.0) - np.log(0.5))).astype(np.float32)
@@ -84,3 +90,18 @@ def compare_dense(gd: np.ndarray, od: np.ndarray, scale: np.ndarray, g: int, wha
     bound = 1e-3 * sc + 1e-6 * np.abs(od) + 1e-30
     bad = err > bound
     assert not bad.any(), f"{what}: {bad.sum()} reconstructed entries off, worst {err[bad].max():.3e}"
+
+
+def spread_units(U: int, count: int = 16) -> list[int]:
+    """count unit indices spread evenly over [0, U), always with the first and the last."""
+    if U <= count:
+        return list(range(U))
+    return sorted({round(i * (U - 1) / (count - 1)) for i in range(count)})
+
+
+def pmap(fn, items, workers: int = 16):
+    """fn over items on a thread pool (the oracle's C calls release the GIL)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(workers, os.cpu_count() or 1))) as ex:
+        return list(ex.map(fn, items))

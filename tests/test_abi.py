@@ -108,6 +108,13 @@ def test_cache_layout_and_host_errors(gear):
     assert L.gear_encode(ctypes.byref(c), ctypes.c_void_p(4096), 2, None, 0, None) == E.GEAR_ERR_INVALID_ARG
     assert L.gear_decode_attn(ctypes.byref(c), ctypes.byref(c), ctypes.c_void_p(4096), 32, ctypes.c_float(0.1),
                               ctypes.c_void_p(4096), 0, None, 0, None) == E.GEAR_ERR_INVALID_ARG  # empty cache
+    # reset empties the host counters and touches nothing else
+    c.n_comp, c.n_buf, c.n_blk, c.blk0_len, c.blk0_rank = 4096, 3, 1, 4096, 4
+    before = (c.codes, c.meta, c.buf, c.k, c.W)
+    assert L.gear_cache_reset(ctypes.byref(c)) == 0
+    assert (c.n_comp, c.n_buf, c.n_blk, c.blk0_len, c.blk0_rank) == (0, 0, 0, 0, 0)
+    assert (c.codes, c.meta, c.buf, c.k, c.W) == before
+    assert L.gear_cache_reset(None) == E.GEAR_ERR_INVALID_ARG
     assert L.gear_decode_attn_ragged(ctypes.byref(c), ctypes.byref(c), ctypes.c_void_p(4096), 32, ctypes.c_float(0.1),
                                      ctypes.c_void_p(4096), 0, None, ctypes.c_void_p(4096), 1 << 20,
                                      None) == E.GEAR_ERR_INVALID_ARG   # no prefill lengths

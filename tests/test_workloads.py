@@ -36,3 +36,20 @@ def test_tiny_spikes_and_channel_scale():
     assert sp.size == round(0.01 * 256 * 128) and np.unique(sp).size == sp.size
     sig = wl.channel_sigma(wl.WORKLOADS["llama7b_layer_encode"], 0)
     assert sig.min() >= 0.5 and sig.max() <= 8.0
+
+
+def test_tiny_draws_true_normals():
+    """The tiny codec workload asks for i.i.d. N(0,1) entries: its values come from
+    numpy's seeded generator (unbounded tails), identical on both sides."""
+    w = wl.WORKLOADS["tiny"]
+    v = wl.kv_unit_np(w, "v", 0, 0, 0)
+    assert v.shape == (256, 128) and abs(v.mean()) < 0.05 and abs(v.std() - 1) < 0.05
+    assert np.abs(v).max() > 3.47    # beyond the bounded Irwin-Hall support
+    k = wl.kv_unit_np(w, "k", 0, 0, 0)
+    sp = wl.spike_positions(w)
+    base = np.random.default_rng([w.seed, wl.S_K, 0, 0, 0]).standard_normal((256, 128), dtype=np.float32)
+    assert np.array_equal(k.reshape(-1)[sp], base.reshape(-1)[sp] * np.float32(10.0))
+    mask = np.ones(256 * 128, bool)
+    mask[sp] = False
+    assert np.array_equal(k.reshape(-1)[mask], base.reshape(-1)[mask])
+    assert np.array_equal(wl.rows_np(w, wl.S_Q, 0, 0, 1), wl.rows_torch(w, wl.S_Q, 0, 0, 1, "cpu").numpy())

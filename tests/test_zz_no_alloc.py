@@ -18,12 +18,12 @@ def _cp(c):
     return ctypes.byref(c.c)
 
 
-def test_noalloc_decode_matches_workspace_decode():
+@pytest.mark.parametrize("B,H,Hq,n0", [(2, 4, 8, 700), (1, 2, 16, 500)])   # 2 and 8 query heads per kv head
+def test_noalloc_decode_matches_workspace_decode(B, H, Hq, n0):
     import kv_cache_compression_gear_b200 as gear
     from kv_cache_compression_gear_b200 import gear as G
     from tests.gpu_helpers import seeded_kv, to_dev
 
-    B, H, Hq, n0 = 2, 4, 8, 700
     p = gear.make_params(bits=4, group_size=64, outlier_frac=0.02, rank=4, buffer_len=5, buffer_rank=2, seed=31)
     kc = gear.Cache(p, B, H, n0 + 16, 4, torch.float16)
     vc = gear.Cache(p, B, H, n0 + 16, 4, torch.float16)
@@ -32,6 +32,7 @@ def test_noalloc_decode_matches_workspace_decode():
     for i in range(7):  # one flush, two tokens left in the buffer
         gear.append_buffer(kc, vc, to_dev(seeded_kv(50 + i, 3, (B, H, 128), "f16"), "f16"),
                            to_dev(seeded_kv(50 + i, 4, (B, H, 128), "f16"), "f16"))
+    assert G.lib.gear_decode_workspace_bytes(_cp(kc), _cp(vc), Hq) <= (4 << 20)   # fits the scratch array
     vmax = float(vc.dense().abs().max())
     tau = 1.0 / math.sqrt(128)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)

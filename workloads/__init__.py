@@ -12,6 +12,11 @@ Generator. Element number e of stream s under seed S draws 64 random bits from a
 the sum of four 16-bit uniforms (the Irwin-Hall approximation of a normal):
     N = (u1 + u2 + u3 + u4 - 131070) * c,   c = 1 / sqrt(4 * (65536^2 - 1) / 12)
 which has mean 0, variance 1 and support |N| <= 3.47.
+
+Small workloads whose description asks for i.i.d. N(0,1) entries (the tiny
+single-head codec) instead draw true standard normals on the CPU from numpy's
+seeded generator (PCG64, ``default_rng``), keyed by (seed, stream, layer, batch,
+head) or (seed, stream, layer, step), and the torch side uploads those values.
 """
 from __future__ import annotations
 
@@ -135,12 +140,13 @@ class Workload:
     seed: int
     k_channel_scale: bool   # K has per-(head, channel) log-uniform std in [0.5, 8]
     spike_frac: float       # fraction of K entries multiplied by 10 (tiny workload)
+    cpu_normal: bool = False   # true N(0,1) draws from numpy's seeded generator (small workloads)
 
 
 WORKLOADS = {
     # one 256 x 128 fp32 K matrix with 1% spiked entries, matching N(0,1) V and q
     "tiny": Workload("tiny", 1, 1, 1, 1, 256, 128, "f32", 4, 64, 0.02, 4, 3, 20, 0, 2,
-                     1001, False, 0.01),
+                     1001, False, 0.01, cpu_normal=True),
     # LLaMA-7B-shaped layer: encode K and V of 32 heads x 4096 tokens, fp16
     "llama7b_layer_encode": Workload("llama7b_layer_encode", 1, 1, 32, 32, 4096, 128, "f16",
                                      4, 64, 0.02, 4, 3, 20, 0, 2, 1002, True, 0.0),
@@ -189,7 +195,10 @@ def kv_unit_np(w: Workload, which: str, layer: int, b: int, h: int, n: int | Non
     """float32 [n][d] exact (dtype-rounded) values of one unit of K or V."""
     n = w.n if n is None else n
     stream = S_K if which == "k" else S_V
-    x = normal_np(w.seed, stream, _unit_index(w, layer, b, h, n)).reshape(n, w.d)
+    if w.cpu_normal:
+        x = np.random.default_rng([w.seed, stream, layer, b, h]).standard_normal((n, w.d), dtype=np.float32)
+    else:
+        x = normal_np(w.seed, stream, _unit_index(w, layer, b, h, n)).reshape(n, w.d)
     if which == "k":
         x = x * channel_sigma(w, layer)[h][None, :]
         sp = spike_positions(w)
@@ -204,6 +213,9 @@ def kv_tensor_torch(w: Workload, which: str, layer: int, device, n: int | None =
     of whole units (bounded temporaries)."""
     import torch
     n = w.n if n is None else n
+    if w.cpu_normal:
+        x = np.stack([kv_unit_np(w, which, layer, b, h, n) for b in range(w.B) for h in range(w.H)])
+        return torch.from_numpy(x.reshape(w.B, w.H, n, w.d)).to(device=device, dtype=torch_dtype(w.dtype))
     stream = S_K if which == "k" else S_V
     out = torch.empty((w.B * w.H, n, w.d), dtype=torch_dtype(w.dtype), device=device)
     sig = torch.from_numpy(channel_sigma(w, layer)).to(device) if which == "k" else None
@@ -230,6 +242,9 @@ def kv_tensor_torch(w: Workload, which: str, layer: int, device, n: int | None =
 
 def rows_np(w: Workload, stream: int, layer: int, step: int, heads: int) -> np.ndarray:
     """float32 [B][heads][d] exact values of a per-step row tensor (q, buffer or new token)."""
+    if w.cpu_normal:
+        x = np.random.default_rng([w.seed, stream, layer, step]).standard_normal((w.B, heads, w.d), dtype=np.float32)
+        return to_dtype_exact_np(x, w.dtype)
     base = ((layer * 1_000_003 + step) * w.B * heads) * w.d
     idx = base + np.arange(w.B * heads * w.d, dtype=np.int64)
     return to_dtype_exact_np(normal_np(w.seed, stream, idx), w.dtype).reshape(w.B, heads, w.d)
@@ -237,6 +252,8 @@ def rows_np(w: Workload, stream: int, layer: int, step: int, heads: int) -> np.n
 
 def rows_torch(w: Workload, stream: int, layer: int, step: int, heads: int, device):
     import torch
+    if w.cpu_normal:
+        return torch.from_numpy(rows_np(w, stream, layer, step, heads)).to(device=device, dtype=torch_dtype(w.dtype))
     base = ((layer * 1_000_003 + step) * w.B * heads) * w.d
     idx = base + torch.arange(w.B * heads * w.d, device=device, dtype=torch.int64)
     return normal_torch(w.seed, stream, idx).view(w.B, heads, w.d).to(torch_dtype(w.dtype))
