@@ -522,8 +522,8 @@ def measure(gear, wl, sc: Scenario, dev, rank, world, steps, warmup, hbm, peak_k
     nflush = sum(1 for r in recs if r[6])
     launches = sum(runner.launches_per_step(r[6]) for r in recs)
     n_comp, n_blk, n_buf = runner.dk[0].n_comp, runner.dk[0].n_blk, runner.dk[0].n_buf
-    ee = runner.e2e(max(3, steps // 4)) if with_e2e else None
-    if ee is not None:
+    ee = runner.e2e(max(3, steps // 4)) if with_e2e else "not measured for this case"
+    if isinstance(ee, tuple):
         ee = tuple(max_over_ranks(v, world, dev) for v in ee[:2]) + ee[2:]
     del runner
     torch.cuda.empty_cache()
@@ -560,12 +560,13 @@ def measure(gear, wl, sc: Scenario, dev, rank, world, steps, warmup, hbm, peak_k
         "roofline": roof, "roofline_other": other,
         "gpu_launches": launches, "clocks": clk,
     }
-    if ee is not None:
+    if isinstance(ee, tuple):
         te, td, h2d, d2h = ee
         res["e2e"] = {"value": round(world * enc_in / te / 1e9, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h, "decode_tokens_per_s": round(world * wd.B / td, 1)}
     else:
-        res["e2e"] = {"value": None, "unit": "GB/s", "skipped": "host memory cannot hold a pinned copy of the inputs"}
+        res["e2e"] = {"value": None, "unit": "GB/s",
+                      "skipped": ee or "host memory cannot hold a pinned copy of the inputs"}
     return res
 
 

@@ -117,7 +117,7 @@ static gear_status encode_block(gear_cache* const* cs, const void* const* kvs, i
   a.grid_e1 = encode_grid(a, sms);
   a.maxc = encode_maxc(a.total_tiles, a.grid_e1, a.tpu);
   const size_t gbytes = align256((size_t)a.U * a.maxc * 128 * 128 * 4);
-  const size_t zbytes = align256((size_t)a.U * 128 * 16 * 4);
+  const size_t zbytes = align256((size_t)a.U * kZSlab);
   if (!ws || ws_bytes < gbytes + zbytes || !aligned(ws, 256)) return GEAR_ERR_WORKSPACE;
   a.gram = reinterpret_cast<float*>(ws);
   a.zbuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gbytes);
@@ -134,7 +134,7 @@ static size_t encode_ws_bytes(const gear_cache* c, int nt, int n) {
   a.total_tiles = (int64_t)a.U * a.tpu;
   const int grid = encode_grid(a, current_sm_count());
   const int maxc = encode_maxc(a.total_tiles, grid, a.tpu);
-  return align256((size_t)a.U * maxc * 128 * 128 * 4) + align256((size_t)a.U * 128 * 16 * 4);
+  return align256((size_t)a.U * maxc * 128 * 128 * 4) + align256((size_t)a.U * kZSlab);
 }
 
 // ------------------------------------------------------------------ append

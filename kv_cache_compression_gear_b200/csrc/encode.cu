@@ -189,6 +189,88 @@ __device__ __forceinline__ int64_t seg_first_cta(int64_t tile, int64_t grid, int
   return ((tile + 1) * grid - 1) / total;
 }
 
+// ---------------------------------------------------------------- top-k
+// Packed 16-bit helpers on |x| bit patterns (non-negative finite fp16/bf16
+// magnitudes order like their bit patterns read as unsigned integers).
+__device__ __forceinline__ uint32_t umax2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// 0xFFFF in each half whose magnitude is >= the threshold's (same half)
+template <typename T>
+__device__ __forceinline__ uint32_t ge_mask2(uint32_t a, uint32_t th2) {
+  uint32_t r;
+  if constexpr (std::is_same<T, __half>::value) asm("set.ge.u32.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(th2));
+  else asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(th2));
+  return r;
+}
+// Sorts 8 values into descending order (19 compare-exchanges, the optimal
+// network for 8 inputs; Knuth, TAOCP vol. 3, 5.3.4).
+template <typename K>
+__device__ __forceinline__ void sort8_desc(K (&v)[8]) {
+  constexpr int kNet[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6}, {5, 7}, {1, 2}, {5, 6},
+                               {0, 4}, {3, 7}, {1, 5}, {2, 6}, {1, 4}, {3, 6}, {2, 4}, {3, 5}, {3, 4}};
+#pragma unroll
+  for (int i = 0; i < 19; ++i) {
+    const K a = v[kNet[i][0]], b = v[kNet[i][1]];
+    v[kNet[i][0]] = max(a, b);
+    v[kNet[i][1]] = min(a, b);
+  }
+}
+
+// Merges two descending lists of 8 into the 8 largest of both, descending:
+// the elementwise maxima against the reversed second list are the 8 largest as
+// a bitonic sequence (Batcher's half-cleaner), which a bitonic merger sorts.
+template <typename K>
+__device__ __forceinline__ void merge8_desc(K (&a)[8], const K (&b)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = max(a[i], b[7 - i]);
+  constexpr int kMerge[12][2] = {{0, 4}, {1, 5}, {2, 6}, {3, 7}, {0, 2}, {1, 3},
+                                 {4, 6}, {5, 7}, {0, 1}, {2, 3}, {4, 5}, {6, 7}};
+#pragma unroll
+  for (int i = 0; i < 12; ++i) {
+    const K x = a[kMerge[i][0]], y = a[kMerge[i][1]];
+    a[kMerge[i][0]] = max(x, y);
+    a[kMerge[i][1]] = min(x, y);
+  }
+}
+
+// Candidates of the per-token top-k for 16-bit inputs (k <= 8): a lower bound
+// theta on the token's k-th largest |x| that costs a few operations per pair,
+// then the exact selection over the few entries with |x| >= theta only.
+// Bound: split the token into 16 blocks of 8 channels (8 per half); the k
+// largest block maxima are k distinct entries, so the k-th largest block
+// maximum is <= the token's k-th largest |x|. Every entry of the top k (|x| >=
+// k-th largest) is therefore a candidate. Returns the candidates of this half as
+// two bit words: bit p of w[i] <-> channel 2(16i + p), bit 16 + p <-> channel
+// 2(16i + p) + 1.
+template <typename T>
+__device__ __forceinline__ void topk_candidates(const uint32_t (&xr)[32], int k, bool valid, uint32_t (&w)[2]) {
+  uint32_t ab[32];
+#pragma unroll
+  for (int p = 0; p < 32; ++p) ab[p] = xr[p] & 0x7FFF7FFFu;
+  uint32_t bm[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t m = umax2(umax2(ab[4 * j], ab[4 * j + 1]), umax2(ab[4 * j + 2], ab[4 * j + 3]));
+    bm[j] = max(m & 0xFFFFu, m >> 16);
+  }
+  sort8_desc(bm);
+  uint32_t other[8];   // the partner half's sorted block maxima
+#pragma unroll
+  for (int i = 0; i < 8; ++i) other[i] = __shfl_xor_sync(0xFFFFFFFFu, bm[i], 1);
+  merge8_desc(bm, other);
+  uint32_t th = bm[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) th = (i == k - 1) ? bm[i] : th;
+  const uint32_t th2 = th | (th << 16);
+  w[0] = w[1] = 0u;
+#pragma unroll
+  for (int p = 0; p < 32; ++p) w[p >> 4] |= ge_mask2<T>(ab[p], th2) & (0x00010001u << (p & 15));
+  if (!valid) w[0] = w[1] = 0u;   // rows past the unit's end select nothing
+}
+
 // One quantizer thread: half h (channels 64h .. 64h+63) of token t of the tile.
 // Writes codes/meta/outliers of the token to the cache and the residual split
 // into the R stage. `valid` is false for tile rows past the unit's last token.
@@ -230,35 +312,58 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
 #pragma unroll
     for (int i = 0; i < KMAX; ++i) top[i] = 0;
     const uint32_t tb0 = 127u - 64u * h;
-#pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      Key key;
-      if constexpr (sizeof(T) == 4) {
-        key = ((uint64_t)(xr[e] & 0x7FFFFFFFu) << 7) | (tb0 - e);
-      } else {
-        uint32_t p = xr[e >> 1];
-        uint32_t ab = (e & 1) ? ((p >> 16) & 0x7FFFu) : (p & 0x7FFFu);
-        key = (ab << 7) | (tb0 - e);
-      }
+    auto insert = [&](Key key) {
 #pragma unroll
       for (int i = 0; i < KMAX; ++i) {   // one max and one min per level
         const Key hi = max(key, top[i]);
         key = min(key, top[i]);
         top[i] = hi;
       }
+    };
+    if constexpr (sizeof(T) == 2 && KMAX <= 8) {
+      // filtered: only the candidates of topk_candidates enter the insertion
+      uint32_t cw[2];
+      topk_candidates<T>(xr, k, valid, cw);
+      const uint8_t* xh = xs + h * 16384;
+      while ((cw[0] | cw[1]) != 0u) {
+        const bool lo = cw[0] != 0u;
+        const uint32_t wv = lo ? cw[0] : cw[1];
+        const int b = __ffs(wv) - 1;
+        if (lo) cw[0] = wv & (wv - 1u); else cw[1] = wv & (wv - 1u);
+        const int e = ((((lo ? 0 : 16) + (b & 15)) << 1) | (b >> 4));   // channel inside the half
+        const uint32_t ab = *reinterpret_cast<const uint16_t*>(xh + swz(t, e >> 3) + (e & 7) * 2) & 0x7FFFu;
+        insert((Key)((ab << 7) | (tb0 - e)));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        Key key;
+        if constexpr (sizeof(T) == 4) {
+          key = ((uint64_t)(xr[e] & 0x7FFFFFFFu) << 7) | (tb0 - e);
+        } else {
+          uint32_t p = xr[e >> 1];
+          uint32_t ab = (e & 1) ? ((p >> 16) & 0x7FFFu) : (p & 0x7FFFu);
+          key = (ab << 7) | (tb0 - e);
+        }
+        insert(key);
+      }
     }
     // snapshot the partner's list before either lane modifies its own
     Key other[KMAX];
 #pragma unroll
     for (int i = 0; i < KMAX; ++i) other[i] = __shfl_xor_sync(0xFFFFFFFFu, top[i], 1);
+    if constexpr (KMAX == 8) {
+      merge8_desc(top, other);   // both lists are sorted descending
+    } else {
 #pragma unroll
-    for (int i = 0; i < KMAX; ++i) {
-      Key key = other[i];
+      for (int i = 0; i < KMAX; ++i) {
+        Key key = other[i];
 #pragma unroll
-      for (int m = 0; m < KMAX; ++m) {
-        const Key hi = max(key, top[m]);
-        key = min(key, top[m]);
-        top[m] = hi;
+        for (int m = 0; m < KMAX; ++m) {
+          const Key hi = max(key, top[m]);
+          key = min(key, top[m]);
+          top[m] = hi;
+        }
       }
     }
     // read the k outlier values (both threads read all k), then patch own half
@@ -474,7 +579,47 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
     } else if (h == 0) {
       put_meta(0, scale[0], mn[0]);
     }
-    if constexpr (KMAX > 0) {
+    if constexpr (KMAX > 0 && KMAX <= 8) {
+      // ascending channel order: sort (channel, value bits) keys by channel
+      // (unused slots sort last); half 0 stores the channels, half 1 the values
+      using SK = typename std::conditional<sizeof(T) == 4, uint64_t, uint32_t>::type;
+      constexpr int kSh = sizeof(T) == 4 ? 32 : 16;
+      SK sk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        sk[i] = (i < KMAX && i < k) ? (((SK)cidx[i < KMAX ? i : 0] << kSh) | (SK)oval_bits[i < KMAX ? i : 0]) : ~(SK)0;
+      if constexpr (KMAX <= 4) {
+        constexpr int kNet4[5][2] = {{0, 1}, {2, 3}, {0, 2}, {1, 3}, {1, 2}};   // optimal network for 4
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+          const SK x = sk[kNet4[i][0]], y = sk[kNet4[i][1]];
+          sk[kNet4[i][0]] = min(x, y);
+          sk[kNet4[i][1]] = max(x, y);
+        }
+      } else {
+        sort8_desc(sk);   // descending; read back from the end
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const SK x = sk[i];
+          sk[i] = sk[7 - i];
+          sk[7 - i] = x;
+        }
+      }
+      if (h == 0) {
+        uint8_t* oi = ten.oidx + row * k;
+#pragma unroll
+        for (int i = 0; i < KMAX; ++i)
+          if (i < k) oi[i] = (uint8_t)(sk[i] >> kSh);
+      } else {
+#pragma unroll
+        for (int i = 0; i < KMAX; ++i) {
+          if (i < k) {
+            if constexpr (sizeof(T) == 4) reinterpret_cast<uint32_t*>(ten.oval)[row * k + i] = (uint32_t)sk[i];
+            else reinterpret_cast<uint16_t*>(ten.oval)[row * k + i] = (uint16_t)sk[i];
+          }
+        }
+      }
+    } else if constexpr (KMAX > 0) {
       if (h == 0 && k > 0) {
         // ascending channel order: selection by rank among the k channels
         uint8_t* oi = ten.oidx + row * k;
@@ -657,6 +802,40 @@ __global__ void __launch_bounds__(E1Cfg<T>::kThreads, 1)
   }
 }
 
+// Channel held by element e of 16-byte chunk m of the spread-code image.
+template <int BITS>
+__device__ __forceinline__ int spread_channel(int m, int e) {
+  if constexpr (BITS == 4) return 8 * m + (e >> 1) + 4 * (e & 1);            // word m: codes i, i + 4
+  else if constexpr (BITS == 2) return 16 * (m >> 1) + 4 * (m & 1) + (e >> 1) + 8 * (e & 1);   // i, i + 8
+  else return 8 * m + 4 * (e >> 2) + 2 * (e & 1) + ((e >> 1) & 1);         // bytes 0, 2 then 1, 3
+}
+
+// Position (chunk, element) of channel c in the spread-code image (inverse of
+// spread_channel).
+__host__ __device__ inline void spread_position(int bits, int c, int& m, int& el) {
+  const int i = c & 7;
+  if (bits == 4) {
+    m = c >> 3;
+    el = 2 * (i & 3) + (i >> 2);
+  } else if (bits == 2) {
+    const int w = c & 15;
+    m = 2 * (c >> 4) + ((w & 7) >> 2);
+    el = 2 * (w & 3) + (w >> 3);
+  } else {
+    const int r = i & 3;
+    m = c >> 3;
+    el = 4 * (i >> 2) + 2 * (r & 1) + (r >> 1);
+  }
+}
+
+// Z (d x r, r <= 16) as a B operand of E3's tensor-core products, K-major
+// (channels contiguous): element (row n, channel c) of one 16-bit part of N
+// rows sits in box c / 64 (N * 128 bytes), row n, 16-byte chunk
+// ((c % 64) / 8) ^ (n % 8) (the 128-byte swizzle), byte 2 (c % 8).
+__host__ __device__ constexpr int zimg_offset(int N, int n, int c) {
+  return (c >> 6) * (N * 128) + n * 128 + ((((c & 63) >> 3) ^ (n & 7)) << 4) + ((c & 7) << 1);
+}
+
 // ================================================================ E2 ======
 // Per unit: M = sym(sum of partial Grams), then T power steps with
 // Cholesky-QR on the r x r Gram. Outputs Rf (cache, scaled 2^-e) and
@@ -698,6 +877,92 @@ struct E2Smem {
     } it;
   } u;
 };
+
+// The unit's slab for E3 (see kZSlab): fp32 Z rows, then for 16-bit inputs
+// the operand images of X Z (16 rows, fp16 hi + lo or bf16 hi + mid + lo) and
+// of C Z (block-diagonal, the codes' spread order, fp16 hi + lo), both scaled
+// by 2^-sh so that max |Z| 2^-sh lies in [8, 16), with S_g (sums of the fp16
+// parts over each group) and the scales; for fp32 inputs the bf16 hi + lo
+// image of R Z (unscaled). Zf [128][16] holds Z on entry; Vf [128][16] is
+// scratch. Called by all threads of the block.
+__device__ void write_z_slab(const EncodeArgs& a, int u, const float* Zf, float* Vf) {
+  const int tid = threadIdx.x, nth = blockDim.x;
+  uint8_t* slab = reinterpret_cast<uint8_t*>(a.zbuf) + (int64_t)u * kZSlab;
+  float* rows = reinterpret_cast<float*>(slab + kSlabRows);
+  for (int e = tid; e < 128 * 16; e += nth) rows[e] = Zf[e];
+  __shared__ float red[32];
+  float m = 0.0f;
+  for (int e = tid; e < 128 * 16; e += nth) m = fmaxf(m, fabsf(Zf[e]));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((tid & 31) == 0) red[tid >> 5] = m;
+  __syncthreads();
+  m = 0.0f;
+  for (int w = 0; w < nth / 32; ++w) m = fmaxf(m, red[w]);
+  const bool wide = a.dtype == GEAR_F32;   // fp32 inputs: bf16 hi + lo, unscaled
+  int sh = 0;
+  if (!wide && m > 0.0f) sh = min(max(((__float_as_int(m) >> 23) & 0xFF) - 127 - 3, -100), 100);
+  const float down = __int_as_float((127 - sh) << 23), up = __int_as_float((127 + sh) << 23);
+  uint8_t* img = slab + kSlabImg;
+  // X Z (or R Z) operand: 16 rows of 128 channels per part, natural order
+  const int parts = wide ? 2 : (a.dtype == GEAR_F16 ? 2 : 3);
+  for (int e = tid; e < 16 * 128; e += nth) {
+    const int n = e >> 7, c = e & 127;
+    float rest = Zf[c * 16 + n] * down;
+    for (int part = 0; part < parts; ++part) {
+      uint16_t bitsv;
+      if (a.dtype == GEAR_F16) {
+        const __half hv = __float2half_rn(rest);
+        bitsv = __half_as_ushort(hv);
+        rest -= __half2float(hv);
+      } else {
+        const __nv_bfloat16 bv = __float2bfloat16_rn(rest);
+        bitsv = __bfloat16_as_ushort(bv);
+        rest -= __bfloat162float(bv);
+      }
+      *reinterpret_cast<uint16_t*>(img + part * 4096 + zimg_offset(16, n, c)) = bitsv;
+    }
+  }
+  if (wide) return;
+  // C Z operand: zero, then each channel's ranks into its group's column block
+  const int G = a.G, RB = a.r_max <= 8 ? 8 : 16, NC = G * RB > 16 ? G * RB : 16;
+  const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
+  uint8_t* zc = img + parts * 4096;
+  for (int e = tid; e < NC * 256 * 2 / 16; e += nth) reinterpret_cast<uint4*>(zc)[e] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  for (int e = tid; e < 128 * 16; e += nth) {
+    const int c = e >> 4, j = e & 15;
+    float v = 0.0f;
+    if (j < RB) {
+      const float z = Zf[c * 16 + j] * down;
+      const __half hi = __float2half_rn(z);
+      const __half lo = __float2half_rn(z - __half2float(hi));
+      int m2, el;
+      spread_position(a.bits, c, m2, el);
+      const int n = (c >> lg) * RB + j;
+      const int off = (m2 >> 3) * (NC * 128) + n * 128 + (((m2 & 7) ^ (n & 7)) << 4) + 2 * el;
+      *reinterpret_cast<__half*>(zc + off) = hi;
+      *reinterpret_cast<__half*>(zc + NC * 256 + off) = lo;
+      v = __half2float(hi) + __half2float(lo);
+    }
+    Vf[e] = v;
+  }
+  __syncthreads();
+  float* Sg = reinterpret_cast<float*>(slab + kSlabS);
+  if (tid < 64) {   // S_g[j]: the group's channels in order
+    const int g = tid >> 4, j = tid & 15;
+    float sum = 0.0f;
+    if (g < G)
+      for (int c = g << lg; c < (g + 1) << lg; ++c) sum += Vf[c * 16 + j];
+    Sg[tid] = sum;
+  }
+  if (tid == 0) {
+    Sg[64] = down;
+    Sg[65] = up;
+    Sg[66] = 0.0f;
+    Sg[67] = 0.0f;
+  }
+}
 
 template <int RM>
 __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a) {
@@ -880,10 +1145,17 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
         for (int j = 0; j < RM; ++j) S.Q[i * RM + j] = wq[j];
       } else {
         const double sL = ldexp(1.0, a.e_blk), sR = ldexp(1.0, -a.e_blk);
-        // Z rows in channel pairs: zbuf[u][i / 2][j][i % 2], the layout E3 copies in one piece
-        float* zrow = a.zbuf + (((int64_t)u * 64 + (i >> 1)) * 16) * 2 + (i & 1);
+        // Z rows (scaled 2^e, 16 ranks, j >= r zero) kept for the slab below;
+        // M is not read again in this step
+        float* Zf = S.M;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) zrow[2 * j] = (j < RM && j < r) ? (float)(zq[j < RM ? j : 0] * sL) : 0.0f;
+        for (int j = 0; j < 16; ++j) {
+          float z = 0.0f;
+#pragma unroll
+          for (int jj = 0; jj < RM; ++jj)
+            if (jj == j && jj < r) z = (float)(zq[jj] * sL);
+          Zf[i * 16 + j] = z;
+        }
         const int rp = rpad_of(a.r_max);
         float* rrow = a.ten[u / a.Uper].rfac + (((int64_t)(u % a.Uper) * a.nblk_max + a.blk) * 128 + i) * rp;
         for (int j = 0; j < rp; ++j) {
@@ -896,38 +1168,38 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
     }
     __syncthreads();
   }
+  write_z_slab(a, u, S.M, S.M + 2048);
 }
 
 // ================================================================ E3 ======
-// L rows: L_t = R_t Z for every token of the block, with R rebuilt as
-// x - fma(code, scale, zero) on every slot; the outlier slots' contribution
-// (x_o - zero) Z[c_o] is then removed again (their residual is 0).
-// One CTA per 128-token tile of one unit, one thread per token. The tile's
-// input rows (the encoder's tensor map: 128-byte swizzled boxes), code rows
-// (16-byte-chunk swizzle) and, for G >= 2, meta rows arrive by tensor copies
-// on one mbarrier; several CTAs per SM overlap one tile's copies with another
-// tile's arithmetic. A thread accumulates channel pairs in f32x2 registers.
-// Codes become floats by the mantissa trick f = 1 + code * 2^-w (w = 8 - pos
-// * bits for the code at position pos of its byte), so that
-// fma(f - 1, scale * 2^w, zero) is exactly fma(code, scale, zero) as long as
-// scale * 2^8 is finite; a token with a larger scale takes a plain loop.
-constexpr int kE3Threads = 128;
+// L rows, L = R Z for every token of the block, on the tensor cores. One CTA
+// per 128-token tile, two threads per token (one per 64 channels). The tile's
+// input rows (E1's tensor map: 128-byte swizzled boxes), code rows
+// (16-byte-chunk swizzle) and meta rows (G >= 2) arrive by tensor copies on one
+// mbarrier; the unit's Z rows (E2, fp32) are read from global memory while
+// they are in flight and turned into 16-bit operand images.
+//
+// 16-bit inputs never rebuild R. With D^ = code * scale + zero per group and
+// R = X - D^ outside the outlier slots (0 there, where the code is 0):
+//   L = X Z - sum_g scale_g (C Z)_g - sum_g zero_g S_g - sum_o (x_o - zero_g(o)) Z[c_o]
+// with C the codes, (C Z)_g the product over the channels of group g and S_g
+// the sum of Z's rows over group g. X Z takes the input tile as it landed (A
+// operand, K-major) against Z split into 16-bit parts; C Z takes the codes
+// spread into fp16 lanes as 1024 + code (one logic operation per pair; the
+// channel order inside each 16-byte chunk is whatever the spread produces, and
+// Z's block-diagonal image follows the same order) against Z split into fp16
+// hi + lo, one column block per group. Z is scaled by a power of two so that the fp16 parts stay
+// in range; the epilogue undoes it exactly. The thread then adds its token's
+// terms: G + 2 products per rank and k outlier corrections.
+//
+// fp32 inputs rebuild R = x - fma(code, scale, zero) per channel (bit-identical
+// to E1's residual, outlier slots 0), split as bf16 hi + lo in E1's residual
+// layout, and take R Z as hi Zhi + hi Zlo + lo Zhi.
+constexpr int kE3Threads = 256;   // two threads per token, one per 64-channel box
 
 struct E3Maps {
   // per tensor: input rows, cache code rows, cache meta rows (G >= 2)
   CUtensorMap x[kMaxBatch], codes[kMaxBatch], meta[kMaxBatch];
-};
-
-template <typename T, int BITS, int RMAX>
-struct E3Cfg {
-  static constexpr int kXB = kTile * 128 * (int)sizeof(T);   // input tile
-  static constexpr int kRow = 16 * BITS;                     // code bytes per token
-  static constexpr int kCB = kTile * kRow;                   // code tile
-  static constexpr int kMB = kTile * 32;                     // meta tile (G <= 4)
-  static constexpr int kZOff = kXB + kCB + kMB;              // Z pairs [64][16] float2
-  static constexpr int kZBytes = 64 * 16 * 8;
-  static constexpr int kBarOff = kZOff + kZBytes;
-  static constexpr int kSmem = kBarOff + 16 + 1024;          // + alignment slack
 };
 
 template <int R>
@@ -935,45 +1207,123 @@ __device__ __forceinline__ int swz_rows(int t) {   // chunk swizzle of R-byte ro
   return ((t * R) >> 7) & (R / 16 - 1);
 }
 
-template <typename T, int BITS, int RMAX>
-__global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_constant__ E3Maps maps, const EncodeArgs a) {
+// Spreads the codes of 32 channels (BITS words) into 4 chunks of eight fp16
+// values, in spread_channel order: each pair is masked into the mantissas of
+// 1024 (one logic operation) and 1024 is subtracted again (exact), so that the
+// products carry no offset (the tensor cores' accumulation error scales with
+// the largest product).
+template <int BITS>
+__device__ __forceinline__ void spread_codes(const uint32_t (&cw)[BITS], uint4 (&ch)[4]) {
+  uint32_t u[16];
+  if constexpr (BITS == 4) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) u[4 * w + i] = ((cw[w] >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
+  } else if constexpr (BITS == 2) {
+#pragma unroll
+    for (int w = 0; w < 2; ++w)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) u[8 * w + i] = ((cw[w] >> (2 * i)) & 0x00030003u) | 0x64006400u;
+  } else {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      u[2 * w] = (cw[w] & 0x00FF00FFu) | 0x64006400u;
+      u[2 * w + 1] = ((cw[w] >> 8) & 0x00FF00FFu) | 0x64006400u;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    __half2 v = *reinterpret_cast<__half2*>(&u[i]);
+    v = __hsub2(v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
+    u[i] = *reinterpret_cast<uint32_t*>(&v);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) ch[j] = make_uint4(u[4 * j], u[4 * j + 1], u[4 * j + 2], u[4 * j + 3]);
+}
+
+// Shared memory of the 16-bit E3 (from a 1024-byte-aligned base). RB columns
+// per group (8 when r <= 8, else 16), NC = max(16, G * RB) columns of C Z.
+template <typename T, int BITS, int RB>
+struct E3ACfg {
+  static constexpr int kParts = std::is_same<T, __half>::value ? 2 : 3;   // X Z: fp16 hi + lo, bf16 hi + mid + lo
+  static constexpr int kX = 0;                         // input tile, 32 KB
+  static constexpr int kC = 32768;                     // spread codes, 32 KB
+  static constexpr int kRow = 16 * BITS;               // code bytes per token
+  static constexpr int kCodes = 65536;                 // code tile
+  static constexpr int kMeta = kCodes + kTile * kRow;  // meta tile (G <= 4)
+  static constexpr int kZx = (kMeta + kTile * 32 + 1023) & ~1023;   // X Z operand: kParts x 4 KB
+  static constexpr int kZc = kZx + kParts * 4096;      // C Z operand: 2 parts x NC x 256 B
+  // then, at kZc + 2 NC 256: S_g [4][16] floats with the scale and its inverse
+  // (1 KB), the fp32 Z rows [128][16] (8 KB) and the barriers
+  static __host__ __device__ constexpr int s_off(int NC) { return kZc + 2 * NC * 256; }
+  static __host__ __device__ constexpr int zr_off(int NC) { return s_off(NC) + 1024; }
+  static __host__ __device__ constexpr int bar_off(int NC) { return zr_off(NC) + 8192; }
+  static __host__ __device__ constexpr int smem(int NC) { return bar_off(NC) + 64 + 1024; }   // + alignment slack
+};
+
+template <typename T, int BITS, int RB>
+__global__ void __launch_bounds__(kE3Threads, 2) encode_lowrank_alg(const __grid_constant__ E3Maps maps,
+                                                                     const EncodeArgs a) {
   using C = E1Cfg<T>;
-  using F = E3Cfg<T, BITS, RMAX>;
-  constexpr int W = 4 * BITS;
-  constexpr int kPerByte = 8 / BITS;
+  using F = E3ACfg<T, BITS, RB>;
+  using P = typename std::conditional<std::is_same<T, __half>::value, __half, __nv_bfloat16>::type;
   extern __shared__ uint8_t e3raw[];
   uint8_t* sm = align_smem_1024(e3raw);
-  uint8_t* xs = sm;
-  uint8_t* cs = sm + F::kXB;
-  uint8_t* ms = cs + F::kCB;
-  float2* Zp = reinterpret_cast<float2*>(sm + F::kZOff);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + F::kBarOff);
-  const int u = blockIdx.y, t0 = blockIdx.x * kTile, t = threadIdx.x;
-  const int G = a.G, k = a.k, r = a.r;
-  const int mrb = meta_row_bytes(G, a.meta_f16);   // meta bytes per token
+  uint8_t* xs = sm + F::kX;
+  uint8_t* cps = sm + F::kC;
+  uint8_t* cs = sm + F::kCodes;
+  uint8_t* ms = sm + F::kMeta;
+  uint8_t* zx = sm + F::kZx;
+  uint8_t* zc = sm + F::kZc;
+  const int G = a.G, k = a.k;
+  const int NC = G * RB > 16 ? G * RB : 16;
+  float* S = reinterpret_cast<float*>(sm + F::s_off(NC));
+  const float* zr = reinterpret_cast<const float*>(sm + F::zr_off(NC));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + F::bar_off(NC));   // [0] tile landed, [1] products done
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + F::bar_off(NC) + 16);
+  const int tid = threadIdx.x, t = tid & 127, h = tid >> 7, warp = tid >> 5;
+  const int u = blockIdx.y, t0 = blockIdx.x * kTile;
+  const int mrb = meta_row_bytes(G, a.meta_f16);
   const bool meta_tma = mrb >= 16;
   const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
   const int tn = u / a.Uper, ul = u % a.Uper;
   const EncodeTensor& ten = a.ten[tn];
-  const int crow = ul * a.n_max + a.t_off + t0;   // cache row of the tile's first token
-  if (t == 0) {
-    mbar_init(bar, 1);
+  const int crow = ul * a.n_max + a.t_off + t0;
+  const uint8_t* slab = reinterpret_cast<const uint8_t*>(a.zbuf) + (int64_t)u * kZSlab;
+  const uint32_t img_bytes = (uint32_t)(F::kParts * 4096 + 2 * NC * 256);
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
     fence_mbarrier_init();
-    mbar_arrive_expect_tx(bar, (uint32_t)(F::kXB + F::kCB + F::kZBytes + (meta_tma ? kTile * mrb : 0)));
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(Zp)),
-                 "l"(a.zbuf + (int64_t)u * (F::kZBytes / 4)), "r"((uint32_t)F::kZBytes), "r"(smem_u32(bar))
-                 : "memory");
-    for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(xs + b * 16384, &maps.x[tn], bar, b * C::kBoxCols, ul * a.n + t0);
-    tma_load_2d(cs, &maps.codes[tn], bar, 0, crow);
-    if (meta_tma) tma_load_2d(ms, &maps.meta[tn], bar, 0, crow);
+    mbar_arrive_expect_tx(&bars[0], (uint32_t)(32768 + kTile * F::kRow + (meta_tma ? kTile * mrb : 0)) +
+                                        img_bytes + (uint32_t)kSlabSBytes + 8192u);
+    for (int b = 0; b < C::kBoxes; ++b)
+      tma_load_2d(xs + b * 16384, &maps.x[tn], &bars[0], b * C::kBoxCols, ul * a.n + t0);
+    tma_load_2d(cs, &maps.codes[tn], &bars[0], 0, crow);
+    if (meta_tma) tma_load_2d(ms, &maps.meta[tn], &bars[0], 0, crow);
+    // the unit's operand images and S_g, written by E2
+    bulk_load(zx, slab + kSlabImg, img_bytes, &bars[0]);
+    bulk_load(S, slab + kSlabS, (uint32_t)kSlabSBytes, &bars[0]);
+    bulk_load(sm + F::zr_off(NC), slab + kSlabRows, 8192u, &bars[0]);
   }
-  // Zp[p][j] = (Z[2p][j], Z[2p + 1][j]) arrives with the tile (E2 writes it in this layout)
+  if (warp == 0) tmem_alloc(tslot, 128);
   const bool valid = t0 + t < a.n;
   const size_t row = (size_t)crow + t;
-  // short meta rows (under 16 bytes) come straight from global memory
+  // this token's outliers (channel, value) and short meta rows, fetched while the tile is in flight
+  constexpr int kOF = 8;
+  int oc[kOF];
+  float ov[kOF];
   float2 szr[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-  if (!meta_tma && valid) {
+  if (h == 0) {
+#pragma unroll
+    for (int i = 0; i < kOF; ++i) {
+      const bool on = valid && i < k;
+      oc[i] = on ? ten.oidx[row * k + i] : 0;
+      ov[i] = on ? Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]) : 0.0f;
+    }
+  }
+  if (!meta_tma && valid && 8 * h < a.r_max) {   // both halves write ranks when r > 8
     if (a.meta_f16) {
       const __half2* mh = reinterpret_cast<const __half2*>(ten.meta) + row * G;
       szr[0] = __half22float2(mh[0]);
@@ -982,74 +1332,269 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
       szr[0] = reinterpret_cast<const float2*>(ten.meta)[row];
     }
   }
-  // the token's first outliers, fetched while the tile is in flight
-  constexpr int kOF = 4;
-  int oc[kOF];
-  float ox[kOF];
-#pragma unroll
-  for (int i = 0; i < kOF; ++i) {
-    const bool on = valid && i < k;
-    oc[i] = on ? ten.oidx[row * k + i] : 0;
-    if constexpr (sizeof(T) == 4) ox[i] = on ? reinterpret_cast<const float*>(ten.oval)[row * k + i] : 0.0f;
-    else ox[i] = on ? Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]) : 0.0f;
-  }
+  tc_fence_before();
   __syncthreads();
-  const bool landed = mbar_wait(bar, 0);
-  if (!landed || !valid) return;
-
-  // this token's meta row: fp32 group gi at byte (8 gi) ^ mx (32-byte rows
-  // swizzled), binary16 group gi at byte 4 gi
-  const uint8_t* mrow = ms + t * mrb;
-  const int mx = mrb == 32 ? ((t >> 2) & 1) << 4 : 0;
-  auto group = [&](int gi) -> float2 {
-    if (!meta_tma) return gi == 0 ? szr[0] : szr[1];
-    if (a.meta_f16) return __half22float2(*reinterpret_cast<const __half2*>(mrow + 4 * gi));
-    return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
-  };
-  bool big = false;
-  for (int gi = 0; gi < G; ++gi) big |= !(group(gi).x <= 0x1p100f);
-  // the code words of 32 channels [32 q, 32 q + 32): 4*BITS bytes of the row
-  auto codes32 = [&](int q, uint32_t (&cw)[BITS]) {
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  bool ok = mbar_wait(&bars[0], 0);
+  ok = __syncthreads_and(ok);
+  if (!ok && tid == 0) mbar_wait(&bars[0], 0);   // let copies still in flight land before the CTA ends
+  const float down = S[64], up = S[65];   // the images' power-of-two scale and its inverse
+  // ---- spread codes of this half row
+  if (ok) {
     const uint8_t* rowp = cs + t * F::kRow;
-    if constexpr (BITS == 2) {
-      const uint2 v = *reinterpret_cast<const uint2*>(rowp + ((((q >> 1) ^ swz_rows<F::kRow>(t)) << 4) | ((q & 1) << 3)));
-      cw[0] = v.x; cw[1] = v.y;
-    } else {
 #pragma unroll
-      for (int h = 0; h < BITS / 4; ++h) {
-        const uint4 v = *reinterpret_cast<const uint4*>(rowp + (((BITS / 4 * q + h) ^ swz_rows<F::kRow>(t)) << 4));
-        cw[4 * h] = v.x; cw[4 * h + 1] = v.y; cw[4 * h + 2] = v.z; cw[4 * h + 3] = v.w;
+    for (int qq = 0; qq < 2; ++qq) {
+      const int q = 2 * h + qq;   // 32-channel block
+      uint32_t cw[BITS];
+      if constexpr (BITS == 2) {
+        const uint2 v =
+            *reinterpret_cast<const uint2*>(rowp + ((((q >> 1) ^ swz_rows<F::kRow>(t)) << 4) | ((q & 1) << 3)));
+        cw[0] = v.x; cw[1] = v.y;
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < BITS / 4; ++hh) {
+          const uint4 v = *reinterpret_cast<const uint4*>(rowp + (((BITS / 4 * q + hh) ^ swz_rows<F::kRow>(t)) << 4));
+          cw[4 * hh] = v.x; cw[4 * hh + 1] = v.y; cw[4 * hh + 2] = v.z; cw[4 * hh + 3] = v.w;
+        }
+      }
+      uint4 ch[4];
+      spread_codes<BITS>(cw, ch);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int m = 4 * q + j;   // chunk 0..15
+        *reinterpret_cast<uint4*>(cps + (m >> 3) * 16384 + swz(t, m & 7)) = ch[j];
       }
     }
-  };
-
-  uint64_t acc[RMAX];
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {
+    // X Z into columns [0, 16): the parts of Z along K
+    constexpr uint32_t kIdX = idesc_f16(128, 16, std::is_same<P, __nv_bfloat16>::value, false, false);
+    const uint32_t xa = smem_u32(xs), za = smem_u32(zx);
+    int m = 0;
 #pragma unroll
-  for (int j = 0; j < RMAX; ++j) acc[j] = 0;
-  // 8 channels [8 jb, 8 jb + 8) of the input row, as floats
-  auto xblock = [&](int jb, float (&xv)[8]) {
-    if constexpr (sizeof(T) == 4) {
+    for (int part = 0; part < F::kParts; ++part)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk, ++m) {
+        const uint64_t ad = smem_desc_sw128(xa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(za + part * 4096 + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+        tc_mma_f16(tmem, ad, bd, kIdX, m == 0 ? 0u : 1u);
+      }
+    // C Z into columns [32, 32 + NC): hi then lo part of Z
+    const uint32_t kIdC = idesc_f16(128, NC, false, false, false);
+    const uint32_t ca = smem_u32(cps), zb = smem_u32(zc);
+    m = 0;
+#pragma unroll
+    for (int part = 0; part < 2; ++part)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk, ++m) {
+        const uint64_t ad = smem_desc_sw128(ca + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd =
+            smem_desc_sw128(zb + part * NC * 256 + (kk >> 2) * (NC * 128) + (kk & 3) * 32, 16, 1024);
+        tc_mma_f16(tmem + 32, ad, bd, kIdC, m == 0 ? 0u : 1u);
+      }
+    tc_commit(&bars[1]);
+  }
+  // ---- epilogue: thread (t, h) writes ranks [8 h, 8 h + 8) of token t
+  if (ok && 8 * h < a.r_max) {
+    bool done = mbar_wait(&bars[1], 0);
+    if (!done) mbar_wait(&bars[1], 0);   // the products must finish before tensor memory is freed
+    tc_fence_after();
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    uint32_t vx[8], vc[4][8];
+    tmem_ld_32x32b_x8(lane_base + 8 * h, vx);
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi)
+      if (gi < G) tmem_ld_32x32b_x8(lane_base + 32 + gi * RB + (RB == 16 ? 8 * h : 0), vc[gi]);
+    tmem_ld_wait();
+    // meta of the token's groups: the tile in shared memory (or the short rows)
+    const uint8_t* mrow = ms + t * mrb;
+    const int mx = mrb == 32 ? ((t >> 2) & 1) << 4 : 0;
+    auto group = [&](int gi) -> float2 {
+      if (!meta_tma) return gi == 0 ? szr[0] : szr[1];
+      if (a.meta_f16) return __half22float2(*reinterpret_cast<const __half2*>(mrow + 4 * gi));
+      return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
+    };
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = __uint_as_float(vx[j]);
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) {
+      if (gi >= G) break;
+      const float2 sz = group(gi);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] -= fmaf(sz.x, __uint_as_float(vc[gi][j]), sz.y * S[gi * 16 + 8 * h + j]);
+    }
+    if (valid && done) {
+      // outlier slots: take (x_o - zero) Z[c_o] back out (their residual is 0)
+      auto fix = [&](int c, float xo) {
+        const float d = (xo - group(c >> lg).y) * down;
+        const float4 z0 = *reinterpret_cast<const float4*>(zr + c * 16 + 8 * h);
+        const float4 z1 = *reinterpret_cast<const float4*>(zr + c * 16 + 8 * h + 4);
+        acc[0] -= d * z0.x; acc[1] -= d * z0.y; acc[2] -= d * z0.z; acc[3] -= d * z0.w;
+        acc[4] -= d * z1.x; acc[5] -= d * z1.y; acc[6] -= d * z1.z; acc[7] -= d * z1.w;
+      };
+      if (h == 0) {
+#pragma unroll
+        for (int i = 0; i < kOF; ++i)
+          if (i < k) fix(oc[i], ov[i]);
+      }
+      for (int i = (h == 0 ? kOF : 0); i < k; ++i)
+        fix(ten.oidx[row * k + i], Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]));
+      const int q1 = min(a.r_max, 8 * h + 8);
+      if (q1 - 8 * h == 8 && (a.r_max & 7) == 0) {   // a whole 16-byte row piece
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 v2 = __floats2half2_rn(acc[2 * j] * up, acc[2 * j + 1] * up);
+          w[j] = *reinterpret_cast<const uint32_t*>(&v2);
+        }
+        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(ten.lfac) + row * a.r_max + 8 * h) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (8 * h + j < q1)
+            reinterpret_cast<__half*>(ten.lfac)[row * a.r_max + 8 * h + j] = __float2half_rn(acc[j] * up);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// fp32 inputs: rebuild R and take R Z as hi Zhi + hi Zlo + lo Zhi.
+template <int BITS>
+struct E3Cfg {
+  static constexpr int kXB = kTile * 128 * 4;          // input tile (4 boxes of 32 channels)
+  static constexpr int kRB = kTile * 128 * 2;          // one bf16 residual image
+  static constexpr int kRow = 16 * BITS;               // code bytes per token
+  static constexpr int kCB = kTile * kRow;             // code tile
+  static constexpr int kMB = kTile * 32;               // meta tile (G <= 4)
+  static constexpr int kX = 0;
+  static constexpr int kRhi = kXB;
+  static constexpr int kRlo = kRhi + kRB;
+  static constexpr int kC = kRlo + kRB;
+  static constexpr int kM = kC + kCB;
+  static constexpr int kZ = (kM + kMB + 1023) & ~1023;   // Z image: bf16 hi | lo, 16 rows each
+  static constexpr int kBar = kZ + 8192;
+  static constexpr int kSmem = kBar + 64 + 1024;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid_constant__ E3Maps maps,
+                                                                    const EncodeArgs a) {
+  using C = E1Cfg<float>;
+  using F = E3Cfg<BITS>;
+  constexpr int kPerByte = 8 / BITS;
+  extern __shared__ uint8_t e3raw[];
+  uint8_t* sm = align_smem_1024(e3raw);
+  uint8_t* xs = sm + F::kX;
+  uint8_t* rhi = sm + F::kRhi;
+  uint8_t* rlo = sm + F::kRlo;
+  uint8_t* cs = sm + F::kC;
+  uint8_t* ms = sm + F::kM;
+  uint8_t* zs = sm + F::kZ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + F::kBar);   // [0] tile landed, [1] product done
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + F::kBar + 16);
+  const int tid = threadIdx.x, t = tid & 127, h = tid >> 7, warp = tid >> 5;
+  const int u = blockIdx.y, t0 = blockIdx.x * kTile;
+  const int G = a.G, k = a.k;
+  const int mrb = meta_row_bytes(G, a.meta_f16);
+  const bool meta_tma = mrb >= 16;
+  const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
+  const int tn = u / a.Uper, ul = u % a.Uper;
+  const EncodeTensor& ten = a.ten[tn];
+  const int crow = ul * a.n_max + a.t_off + t0;
+  const uint8_t* slab = reinterpret_cast<const uint8_t*>(a.zbuf) + (int64_t)u * kZSlab;
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbarrier_init();
+    mbar_arrive_expect_tx(&bars[0], (uint32_t)(F::kXB + F::kCB + (meta_tma ? kTile * mrb : 0) + 8192));
+    for (int b = 0; b < C::kBoxes; ++b)
+      tma_load_2d(xs + b * 16384, &maps.x[tn], &bars[0], b * C::kBoxCols, ul * a.n + t0);
+    tma_load_2d(cs, &maps.codes[tn], &bars[0], 0, crow);
+    if (meta_tma) tma_load_2d(ms, &maps.meta[tn], &bars[0], 0, crow);
+    bulk_load(zs, slab + kSlabImg, 8192u, &bars[0]);   // Z image, bf16 hi | lo (E2)
+  }
+  if (warp == 0) tmem_alloc(tslot, 32);
+  const bool valid = t0 + t < a.n;
+  const size_t row = (size_t)crow + t;
+  float2 szr[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+  if (!meta_tma && valid) szr[0] = reinterpret_cast<const float2*>(ten.meta)[row];
+  constexpr int kOF = 8;
+  int oc[kOF];
+#pragma unroll
+  for (int i = 0; i < kOF; ++i) oc[i] = (valid && i < k) ? ten.oidx[row * k + i] : -1;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  bool ok = mbar_wait(&bars[0], 0);
+  ok = __syncthreads_and(ok);
+  if (!ok && tid == 0) mbar_wait(&bars[0], 0);   // let copies still in flight land before the CTA ends
+
+  if (ok && valid) {
+    const uint8_t* mrow = ms + t * mrb;
+    const int mx = mrb == 32 ? ((t >> 2) & 1) << 4 : 0;
+    auto group = [&](int gi) -> float2 {
+      if (!meta_tma) return gi == 0 ? szr[0] : szr[1];
+      return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
+    };
+    bool big = false;
+    for (int gi = 0; gi < G; ++gi) big |= !(group(gi).x <= 0x1p100f);
+    auto codes32 = [&](int q, uint32_t (&cw)[BITS]) {
+      const uint8_t* rowp = cs + t * F::kRow;
+      if constexpr (BITS == 2) {
+        const uint2 v =
+            *reinterpret_cast<const uint2*>(rowp + ((((q >> 1) ^ swz_rows<F::kRow>(t)) << 4) | ((q & 1) << 3)));
+        cw[0] = v.x; cw[1] = v.y;
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < BITS / 4; ++hh) {
+          const uint4 v = *reinterpret_cast<const uint4*>(rowp + (((BITS / 4 * q + hh) ^ swz_rows<F::kRow>(t)) << 4));
+          cw[4 * hh] = v.x; cw[4 * hh + 1] = v.y; cw[4 * hh + 2] = v.z; cw[4 * hh + 3] = v.w;
+        }
+      }
+    };
+    auto xblock = [&](int jb, float (&xv)[8]) {
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
         const uint4 v = *reinterpret_cast<const uint4*>(xs + (jb >> 2) * 16384 + swz(t, 2 * (jb & 3) + hq));
         xv[4 * hq] = __uint_as_float(v.x); xv[4 * hq + 1] = __uint_as_float(v.y);
         xv[4 * hq + 2] = __uint_as_float(v.z); xv[4 * hq + 3] = __uint_as_float(v.w);
       }
-    } else {
-      const uint4 v = *reinterpret_cast<const uint4*>(xs + (jb >> 3) * 16384 + swz(t, jb & 7));
-      const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
+    };
+    auto put = [&](int jb, const float (&rr)[8]) {
+      uint32_t h4[4], l4[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = Elem16<T>::to_f2(pr[q]);
-        xv[2 * q] = f.x; xv[2 * q + 1] = f.y;
+      for (int p = 0; p < 4; ++p) {
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(rr[2 * p], rr[2 * p + 1]);
+        const uint32_t hbits = *reinterpret_cast<const uint32_t*>(&hb);
+        const uint64_t hv = f2_pack(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u));
+        const uint64_t lv = f2_sub(f2_pack(rr[2 * p], rr[2 * p + 1]), hv);
+        const __nv_bfloat162 lb = __floats2bfloat162_rn(f2_lo(lv), f2_hi(lv));
+        h4[p] = hbits;
+        l4[p] = *reinterpret_cast<const uint32_t*>(&lb);
       }
-    }
-  };
-  if (!big) {
+      const uint32_t off = (uint32_t)((jb >> 3) * 16384) + swz(t, jb & 7);
+      *reinterpret_cast<uint4*>(rhi + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+      *reinterpret_cast<uint4*>(rlo + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    };
     const uint32_t one = a.one_bits;
     const uint64_t one2 = f2_pack(1.0f, 1.0f);
+    constexpr int kCpw = 32 / BITS;
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {   // 32 channels per pass, one group (g >= 32)
+    for (int q = 2 * h; q < 2 * h + 2; ++q) {   // 32 channels per pass, one group (g >= 32)
       uint32_t cw[BITS];
       codes32(q, cw);
       const float2 sz = group((32 * q) >> lg);
@@ -1057,100 +1602,101 @@ __global__ void __launch_bounds__(kE3Threads, 4) encode_lowrank(const __grid_con
 #pragma unroll
       for (int bq = 0; bq < 4; ++bq) {
         const int jb = 4 * q + bq;
-        float xv[8];
+        float xv[8], rr[8];
         xblock(jb, xv);
-        float f[8];   // the block's 8 codes as 1 + code * 2^-w
-        if constexpr (BITS == 4) {
-          CodeFloats<4>::word(cw[bq], f, one);
-        } else if constexpr (BITS == 2) {
-          float ff[16];
-          CodeFloats<2>::word(cw[bq >> 1] >> (16 * (bq & 1)), ff, one);
+        if (!big) {
+          float f[8];   // the block's 8 codes as 1 + code * 2^-w
+          if constexpr (BITS == 4) {
+            CodeFloats<4>::word(cw[bq], f, one);
+          } else if constexpr (BITS == 2) {
+            float ff[16];
+            CodeFloats<2>::word(cw[bq >> 1] >> (16 * (bq & 1)), ff, one);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = ff[e];
+            for (int e = 0; e < 8; ++e) f[e] = ff[e];
+          } else {
+            float fa[4], fb[4];
+            CodeFloats<8>::word(cw[2 * bq], fa, one);
+            CodeFloats<8>::word(cw[2 * bq + 1], fb, one);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { f[e] = fa[e]; f[4 + e] = fb[e]; }
+          }
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const int cl = 2 * p;
+            const uint64_t w2 = f2_pack((float)(1 << (8 - (cl % kPerByte) * BITS)),
+                                        (float)(1 << (8 - ((cl + 1) % kPerByte) * BITS)));
+            const uint64_t cf = f2_sub(f2_pack(f[cl], f[cl + 1]), one2);
+            const uint64_t dh = f2_fma(cf, f2_mul(sc2, w2), zr2);
+            const uint64_t rv = f2_sub(f2_pack(xv[cl], xv[cl + 1]), dh);
+            rr[cl] = f2_lo(rv);
+            rr[cl + 1] = f2_hi(rv);
+          }
         } else {
-          float fa[4], fb[4];
-          CodeFloats<8>::word(cw[2 * bq], fa, one);
-          CodeFloats<8>::word(cw[2 * bq + 1], fb, one);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) { f[e] = fa[e]; f[4 + e] = fb[e]; }
-        }
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const int cl = 2 * p;   // channel inside the block; 8*jb is a whole number of bytes
-          const uint64_t w2 = f2_pack((float)(1 << (8 - (cl % kPerByte) * BITS)),
-                                      (float)(1 << (8 - ((cl + 1) % kPerByte) * BITS)));
-          const uint64_t cf = f2_sub(f2_pack(f[cl], f[cl + 1]), one2);
-          const uint64_t dh = f2_fma(cf, f2_mul(sc2, w2), zr2);
-          const uint64_t rr = f2_sub(f2_pack(xv[cl], xv[cl + 1]), dh);
-          const float4* zq = reinterpret_cast<const float4*>(Zp + (4 * jb + p) * 16);
-#pragma unroll
-          for (int j = 0; j < RMAX; j += 2) {
-            const float4 z = zq[j >> 1];
-            acc[j] = f2_fma(rr, f2_pack(z.x, z.y), acc[j]);
-            acc[j + 1] = f2_fma(rr, f2_pack(z.z, z.w), acc[j + 1]);
-          }
-        }
-      }
-    }
-  } else {
-    constexpr int kCpw = 32 / BITS;
-#pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-      uint32_t cw[BITS];
-      codes32(q, cw);
-      const float2 sz = group((32 * q) >> lg);
-#pragma unroll
-      for (int bq = 0; bq < 4; ++bq) {
-        const int jb = 4 * q + bq;
-        float xv[8];
-        xblock(jb, xv);
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          float rr[2];
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int c = 8 * bq + 2 * p + e2;   // channel inside the 32
+          for (int e = 0; e < 8; ++e) {
+            const int c = 8 * bq + e;
             const float code = (float)((cw[c / kCpw] >> (BITS * (c % kCpw))) & ((1u << BITS) - 1u));
-            rr[e2] = __fsub_rn(xv[2 * p + e2], __fmaf_rn(code, sz.x, sz.y));
+            rr[e] = __fsub_rn(xv[e], __fmaf_rn(code, sz.x, sz.y));
           }
-          const uint64_t rv = f2_pack(rr[0], rr[1]);
-#pragma unroll
-          for (int j = 0; j < RMAX; ++j)
-            acc[j] = f2_fma(rv, *reinterpret_cast<const uint64_t*>(&Zp[(4 * jb + p) * 16 + j]), acc[j]);
         }
+        put(jb, rr);
       }
     }
-  }
-  // outlier slots: their residual is zero; remove what the loop added
-  for (int i = 0; i < k; ++i) {
-    int c;
-    float x;
-    if (i < kOF) {
+    for (int i = 0; i < k; ++i) {   // outlier slots of this half: residual 0
+      int c = 0;
+      if (i < kOF) {
 #pragma unroll
-      for (int i2 = 0; i2 < kOF; ++i2)
-        if (i2 == i) { c = oc[i2]; x = ox[i2]; }
-    } else {
-      c = ten.oidx[row * k + i];
-      if constexpr (sizeof(T) == 4) x = reinterpret_cast<const float*>(ten.oval)[row * k + i];
-      else x = Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]);
-    }
-    const float2 sz = group(c >> lg);
-    const float rr = __fsub_rn(x, __fmaf_rn(0.0f, sz.x, sz.y));
-#pragma unroll
-    for (int j = 0; j < RMAX; ++j) {
-      const float2 z = Zp[(c >> 1) * 16 + j];
-      const float v = rr * ((c & 1) ? z.y : z.x);
-      acc[j] = f2_sub(acc[j], (c & 1) ? f2_pack(0.0f, v) : f2_pack(v, 0.0f));
+        for (int i2 = 0; i2 < kOF; ++i2)
+          if (i2 == i) c = oc[i2];
+      } else {
+        c = ten.oidx[row * k + i];
+      }
+      if ((c >> 6) != h) continue;
+      const uint32_t off = (uint32_t)(h * 16384) + swz(t, (c & 63) >> 3) + (c & 7) * 2;
+      *reinterpret_cast<uint16_t*>(rhi + off) = 0;
+      *reinterpret_cast<uint16_t*>(rlo + off) = 0;
     }
   }
-  for (int q = 0; q < a.r_max; ++q) {
-    float v = 0.0f;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (ok && tid == 0) {
+    constexpr uint32_t kIdesc = idesc_f16(128, 16, true, false, false);
+    const uint32_t ah = smem_u32(rhi), al = smem_u32(rlo), zb = smem_u32(zs);
+    int m = 0;
 #pragma unroll
-    for (int j = 0; j < RMAX; ++j)
-      if (j == q) v = f2_lo(acc[j]) + f2_hi(acc[j]);
-    if (q >= r) v = 0.0f;
-    if constexpr (sizeof(T) == 4) reinterpret_cast<float*>(ten.lfac)[row * a.r_max + q] = v;
-    else reinterpret_cast<__half*>(ten.lfac)[row * a.r_max + q] = __float2half_rn(v);
+    for (int part = 0; part < 3; ++part) {   // hi Zhi, hi Zlo, lo Zhi
+      const uint32_t abase = part == 2 ? al : ah;
+      const uint32_t bbase = zb + (part == 1 ? 4096 : 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk, ++m) {
+        const uint64_t ad = smem_desc_sw128(abase + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(bbase + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+        tc_mma_f16(tmem, ad, bd, kIdesc, m == 0 ? 0u : 1u);
+      }
+    }
+    tc_commit(&bars[1]);
+  }
+  if (ok && 8 * h < a.r_max) {
+    bool done = mbar_wait(&bars[1], 0);
+    if (!done) mbar_wait(&bars[1], 0);   // the product must finish before tensor memory is freed
+    tc_fence_after();
+    uint32_t v[8];
+    tmem_ld_32x32b_x8(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 8 * h, v);
+    tmem_ld_wait();
+    if (valid && done) {
+      const int q1 = min(a.r_max, 8 * h + 8);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (8 * h + j < q1) reinterpret_cast<float*>(ten.lfac)[row * a.r_max + 8 * h + j] = __uint_as_float(v[j]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
   }
 }
 
@@ -1183,10 +1729,10 @@ static cudaError_t launch_e1_b(const XMaps& map, const EncodeArgs& a, int grid, 
   }
 }
 
-template <typename T, int BITS, int RMAX>
-static cudaError_t launch_e3(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
-  auto kern = encode_lowrank<T, BITS, RMAX>;
-  constexpr int smem = E3Cfg<T, BITS, RMAX>::kSmem;
+template <typename T, int BITS, int RB>
+static cudaError_t launch_e3a(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
+  auto kern = encode_lowrank_alg<T, BITS, RB>;
+  const int smem = E3ACfg<T, BITS, RB>::smem(a.G * RB > 16 ? a.G * RB : 16);
   static std::atomic<int> smem_set[kMaxDevices];
   cudaError_t e = ensure_smem_limit(kern, smem, smem_set);
   if (e != cudaSuccess) return e;
@@ -1194,20 +1740,33 @@ static cudaError_t launch_e3(const E3Maps& maps, const EncodeArgs& a, dim3 grid,
   return cudaGetLastError();
 }
 
-template <typename T, int BITS>
-static cudaError_t launch_e3_r(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
-  if (a.r <= 4) return launch_e3<T, BITS, 4>(maps, a, grid, st);
-  if (a.r <= 8) return launch_e3<T, BITS, 8>(maps, a, grid, st);
-  return launch_e3<T, BITS, 16>(maps, a, grid, st);
+template <int BITS>
+static cudaError_t launch_e3f(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
+  auto kern = encode_lowrank_f32<BITS>;
+  constexpr int smem = E3Cfg<BITS>::kSmem;
+  static std::atomic<int> smem_set[kMaxDevices];
+  cudaError_t e = ensure_smem_limit(kern, smem, smem_set);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kE3Threads, smem, st>>>(maps, a);
+  return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_e3_b(const E3Maps& maps, const EncodeArgs& a, cudaStream_t st) {
   dim3 grid(a.tpu, a.U);
-  switch (a.bits) {
-    case 2: return launch_e3_r<T, 2>(maps, a, grid, st);
-    case 4: return launch_e3_r<T, 4>(maps, a, grid, st);
-    default: return launch_e3_r<T, 8>(maps, a, grid, st);
+  if constexpr (sizeof(T) == 4) {
+    switch (a.bits) {
+      case 2: return launch_e3f<2>(maps, a, grid, st);
+      case 4: return launch_e3f<4>(maps, a, grid, st);
+      default: return launch_e3f<8>(maps, a, grid, st);
+    }
+  } else {
+    const bool r8 = a.r_max <= 8;
+    switch (a.bits) {
+      case 2: return r8 ? launch_e3a<T, 2, 8>(maps, a, grid, st) : launch_e3a<T, 2, 16>(maps, a, grid, st);
+      case 4: return r8 ? launch_e3a<T, 4, 8>(maps, a, grid, st) : launch_e3a<T, 4, 16>(maps, a, grid, st);
+      default: return r8 ? launch_e3a<T, 8, 8>(maps, a, grid, st) : launch_e3a<T, 8, 16>(maps, a, grid, st);
+    }
   }
 }
 

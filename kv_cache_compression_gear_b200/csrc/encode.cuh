@@ -11,6 +11,15 @@ namespace gear {
 // u % Uper of tensor u / Uper.
 constexpr int kMaxBatch = 16;
 
+// Per-unit "Z slab" that E2 writes for E3 (bytes): the fp32 rows of Z
+// [128 channels][16 ranks], then S_g [4][16] floats with the power-of-two
+// scale of the images and its inverse, then the tensor-core operand images.
+constexpr int kSlabRows = 0;
+constexpr int kSlabS = 8192;          // 64 floats, then down, up (272 bytes in all)
+constexpr int kSlabSBytes = 272;
+constexpr int kSlabImg = 9216;        // X Z parts (3 x 4 KB at most), then C Z parts (2 x 16 KB at most)
+constexpr int kZSlab = kSlabImg + 3 * 4096 + 2 * 16384;
+
 struct EncodeTensor {
   const void* kv;    // input rows [Uper][n][128], cache dtype
   uint32_t* codes;   // the tensor's cache arrays
@@ -33,7 +42,7 @@ struct EncodeArgs {
   uint32_t one_bits;     // 0x3F800000 (1.0f), kept in a register by the kernels
   int32_t n_max, nblk_max, W, G, r_max;
   int32_t meta_f16;      // scale and zero stored as binary16
-  // workspace: partial Grams [U][maxc][128][128] and Z [U][64][16][2] (channel pairs)
+  // workspace: partial Grams [U][maxc][128][128] and Z slabs [U][kZSlab bytes] (E3 operands)
   float* gram;
   float* zbuf;
   // tiling of E1

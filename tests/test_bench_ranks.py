@@ -50,7 +50,13 @@ def test_reference_arm_runs_on_rank0_only(capsys):
 
 
 def test_both_arms_report_the_same_config():
+    """The headline is the 2-bit batch-64 workload (the largest fp16 configuration);
+    both arms name it, and the lines beside it name their own workloads."""
     c = bench.bench_config(1)
-    assert c["workload"] == "llama7b_layer_encode + decode_b16_ctx8192"
-    assert c["encode"]["tokens"] == 4096 and c["decode"]["context"] == 8192
+    assert c["workload"] == "twobit_b64_ctx8192"
+    assert c["encode"]["batch"] == 64 and c["encode"]["bits"] == 2 and c["decode"]["context"] == 8192
     assert bench.bench_config(4)["parallelism"] == "replicas x4"
+    names = [sc.name for sc in bench.BESIDE]
+    assert names == ["llama3_8b_gqa", "llama7b_layer_encode + decode_b16_ctx8192"]
+    g = bench.scenario_config(bench.BESIDE[0], 1)
+    assert g["encode"]["layers"] == 32 and g["decode"]["q_heads"] == 32 and g["decode"]["buffer"] == 20
