@@ -1247,10 +1247,9 @@ __device__ __forceinline__ void spread_codes(const uint32_t (&cw)[BITS], uint4 (
 template <typename T, int BITS, int RB>
 struct E3ACfg {
   static constexpr int kParts = std::is_same<T, __half>::value ? 2 : 3;   // X Z: fp16 hi + lo, bf16 hi + mid + lo
-  static constexpr int kX = 0;                         // input tile, 32 KB
-  static constexpr int kC = 32768;                     // spread codes, 32 KB
+  static constexpr int kX = 0;                         // input tile, then the spread codes, 32 KB
   static constexpr int kRow = 16 * BITS;               // code bytes per token
-  static constexpr int kCodes = 65536;                 // code tile
+  static constexpr int kCodes = 32768;                 // code tile
   static constexpr int kMeta = kCodes + kTile * kRow;  // meta tile (G <= 4)
   static constexpr int kZx = (kMeta + kTile * 32 + 1023) & ~1023;   // X Z operand: kParts x 4 KB
   static constexpr int kZc = kZx + kParts * 4096;      // C Z operand: 2 parts x NC x 256 B
@@ -1263,7 +1262,7 @@ struct E3ACfg {
 };
 
 template <typename T, int BITS, int RB>
-__global__ void __launch_bounds__(kE3Threads, 2) encode_lowrank_alg(const __grid_constant__ E3Maps maps,
+__global__ void __launch_bounds__(kE3Threads, 3) encode_lowrank_alg(const __grid_constant__ E3Maps maps,
                                                                      const EncodeArgs a) {
   using C = E1Cfg<T>;
   using F = E3ACfg<T, BITS, RB>;
@@ -1271,7 +1270,7 @@ __global__ void __launch_bounds__(kE3Threads, 2) encode_lowrank_alg(const __grid
   extern __shared__ uint8_t e3raw[];
   uint8_t* sm = align_smem_1024(e3raw);
   uint8_t* xs = sm + F::kX;
-  uint8_t* cps = sm + F::kC;
+  uint8_t* cps = xs;   // the spread codes overwrite the input tile once X Z is done
   uint8_t* cs = sm + F::kCodes;
   uint8_t* ms = sm + F::kMeta;
   uint8_t* zx = sm + F::kZx;
@@ -1340,8 +1339,28 @@ __global__ void __launch_bounds__(kE3Threads, 2) encode_lowrank_alg(const __grid
   ok = __syncthreads_and(ok);
   if (!ok && tid == 0) mbar_wait(&bars[0], 0);   // let copies still in flight land before the CTA ends
   const float down = S[64], up = S[65];   // the images' power-of-two scale and its inverse
-  // ---- spread codes of this half row
+  // ---- X Z into columns [0, 16): the input tile against the parts of Z along K
+  if (ok && tid == 0) {
+    tc_fence_after();
+    constexpr uint32_t kIdX = idesc_f16(128, 16, std::is_same<P, __nv_bfloat16>::value, false, false);
+    const uint32_t xa = smem_u32(xs), za = smem_u32(zx);
+    int m = 0;
+#pragma unroll
+    for (int part = 0; part < F::kParts; ++part)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk, ++m) {
+        const uint64_t ad = smem_desc_sw128(xa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(za + part * 4096 + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+        tc_mma_f16(tmem, ad, bd, kIdX, m == 0 ? 0u : 1u);
+      }
+    tc_commit(&bars[1]);
+  }
+  // ---- spread codes of this half row, written over the input tile once X Z has read it
+  bool xz_done = true;
   if (ok) {
+    xz_done = mbar_wait(&bars[1], 0);
+    if (!xz_done) mbar_wait(&bars[1], 0);   // nothing may overwrite the tile while the product reads it
+    tc_fence_after();
     const uint8_t* rowp = cs + t * F::kRow;
 #pragma unroll
     for (int qq = 0; qq < 2; ++qq) {
@@ -1372,22 +1391,10 @@ __global__ void __launch_bounds__(kE3Threads, 2) encode_lowrank_alg(const __grid
   __syncthreads();
   tc_fence_after();
   if (ok && tid == 0) {
-    // X Z into columns [0, 16): the parts of Z along K
-    constexpr uint32_t kIdX = idesc_f16(128, 16, std::is_same<P, __nv_bfloat16>::value, false, false);
-    const uint32_t xa = smem_u32(xs), za = smem_u32(zx);
-    int m = 0;
-#pragma unroll
-    for (int part = 0; part < F::kParts; ++part)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk, ++m) {
-        const uint64_t ad = smem_desc_sw128(xa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd = smem_desc_sw128(za + part * 4096 + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
-        tc_mma_f16(tmem, ad, bd, kIdX, m == 0 ? 0u : 1u);
-      }
     // C Z into columns [32, 32 + NC): hi then lo part of Z
     const uint32_t kIdC = idesc_f16(128, NC, false, false, false);
     const uint32_t ca = smem_u32(cps), zb = smem_u32(zc);
-    m = 0;
+    int m = 0;
 #pragma unroll
     for (int part = 0; part < 2; ++part)
 #pragma unroll
@@ -1401,8 +1408,8 @@ __global__ void __launch_bounds__(kE3Threads, 2) encode_lowrank_alg(const __grid
   }
   // ---- epilogue: thread (t, h) writes ranks [8 h, 8 h + 8) of token t
   if (ok && 8 * h < a.r_max) {
-    bool done = mbar_wait(&bars[1], 0);
-    if (!done) mbar_wait(&bars[1], 0);   // the products must finish before tensor memory is freed
+    bool done = mbar_wait(&bars[1], 1) && xz_done;
+    if (!done) mbar_wait(&bars[1], 1);   // the products must finish before tensor memory is freed
     tc_fence_after();
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint32_t vx[8], vc[4][8];
