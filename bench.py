@@ -329,13 +329,17 @@ def dec_alg_bytes(w, n_comp: int, n_blk: int, n_buf: int, layers: int) -> int:
 class Runner:
     """Holds the device state of one scenario and runs its steps."""
 
-    def __init__(self, gear, wl, sc: Scenario, dev, rank: int, n_steps_total: int, batch_override=None):
+    def __init__(self, gear, wl, sc: Scenario, dev, rank: int, n_steps_total: int, batch_override=None,
+                 layers_override=None):
         import torch
         self.gear, self.wl, self.sc, self.dev = gear, wl, sc, dev
         we, wd = wl.WORKLOADS[sc.enc], wl.WORKLOADS[sc.dec]
         if batch_override:
             we = dataclasses.replace(we, B=batch_override)
             wd = dataclasses.replace(wd, B=batch_override) if not sc.same else we
+        if layers_override:
+            we = dataclasses.replace(we, layers=layers_override)
+            wd = dataclasses.replace(wd, layers=layers_override) if not sc.same else we
         self.we, self.wd = we, wd
         dt = wl.torch_dtype(we.dtype)
         # ---- encode inputs and caches (per layer: K and V); rank r selects the data
@@ -496,9 +500,9 @@ TRAFFIC_BYTES = {
 
 
 def measure(gear, wl, sc: Scenario, dev, rank, world, steps, warmup, hbm, peak_kind, batch_override=None,
-            with_e2e=True):
+            with_e2e=True, layers_override=None):
     import torch
-    runner = Runner(gear, wl, sc, dev, rank, warmup + steps + 1, batch_override)
+    runner = Runner(gear, wl, sc, dev, rank, warmup + steps + 1, batch_override, layers_override)
     we, wd = runner.we, runner.wd
     for _ in range(warmup):
         runner.step(None)
@@ -578,6 +582,13 @@ def run_gpu(args, rank: int, world: int):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     hbm, peak_kind = peaks()
+    if args.profile_case:
+        sc = [b for b in BESIDE if b.enc == args.profile_case][0]
+        res = measure(gear, wl, sc, dev, rank, world, args.steps, args.warmup, hbm, peak_kind,
+                      layers_override=2 if sc.enc == "llama3_8b_gqa" else None, with_e2e=False)
+        if rank == 0:
+            print(json.dumps({"profile_case": scenario_config(sc, world), **res}), flush=True)
+        return
     if args.batch_override:
         # a smaller batch of the headline workload, for counter captures only (not a bench value)
         res = measure(gear, wl, HEADLINE, dev, rank, world, args.steps, args.warmup, hbm, peak_kind,
@@ -689,6 +700,9 @@ def main():
     ap.add_argument("--impl", default="gear", choices=["gear", "reference"])
     ap.add_argument("--batch-override", type=int, default=None,
                     help="run only the headline workload at this batch (a small case for counter captures)")
+    ap.add_argument("--profile-case", default=None, choices=["llama3_8b_gqa", "llama7b_layer_encode"],
+                    help="run only this workload beside the headline (the GQA cache with 2 of its 32 layers), "
+                         "a small case for counter captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -73,6 +73,19 @@ typedef enum { GEAR_F16 = 0, GEAR_BF16 = 1, GEAR_F32 = 2 } gear_dtype;
  *               binary16, rounded to nearest even, with the codes decided
  *               against the stored values (a byte-lean layout: 4 instead of
  *               8 bytes per group; fp16 caches only, else UNSUPPORTED).
+ *  channel_groups 0: the quantizer groups g channels of a token (default);
+ *               1: the KIVI-combined key quantizer -- every channel gets its
+ *               own (scale, zero) over each group of g consecutive tokens of a
+ *               block (the last group of the block written by gear_encode may
+ *               be shorter); outliers stay per token and are left out of the
+ *               groups' min/max (GEAR: An Efficient KV Cache Compression
+ *               Recipe ..., Cites list, KIVI entries: the buffer must be at
+ *               least the group size; the same page's citing works, TailorKV
+ *               entry: keys per channel, values per token). Requires a 16-bit
+ *               cache, meta_f16 = 0, g in {32, 64, 128} and a buffer_len that
+ *               is a multiple of g (>= g), so that every flushed buffer is
+ *               whole groups (else INVALID_ARG / UNSUPPORTED). In decode such a
+ *               cache serves as the K cache, with a V cache of channel_groups 0.
  *  seed         seeds the power-iteration start matrix Q0 (d x r): entry
  *               (i, j) is the (i*r + j)-th output of the splitmix64 stream
  *               whose state starts at `seed` (Steele, Lea & Flood, OOPSLA
@@ -86,6 +99,7 @@ typedef struct gear_params {
   int32_t buffer_len;
   int32_t buffer_rank;
   int32_t meta_f16;
+  int32_t channel_groups;
   uint64_t seed;
 } gear_params;
 
@@ -102,6 +116,11 @@ typedef struct gear_params {
  *   meta   float  [U][n_max][G][2]   G = d/g; (scale, zero) of each group,
  *                                    zero = group minimum over non-outliers
  *                                    (binary16 [U][n_max][G][2] if meta_f16).
+ *                                    With channel_groups: float
+ *                                    [U][S][d][2], S = ceil(n_max/g) + 1 token
+ *                                    groups; token t of block 0 is in group
+ *                                    t / g, token t of a flushed block in group
+ *                                    ceil(blk0_len/g) + (t - blk0_len) / g.
  *   oidx   uint8  [U][n_max][k]      outlier channels, ascending.
  *   oval   dtype  [U][n_max][k]      outlier values, bit-exact input copies.
  *   lfac   f16|f32[U][n_max][r_max]  L rows, stored as L * 2^e_blk.

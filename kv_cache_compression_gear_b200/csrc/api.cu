@@ -50,7 +50,10 @@ static Layout cache_layout(const gear_params* p, int B, int H, int d, int n_max,
   const int rm = rmax > 0 ? rmax : 1;
   size_t off = 0;
   L.codes = off; off = align256(off + U * n_max * W * 4);
-  L.meta = off;  off = align256(off + U * n_max * G * (size_t)meta_row_bytes(1, p->meta_f16));
+  if (p->channel_groups)   // [U][slots][d][2] fp32, one slot per token group
+    L.meta = off, off = align256(off + U * (size_t)channel_group_slots(n_max, p->group_size) * d * 8);
+  else
+    L.meta = off, off = align256(off + U * n_max * G * (size_t)meta_row_bytes(1, p->meta_f16));
   L.oidx = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1));
   L.oval = off;  off = align256(off + U * n_max * (size_t)(k > 0 ? k : 1) * esize(dt));
   L.lfac = off;  off = align256(off + U * n_max * rm * (dt == GEAR_F32 ? 4 : 2));
@@ -81,6 +84,15 @@ static bool same_shape(const gear_cache* a, const gear_cache* b) {
          memcmp(&a->p, &b->p, sizeof(gear_params)) == 0;
 }
 
+// True when k and v can serve as the K and V caches of one layer: identical
+// parameters, except that K may use per-channel key groups (the KIVI-combined
+// quantizer) while V keeps per-token groups.
+static bool kv_params_match(const gear_cache* k, const gear_cache* v) {
+  gear_params pk = k->p;
+  pk.channel_groups = v->p.channel_groups;
+  return v->p.channel_groups == 0 && memcmp(&pk, &v->p, sizeof(gear_params)) == 0;
+}
+
 // Encodes n tokens per unit of kvs[i] into cs[i] (i < nt <= kMaxBatch, all of
 // one shape) as block `blk` at token offset t_off, in one launch per kernel.
 static gear_status encode_block(gear_cache* const* cs, const void* const* kvs, int nt, int n, int t_off, int blk,
@@ -109,6 +121,12 @@ static gear_status encode_block(gear_cache* const* cs, const void* const* kvs, i
   a.G = c->G;
   a.r_max = c->r_max;
   a.meta_f16 = c->p.meta_f16;
+  a.ch = c->p.channel_groups;
+  if (a.ch) {
+    a.ch_slots = channel_group_slots(c->n_max, a.g);
+    // block 0 (possibly ending in a shorter group), then whole groups per flushed block
+    a.slot0 = blk == 0 ? 0 : (c->blk0_len + a.g - 1) / a.g + (t_off - c->blk0_len) / a.g;
+  }
   for (int i = 0; i < nt; ++i)
     a.ten[i] = EncodeTensor{kvs[i], cs[i]->codes, cs[i]->meta, cs[i]->oidx, cs[i]->oval, cs[i]->lfac, cs[i]->rfac};
   a.tpu = (n + 127) / 128;
@@ -186,6 +204,11 @@ gear_status gear_validate_params(const gear_params* p, int32_t d) {
   if ((p->rank > 0 || p->buffer_rank > 0) && p->power_iters < 1) return GEAR_ERR_INVALID_ARG;
   if (p->power_iters < 0) return GEAR_ERR_INVALID_ARG;
   if (p->meta_f16 != 0 && p->meta_f16 != 1) return GEAR_ERR_INVALID_ARG;
+  if (p->channel_groups != 0 && p->channel_groups != 1) return GEAR_ERR_INVALID_ARG;
+  if (p->channel_groups) {   // whole token groups in every flushed buffer; the buffer at least one group
+    if (p->buffer_len < p->group_size || p->buffer_len % p->group_size != 0) return GEAR_ERR_INVALID_ARG;
+    if (p->meta_f16) return GEAR_ERR_UNSUPPORTED;
+  }
   if (d != 128) return GEAR_ERR_UNSUPPORTED;
   if (p->group_size < 32) return GEAR_ERR_UNSUPPORTED;
   if (gear_num_outliers(p->outlier_frac, d) > 16) return GEAR_ERR_UNSUPPORTED;
@@ -197,6 +220,7 @@ size_t gear_cache_bytes(const gear_params* p, int32_t B, int32_t H, int32_t d, i
   if (gear_validate_params(p, d) != GEAR_OK) return 0;
   if (B <= 0 || H <= 0 || n_max <= 0 || nblk_max <= 0 || dtype < GEAR_F16 || dtype > GEAR_F32) return 0;
   if (p->meta_f16 && dtype != GEAR_F16) return 0;
+  if (p->channel_groups && dtype == GEAR_F32) return 0;
   return cache_layout(p, B, H, d, n_max, nblk_max, dtype).total;
 }
 
@@ -209,6 +233,7 @@ gear_status gear_cache_init(gear_cache* c, const gear_params* p, int32_t B, int3
     return GEAR_ERR_INVALID_ARG;
   if (!aligned(dev, 256)) return GEAR_ERR_INVALID_ARG;
   if (p->meta_f16 && dtype != GEAR_F16) return GEAR_ERR_UNSUPPORTED;   // binary16 metadata of fp16 input only
+  if (p->channel_groups && dtype == GEAR_F32) return GEAR_ERR_UNSUPPORTED;   // per-channel keys of 16-bit caches
   if ((size_t)B * H * round_nmax(n_max) >= ((size_t)1 << 31)) return GEAR_ERR_UNSUPPORTED;
   Layout L = cache_layout(p, B, H, d, n_max, nblk_max, dtype);
   if (bytes < L.total) return GEAR_ERR_CAPACITY;
@@ -296,7 +321,7 @@ static gear_status decode_args(const gear_cache* k, const gear_cache* v, int32_t
   if (!cache_ok(k) || !cache_ok(v)) return GEAR_ERR_INVALID_ARG;
   if (k->B != v->B || k->H != v->H || k->dtype != v->dtype || k->n_comp != v->n_comp || k->n_buf != v->n_buf ||
       k->n_blk != v->n_blk || k->blk0_len != v->blk0_len || k->n_max != v->n_max || k->nblk_max != v->nblk_max ||
-      memcmp(&k->p, &v->p, sizeof(gear_params)) != 0)
+      !kv_params_match(k, v))
     return GEAR_ERR_INVALID_ARG;
   if (Hq <= 0 || Hq % k->H != 0 || Hq / k->H > 8) return GEAR_ERR_INVALID_ARG;
   if (k->n_comp + k->n_buf == 0) return GEAR_ERR_INVALID_ARG;
@@ -307,6 +332,9 @@ static gear_status decode_args(const gear_cache* k, const gear_cache* v, int32_t
   a.B = k->B; a.H = k->H; a.Hq = Hq; a.hq = Hq / k->H;
   a.bits = k->p.bits; a.g = k->p.group_size; a.G = k->G; a.W = k->W; a.k = k->k; a.r_max = k->r_max;
   a.meta_f16 = k->p.meta_f16;
+  a.kc = k->p.channel_groups;
+  a.ch_slots = a.kc ? channel_group_slots(k->n_max, k->p.group_size) : 0;
+  if (a.kc && a.hq > 4) return GEAR_ERR_UNSUPPORTED;   // per-channel key groups: up to 4 query heads per kv head
   a.n_max = k->n_max; a.nblk_max = k->nblk_max; a.n_b = k->p.buffer_len;
   a.n_comp = k->n_comp; a.n_buf = k->n_buf;
   a.blk0_len = k->blk0_len; a.blk0_rank = k->blk0_rank; a.buffer_rank = k->p.buffer_rank;
@@ -362,7 +390,7 @@ gear_status gear_append_buffer(gear_cache* k, gear_cache* v, const void* k_new, 
                                size_t ws_bytes, void* stream) {
   if (!cache_ok(k) || !cache_ok(v) || !k_new || !v_new) return GEAR_ERR_INVALID_ARG;
   if (k->B != v->B || k->H != v->H || k->dtype != v->dtype || k->n_comp != v->n_comp || k->n_buf != v->n_buf ||
-      k->n_blk != v->n_blk || memcmp(&k->p, &v->p, sizeof(gear_params)) != 0)
+      k->n_blk != v->n_blk || !kv_params_match(k, v))
     return GEAR_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   const int n_b = k->p.buffer_len;
@@ -413,6 +441,8 @@ gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream)
   a.U = c->B * c->H;
   a.bits = c->p.bits; a.g = c->p.group_size; a.G = c->G; a.W = c->W; a.k = c->k; a.r_max = c->r_max;
   a.meta_f16 = c->p.meta_f16;
+  a.ch = c->p.channel_groups;
+  a.ch_slots = a.ch ? channel_group_slots(c->n_max, c->p.group_size) : 0;
   a.n_max = c->n_max; a.nblk_max = c->nblk_max; a.n_b = c->p.buffer_len;
   a.n_comp = c->n_comp; a.n_buf = c->n_buf;
   a.blk0_len = c->blk0_len; a.blk0_rank = c->blk0_rank; a.buffer_rank = c->p.buffer_rank;

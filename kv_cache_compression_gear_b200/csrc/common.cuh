@@ -97,6 +97,10 @@ struct CodeFloats {
 // Bytes of G groups' (scale, zero) pairs: fp32 pairs, or binary16 pairs.
 __host__ __device__ constexpr int meta_row_bytes(int G, int meta_f16) { return G * (meta_f16 ? 4 : 8); }
 
+// Token-group slots of a cache with per-channel key groups of g tokens: block
+// 0 may end in a shorter group, every flushed block holds whole groups.
+__host__ __device__ constexpr int channel_group_slots(int n_max, int g) { return (n_max + g - 1) / g + 1; }
+
 // Row length of the stored Rf factors: r_max rounded up to a multiple of 4, so
 // that one channel's row is a whole number of 16-byte vectors.
 __host__ __device__ constexpr int rpad_of(int r_max) { return (r_max + 3) & ~3; }

@@ -7,6 +7,12 @@
 
 namespace gear {
 
+constexpr int kDTile = 32;       // tokens per decode tile (one per lane)
+// token stride of one group's value weights in shared memory: the two tokens
+// and G groups a value-loop step reads fall in distinct banks
+constexpr int kWStride = kDTile + 2;
+constexpr int kMaxR = 16;        // largest rank
+
 // One compressed tensor as the decode kernels see it.
 struct CacheView {
   const uint32_t* codes;
@@ -47,6 +53,7 @@ struct DecodeArgs {
   int32_t B, H, Hq, hq;   // hq = Hq / H query heads per kv head
   int32_t bits, g, G, W, k, r_max;
   int32_t meta_f16;       // (scale, zero) pairs stored as binary16
+  int32_t kc, ch_slots;   // K quantized per channel over token groups; token-group slots per unit
   int32_t n_max, nblk_max, n_b;
   int32_t n_comp, n_buf;
   int32_t blk0_len, blk0_rank, buffer_rank;
@@ -68,11 +75,18 @@ struct DenseArgs {
   int32_t dtype;
   int32_t U, bits, g, G, W, k, r_max, n_max, nblk_max, n_b;
   int32_t meta_f16;
+  int32_t ch, ch_slots;   // per-channel key groups: meta per token-group slot
   int32_t n_comp, n_buf, blk0_len, blk0_rank, buffer_rank;
   float* out;             // [U][n_comp + n_buf][128]
 };
 
 void decode_plan(DecodeArgs& a, int num_sms);
+// decode_warp launches for each cache dtype (decode_f16.cu, decode_bf16.cu, decode_f32.cu)
+cudaError_t decode_warp_launch_f16(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st);
+cudaError_t decode_warp_launch_bf16(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st);
+cudaError_t decode_warp_launch_f32(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st);
+// K caches with per-channel key groups, fp16 or bf16 (decode_kc.cu)
+cudaError_t decode_warp_launch_kc(const DecodeMaps& maps, const DecodeArgs& a, cudaStream_t st);
 size_t decode_workspace_bytes(int B, int Hq, int nsplit);
 cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t st);
 cudaError_t dense_launch(const DenseArgs& a, cudaStream_t st);

@@ -141,6 +141,14 @@ __device__ __forceinline__ uint64_t div_pair_fast(uint64_t a, uint64_t s2n, uint
 __device__ __forceinline__ uint64_t div_pair_slow(uint64_t a, float s) {
   return f2_pack(__fdiv_rn(f2_lo(a), s), __fdiv_rn(f2_hi(a), s));
 }
+__device__ __forceinline__ uint64_t div_pair_slow2(uint64_t a, float s0, float s1) {
+  return f2_pack(__fdiv_rn(f2_lo(a), s0), __fdiv_rn(f2_hi(a), s1));
+}
+
+// Barrier among `count` threads (whole warps) under id (1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 // ================================================================ E1 ======
 // Shared-memory map of E1 (dynamic, 1024-byte aligned):
@@ -170,6 +178,12 @@ struct E1Cfg {
   static constexpr int kBoxes = 128 / kBoxCols;
   static constexpr uint32_t kBarOff = kNX * kXBytes + kNR * kRBytes;
   static constexpr uint32_t kSmem = kBarOff + 256 + 1024;     // + alignment slack
+  // per-channel key groups: per quantizer group, the column min/max partials
+  // [4 x 32-token blocks][64 channel pairs] (2 KB), then the channels'
+  // (zero, scale, 1/scale, fast) of up to 4 token groups (8 KB)
+  static constexpr uint32_t kChOff = kBarOff + 256;
+  static constexpr uint32_t kChBytes = 10240;
+  static constexpr uint32_t kSmemCh = kSmem + kGroups * kChBytes;
 };
 
 struct XMaps {
@@ -274,9 +288,10 @@ __device__ __forceinline__ void topk_candidates(const uint32_t (&xr)[32], int k,
 // One quantizer thread: half h (channels 64h .. 64h+63) of token t of the tile.
 // Writes codes/meta/outliers of the token to the cache and the residual split
 // into the R stage. `valid` is false for tile rows past the unit's last token.
-template <typename T, int BITS, int KMAX>
+template <typename T, int BITS, int KMAX, bool CH>
 __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, uint8_t* rs, int t, int h,
-                                              bool valid, int u, int tok, uint64_t* x_release) {
+                                              bool valid, int u, int tok, uint64_t* x_release, uint8_t* chs,
+                                              int group, int t0) {
   constexpr int kCodesPerWord = 32 / BITS;
   constexpr int kWordsHalf = 64 * BITS / 32;
   const float levels = (float)((1 << BITS) - 1);
@@ -407,15 +422,72 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       xr[4 * j + 0] = v.x; xr[4 * j + 1] = v.y; xr[4 * j + 2] = v.z; xr[4 * j + 3] = v.w;
     }
   }
-  // the X stage is not read again: hand it back to the producer
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(x_release);
+  if constexpr (!CH) {
+    // the X stage is not read again: hand it back to the producer
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(x_release);
+  }
+
+  // ---------------- per-channel key groups (KIVI-combined) -----------------
+  // Every channel gets its own (zero, scale) over each group of g consecutive
+  // tokens; the tile's 128 rows (outlier slots now NaN, which min/max ignore)
+  // are read column-wise by the group's 256 threads, one channel pair and one
+  // 32-token block each, after all rows are patched.
+  float4* prm = reinterpret_cast<float4*>(chs + 2048);
+  if constexpr (CH) {
+    const int qid = 2 * t + h;
+    uint2* part = reinterpret_cast<uint2*>(chs);
+    named_barrier_sync(1 + group, kQThreads);
+    {
+      const int cp = qid & 63, sb = qid >> 6;
+      const int nval = min(a.n - t0, kTile);
+      const uint32_t nan2 = (uint32_t)Elem16<T>::kNaN * 0x10001u;
+      uint32_t lo2 = nan2, hi2 = nan2;
+      const uint8_t* col = xs + (cp >> 5) * 16384 + (cp & 3) * 4;
+      for (int r = 32 * sb; r < 32 * sb + 32; ++r) {
+        if (r >= nval) break;
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(col + swz(r, (cp & 31) >> 2));
+        lo2 = pair_min<T>(lo2, v);
+        hi2 = pair_max<T>(hi2, v);
+      }
+      part[sb * 64 + cp] = make_uint2(lo2, hi2);
+    }
+    named_barrier_sync(1 + group, kQThreads);
+    // the X stage is not read again: hand it back to the producer
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(x_release);
+    {
+      const int ng = kTile / a.g, sbg = a.g / 32;
+      const EncodeTensor& ten = a.ten[u / a.Uper];
+      const size_t slot_row = ((size_t)(u % a.Uper) * a.ch_slots + a.slot0 + t0 / a.g) * 128;
+      for (int e = qid; e < ng * 128; e += kQThreads) {
+        const int j = e >> 7, c = e & 127;
+        float mnc = __uint_as_float(0x7FC00000u), mxc = mnc;
+        for (int sb = j * sbg; sb < (j + 1) * sbg; ++sb) {
+          const uint2 pr = part[sb * 64 + (c >> 1)];
+          const float2 l = Elem16<T>::to_f2(pr.x), hv = Elem16<T>::to_f2(pr.y);
+          mnc = fminf(mnc, (c & 1) ? l.y : l.x);
+          mxc = fmaxf(mxc, (c & 1) ? hv.y : hv.x);
+        }
+        if (isnan(mnc)) { mnc = 0.0f; mxc = 0.0f; }   // no non-outlier entry
+        mnc = __fadd_rn(mnc, 0.0f);                    // -0 -> +0
+        mxc = __fadd_rn(mxc, 0.0f);
+        const float sc = __fdiv_rn(__fsub_rn(mxc, mnc), levels);
+        const bool fst = (sc >= 0x1p-100f && sc <= 0x1p100f) || sc == 0.0f;
+        prm[j * 128 + c] = make_float4(mnc, sc, sc == 0.0f ? 0.0f : __frcp_rn(sc), fst ? 1.0f : 0.0f);
+        if (t0 + j * a.g < a.n)   // a group with tokens of this block: its meta to the cache
+          reinterpret_cast<float2*>(ten.meta)[slot_row + (size_t)j * 128 + c] = make_float2(sc, mnc);
+      }
+    }
+    named_barrier_sync(1 + group, kQThreads);
+  }
 
   // ---------------- group min / max over non-outliers ----------------------
   // Two 32-channel sub-halves; combined for g >= 64, and with the partner for
   // g = 128. NaN (outlier) operands are ignored by min/max.
-  float mn[2], mx[2];
-  if constexpr (sizeof(T) == 4) {
+  float mn[2] = {0.0f, 0.0f}, mx[2] = {0.0f, 0.0f};
+  if constexpr (CH) {
+  } else if constexpr (sizeof(T) == 4) {
 #pragma unroll
     for (int sh = 0; sh < 2; ++sh) {
       float lo = __uint_as_float(0x7FC00000u), hi = lo;
@@ -441,19 +513,19 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       mx[sh] = fmaxf(u2.x, u2.y);
     }
   }
-  if (a.g >= 64) {
+  if (!CH && a.g >= 64) {
     mn[0] = mn[1] = fminf(mn[0], mn[1]);
     mx[0] = mx[1] = fmaxf(mx[0], mx[1]);
   }
-  if (a.g == 128) {
+  if (!CH && a.g == 128) {
     float om = __shfl_xor_sync(0xFFFFFFFFu, mn[0], 1), oM = __shfl_xor_sync(0xFFFFFFFFu, mx[0], 1);
     mn[0] = mn[1] = fminf(mn[0], om);
     mx[0] = mx[1] = fmaxf(mx[0], oM);
   }
-  float scale[2], y[2];
-  bool fast[2];
+  float scale[2] = {0.0f, 0.0f}, y[2] = {0.0f, 0.0f};
+  bool fast[2] = {true, true};
 #pragma unroll
-  for (int sh = 0; sh < 2; ++sh) {
+  for (int sh = 0; sh < 2 && !CH; ++sh) {
     if (isnan(mn[sh])) { mn[sh] = 0.0f; mx[sh] = 0.0f; }   // group made of outliers only
     mn[sh] = __fadd_rn(mn[sh], 0.0f);                      // -0 -> +0
     mx[sh] = __fadd_rn(mx[sh], 0.0f);
@@ -474,14 +546,12 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
   // one pair of channels (2p, 2p + 1); DIV is the division of the pair. The
   // residual split (hi = bf16(R), lo = bf16(R - hi)) comes back packed in ho, lo.
   auto qpair = [&](const int p, const uint64_t mnv, const uint64_t sc2, auto div, uint32_t& ho, uint32_t& lo) {
-    const int sh = p >> 4;
     float x0, x1;
     if constexpr (sizeof(T) == 4) {
-      x0 = fmaxf(__uint_as_float(xr[2 * p]), mn[sh]);       // NaN -> zero point
-      x1 = fmaxf(__uint_as_float(xr[2 * p + 1]), mn[sh]);
+      x0 = fmaxf(__uint_as_float(xr[2 * p]), f2_lo(mnv));       // NaN -> zero point
+      x1 = fmaxf(__uint_as_float(xr[2 * p + 1]), f2_hi(mnv));
     } else {
-      uint32_t m2 = Elem16<T>::from_f(mn[sh]);
-      m2 |= m2 << 16;
+      const uint32_t m2 = Elem16<T>::from_f(f2_lo(mnv)) | (Elem16<T>::from_f(f2_hi(mnv)) << 16);
       const float2 f = Elem16<T>::to_f2(pair_max<T>(xr[p], m2));  // NaN -> zero point
       x0 = f.x; x1 = f.y;
     }
@@ -521,8 +591,29 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       *reinterpret_cast<uint4*>(ph + 32768) = make_uint4(0u, 0u, 0u, 0u);
     }
   };
+  if constexpr (CH) {
+    // per channel: the (zero, scale, 1/scale) of the token's group
+    const float4* pj = prm + (t / a.g) * 128 + 64 * h;
 #pragma unroll
-  for (int sh = 0; sh < 2; ++sh) {
+    for (int jj = 0; jj < 8; ++jj) {
+      uint32_t h4[4], l4[4];
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp) {
+        const int p = 4 * jj + pp;
+        const float4 P0 = pj[2 * p], P1 = pj[2 * p + 1];
+        const uint64_t mnv = f2_pack(P0.x, P1.x), sc2 = f2_pack(P0.y, P1.y);
+        if (P0.w != 0.0f && P1.w != 0.0f) {
+          const uint64_t y2 = f2_pack(P0.z, P1.z), s2n = f2_pack(-P0.y, -P1.y);
+          qpair(p, mnv, sc2, [&](uint64_t av) { return div_pair_fast(av, s2n, y2); }, h4[pp], l4[pp]);
+        } else {
+          qpair(p, mnv, sc2, [&](uint64_t av) { return div_pair_slow2(av, P0.y, P1.y); }, h4[pp], l4[pp]);
+        }
+      }
+      chunk_out(jj, h4, l4);
+    }
+  }
+#pragma unroll
+  for (int sh = 0; sh < 2 && !CH; ++sh) {
     const uint64_t mnv = f2_pack(mn[sh], mn[sh]);
     const uint64_t sc2 = f2_pack(scale[sh], scale[sh]);
     if (fast[sh]) {
@@ -571,7 +662,9 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
       if (a.meta_f16) reinterpret_cast<__half2*>(ten.meta)[row * a.G + gi] = __floats2half2_rn(sc, z);   // exact
       else reinterpret_cast<float2*>(ten.meta)[row * a.G + gi] = make_float2(sc, z);
     };
-    if (gsz == 32) {
+    if (CH) {
+      // per-channel groups: the meta was written by the column pass
+    } else if (gsz == 32) {
       put_meta(2 * h, scale[0], mn[0]);
       put_meta(2 * h + 1, scale[1], mn[1]);
     } else if (gsz == 64) {
@@ -641,7 +734,7 @@ __device__ __forceinline__ void quantize_half(const EncodeArgs& a, uint8_t* xs, 
   }
 }
 
-template <typename T, int BITS, int KMAX>
+template <typename T, int BITS, int KMAX, bool CH>
 __global__ void __launch_bounds__(E1Cfg<T>::kThreads, 1)
     encode_quant_gram(const __grid_constant__ XMaps maps, const EncodeArgs a) {
   using C = E1Cfg<T>;
@@ -783,8 +876,8 @@ __global__ void __launch_bounds__(E1Cfg<T>::kThreads, 1)
       ok = mbar_wait(&bars->x_full[s], (it / C::kNX) & 1);
       ok = ok && mbar_wait(&bars->r_empty[sr], ((it / kNR) & 1) ^ 1);
       if (!ok || bars->abort_flag) { ok = false; break; }
-      quantize_half<T, BITS, KMAX>(a, xst + s * C::kXBytes, rst + sr * kRBytes, t, h, t0 + t < a.n, u, t0 + t,
-                                   &bars->x_empty[s]);
+      quantize_half<T, BITS, KMAX, CH>(a, xst + s * C::kXBytes, rst + sr * kRBytes, t, h, t0 + t < a.n, u, t0 + t,
+                                       &bars->x_empty[s], smem + C::kChOff + group * C::kChBytes, group, t0);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->r_full[sr]);
@@ -899,7 +992,7 @@ __device__ void write_z_slab(const EncodeArgs& a, int u, const float* Zf, float*
   __syncthreads();
   m = 0.0f;
   for (int w = 0; w < nth / 32; ++w) m = fmaxf(m, red[w]);
-  const bool wide = a.dtype == GEAR_F32;   // fp32 inputs: bf16 hi + lo, unscaled
+  const bool wide = a.dtype == GEAR_F32 || a.ch;   // the rebuilding pass: bf16 hi + lo, unscaled
   int sh = 0;
   if (!wide && m > 0.0f) sh = min(max(((__float_as_int(m) >> 23) & 0xFF) - 127 - 3, -100), 100);
   const float down = __int_as_float((127 - sh) << 23), up = __int_as_float((127 + sh) << 23);
@@ -911,7 +1004,7 @@ __device__ void write_z_slab(const EncodeArgs& a, int u, const float* Zf, float*
     float rest = Zf[c * 16 + n] * down;
     for (int part = 0; part < parts; ++part) {
       uint16_t bitsv;
-      if (a.dtype == GEAR_F16) {
+      if (a.dtype == GEAR_F16 && !wide) {
         const __half hv = __float2half_rn(rest);
         bitsv = __half_as_ushort(hv);
         rest -= __half2float(hv);
@@ -1259,6 +1352,7 @@ struct E3ACfg {
   static __host__ __device__ constexpr int zr_off(int NC) { return s_off(NC) + 1024; }
   static __host__ __device__ constexpr int bar_off(int NC) { return zr_off(NC) + 8192; }
   static __host__ __device__ constexpr int smem(int NC) { return bar_off(NC) + 64 + 1024; }   // + alignment slack
+  // three barriers (24 bytes), the tensor-memory slot at +32
 };
 
 template <typename T, int BITS, int RB>
@@ -1279,196 +1373,234 @@ __global__ void __launch_bounds__(kE3Threads, 3) encode_lowrank_alg(const __grid
   const int NC = G * RB > 16 ? G * RB : 16;
   float* S = reinterpret_cast<float*>(sm + F::s_off(NC));
   const float* zr = reinterpret_cast<const float*>(sm + F::zr_off(NC));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + F::bar_off(NC));   // [0] tile landed, [1] products done
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + F::bar_off(NC) + 16);
+  // [0] tile landed (one phase per tile), [1] products done (two phases per tile), [2] unit operands landed
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + F::bar_off(NC));
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + F::bar_off(NC) + 32);
   const int tid = threadIdx.x, t = tid & 127, h = tid >> 7, warp = tid >> 5;
-  const int u = blockIdx.y, t0 = blockIdx.x * kTile;
+  const int u = blockIdx.y;
+  const int tile0 = blockIdx.x * a.e3_tpc;
+  const int ntile = min(a.e3_tpc, a.tpu - tile0);
   const int mrb = meta_row_bytes(G, a.meta_f16);
   const bool meta_tma = mrb >= 16;
   const int lg = a.g == 32 ? 5 : (a.g == 64 ? 6 : 7);
   const int tn = u / a.Uper, ul = u % a.Uper;
   const EncodeTensor& ten = a.ten[tn];
-  const int crow = ul * a.n_max + a.t_off + t0;
   const uint8_t* slab = reinterpret_cast<const uint8_t*>(a.zbuf) + (int64_t)u * kZSlab;
   const uint32_t img_bytes = (uint32_t)(F::kParts * 4096 + 2 * NC * 256);
+  const uint32_t tile_bytes = (uint32_t)(32768 + kTile * F::kRow + (meta_tma ? kTile * mrb : 0));
+  // the tile's input rows, code rows and meta rows (one phase of bars[0])
+  auto issue_tile = [&](int it) {
+    const int tt0 = (tile0 + it) * kTile;
+    const int crow = ul * a.n_max + a.t_off + tt0;
+    mbar_arrive_expect_tx(&bars[0], tile_bytes);
+    for (int b = 0; b < C::kBoxes; ++b)
+      tma_load_2d(xs + b * 16384, &maps.x[tn], &bars[0], b * C::kBoxCols, ul * a.n + tt0);
+    tma_load_2d(cs, &maps.codes[tn], &bars[0], 0, crow);
+    if (meta_tma) tma_load_2d(ms, &maps.meta[tn], &bars[0], 0, crow);
+  };
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
+    mbar_init(&bars[2], 1);
     fence_mbarrier_init();
-    mbar_arrive_expect_tx(&bars[0], (uint32_t)(32768 + kTile * F::kRow + (meta_tma ? kTile * mrb : 0)) +
-                                        img_bytes + (uint32_t)kSlabSBytes + 8192u);
-    for (int b = 0; b < C::kBoxes; ++b)
-      tma_load_2d(xs + b * 16384, &maps.x[tn], &bars[0], b * C::kBoxCols, ul * a.n + t0);
-    tma_load_2d(cs, &maps.codes[tn], &bars[0], 0, crow);
-    if (meta_tma) tma_load_2d(ms, &maps.meta[tn], &bars[0], 0, crow);
-    // the unit's operand images and S_g, written by E2
-    bulk_load(zx, slab + kSlabImg, img_bytes, &bars[0]);
-    bulk_load(S, slab + kSlabS, (uint32_t)kSlabSBytes, &bars[0]);
-    bulk_load(sm + F::zr_off(NC), slab + kSlabRows, 8192u, &bars[0]);
+    // the unit's operand images, S_g and fp32 Z rows, written by E2
+    mbar_arrive_expect_tx(&bars[2], img_bytes + (uint32_t)kSlabSBytes + 8192u);
+    bulk_load(zx, slab + kSlabImg, img_bytes, &bars[2]);
+    bulk_load(S, slab + kSlabS, (uint32_t)kSlabSBytes, &bars[2]);
+    bulk_load(sm + F::zr_off(NC), slab + kSlabRows, 8192u, &bars[2]);
+    issue_tile(0);
   }
   if (warp == 0) tmem_alloc(tslot, 128);
-  const bool valid = t0 + t < a.n;
-  const size_t row = (size_t)crow + t;
-  // this token's outliers (channel, value) and short meta rows, fetched while the tile is in flight
-  constexpr int kOF = 8;
-  int oc[kOF];
-  float ov[kOF];
-  float2 szr[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-  if (h == 0) {
-#pragma unroll
-    for (int i = 0; i < kOF; ++i) {
-      const bool on = valid && i < k;
-      oc[i] = on ? ten.oidx[row * k + i] : 0;
-      ov[i] = on ? Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]) : 0.0f;
-    }
-  }
-  if (!meta_tma && valid && 8 * h < a.r_max) {   // both halves write ranks when r > 8
-    if (a.meta_f16) {
-      const __half2* mh = reinterpret_cast<const __half2*>(ten.meta) + row * G;
-      szr[0] = __half22float2(mh[0]);
-      if (G == 2) szr[1] = __half22float2(mh[1]);
-    } else {
-      szr[0] = reinterpret_cast<const float2*>(ten.meta)[row];
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  bool ok = mbar_wait(&bars[0], 0);
-  ok = __syncthreads_and(ok);
-  if (!ok && tid == 0) mbar_wait(&bars[0], 0);   // let copies still in flight land before the CTA ends
+  bool ok = __syncthreads_and(mbar_wait(&bars[2], 0));
   const float down = S[64], up = S[65];   // the images' power-of-two scale and its inverse
-  // ---- X Z into columns [0, 16): the input tile against the parts of Z along K
-  if (ok && tid == 0) {
-    tc_fence_after();
-    constexpr uint32_t kIdX = idesc_f16(128, 16, std::is_same<P, __nv_bfloat16>::value, false, false);
-    const uint32_t xa = smem_u32(xs), za = smem_u32(zx);
-    int m = 0;
+  int issued = 1;                          // tiles whose loads were issued
+  for (int it = 0; it < ntile && ok; ++it) {
+    const int t0 = (tile0 + it) * kTile;
+    const bool valid = t0 + t < a.n;
+    const size_t row = (size_t)(ul * a.n_max + a.t_off + t0) + t;
+    // this token's outliers (channel, value) and short meta rows, fetched while the tile is in flight
+    constexpr int kOF = 8;
+    int oc[kOF];
+    float ov[kOF];
+    float2 sz[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                    make_float2(0.0f, 0.0f)};
+    if (h == 0) {
 #pragma unroll
-    for (int part = 0; part < F::kParts; ++part)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk, ++m) {
-        const uint64_t ad = smem_desc_sw128(xa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd = smem_desc_sw128(za + part * 4096 + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
-        tc_mma_f16(tmem, ad, bd, kIdX, m == 0 ? 0u : 1u);
+      for (int i = 0; i < kOF; ++i) {
+        const bool on = valid && i < k;
+        oc[i] = on ? ten.oidx[row * k + i] : 0;
+        ov[i] = on ? Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]) : 0.0f;
       }
-    tc_commit(&bars[1]);
-  }
-  // ---- spread codes of this half row, written over the input tile once X Z has read it
-  bool xz_done = true;
-  if (ok) {
-    xz_done = mbar_wait(&bars[1], 0);
+    }
+    if (!meta_tma && valid && 8 * h < a.r_max) {   // both halves write ranks when r > 8
+      if (a.meta_f16) {
+        const __half2* mh = reinterpret_cast<const __half2*>(ten.meta) + row * G;
+        sz[0] = __half22float2(mh[0]);
+        if (G == 2) sz[1] = __half22float2(mh[1]);
+      } else {
+        sz[0] = reinterpret_cast<const float2*>(ten.meta)[row];
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(&bars[0], it & 1));
+    if (!ok) break;
+    // ---- X Z into columns [0, 16): the input tile against the parts of Z along K
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t kIdX = idesc_f16(128, 16, std::is_same<P, __nv_bfloat16>::value, false, false);
+      const uint32_t xa = smem_u32(xs), za = smem_u32(zx);
+      int m = 0;
+#pragma unroll
+      for (int part = 0; part < F::kParts; ++part)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk, ++m) {
+          const uint64_t ad = smem_desc_sw128(xa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(za + part * 4096 + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+          tc_mma_f16(tmem, ad, bd, kIdX, m == 0 ? 0u : 1u);
+        }
+      tc_commit(&bars[1]);
+    }
+    // ---- the meta of the token's groups into registers (the tile's meta rows
+    // are overwritten by the next tile's loads before the epilogue ends)
+    if (meta_tma && valid && 8 * h < a.r_max) {
+      const uint8_t* mrow = ms + t * mrb;
+      const int mx = mrb == 32 ? ((t >> 2) & 1) << 4 : 0;
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi)
+        if (gi < G)
+          sz[gi] = a.meta_f16 ? __half22float2(*reinterpret_cast<const __half2*>(mrow + 4 * gi))
+                              : *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
+    }
+    // ---- spread codes of this half row, written over the input tile once X Z has read it
+    const bool xz_done = mbar_wait(&bars[1], 0);
     if (!xz_done) mbar_wait(&bars[1], 0);   // nothing may overwrite the tile while the product reads it
     tc_fence_after();
-    const uint8_t* rowp = cs + t * F::kRow;
+    {
+      const uint8_t* rowp = cs + t * F::kRow;
 #pragma unroll
-    for (int qq = 0; qq < 2; ++qq) {
-      const int q = 2 * h + qq;   // 32-channel block
-      uint32_t cw[BITS];
-      if constexpr (BITS == 2) {
-        const uint2 v =
-            *reinterpret_cast<const uint2*>(rowp + ((((q >> 1) ^ swz_rows<F::kRow>(t)) << 4) | ((q & 1) << 3)));
-        cw[0] = v.x; cw[1] = v.y;
-      } else {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * h + qq;   // 32-channel block
+        uint32_t cw[BITS];
+        if constexpr (BITS == 2) {
+          const uint2 v =
+              *reinterpret_cast<const uint2*>(rowp + ((((q >> 1) ^ swz_rows<F::kRow>(t)) << 4) | ((q & 1) << 3)));
+          cw[0] = v.x; cw[1] = v.y;
+        } else {
 #pragma unroll
-        for (int hh = 0; hh < BITS / 4; ++hh) {
-          const uint4 v = *reinterpret_cast<const uint4*>(rowp + (((BITS / 4 * q + hh) ^ swz_rows<F::kRow>(t)) << 4));
-          cw[4 * hh] = v.x; cw[4 * hh + 1] = v.y; cw[4 * hh + 2] = v.z; cw[4 * hh + 3] = v.w;
+          for (int hh = 0; hh < BITS / 4; ++hh) {
+            const uint4 v =
+                *reinterpret_cast<const uint4*>(rowp + (((BITS / 4 * q + hh) ^ swz_rows<F::kRow>(t)) << 4));
+            cw[4 * hh] = v.x; cw[4 * hh + 1] = v.y; cw[4 * hh + 2] = v.z; cw[4 * hh + 3] = v.w;
+          }
         }
-      }
-      uint4 ch[4];
-      spread_codes<BITS>(cw, ch);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int m = 4 * q + j;   // chunk 0..15
-        *reinterpret_cast<uint4*>(cps + (m >> 3) * 16384 + swz(t, m & 7)) = ch[j];
-      }
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (ok && tid == 0) {
-    // C Z into columns [32, 32 + NC): hi then lo part of Z
-    const uint32_t kIdC = idesc_f16(128, NC, false, false, false);
-    const uint32_t ca = smem_u32(cps), zb = smem_u32(zc);
-    int m = 0;
-#pragma unroll
-    for (int part = 0; part < 2; ++part)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk, ++m) {
-        const uint64_t ad = smem_desc_sw128(ca + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd =
-            smem_desc_sw128(zb + part * NC * 256 + (kk >> 2) * (NC * 128) + (kk & 3) * 32, 16, 1024);
-        tc_mma_f16(tmem + 32, ad, bd, kIdC, m == 0 ? 0u : 1u);
-      }
-    tc_commit(&bars[1]);
-  }
-  // ---- epilogue: thread (t, h) writes ranks [8 h, 8 h + 8) of token t
-  if (ok && 8 * h < a.r_max) {
-    bool done = mbar_wait(&bars[1], 1) && xz_done;
-    if (!done) mbar_wait(&bars[1], 1);   // the products must finish before tensor memory is freed
-    tc_fence_after();
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    uint32_t vx[8], vc[4][8];
-    tmem_ld_32x32b_x8(lane_base + 8 * h, vx);
-#pragma unroll
-    for (int gi = 0; gi < 4; ++gi)
-      if (gi < G) tmem_ld_32x32b_x8(lane_base + 32 + gi * RB + (RB == 16 ? 8 * h : 0), vc[gi]);
-    tmem_ld_wait();
-    // meta of the token's groups: the tile in shared memory (or the short rows)
-    const uint8_t* mrow = ms + t * mrb;
-    const int mx = mrb == 32 ? ((t >> 2) & 1) << 4 : 0;
-    auto group = [&](int gi) -> float2 {
-      if (!meta_tma) return gi == 0 ? szr[0] : szr[1];
-      if (a.meta_f16) return __half22float2(*reinterpret_cast<const __half2*>(mrow + 4 * gi));
-      return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
-    };
-    float acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = __uint_as_float(vx[j]);
-#pragma unroll
-    for (int gi = 0; gi < 4; ++gi) {
-      if (gi >= G) break;
-      const float2 sz = group(gi);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] -= fmaf(sz.x, __uint_as_float(vc[gi][j]), sz.y * S[gi * 16 + 8 * h + j]);
-    }
-    if (valid && done) {
-      // outlier slots: take (x_o - zero) Z[c_o] back out (their residual is 0)
-      auto fix = [&](int c, float xo) {
-        const float d = (xo - group(c >> lg).y) * down;
-        const float4 z0 = *reinterpret_cast<const float4*>(zr + c * 16 + 8 * h);
-        const float4 z1 = *reinterpret_cast<const float4*>(zr + c * 16 + 8 * h + 4);
-        acc[0] -= d * z0.x; acc[1] -= d * z0.y; acc[2] -= d * z0.z; acc[3] -= d * z0.w;
-        acc[4] -= d * z1.x; acc[5] -= d * z1.y; acc[6] -= d * z1.z; acc[7] -= d * z1.w;
-      };
-      if (h == 0) {
-#pragma unroll
-        for (int i = 0; i < kOF; ++i)
-          if (i < k) fix(oc[i], ov[i]);
-      }
-      for (int i = (h == 0 ? kOF : 0); i < k; ++i)
-        fix(ten.oidx[row * k + i], Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]));
-      const int q1 = min(a.r_max, 8 * h + 8);
-      if (q1 - 8 * h == 8 && (a.r_max & 7) == 0) {   // a whole 16-byte row piece
-        uint32_t w[4];
+        uint4 ch[4];
+        spread_codes<BITS>(cw, ch);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const __half2 v2 = __floats2half2_rn(acc[2 * j] * up, acc[2 * j + 1] * up);
-          w[j] = *reinterpret_cast<const uint32_t*>(&v2);
+          const int m = 4 * q + j;   // chunk 0..15
+          *reinterpret_cast<uint4*>(cps + (m >> 3) * 16384 + swz(t, m & 7)) = ch[j];
         }
-        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(ten.lfac) + row * a.r_max + 8 * h) =
-            make_uint4(w[0], w[1], w[2], w[3]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (8 * h + j < q1)
-            reinterpret_cast<__half*>(ten.lfac)[row * a.r_max + 8 * h + j] = __float2half_rn(acc[j] * up);
       }
     }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(xz_done);
+    tc_fence_after();
+    if (ok && tid == 0) {
+      // C Z into columns [32, 32 + NC): hi then lo part of Z
+      const uint32_t kIdC = idesc_f16(128, NC, false, false, false);
+      const uint32_t ca = smem_u32(cps), zb = smem_u32(zc);
+      int m = 0;
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk, ++m) {
+          const uint64_t ad = smem_desc_sw128(ca + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(zb + part * NC * 256 + (kk >> 2) * (NC * 128) + (kk & 3) * 32, 16, 1024);
+          tc_mma_f16(tmem + 32, ad, bd, kIdC, m == 0 ? 0u : 1u);
+        }
+      tc_commit(&bars[1]);
+    }
+    if (!ok) break;
+    bool done = mbar_wait(&bars[1], 1);
+    if (!done) mbar_wait(&bars[1], 1);   // the products must finish before their buffers are reused
+    ok = __syncthreads_and(done);
+    if (!ok) break;
+    tc_fence_after();
+    // the tile's shared buffers are free: the next tile loads during this epilogue
+    if (tid == 0 && it + 1 < ntile) {
+      issue_tile(it + 1);
+      ++issued;
+    }
+    // ---- epilogue: thread (t, h) writes ranks [8 h, 8 h + 8) of token t
+    if (8 * h < a.r_max) {
+      const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+      uint32_t vx[8], vc[4][8];
+      tmem_ld_32x32b_x8(lane_base + 8 * h, vx);
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi)
+        if (gi < G) tmem_ld_32x32b_x8(lane_base + 32 + gi * RB + (RB == 16 ? 8 * h : 0), vc[gi]);
+      tmem_ld_wait();
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = __uint_as_float(vx[j]);
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) {
+        if (gi >= G) break;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          acc[j] -= fmaf(sz[gi].x, __uint_as_float(vc[gi][j]), sz[gi].y * S[gi * 16 + 8 * h + j]);
+      }
+      if (valid) {
+        // outlier slots: take (x_o - zero) Z[c_o] back out (their residual is 0)
+        auto fix = [&](int c, float xo) {
+          float zero_o = 0.0f;
+#pragma unroll
+          for (int gi = 0; gi < 4; ++gi)
+            if (gi == (c >> lg)) zero_o = sz[gi].y;
+          const float d = (xo - zero_o) * down;
+          const float4 z0 = *reinterpret_cast<const float4*>(zr + c * 16 + 8 * h);
+          const float4 z1 = *reinterpret_cast<const float4*>(zr + c * 16 + 8 * h + 4);
+          acc[0] -= d * z0.x; acc[1] -= d * z0.y; acc[2] -= d * z0.z; acc[3] -= d * z0.w;
+          acc[4] -= d * z1.x; acc[5] -= d * z1.y; acc[6] -= d * z1.z; acc[7] -= d * z1.w;
+        };
+        if (h == 0) {
+#pragma unroll
+          for (int i = 0; i < kOF; ++i)
+            if (i < k) fix(oc[i], ov[i]);
+        }
+        for (int i = (h == 0 ? kOF : 0); i < k; ++i)
+          fix(ten.oidx[row * k + i], Elem16<T>::lo(reinterpret_cast<const uint16_t*>(ten.oval)[row * k + i]));
+        const int q1 = min(a.r_max, 8 * h + 8);
+        if (q1 - 8 * h == 8 && (a.r_max & 7) == 0) {   // a whole 16-byte row piece
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const __half2 v2 = __floats2half2_rn(acc[2 * j] * up, acc[2 * j + 1] * up);
+            w[j] = *reinterpret_cast<const uint32_t*>(&v2);
+          }
+          *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(ten.lfac) + row * a.r_max + 8 * h) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (8 * h + j < q1)
+              reinterpret_cast<__half*>(ten.lfac)[row * a.r_max + 8 * h + j] = __float2half_rn(acc[j] * up);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();   // tensor memory read before the next tile's products overwrite it
+    tc_fence_after();
+  }
+  if (!ok && tid == 0) {
+    // a bounded wait gave up (error word set): let the copies still in flight land
+    mbar_wait(&bars[2], 0);
+    mbar_wait(&bars[0], (issued - 1) & 1);   // every earlier tile load was waited for
   }
   tc_fence_before();
   __syncthreads();
@@ -1478,10 +1610,12 @@ __global__ void __launch_bounds__(kE3Threads, 3) encode_lowrank_alg(const __grid
   }
 }
 
-// fp32 inputs: rebuild R and take R Z as hi Zhi + hi Zlo + lo Zhi.
-template <int BITS>
+// fp32 inputs, and keys with per-channel groups (CH): rebuild R and take R Z
+// as hi Zhi + hi Zlo + lo Zhi. With CH the tile's token groups' per-channel
+// (scale, zero) arrive by one bulk copy of their slots (1 KB each).
+template <typename T, int BITS>
 struct E3Cfg {
-  static constexpr int kXB = kTile * 128 * 4;          // input tile (4 boxes of 32 channels)
+  static constexpr int kXB = kTile * 128 * (int)sizeof(T);   // input tile (128-byte boxes)
   static constexpr int kRB = kTile * 128 * 2;          // one bf16 residual image
   static constexpr int kRow = 16 * BITS;               // code bytes per token
   static constexpr int kCB = kTile * kRow;             // code tile
@@ -1496,11 +1630,11 @@ struct E3Cfg {
   static constexpr int kSmem = kBar + 64 + 1024;
 };
 
-template <int BITS>
-__global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid_constant__ E3Maps maps,
-                                                                    const EncodeArgs a) {
-  using C = E1Cfg<float>;
-  using F = E3Cfg<BITS>;
+template <typename T, int BITS, bool CH>
+__global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_rebuild(const __grid_constant__ E3Maps maps,
+                                                                        const EncodeArgs a) {
+  using C = E1Cfg<T>;
+  using F = E3Cfg<T, BITS>;
   constexpr int kPerByte = 8 / BITS;
   extern __shared__ uint8_t e3raw[];
   uint8_t* sm = align_smem_1024(e3raw);
@@ -1522,22 +1656,27 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
   const EncodeTensor& ten = a.ten[tn];
   const int crow = ul * a.n_max + a.t_off + t0;
   const uint8_t* slab = reinterpret_cast<const uint8_t*>(a.zbuf) + (int64_t)u * kZSlab;
+  // CH: the slots of the tile's token groups (those past the cache's slots hold no token of the tile)
+  const int slot_t = a.slot0 + t0 / a.g;
+  const int ngt = CH ? min(kTile / a.g, a.ch_slots - slot_t) : 0;
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     fence_mbarrier_init();
-    mbar_arrive_expect_tx(&bars[0], (uint32_t)(F::kXB + F::kCB + (meta_tma ? kTile * mrb : 0) + 8192));
+    const uint32_t mbytes = CH ? (uint32_t)ngt * 1024u : (meta_tma ? (uint32_t)(kTile * mrb) : 0u);
+    mbar_arrive_expect_tx(&bars[0], (uint32_t)(F::kXB + F::kCB + 8192) + mbytes);
     for (int b = 0; b < C::kBoxes; ++b)
       tma_load_2d(xs + b * 16384, &maps.x[tn], &bars[0], b * C::kBoxCols, ul * a.n + t0);
     tma_load_2d(cs, &maps.codes[tn], &bars[0], 0, crow);
-    if (meta_tma) tma_load_2d(ms, &maps.meta[tn], &bars[0], 0, crow);
+    if (CH) bulk_load(ms, ten.meta + ((size_t)ul * a.ch_slots + slot_t) * 256, mbytes, &bars[0]);
+    else if (meta_tma) tma_load_2d(ms, &maps.meta[tn], &bars[0], 0, crow);
     bulk_load(zs, slab + kSlabImg, 8192u, &bars[0]);   // Z image, bf16 hi | lo (E2)
   }
   if (warp == 0) tmem_alloc(tslot, 32);
   const bool valid = t0 + t < a.n;
   const size_t row = (size_t)crow + t;
   float2 szr[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-  if (!meta_tma && valid) szr[0] = reinterpret_cast<const float2*>(ten.meta)[row];
+  if (!CH && !meta_tma && valid) szr[0] = reinterpret_cast<const float2*>(ten.meta)[row];
   constexpr int kOF = 8;
   int oc[kOF];
 #pragma unroll
@@ -1555,10 +1694,17 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
     const int mx = mrb == 32 ? ((t >> 2) & 1) << 4 : 0;
     auto group = [&](int gi) -> float2 {
       if (!meta_tma) return gi == 0 ? szr[0] : szr[1];
+      if (a.meta_f16) return __half22float2(*reinterpret_cast<const __half2*>(mrow + 4 * gi));
       return *reinterpret_cast<const float2*>(mrow + ((gi << 3) ^ mx));
     };
+    // CH: (scale, zero) of channel c in the token's group
+    const float2* cmeta = reinterpret_cast<const float2*>(ms) + (t / a.g) * 128;
     bool big = false;
-    for (int gi = 0; gi < G; ++gi) big |= !(group(gi).x <= 0x1p100f);
+    if (CH) {
+      for (int c = 64 * h; c < 64 * h + 64; ++c) big |= !(cmeta[c].x <= 0x1p100f);
+    } else {
+      for (int gi = 0; gi < G; ++gi) big |= !(group(gi).x <= 0x1p100f);
+    }
     auto codes32 = [&](int q, uint32_t (&cw)[BITS]) {
       const uint8_t* rowp = cs + t * F::kRow;
       if constexpr (BITS == 2) {
@@ -1574,11 +1720,21 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
       }
     };
     auto xblock = [&](int jb, float (&xv)[8]) {
+      if constexpr (sizeof(T) == 4) {
 #pragma unroll
-      for (int hq = 0; hq < 2; ++hq) {
-        const uint4 v = *reinterpret_cast<const uint4*>(xs + (jb >> 2) * 16384 + swz(t, 2 * (jb & 3) + hq));
-        xv[4 * hq] = __uint_as_float(v.x); xv[4 * hq + 1] = __uint_as_float(v.y);
-        xv[4 * hq + 2] = __uint_as_float(v.z); xv[4 * hq + 3] = __uint_as_float(v.w);
+        for (int hq = 0; hq < 2; ++hq) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xs + (jb >> 2) * 16384 + swz(t, 2 * (jb & 3) + hq));
+          xv[4 * hq] = __uint_as_float(v.x); xv[4 * hq + 1] = __uint_as_float(v.y);
+          xv[4 * hq + 2] = __uint_as_float(v.z); xv[4 * hq + 3] = __uint_as_float(v.w);
+        }
+      } else {
+        const uint4 v = *reinterpret_cast<const uint4*>(xs + (jb >> 3) * 16384 + swz(t, jb & 7));
+        const uint32_t pr[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = Elem16<T>::to_f2(pr[q]);
+          xv[2 * q] = f.x; xv[2 * q + 1] = f.y;
+        }
       }
     };
     auto put = [&](int jb, const float (&rr)[8]) {
@@ -1604,8 +1760,8 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
     for (int q = 2 * h; q < 2 * h + 2; ++q) {   // 32 channels per pass, one group (g >= 32)
       uint32_t cw[BITS];
       codes32(q, cw);
-      const float2 sz = group((32 * q) >> lg);
-      const uint64_t sc2 = f2_pack(sz.x, sz.x), zr2 = f2_pack(sz.y, sz.y);
+      const float2 sz = CH ? make_float2(0.0f, 0.0f) : group((32 * q) >> lg);
+      uint64_t sc2 = f2_pack(sz.x, sz.x), zr2 = f2_pack(sz.y, sz.y);
 #pragma unroll
       for (int bq = 0; bq < 4; ++bq) {
         const int jb = 4 * q + bq;
@@ -1630,6 +1786,11 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
             const int cl = 2 * p;
+            if (CH) {   // per-channel (scale, zero) of the pair
+              const float2 m0 = cmeta[8 * jb + cl], m1 = cmeta[8 * jb + cl + 1];
+              sc2 = f2_pack(m0.x, m1.x);
+              zr2 = f2_pack(m0.y, m1.y);
+            }
             const uint64_t w2 = f2_pack((float)(1 << (8 - (cl % kPerByte) * BITS)),
                                         (float)(1 << (8 - ((cl + 1) % kPerByte) * BITS)));
             const uint64_t cf = f2_sub(f2_pack(f[cl], f[cl + 1]), one2);
@@ -1643,7 +1804,8 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
           for (int e = 0; e < 8; ++e) {
             const int c = 8 * bq + e;
             const float code = (float)((cw[c / kCpw] >> (BITS * (c % kCpw))) & ((1u << BITS) - 1u));
-            rr[e] = __fsub_rn(xv[e], __fmaf_rn(code, sz.x, sz.y));
+            const float2 m = CH ? cmeta[32 * q + c] : sz;
+            rr[e] = __fsub_rn(xv[e], __fmaf_rn(code, m.x, m.y));
           }
         }
         put(jb, rr);
@@ -1696,7 +1858,10 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
       const int q1 = min(a.r_max, 8 * h + 8);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (8 * h + j < q1) reinterpret_cast<float*>(ten.lfac)[row * a.r_max + 8 * h + j] = __uint_as_float(v[j]);
+        if (8 * h + j < q1) {
+          if constexpr (sizeof(T) == 4) reinterpret_cast<float*>(ten.lfac)[row * a.r_max + 8 * h + j] = __uint_as_float(v[j]);
+          else reinterpret_cast<__half*>(ten.lfac)[row * a.r_max + 8 * h + j] = __float2half_rn(__uint_as_float(v[j]));
+        }
     }
   }
   tc_fence_before();
@@ -1708,23 +1873,32 @@ __global__ void __launch_bounds__(kE3Threads, 1) encode_lowrank_f32(const __grid
 }
 
 // ================================================================ host =====
-template <typename T, int BITS, int KMAX>
+template <typename T, int BITS, int KMAX, bool CH>
 static cudaError_t launch_e1(const XMaps& map, const EncodeArgs& a, int grid, cudaStream_t st) {
-  auto kern = encode_quant_gram<T, BITS, KMAX>;
+  auto kern = encode_quant_gram<T, BITS, KMAX, CH>;
+  constexpr uint32_t smem = CH ? E1Cfg<T>::kSmemCh : E1Cfg<T>::kSmem;
   static std::atomic<int> smem_set[kMaxDevices];   // per device: the limit is a per-device setting
-  cudaError_t e = ensure_smem_limit(kern, E1Cfg<T>::kSmem, smem_set);
+  cudaError_t e = ensure_smem_limit(kern, (int)smem, smem_set);
   if (e != cudaSuccess) return e;
-  kern<<<grid, E1Cfg<T>::kThreads, E1Cfg<T>::kSmem, st>>>(map, a);
+  kern<<<grid, E1Cfg<T>::kThreads, smem, st>>>(map, a);
   return cudaGetLastError();
+}
+
+template <typename T, int BITS, bool CH>
+static cudaError_t launch_e1_kc(const XMaps& map, const EncodeArgs& a, int grid, cudaStream_t st) {
+  if (a.k == 0) return launch_e1<T, BITS, 0, CH>(map, a, grid, st);
+  if (a.k == 3) return launch_e1<T, BITS, 3, CH>(map, a, grid, st);
+  if (a.k <= 4) return launch_e1<T, BITS, 4, CH>(map, a, grid, st);
+  if (a.k <= 8) return launch_e1<T, BITS, 8, CH>(map, a, grid, st);
+  return launch_e1<T, BITS, 16, CH>(map, a, grid, st);
 }
 
 template <typename T, int BITS>
 static cudaError_t launch_e1_k(const XMaps& map, const EncodeArgs& a, int grid, cudaStream_t st) {
-  if (a.k == 0) return launch_e1<T, BITS, 0>(map, a, grid, st);
-  if (a.k == 3) return launch_e1<T, BITS, 3>(map, a, grid, st);
-  if (a.k <= 4) return launch_e1<T, BITS, 4>(map, a, grid, st);
-  if (a.k <= 8) return launch_e1<T, BITS, 8>(map, a, grid, st);
-  return launch_e1<T, BITS, 16>(map, a, grid, st);
+  if constexpr (sizeof(T) == 2) {   // per-channel key groups: 16-bit caches only
+    if (a.ch) return launch_e1_kc<T, BITS, true>(map, a, grid, st);
+  }
+  return launch_e1_kc<T, BITS, false>(map, a, grid, st);
 }
 
 template <typename T>
@@ -1747,10 +1921,10 @@ static cudaError_t launch_e3a(const E3Maps& maps, const EncodeArgs& a, dim3 grid
   return cudaGetLastError();
 }
 
-template <int BITS>
+template <typename T, int BITS, bool CH>
 static cudaError_t launch_e3f(const E3Maps& maps, const EncodeArgs& a, dim3 grid, cudaStream_t st) {
-  auto kern = encode_lowrank_f32<BITS>;
-  constexpr int smem = E3Cfg<BITS>::kSmem;
+  auto kern = encode_lowrank_rebuild<T, BITS, CH>;
+  constexpr int smem = E3Cfg<T, BITS>::kSmem;
   static std::atomic<int> smem_set[kMaxDevices];
   cudaError_t e = ensure_smem_limit(kern, smem, smem_set);
   if (e != cudaSuccess) return e;
@@ -1763,11 +1937,18 @@ static cudaError_t launch_e3_b(const E3Maps& maps, const EncodeArgs& a, cudaStre
   dim3 grid(a.tpu, a.U);
   if constexpr (sizeof(T) == 4) {
     switch (a.bits) {
-      case 2: return launch_e3f<2>(maps, a, grid, st);
-      case 4: return launch_e3f<4>(maps, a, grid, st);
-      default: return launch_e3f<8>(maps, a, grid, st);
+      case 2: return launch_e3f<float, 2, false>(maps, a, grid, st);
+      case 4: return launch_e3f<float, 4, false>(maps, a, grid, st);
+      default: return launch_e3f<float, 8, false>(maps, a, grid, st);
+    }
+  } else if (a.ch) {
+    switch (a.bits) {
+      case 2: return launch_e3f<T, 2, true>(maps, a, grid, st);
+      case 4: return launch_e3f<T, 4, true>(maps, a, grid, st);
+      default: return launch_e3f<T, 8, true>(maps, a, grid, st);
     }
   } else {
+    grid.x = (a.tpu + a.e3_tpc - 1) / a.e3_tpc;   // e3_tpc tiles per CTA
     const bool r8 = a.r_max <= 8;
     switch (a.bits) {
       case 2: return r8 ? launch_e3a<T, 2, 8>(maps, a, grid, st) : launch_e3a<T, 2, 16>(maps, a, grid, st);
@@ -1832,6 +2013,14 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
   }
   XMaps xm;
   memcpy(xm.x, m3.x, sizeof(xm.x));
+  // E3 (16-bit inputs): consecutive tiles of one unit per CTA, so that the
+  // unit's operands load once per CTA; at least two waves of three CTAs per SM
+  {
+    const int64_t waves2 = (int64_t)num_sms * 3 * 2;
+    int64_t tpc = a.total_tiles / (waves2 > 0 ? waves2 : 1);
+    a.e3_tpc = (int)(tpc < 1 ? 1 : (tpc > 8 ? 8 : tpc));
+    if (a.e3_tpc > a.tpu) a.e3_tpc = a.tpu;
+  }
 
   const int grid = a.grid_e1;
   cudaError_t e;

@@ -42,6 +42,9 @@ struct EncodeArgs {
   uint32_t one_bits;     // 0x3F800000 (1.0f), kept in a register by the kernels
   int32_t n_max, nblk_max, W, G, r_max;
   int32_t meta_f16;      // scale and zero stored as binary16
+  int32_t ch;            // per-channel key groups of g tokens (meta per token-group slot)
+  int32_t ch_slots;      // token-group slots per unit of the cache (ch)
+  int32_t slot0;         // slot of this block's first token group (ch)
   // workspace: partial Grams [U][maxc][128][128] and Z slabs [U][kZSlab bytes] (E3 operands)
   float* gram;
   float* zbuf;
@@ -50,6 +53,7 @@ struct EncodeArgs {
   int64_t total_tiles;   // U * tpu
   int32_t grid_e1;       // persistent CTAs of E1
   int32_t maxc;          // partial-Gram slots per unit
+  int32_t e3_tpc;        // consecutive 128-token tiles per CTA of the low-rank pass (16-bit inputs)
   EncodeTensor ten[kMaxBatch];
 };
 

@@ -27,7 +27,8 @@ _TORCH = {v: k for k, v in _DT.items()}
 class GearParams(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("outlier_frac", ctypes.c_float),
                 ("rank", ctypes.c_int32), ("power_iters", ctypes.c_int32), ("buffer_len", ctypes.c_int32),
-                ("buffer_rank", ctypes.c_int32), ("meta_f16", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+                ("buffer_rank", ctypes.c_int32), ("meta_f16", ctypes.c_int32), ("channel_groups", ctypes.c_int32),
+                ("seed", ctypes.c_uint64)]
 
 
 class GearCacheStruct(ctypes.Structure):
@@ -104,8 +105,9 @@ def _stream_ptr(stream=None):
 
 
 def make_params(bits=4, group_size=64, outlier_frac=0.02, rank=4, power_iters=3, buffer_len=20, buffer_rank=2,
-                seed=0, meta_f16=False) -> GearParams:
-    return GearParams(bits, group_size, outlier_frac, rank, power_iters, buffer_len, buffer_rank, int(meta_f16), seed)
+                seed=0, meta_f16=False, channel_groups=False) -> GearParams:
+    return GearParams(bits, group_size, outlier_frac, rank, power_iters, buffer_len, buffer_rank, int(meta_f16),
+                      int(channel_groups), seed)
 
 
 class _Workspace:
@@ -191,8 +193,11 @@ class Cache:
         rp = (c.r_max + 3) // 4 * 4
         return {
             "codes": self._view(c.codes, U * n * c.W, torch.int32).view(U, n, c.W),
-            "meta": self._view(c.meta, U * n * c.G * 2, torch.float16 if c.p.meta_f16 else torch.float32)
-            .view(U, n, c.G, 2),
+            # per-channel key groups: [U][ceil(n_max / g) + 1 slots][d][2]
+            "meta": (self._view(c.meta, U * (-(-n // c.p.group_size) + 1) * c.d * 2, torch.float32)
+                     .view(U, -1, c.d, 2) if c.p.channel_groups else
+                     self._view(c.meta, U * n * c.G * 2, torch.float16 if c.p.meta_f16 else torch.float32)
+                     .view(U, n, c.G, 2)),
             "oidx": self._view(c.oidx, U * n * k, torch.uint8).view(U, n, k),
             "oval": self._view(c.oval, U * n * k, self.dtype).view(U, n, k),
             "lfac": self._view(c.lfac, U * n * c.r_max, ld).view(U, n, c.r_max),

@@ -58,6 +58,10 @@ def lib():
                                          P, P, P, P, P, P, P, P]
         L.oracle_reconstruct_unit.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
         L.oracle_attention.argtypes = [P, P, P, i32, i32, ctypes.c_double, P]
+        L.oracle_quantize_channels.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P]
+        L.oracle_encode_unit_channels.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, ctypes.c_uint64,
+                                                  P, P, P, P, P, P, P, P]
+        L.oracle_reconstruct_unit_channels.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -81,6 +85,7 @@ class Params:
     buffer_rank: int = 2
     seed: int = 0
     meta_f16: bool = False   # scale and zero stored as binary16 (byte-lean metadata)
+    channel_groups: bool = False   # KIVI-combined keys: per-channel groups of group_size tokens
 
 
 def num_outliers(s: float, d: int) -> int:
@@ -144,12 +149,40 @@ class Unit:
     rank: int = 0
 
 
+def quantize_channels(X: np.ndarray, bits: int, g: int, is_out: np.ndarray):
+    """Per-channel min-max quantization over groups of g consecutive tokens (the
+    KIVI-combined key quantizer): returns (codes u32[n][W], scale f32[ng][d],
+    zero f32[ng][d], resid f32[n][d])."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    n, d = X.shape
+    ng = (n + g - 1) // g
+    m = np.ascontiguousarray(is_out, dtype=np.int8)
+    codes = np.zeros((n, d * bits // 32), np.uint32)
+    scale = np.zeros((ng, d), np.float32)
+    zero = np.zeros((ng, d), np.float32)
+    resid = np.zeros((n, d), np.float32)
+    lib().oracle_quantize_channels(_p(X), n, d, bits, g, _p(m), _p(codes), _p(scale), _p(zero), _p(resid))
+    return codes, scale, zero, resid
+
+
 def encode_unit(X: np.ndarray, p: Params, rank: int | None = None) -> Unit:
-    """Steps 1-5 on one unit X [n][d] (float32 holding the exact input values)."""
+    """Steps 1-5 on one unit X [n][d] (float32 holding the exact input values).
+    With p.channel_groups the quantizer is the KIVI-combined key quantizer and
+    scale/zero are [ceil(n/g)][d]."""
     X = np.ascontiguousarray(X, dtype=np.float32)
     n, d = X.shape
     r = p.rank if rank is None else rank
     k = num_outliers(p.outlier_frac, d)
+    if p.channel_groups:
+        ng = (n + p.group_size - 1) // p.group_size
+        u = Unit(codes=np.zeros((n, d * p.bits // 32), np.uint32), scale=np.zeros((ng, d), np.float32),
+                 zero=np.zeros((ng, d), np.float32), oidx=np.zeros((n, k), np.int32),
+                 oval=np.zeros((n, k), np.float32), resid=np.zeros((n, d), np.float32),
+                 L=np.zeros((n, r), np.float64), Rf=np.zeros((d, r), np.float64), rank=r)
+        lib().oracle_encode_unit_channels(_p(X), n, d, p.bits, p.group_size, k, r, p.power_iters,
+                                          ctypes.c_uint64(p.seed), _p(u.codes), _p(u.scale), _p(u.zero),
+                                          _p(u.oidx), _p(u.oval), _p(u.resid), _p(u.L), _p(u.Rf))
+        return u
     W = d * p.bits // 32
     G = d // p.group_size
     u = Unit(codes=np.zeros((n, W), np.uint32), scale=np.zeros((n, G), np.float32),
@@ -168,8 +201,9 @@ def reconstruct_unit(u: Unit, p: Params) -> np.ndarray:
     d = u.resid.shape[1]
     k = u.oidx.shape[1]
     Xh = np.zeros((n, d), dtype=np.float64)
-    lib().oracle_reconstruct_unit(n, d, p.bits, p.group_size, k, u.rank, _p(u.codes), _p(u.scale),
-                                  _p(u.zero), _p(u.oidx), _p(u.oval), _p(u.L), _p(u.Rf), _p(Xh))
+    fn = lib().oracle_reconstruct_unit_channels if p.channel_groups else lib().oracle_reconstruct_unit
+    fn(n, d, p.bits, p.group_size, k, u.rank, _p(u.codes), _p(u.scale), _p(u.zero), _p(u.oidx), _p(u.oval),
+       _p(u.L), _p(u.Rf), _p(Xh))
     return Xh
 
 

@@ -130,6 +130,63 @@ void oracle_quantize_token(const float* x, int32_t d, int32_t bits, int32_t g,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Step 2, KIVI-combined variant (keys): per-channel groups across tokens.   */
+/* [cites] KIVI entries: combining GEAR with KIVI requires a buffer at least */
+/* as large as the group size; the same page's list of works citing GEAR,    */
+/* TailorKV entry: KIVI quantizes keys per channel and values per token.     */
+/* Reading: the                                                              */
+/* tokens of a block form groups of g consecutive tokens (the last group may */
+/* be shorter); within each group every channel gets its own min-max         */
+/* quantizer over the group's non-outlier entries, with the same formulas as */
+/* oracle_quantize_token (zero point = minimum, -0 stored as +0, codes       */
+/* rounded half to even, code 0 at outlier slots and where scale is 0).      */
+/* X is n x d; is_out marks outlier entries (n x d); codes are packed per    */
+/* token as in the per-token quantizer; scale and zero are [ngroups][d].     */
+/* ------------------------------------------------------------------------ */
+void oracle_quantize_channels(const float* X, int32_t n, int32_t d, int32_t bits, int32_t g,
+                              const char* is_out, uint32_t* codes, float* scale_out, float* zero_out,
+                              float* resid_out) {
+  const int32_t levels = (1 << bits) - 1;
+  const int32_t words = d * bits / 32;
+  for (size_t w = 0; w < (size_t)n * words; ++w) codes[w] = 0u;
+  const int32_t ngroups = (n + g - 1) / g;
+  for (int32_t j = 0; j < ngroups; ++j) {
+    const int32_t t0 = j * g, t1 = (t0 + g < n) ? t0 + g : n;
+    for (int32_t c = 0; c < d; ++c) {
+      int have = 0;
+      float mn = 0.0f, mx = 0.0f;
+      for (int32_t t = t0; t < t1; ++t) {
+        if (is_out[(size_t)t * d + c]) continue;
+        float x = X[(size_t)t * d + c];
+        if (!have) { mn = x; mx = x; have = 1; }
+        if (x < mn) mn = x;
+        if (x > mx) mx = x;
+      }
+      mn = mn + 0.0f;
+      mx = mx + 0.0f;
+      float scale = (mx - mn) / (float)levels;
+      scale_out[(size_t)j * d + c] = scale;
+      zero_out[(size_t)j * d + c] = mn;
+      for (int32_t t = t0; t < t1; ++t) {
+        uint32_t code = 0u;
+        const int out = is_out[(size_t)t * d + c];
+        if (!out && scale != 0.0f) {
+          float q = (X[(size_t)t * d + c] - mn) / scale;
+          float qr = nearbyintf(q);
+          if (qr < 0.0f) qr = 0.0f;
+          if (qr > (float)levels) qr = (float)levels;
+          code = (uint32_t)qr;
+        }
+        int32_t bit = c * bits;
+        codes[(size_t)t * words + bit / 32] |= code << (bit % 32);
+        float dh = fmaf((float)code, scale, mn);
+        resid_out[(size_t)t * d + c] = out ? 0.0f : X[(size_t)t * d + c] - dh;
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Step 4: seeded start matrix of the power iteration. splitmix64 as         */
 /* published by Steele, Lea & Flood (OOPSLA 2014, "Fast splittable          */
 /* pseudorandom number generators"): the state advances by the golden-ratio */
@@ -241,6 +298,32 @@ void oracle_encode_unit(const float* X, int32_t n, int32_t d, int32_t bits, int3
   }
 }
 
+/* The KIVI-combined key encoding of one unit: steps 1 (per token), 2 with  */
+/* per-channel token groups of g (oracle_quantize_channels), 3-5 as above.  */
+/* scale and zero are [ceil(n/g)][d].                                        */
+void oracle_encode_unit_channels(const float* X, int32_t n, int32_t d, int32_t bits, int32_t g,
+                                 int32_t k, int32_t r, int32_t T, uint64_t seed, uint32_t* codes,
+                                 float* scale, float* zero, int32_t* oidx, float* oval, float* resid,
+                                 double* L, double* Rf) {
+  char* is_out = (char*)calloc((size_t)n * d, 1);
+  for (int32_t t = 0; t < n; ++t) {
+    const float* x = X + (size_t)t * d;
+    oracle_select_outliers(x, d, k, oidx + (size_t)t * k);
+    for (int32_t i = 0; i < k; ++i) {
+      oval[(size_t)t * k + i] = x[oidx[(size_t)t * k + i]];
+      is_out[(size_t)t * d + oidx[(size_t)t * k + i]] = 1;
+    }
+  }
+  oracle_quantize_channels(X, n, d, bits, g, is_out, codes, scale, zero, resid);
+  free(is_out);
+  if (r > 0) {
+    double* q0 = (double*)malloc(sizeof(double) * (size_t)d * (size_t)r);
+    oracle_start_matrix(seed, d, r, q0);
+    oracle_power_iteration(resid, n, d, r, T, q0, L, Rf);
+    free(q0);
+  }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Step 6: reconstruction, X ~ D + L Rf^T with the outlier slots holding    */
 /* their exact values ([cites] LoftQ and Zafrir et al. entries: the low-rank */
@@ -261,6 +344,27 @@ void oracle_reconstruct_unit(int32_t n, int32_t d, int32_t bits, int32_t g, int3
       int32_t grp = c / g;
       double v = (double)fmaf((float)code, scale[(size_t)t * G + grp], zero[(size_t)t * G + grp]);
       for (int32_t j = 0; j < r; ++j) v += L[(size_t)t * r + j] * Rf[(size_t)c * r + j];
+      Xhat[(size_t)t * d + c] = v;
+    }
+    for (int32_t i = 0; i < k; ++i)
+      Xhat[(size_t)t * d + oidx[(size_t)t * k + i]] = (double)oval[(size_t)t * k + i];
+  }
+}
+
+/* Step 6 for a KIVI-combined key unit: the group of token t is t / g.      */
+void oracle_reconstruct_unit_channels(int32_t n, int32_t d, int32_t bits, int32_t g, int32_t k,
+                                      int32_t r, const uint32_t* codes, const float* scale,
+                                      const float* zero, const int32_t* oidx, const float* oval,
+                                      const double* L, const double* Rf, double* Xhat) {
+  const int32_t words = d * bits / 32;
+  const uint32_t mask = (1u << bits) - 1u;
+  for (int32_t t = 0; t < n; ++t) {
+    const int32_t j = t / g;
+    for (int32_t c = 0; c < d; ++c) {
+      int32_t bit = c * bits;
+      uint32_t code = (codes[(size_t)t * words + bit / 32] >> (bit % 32)) & mask;
+      double v = (double)fmaf((float)code, scale[(size_t)j * d + c], zero[(size_t)j * d + c]);
+      for (int32_t q = 0; q < r; ++q) v += L[(size_t)t * r + q] * Rf[(size_t)c * r + q];
       Xhat[(size_t)t * d + c] = v;
     }
     for (int32_t i = 0; i < k; ++i)

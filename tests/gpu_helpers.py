@@ -14,7 +14,7 @@ TORCH_DT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
 def oracle_params(p) -> oracle.Params:
     return oracle.Params(bits=p.bits, group_size=p.group_size, outlier_frac=p.outlier_frac, rank=p.rank,
                          power_iters=p.power_iters, buffer_len=p.buffer_len, buffer_rank=p.buffer_rank, seed=p.seed,
-                         meta_f16=bool(p.meta_f16))
+                         meta_f16=bool(p.meta_f16), channel_groups=bool(p.channel_groups))
 
 
 def seeded_kv(seed: int, stream: int, shape, dtype: str, channel_scale: bool = False,

@@ -409,3 +409,120 @@ def test_ragged_prefill_all_padding():
     vc.append(2 * row)
     out = oracle.decode_attn(kc, vc, q, 0.1, prefill_len=[0, 0])
     np.testing.assert_allclose(out[:, 0], 2 * row[:, 0], rtol=0, atol=1e-12)   # one real token: its value
+
+
+# ------------------------------------ KIVI-combined keys: per-channel token groups
+def textbook_channel_groups(x: np.ndarray, bits: int, g: int):
+    """Independent restatement: per channel, min-max over each group of g
+    consecutive tokens (last group shorter), binary32 arithmetic, ties to even."""
+    n, d = x.shape
+    L = np.float32(2 ** bits - 1)
+    codes = np.zeros((n, d), np.uint32)
+    ng = (n + g - 1) // g
+    scale = np.zeros((ng, d), np.float32)
+    zero = np.zeros((ng, d), np.float32)
+    for j in range(ng):
+        xs = x[j * g:(j + 1) * g]
+        mn = xs.min(axis=0) + np.float32(0.0)
+        mx = xs.max(axis=0) + np.float32(0.0)
+        sc = (mx - mn) / L
+        with np.errstate(divide="ignore", invalid="ignore"):
+            q = np.where(sc > 0, np.rint((xs - mn) / sc), 0).astype(np.float32)
+        codes[j * g:(j + 1) * g] = np.clip(q, 0, L).astype(np.uint32)
+        scale[j], zero[j] = sc, mn
+    return codes, scale, zero
+
+
+@pytest.mark.parametrize("bits,g,n", [(2, 32, 128), (4, 64, 200), (8, 32, 77), (4, 128, 256), (2, 64, 1)])
+def test_channel_groups_s0_r0_is_textbook_per_channel_quantization(bits, g, n):
+    x = (RNG.standard_normal((n, 128)) * np.exp(RNG.uniform(-1, 2, size=(1, 128)))).astype(np.float32)
+    x[:, 5] = 0.75              # a constant channel: scale 0 in every group
+    p = Params(bits=bits, group_size=g, outlier_frac=0.0, rank=0, channel_groups=True)
+    u = oracle.encode_unit(x, p)
+    codes, scale, zero = textbook_channel_groups(x, bits, g)
+    assert np.array_equal(unpack_codes(u.codes, 128, bits), codes)
+    assert np.array_equal(u.scale, scale) and np.array_equal(u.zero, zero)
+    assert u.scale.shape == ((n + g - 1) // g, 128)
+    dh = oracle.reconstruct_unit(u, p).astype(np.float32)
+    grp = np.arange(n) // g
+    want = np.float32(codes.astype(np.float64) * scale[grp].astype(np.float64) + zero[grp].astype(np.float64))
+    assert np.array_equal(dh, want)
+
+
+@pytest.mark.parametrize("bits,g", [(2, 32), (4, 64), (8, 32)])
+def test_channel_groups_equal_per_token_quantizer_of_the_transpose(bits, g):
+    """Per-channel groups of g tokens of X are per-token groups of g entries of X^T:
+    the per-token quantizer (pinned above against the textbook) on the rows of X^T
+    must give the same codes, scales and zero points."""
+    n = 4 * g
+    x = (RNG.standard_normal((n, 128)) * 3).astype(np.float16).astype(np.float32)
+    u = oracle.encode_unit(x, Params(bits=bits, group_size=g, outlier_frac=0.0, rank=0, channel_groups=True))
+    codes = unpack_codes(u.codes, 128, bits)
+    for c in range(0, 128, 13):
+        tc, ts, tz, _, _ = oracle.quantize_token(np.ascontiguousarray(x[:, c]), bits, g, np.zeros(0, np.int32))
+        assert np.array_equal(unpack_codes(tc, n, bits), codes[:, c])
+        assert np.array_equal(ts, u.scale[:, c]) and np.array_equal(tz, u.zero[:, c])
+
+
+@pytest.mark.parametrize("bits,g,s,n", [(2, 32, 0.05, 160), (4, 64, 0.02, 300), (4, 32, 0.1, 45)])
+def test_channel_groups_invariants(bits, g, s, n):
+    d = 128
+    x = (RNG.standard_normal((n, d)) * np.exp(RNG.uniform(np.log(0.5), np.log(8), size=(1, d))))
+    x = x.astype(np.float16).astype(np.float32)
+    p = Params(bits=bits, group_size=g, outlier_frac=s, rank=0, channel_groups=True)
+    u = oracle.encode_unit(x, p)
+    L = 2 ** bits - 1
+    codes = unpack_codes(u.codes, d, bits)
+    out_mask = np.zeros((n, d), bool)
+    np.put_along_axis(out_mask, u.oidx.astype(np.int64), True, axis=1)
+    # outliers per token as in GEAR: the same selection, exact values, code 0, zero residual
+    for t in range(0, n, 7):
+        assert np.array_equal(u.oidx[t], oracle.select_outliers(x[t], oracle.num_outliers(s, d)))
+    assert np.array_equal(u.oval, np.take_along_axis(x, u.oidx.astype(np.int64), axis=1))
+    assert np.all(codes[out_mask] == 0) and np.all(u.resid[out_mask] == 0)
+    grp = np.arange(n) // g
+    for j in range((n + g - 1) // g):
+        rows = grp == j
+        for c in range(d):
+            vals = x[rows, c][~out_mask[rows, c]]
+            if vals.size == 0:
+                assert u.scale[j, c] == 0 and u.zero[j, c] == 0
+                continue
+            assert u.zero[j, c] == vals.min() + np.float32(0)
+            if u.scale[j, c] > 0:
+                cc = codes[rows, c][~out_mask[rows, c]]
+                assert cc[np.argmin(vals)] == 0 and cc[np.argmax(vals)] == L
+    dh = oracle.reconstruct_unit(u, p).astype(np.float32)
+    err = np.abs(x.astype(np.float64) - dh.astype(np.float64))
+    bound = u.scale[grp].astype(np.float64) * (0.5 + L * 2.0 ** -22) + 0.5 * np.spacing(np.abs(dh)).astype(np.float64)
+    assert np.all(err[~out_mask] <= bound[~out_mask])
+    assert np.array_equal(dh[out_mask], x[out_mask])
+
+
+def test_channel_groups_flush_protocol_and_low_rank():
+    """A buffer of n_b = 2g tokens flushes as whole groups; the flushed block equals a
+    standalone per-channel encode, and attention over the cache is textbook attention
+    over the reconstruction."""
+    B, H, d, g = 1, 2, 128, 32
+    p = Params(bits=2, group_size=g, outlier_frac=0.05, rank=4, buffer_len=2 * g, buffer_rank=2, seed=5,
+               channel_groups=True)
+    kc = oracle.Cache(p, B, H, d)
+    X0 = RNG.standard_normal((B, H, 70, d)).astype(np.float32)   # block 0 ends in a partial group
+    kc.encode(X0)
+    assert kc.blocks[0][0].scale.shape == (3, d)
+    rows = [RNG.standard_normal((B, H, d)).astype(np.float32) for _ in range(2 * g + 3)]
+    for row in rows:
+        kc.append(row)
+    assert kc.n_comp == 70 + 2 * g and len(kc.buffer) == 3
+    blk = np.stack(rows[:2 * g], 2)
+    for h in range(H):
+        alone = oracle.encode_unit(blk[0, h], p, rank=2)
+        got = kc.blocks[1][h]
+        assert np.array_equal(got.codes, alone.codes) and np.array_equal(got.scale, alone.scale)
+        assert got.scale.shape == (2, d)
+    # the low-rank factors shrink the residual of the key block
+    u = kc.blocks[0][0]
+    rec = oracle.reconstruct_unit(u, p)
+    nol = oracle.reconstruct_unit(oracle.Unit(u.codes, u.scale, u.zero, u.oidx, u.oval, u.resid,
+                                              u.L[:, :0], u.Rf[:, :0], 0), p)
+    assert np.linalg.norm(rec - X0[0, 0]) < np.linalg.norm(nol - X0[0, 0])
