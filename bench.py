@@ -617,49 +617,59 @@ def run_gpu(args, rank: int, world: int):
         line["gear_l"] = variant_measure(gear, wl, we, wd, dev, max(3, args.steps // 2), hbm, s=0.0)
         line["meta_f16"] = variant_measure(gear, wl, we, wd, dev, max(3, args.steps // 2), hbm, s=we.s,
                                            meta_f16=True)
+        line["kivi_keys"] = variant_measure(gear, wl, we, wd, dev, max(3, args.steps // 2), hbm, s=we.s,
+                                            kivi=True)
         line["cpu_baseline"] = cpu_baseline(HEADLINE)
         for sc in BESIDE:
             line["configs"][sc.name]["cpu_baseline"] = cpu_baseline(sc)
     print(json.dumps(line), flush=True)
 
 
-def variant_measure(gear, wl, we, wd, dev, reps, hbm, s, meta_f16=False):
+def variant_measure(gear, wl, we, wd, dev, reps, hbm, s, meta_f16=False, kivi=False):
     """The same two workloads with another outlier fraction s (s = 0 is the pages'
-    GEAR-L: group-wise quantization plus low rank, no outliers) or with binary16
-    metadata, timed like the main stages (CUDA events, L2 flushed before each timed
-    launch sequence). Reported beside GEAR; not the headline."""
+    GEAR-L: group-wise quantization plus low rank, no outliers), with binary16
+    metadata, or (kivi) with the KIVI-combined keys (per-channel groups of g tokens;
+    values per token; a buffer of whole groups), timed like the main stages (CUDA
+    events, L2 flushed before each timed launch sequence). Reported beside GEAR;
+    not the headline."""
     import torch
     w0e = dataclasses.replace(we, s=s)
     w0d = dataclasses.replace(wd, s=s)
+    if kivi:   # the buffer holds whole key groups
+        w0e = dataclasses.replace(w0e, buffer_len=we.group)
+        w0d = dataclasses.replace(w0d, buffer_len=wd.group)
 
-    def params(w):
+    def params(w, which="v"):
         return gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank,
                                 power_iters=w.iters, buffer_len=w.buffer_len, buffer_rank=w.buffer_rank,
-                                seed=w.seed, meta_f16=meta_f16)
+                                seed=w.seed, meta_f16=meta_f16, channel_groups=kivi and which == "k")
 
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    # encode: K and V of the layer in one batched encode
+    # encode: K and V of the layer in one batched encode (two encodes when the
+    # keys take per-channel groups: the batch wants one parameter set)
     xs = [wl.kv_tensor_torch(w0e, which, 0, dev) for which in ("k", "v")]
-    pe = params(w0e)
-    cs = [gear.Cache(pe, w0e.B, w0e.H, w0e.n, 1, torch.float16, dev) for _ in range(2)]
+    cs = [gear.Cache(params(w0e, which), w0e.B, w0e.H, w0e.n, 1, torch.float16, dev) for which in ("k", "v")]
     enc = []
     for it in range(reps + 3):
         for c in cs:
-            c.c.n_comp = c.c.n_buf = c.c.n_blk = c.c.blk0_len = c.c.blk0_rank = 0
+            c.reset()
         flush.fill_(it & 0xFF)
         a, b = ev(), ev()
         a.record()
-        gear.encode_batch(cs, xs)
+        if kivi:
+            for c, x in zip(cs, xs):
+                c.encode(x)
+        else:
+            gear.encode_batch(cs, xs)
         b.record()
         torch.cuda.synchronize()
         if it >= 3:
             enc.append(a.elapsed_time(b))
     del xs, cs
     # decode: compressed context + full buffer
-    pd = params(w0d)
-    dk = gear.Cache(pd, w0d.B, w0d.H, w0d.n + w0d.buffer_len, 2, torch.float16, dev)
-    dv = gear.Cache(pd, w0d.B, w0d.H, w0d.n + w0d.buffer_len, 2, torch.float16, dev)
+    dk = gear.Cache(params(w0d, "k"), w0d.B, w0d.H, w0d.n + w0d.buffer_len, 2, torch.float16, dev)
+    dv = gear.Cache(params(w0d, "v"), w0d.B, w0d.H, w0d.n + w0d.buffer_len, 2, torch.float16, dev)
     for c, which in ((dk, "k"), (dv, "v")):
         t = wl.kv_tensor_torch(w0d, which, 0, dev)
         c.encode(t)
@@ -685,7 +695,11 @@ def variant_measure(gear, wl, we, wd, dev, reps, hbm, s, meta_f16=False):
     ptb = per_token_bytes(w0d, meta_f16)
     dec_alg = (2 * w0d.B * w0d.H * w0d.n * ptb + 2 * w0d.B * w0d.H * w0d.rank * 128 * 4
                + 2 * w0d.B * w0d.H * w0d.buffer_fill * 128 * 2 + 2 * w0d.B * w0d.Hq * 128 * 2)
-    return {"s": s, "meta_f16": bool(meta_f16), "encode_ms": round(enc_ms, 4),
+    if kivi:   # keys: per-channel (scale, zero) of a token group instead of per-token groups
+        ptb_k = ptb - (w0d.d // w0d.group) * 8 + (w0d.d * 8) // w0d.group
+        dec_alg = (w0d.B * w0d.H * w0d.n * (ptb + ptb_k) + 2 * w0d.B * w0d.H * w0d.rank * 128 * 4
+                   + 2 * w0d.B * w0d.H * w0d.buffer_fill * 128 * 2 + 2 * w0d.B * w0d.Hq * 128 * 2)
+    return {"s": s, "meta_f16": bool(meta_f16), "kivi_keys": bool(kivi), "encode_ms": round(enc_ms, 4),
             "encode_gbs": round(enc_in / enc_ms / 1e6, 3),
             "decode_ms": round(dec_ms, 4), "decode_tokens_per_s": round(w0d.B / dec_ms * 1e3, 1),
             "decode_hbm_frac": round(dec_alg / dec_ms / 1e6 / hbm, 4),

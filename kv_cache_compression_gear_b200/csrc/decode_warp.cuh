@@ -188,33 +188,39 @@ __device__ __forceinline__ void meta_row(const uint8_t* mrow, int G, int mx, flo
 // rank <= 4 block needs one load per outlier. All loads are issued together.
 // Three slots cover s <= 2 % of 128 channels; more outliers take the general loop.
 constexpr int kFast = 3;
-template <typename T, bool MF, bool ZC = false>
+template <typename T, bool MF, bool ZC = false, int NS = kFast, int NR = 4>
 __device__ __forceinline__ void outlier_fixes(const uint8_t* rest, int oval_off, const uint8_t* mrow, int mx, int t,
-                                              int k, int lg, const float (&lt)[4], const float* rf, int rp,
-                                              int (&cix)[kFast], float (&fix)[kFast], const float* zc = nullptr) {
-  float xo[kFast], zr[kFast];
-  float4 rv[kFast];
+                                              int k, int lg, const float (&lt)[NR], const float* rf, int rp,
+                                              int (&cix)[NS], float (&fix)[NS], const float* zc = nullptr,
+                                              int i0 = 0) {
+  float xo[NS], zr[NS];
+  float4 rv[NS][NR / 4];
 #pragma unroll
-  for (int i = 0; i < kFast; ++i) {
-    const bool on = i < k;
-    cix[i] = on ? rest[t * k + i] : 0;
-    xo[i] = on ? (float)reinterpret_cast<const T*>(rest + oval_off)[t * k + i] : 0.0f;
+  for (int i = 0; i < NS; ++i) {
+    const bool on = i0 + i < k;
+    cix[i] = on ? rest[t * k + i0 + i] : 0;
+    xo[i] = on ? (float)reinterpret_cast<const T*>(rest + oval_off)[t * k + i0 + i] : 0.0f;
   }
 #pragma unroll
-  for (int i = 0; i < kFast; ++i) {
-    const bool on = i < k;
+  for (int i = 0; i < NS; ++i) {
+    const bool on = i0 + i < k;
     // the zero point at the outlier's channel: per channel (ZC) or of its group
     zr[i] = on ? (ZC ? zc[cix[i]] : meta_at<MF>(mrow, cix[i] >> lg, mx).y) : 0.0f;
-    rv[i] = on ? __ldg(reinterpret_cast<const float4*>(rf + cix[i] * rp)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int q = 0; q < NR / 4; ++q)
+      rv[i][q] = on ? __ldg(reinterpret_cast<const float4*>(rf + cix[i] * rp) + q) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
 #pragma unroll
-  for (int i = 0; i < kFast; ++i) {
+  for (int i = 0; i < NS; ++i) {
     float lr = 0.0f;
-    lr = fmaf(lt[0], rv[i].x, lr);
-    lr = fmaf(lt[1], rv[i].y, lr);
-    lr = fmaf(lt[2], rv[i].z, lr);
-    lr = fmaf(lt[3], rv[i].w, lr);
-    fix[i] = i < k ? xo[i] - (zr[i] + lr) : 0.0f;
+#pragma unroll
+    for (int q = 0; q < NR / 4; ++q) {
+      lr = fmaf(lt[4 * q], rv[i][q].x, lr);
+      lr = fmaf(lt[4 * q + 1], rv[i][q].y, lr);
+      lr = fmaf(lt[4 * q + 2], rv[i][q].z, lr);
+      lr = fmaf(lt[4 * q + 3], rv[i][q].w, lr);
+    }
+    fix[i] = i0 + i < k ? xo[i] - (zr[i] + lr) : 0.0f;
   }
 }
 
@@ -735,6 +741,23 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
               for (int i = 0; i < kFast; ++i)
 #pragma unroll
                 for (int hh = 0; hh < HQ; ++hh) s_[hh] = fmaf(qw_s[hh * 128 + cix[i]] * CF::weight(cix[i]), fx[i], s_[hh]);
+            } else if (k <= 8 && rb <= 8) {
+              // the token's L row once, then outliers four at a time
+              float l8[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) l8[j] = j < kRReg ? lt[j] : (j < rb ? l_at<T>(tkr + L.lf, t, j, rm) : 0.0f);
+#pragma unroll
+              for (int i0 = 0; i0 < 8; i0 += 4) {
+                if (i0 >= k) break;
+                int cix[4];
+                float fx[4];
+                outlier_fixes<T, MF, KC, 4, 8>(tkr, L.oval, kmrow, mx, t, k, lg, l8, rfk, rp, cix, fx, zk_s, i0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                  for (int hh = 0; hh < HQ; ++hh)
+                    s_[hh] = fmaf(qw_s[hh * 128 + cix[i]] * CF::weight(cix[i]), fx[i], s_[hh]);
+              }
             } else {
               for (int i = 0; i < k; ++i) {
                 const int c = tkr[t * k + i];
@@ -794,6 +817,22 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
                 if (i < k)
 #pragma unroll
                   for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + cix[i], p[hh] * fx[i]);
+            } else if (k <= 8 && rb <= 8) {
+              float l8[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) l8[j] = j < kRReg ? lv[j] : (j < rb ? l_at<T>(tvr + L.lf, t, j, rm) : 0.0f);
+#pragma unroll
+              for (int i0 = 0; i0 < 8; i0 += 4) {
+                if (i0 >= k) break;
+                int cix[4];
+                float fx[4];
+                outlier_fixes<T, MF, false, 4, 8>(tvr, L.oval, vmrow, mx, t, k, lg, l8, rfv, rp, cix, fx, nullptr, i0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  if (i0 + i < k)
+#pragma unroll
+                    for (int hh = 0; hh < HQ; ++hh) red_add_gpu(part_row + hh * hstride + 2 + cix[i], p[hh] * fx[i]);
+              }
             } else {
               for (int i = 0; i < k; ++i) {
                 const int c = tvr[t * k + i];

@@ -170,3 +170,29 @@ def test_encode_batch_host_errors(gear):
     assert L.gear_encode_batch(2, ptrs(caches[:2]), xs(2), 2000, None, 0, None) == E.GEAR_ERR_CAPACITY
     assert L.gear_encode_batch(2, ptrs(caches[:2]), xs(2), 2, None, 0, None) == E.GEAR_ERR_INVALID_ARG  # rank 4 > n
     assert all(c.n_comp == 0 for c in caches)
+
+
+def test_channel_groups_validation_and_layout(gear):
+    """Per-channel key groups (the KIVI-combined quantizer): the buffer holds whole
+    groups (at least one), 16-bit caches only, no binary16 metadata; the meta array
+    holds one 1 KB slot per token group."""
+    L, E = gear.lib, gear.gear
+    ok = gear.make_params(group_size=64, buffer_len=128, channel_groups=True)
+    assert L.gear_validate_params(ctypes.byref(ok), 128) == 0
+    for kw, want in [(dict(buffer_len=32), E.GEAR_ERR_INVALID_ARG),     # shorter than a group
+                     (dict(buffer_len=96), E.GEAR_ERR_INVALID_ARG),     # not whole groups
+                     (dict(buffer_len=128, meta_f16=True), E.GEAR_ERR_UNSUPPORTED)]:
+        bad = gear.make_params(group_size=64, channel_groups=True, **kw)
+        assert L.gear_validate_params(ctypes.byref(bad), 128) == want, kw
+    bad = gear.make_params(group_size=64, buffer_len=128)
+    bad.channel_groups = 2
+    assert L.gear_validate_params(ctypes.byref(bad), 128) == E.GEAR_ERR_INVALID_ARG
+    assert L.gear_cache_bytes(ctypes.byref(ok), 1, 4, 128, 1000, 2, 2) == 0            # fp32 cache
+    c = gear.GearCacheStruct()
+    fake = ctypes.c_void_p(1 << 40)
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(ok), 1, 4, 128, 1000, 2, 2, fake, 1 << 30) == \
+        E.GEAR_ERR_UNSUPPORTED
+    nbytes = L.gear_cache_bytes(ctypes.byref(ok), 1, 4, 128, 1000, 2, 0)
+    assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(ok), 1, 4, 128, 1000, 2, 0, fake, nbytes) == 0
+    slots = -(-c.n_max // 64) + 1                # n_max is rounded up to 1024
+    assert c.n_max == 1024 and c.oidx - c.meta >= 4 * slots * 128 * 8
