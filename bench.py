@@ -494,8 +494,13 @@ class Runner:
 # stage's dominant kernel, from one ncu capture each (profiles/), keyed by
 # (scenario, stage); an entry is removed whenever its kernel changes, until it is
 # captured again.
+# The 2-bit batch-64 workload's traffic comes from a capture of the same step at
+# batch 4 (1/16 of the units), scaled by 16: every kernel's traffic is per unit.
 TRAFFIC_BYTES = {
-    (f"{ENC} + {DEC}", "decode"): 830936064 + 7828224,
+    # encode stage: E1 539145984 + 175796224, E2 26292736, E3 723998208 + 30295040 bytes at batch 4
+    ("twobit_b64_ctx8192", "encode"): 16 * (539145984 + 175796224 + 26292736 + 723998208 + 30295040),
+    # decode_warp 213756928 + 757504 bytes at batch 4
+    ("twobit_b64_ctx8192", "decode"): 16 * (213756928 + 757504),
 }
 
 
