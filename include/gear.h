@@ -28,7 +28,8 @@
  *    fp16 for 16-bit caches and fp32 for fp32 caches; Rf is always fp32.
  *  - Shapes are row-major, innermost dimension last, densely packed.
  *  - One "unit" is one (batch b, kv-head h) matrix; units are indexed
- *    u = b*H + h. Every unit of a cache holds the same number of tokens.
+ *    u = b*H + h. Every unit of a contiguous cache holds the same number of
+ *    tokens; a paged cache (gear_paged_cache_init) keeps counts per batch row.
  */
 #ifndef GEAR_H_
 #define GEAR_H_
@@ -155,6 +156,14 @@ typedef struct gear_cache {
   int32_t blk0_len;   /* tokens in block 0 (0 while n_blk == 0)      */
   int32_t blk0_rank;  /* rank of block 0                             */
   int32_t reserved1;
+  /* paged layout (gear_paged_cache_init); all zero for a contiguous cache */
+  int32_t page_tokens;    /* P: tokens per page, a multiple of 32         */
+  int32_t num_pages;      /* pages in the pool                            */
+  int32_t pages_per_row;  /* block-table row length                       */
+  int32_t reserved2;
+  int32_t* table;         /* device [B][pages_per_row] pool page of each logical page, -1 if none */
+  int32_t* rows;          /* device [3][B] per row: block-0 length, blocks, buffer fill */
+  int32_t* host;          /* host, caller-owned: see gear_paged_host_ints  */
 } gear_cache;
 
 /* Number of outliers kept per token: k = ceil(s*d - 1e-9), computed in double
@@ -221,7 +230,8 @@ size_t gear_decode_workspace_bytes(const gear_cache* k, const gear_cache* v, int
  * tokens, with h = j / (Hq / H) (grouped-query sharing).
  *   q    [B][Hq][d], cache dtype.       out  [B][Hq][d], out_dtype
  *   out_dtype is the cache dtype or GEAR_F32.
- * k and v must have identical geometry and counters; Hq % H == 0.
+ * k and v must have identical geometry, counters and parameters, except that
+ * k may have channel_groups = 1 where v has 0; Hq % H == 0.
  * Errors: INVALID_ARG, WORKSPACE, CUDA. */
 gear_status gear_decode_attn(const gear_cache* k, const gear_cache* v, const void* q,
                              int32_t Hq, float softmax_scale, void* out, gear_dtype out_dtype,
@@ -284,6 +294,91 @@ gear_status gear_append_buffer(gear_cache* k, gear_cache* v, const void* k_new,
  * out_f32 [B][H][n_comp + n_buf][d] fp32 (compressed tokens first, then the
  * buffer). Errors: INVALID_ARG, CUDA. */
 gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream);
+
+/* ------------------------------------------------------------ paged layout
+ * Serving integration (GEAR: Efficient KV Cache Compression for LLM Inference,
+ * Q5 on integration into real-time inference systems; the pages give no
+ * layout, so this one is the library's own). In a paged cache every batch row
+ * b (one sequence: its H units) has its own counters -- block-0 length, number
+ * of blocks, buffer fill -- so that rows join (gear_encode_rows), grow
+ * (gear_append_rows, flushing each row's buffer when that row's buffer is
+ * full) and leave (gear_release_rows) independently. The per-token arrays
+ * (codes, meta, oidx, oval, lfac) live in a pool of num_pages pages of P
+ * tokens; a row's compressed tokens are numbered from 0 as in a contiguous
+ * cache (block 0, then n_b per flushed block) and token t of row b, head h is
+ * pool row (table[b][t / P] * H + h) * P + t % P. The library hands pages out
+ * from the pool as rows grow and takes them back on release. Per-token arrays
+ * are laid out as in a contiguous cache with [U][n_max] replaced by
+ * [num_pages][H][P]; rfac [U][nblk_max][d][r_pad] and buf [U][n_b][d] stay per
+ * unit; then table [B][pages_per_row] and rows [3][B] (int32).
+ * The cache-level counters n_comp, n_buf and n_blk hold the maxima over rows;
+ * blk0_len is 0 (per row) and blk0_rank is p.rank.
+ * gear_decode_attn, gear_decode_attn_ragged and gear_decode_attn_noalloc take
+ * paged caches (both K and V paged, built by the same calls on the same rows,
+ * so that their counters and tables agree; INVALID_ARG otherwise): each row
+ * attends over its own tokens, a row without tokens gets an output of 0.
+ * The work split covers the longest row, so rows shorter than it leave part
+ * of their share idle. gear_encode, gear_encode_batch, gear_append_buffer,
+ * gear_cache_reset and gear_decode_dense return UNSUPPORTED on a paged cache.
+ * Limits: channel_groups = 0; P a multiple of 32 (a decode tile of 32 tokens
+ * never spans two pages). */
+
+/* Host int32 entries a paged cache keeps in caller memory:
+ * 3*B counters (block-0 length, blocks, buffer fill per row), the table
+ * mirror [B][pages_per_row], a stack of free pages [num_pages] and its
+ * height (1). The host array must stay alive and untouched while the cache
+ * is used. */
+size_t gear_paged_host_ints(int32_t B, int32_t pages_per_row, int32_t num_pages);
+
+/* Device bytes of a paged cache (0 on bad args). A row holds at most
+ * page_tokens * pages_per_row compressed tokens and nblk_max blocks. */
+size_t gear_paged_cache_bytes(const gear_params* p, int32_t B, int32_t H, int32_t d, int32_t page_tokens,
+                              int32_t num_pages, int32_t pages_per_row, int32_t nblk_max, gear_dtype dtype);
+
+/* Lays a paged cache out in [dev, dev + bytes) (256-byte aligned) with host
+ * state in host[0 .. host_ints). Every row starts empty and every page free.
+ * Enqueues two memsets on `stream` (counters to 0, table to -1).
+ * Errors: INVALID_ARG (null, misaligned, bad geometry, P % 32 != 0,
+ * channel_groups), UNSUPPORTED (d != 128, pool rows >= 2^31), CAPACITY (bytes
+ * or host_ints too small), CUDA. */
+gear_status gear_paged_cache_init(gear_cache* c, const gear_params* p, int32_t B, int32_t H, int32_t d,
+                                  int32_t page_tokens, int32_t num_pages, int32_t pages_per_row, int32_t nblk_max,
+                                  gear_dtype dtype, void* dev, size_t bytes, int32_t* host, size_t host_ints,
+                                  void* stream);
+
+/* Workspace bytes gear_encode_rows needs for nrows rows of n tokens. */
+size_t gear_encode_rows_workspace_bytes(const gear_cache* c, int32_t nrows, int32_t n);
+
+/* Encodes kv [nrows][H][n][d] (cache dtype, 16-byte aligned) as block 0 of
+ * the empty rows rows[0 .. nrows) (HOST array of distinct row indices), with
+ * rank p.rank -- the computation of gear_encode, row by row. Takes
+ * ceil(n / P) pages per row from the pool. The codec runs on a contiguous
+ * copy in the workspace, which a scatter kernel then moves into the pages.
+ * Errors: INVALID_ARG (not paged, bad or repeated row, row not empty,
+ * rank > n), CAPACITY (n > P * pages_per_row, too few free pages),
+ * WORKSPACE, CUDA. */
+gear_status gear_encode_rows(gear_cache* c, const int32_t* rows, int32_t nrows, const void* kv, int32_t n,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes gear_append_rows needs (covers a flush of every row). */
+size_t gear_append_rows_workspace_bytes(const gear_cache* k);
+
+/* Appends one token to each of the rows rows[0 .. nrows) (HOST array of
+ * distinct, already encoded rows): k_new/v_new [nrows][H][d], cache dtype.
+ * A listed row whose buffer holds n_b tokens is flushed first: its buffer is
+ * compressed as that row's next block with rank buffer_rank and the buffer
+ * emptied (Q3, streaming strategy, row by row), taking pages from the pool as
+ * needed. Rows not listed are left as they are.
+ * Errors: INVALID_ARG (caches not a matching paged pair, bad, repeated or
+ * unencoded row), CAPACITY (a flush past P * pages_per_row tokens or nblk_max
+ * blocks, too few free pages), WORKSPACE, CUDA. */
+gear_status gear_append_rows(gear_cache* k, gear_cache* v, const int32_t* rows, int32_t nrows, const void* k_new,
+                             const void* v_new, void* workspace, size_t ws_bytes, void* stream);
+
+/* Empties the rows rows[0 .. nrows) (HOST array) and returns their pages to
+ * the pool; the rows can then be encoded again. Enqueues the counter and
+ * table updates on `stream`. Errors: INVALID_ARG, CUDA. */
+gear_status gear_release_rows(gear_cache* c, const int32_t* rows, int32_t nrows, void* stream);
 
 /* Reads (host, synchronous) and clears the device-side error word that
  * kernels set instead of trapping (GEAR_ERR_* value, 0 if none). */

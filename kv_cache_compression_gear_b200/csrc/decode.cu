@@ -102,7 +102,7 @@ cudaError_t decode_launch(const DecodeArgs& a, cudaStream_t st) {
     if (a.n_comp > 0) {
       PFN_encodeTiled enc = tensor_map_encoder();
       if (!enc) return cudaErrorNotSupported;
-      const uint64_t rows = (uint64_t)a.B * a.H * a.n_max;
+      const uint64_t rows = a.table ? (uint64_t)a.num_pages * a.H * a.page_tokens : (uint64_t)a.B * a.H * a.n_max;
       bool ok = cache_row_map(enc, &maps.kc, a.K.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kDTile) &&
                 cache_row_map(enc, &maps.vc, a.V.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.W, rows, kDTile);
       // meta rows of 16 bytes or more come by tensor copy, as 32-bit words

@@ -64,6 +64,13 @@ struct DecodeArgs {
   int32_t out_dtype;
   float* part;            // [B][Hq][nsplit][130] partial (m, l, acc[128]) per warp that meets the unit
   const int32_t* plen;    // [B] device: real tokens at the head of block 0 per batch row, or null (all)
+  // paged layout (null table: contiguous). Token t of row b, head h is row
+  // (table[b * ppr + t / page_tokens] * H + h) * page_tokens + t % page_tokens
+  // of the per-token arrays; rows [3][B] holds each row's block-0 length,
+  // blocks and buffer fill (n_comp and n_buf above are the maxima over rows).
+  const int32_t* table;
+  const int32_t* rows;
+  int32_t page_tokens, ppr, num_pages;
   int32_t seg_tokens;     // compressed tokens per warp (a multiple of 32); 0 without any
   int32_t nsplit;         // partial rows per unit: at most ceil(n_comp / seg_tokens) + 1 warps meet a unit
   int32_t total_splits;   // warps: ceil(units * n_comp / seg_tokens), or units without compressed tokens

@@ -64,11 +64,12 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ int block_of(const DecodeArgs& a, int t) {
-  return t < a.blk0_len ? 0 : 1 + (t - a.blk0_len) / a.n_b;
+// blocks of a unit whose block 0 holds b0 tokens
+__device__ __forceinline__ int block_of(const DecodeArgs& a, int b0, int t) {
+  return t < b0 ? 0 : 1 + (t - b0) / a.n_b;
 }
-__device__ __forceinline__ int block_end(const DecodeArgs& a, int b) {
-  return b == 0 ? a.blk0_len : a.blk0_len + b * a.n_b;
+__device__ __forceinline__ int block_end(const DecodeArgs& a, int b0, int b) {
+  return b == 0 ? b0 : b0 + b * a.n_b;
 }
 
 // Bulk copy global -> shared, completing on an mbarrier (no multicast).
@@ -289,12 +290,21 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
   // One segment: compressed tokens [c0, c1) of `unit` (maybe none), then the
   // unit's buffer if with_buf, into partial row sp of the unit. Returns false if
   // a bounded wait gave up (the error word is set; nothing is written).
-  auto segment = [&](const int unit, const int c0, const int c1, const int sp, const bool with_buf) -> bool {
+  auto segment = [&](const int unit, const int c0, const int c1_run, const int sp, const bool with_buf) -> bool {
     const int b = unit / a.H, h = unit % a.H;
+    // this row's block-0 length, compressed tokens and buffer fill (paged
+    // layout: per row, the run cut to the row's own tokens)
+    int b0 = a.blk0_len, nbuf = a.n_buf, c1 = c1_run;
+    if (a.rows) {
+      b0 = __ldg(a.rows + b);
+      const int nblk = __ldg(a.rows + a.B + b);
+      nbuf = __ldg(a.rows + 2 * a.B + b);
+      c1 = max(c0, min(c1_run, nblk > 0 ? b0 + (nblk - 1) * a.n_b : 0));
+    }
     const bool comp = c1 > c0;
-    // right-padded prefill: block-0 tokens [pl, blk0_len) of this batch row are
+    // right-padded prefill: block-0 tokens [pl, b0) of this batch row are
     // padding and take no part in the softmax
-    const int pl = a.plen ? min(max(__ldg(a.plen + b), 0), a.blk0_len) : a.blk0_len;
+    const int pl = a.plen ? min(max(__ldg(a.plen + b), 0), b0) : b0;
     // this split's partial row of query head hh: part_row + hh * hstride
     float* part_row = a.part + (((size_t)b * a.Hq + (size_t)h * HQ) * a.nsplit + sp) * 130;
     const size_t hstride = (size_t)a.nsplit * 130;
@@ -424,7 +434,13 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
             break;
         }
       }
-      const size_t row0 = (size_t)unit * a.n_max;   // row of the unit's token 0
+      const size_t row0 = (size_t)unit * a.n_max;   // row of the unit's token 0 (contiguous layout)
+      // paged layout: the row of token t (a 32-token tile never spans two pages)
+      auto token_row = [&](int t) -> size_t {
+        if (!a.table) return row0 + t;
+        const int pg = min(max(__ldg(a.table + (size_t)b * a.ppr + t / a.page_tokens), 0), a.num_pages - 1);
+        return ((size_t)pg * a.H + h) * a.page_tokens + t % a.page_tokens;
+      };
       // Brings tokens [t, t + nt) of the unit into stage s. A whole, 32-aligned
       // tile is all copies; another one (a block boundary or the split's end)
       // takes codes and meta by tensor copy (rows past nt are read and ignored)
@@ -434,7 +450,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         if (lane == 0) mbar_arrive_expect_tx(&bars[s], (uint32_t)(full ? L.tx_full : L.tx_part));
         __syncwarp();
         const uint32_t bar = smem_u32(&bars[s]);
-        const size_t row = row0 + t;
+        const size_t row = token_row(t);
         if (my_map) {
           fence_proxy_async_smem();
           tensor_copy(my_dst + s * my_sst, my_map, bar, (int32_t)row);
@@ -464,8 +480,8 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
       };
 
       // blocks: block 0 = [0, blk0_len), then n_b tokens each; tracked incrementally
-      int blk = block_of(a, c0);
-      int bend = block_end(a, blk);
+      int blk = block_of(a, b0, c0);
+      int bend = block_end(a, b0, blk);
       const float* rfk = nullptr;
       const float* rfv = nullptr;
       // KC: slot and end of the key token group holding token t of block b
@@ -474,10 +490,10 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
         if (b == 0) {
           const int j = t / a.g;
           slot = j;
-          gend = min((j + 1) * a.g, a.blk0_len);
+          gend = min((j + 1) * a.g, b0);
         } else {
-          const int bs = block_end(a, b - 1), j = (t - bs) / a.g;
-          slot = (a.blk0_len + a.g - 1) / a.g + (b - 1) * (a.n_b / a.g) + j;
+          const int bs = block_end(a, b0, b - 1), j = (t - bs) / a.g;
+          slot = (b0 + a.g - 1) / a.g + (b - 1) * (a.n_b / a.g) + j;
           gend = bs + (j + 1) * a.g;
         }
       };
@@ -546,13 +562,13 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
 
       int t0 = c0, cur_blk = -1;
       while (t0 < c1) {
-        if (t0 >= bend) { ++blk; bend = block_end(a, blk); }
+        if (t0 >= bend) { ++blk; bend = block_end(a, b0, blk); }
         const int t1 = next_end(t0, bend, blk);
         const int nt = t1 - t0;
         const int s = it & 1;
         if (t1 < c1) {   // prefetch the next tile into the other stage
           const int b2 = t1 >= bend ? blk + 1 : blk;
-          issue(s ^ 1, t1, next_end(t1, block_end(a, b2), b2) - t1);
+          issue(s ^ 1, t1, next_end(t1, block_end(a, b0, b2), b2) - t1);
         }
         const bool landed = mbar_wait(&bars[s], (uint32_t)(it >> 1) & 1u);
         if (!__all_sync(0xFFFFFFFFu, landed)) {
@@ -631,7 +647,7 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
 
         // ---------------- scores: lane = token
         const int t = lane;
-        const bool live = t < nt && (t0 + t < pl || t0 + t >= a.blk0_len);
+        const bool live = t < nt && (t0 + t < pl || t0 + t >= b0);
         const uint8_t* kmrow = tkm + t * mrb;
         const uint8_t* vmrow = tvm + t * mrb;
         float s_[HQ];
@@ -908,8 +924,8 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
     if (with_buf) {
       // ---------------- the streaming buffer: exact tokens, lane = token for keys
       const size_t brow = (size_t)unit * a.n_b;
-      for (int t0 = 0; t0 < a.n_buf; t0 += kDTile) {
-        const int nt = min(kDTile, a.n_buf - t0);
+      for (int t0 = 0; t0 < nbuf; t0 += kDTile) {
+        const int nt = min(kDTile, nbuf - t0);
         const bool live = lane < nt;
         float s[HQ];
 #pragma unroll

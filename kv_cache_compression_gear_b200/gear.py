@@ -39,7 +39,9 @@ class GearCacheStruct(ctypes.Structure):
                 ("oval", ctypes.c_void_p), ("lfac", ctypes.c_void_p), ("rfac", ctypes.c_void_p),
                 ("buf", ctypes.c_void_p), ("n_comp", ctypes.c_int32), ("n_buf", ctypes.c_int32),
                 ("n_blk", ctypes.c_int32), ("blk0_len", ctypes.c_int32), ("blk0_rank", ctypes.c_int32),
-                ("reserved1", ctypes.c_int32)]
+                ("reserved1", ctypes.c_int32), ("page_tokens", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("pages_per_row", ctypes.c_int32), ("reserved2", ctypes.c_int32), ("table", ctypes.c_void_p),
+                ("rows", ctypes.c_void_p), ("host", ctypes.c_void_p)]
 
 
 class GearError(RuntimeError):
@@ -73,6 +75,14 @@ def _load():
         "gear_append_workspace_bytes": (S, [pc]),
         "gear_append_buffer": (i32, [pc, pc, P, P, P, S, P]),
         "gear_decode_dense": (i32, [pc, P, P]),
+        "gear_paged_host_ints": (S, [i32, i32, i32]),
+        "gear_paged_cache_bytes": (S, [pp, i32, i32, i32, i32, i32, i32, i32, i32]),
+        "gear_paged_cache_init": (i32, [pc, pp, i32, i32, i32, i32, i32, i32, i32, i32, P, S, P, S, P]),
+        "gear_encode_rows_workspace_bytes": (S, [pc, i32, i32]),
+        "gear_encode_rows": (i32, [pc, P, i32, P, i32, P, S, P]),
+        "gear_append_rows_workspace_bytes": (S, [pc]),
+        "gear_append_rows": (i32, [pc, pc, P, i32, P, P, P, S, P]),
+        "gear_release_rows": (i32, [pc, P, i32, P]),
         "gear_get_device_status": (i32, [ctypes.POINTER(i32)]),
         "gear_selftest_wait_timeout": (i32, [ctypes.c_uint32, P]),
         "gear_status_string": (ctypes.c_char_p, [i32]),
@@ -204,6 +214,109 @@ class Cache:
             "rfac": self._view(c.rfac, U * c.nblk_max * c.d * rp, torch.float32).view(U, c.nblk_max, c.d, rp),
             "buf": self._view(c.buf, U * c.p.buffer_len * c.d, self.dtype).view(U, c.p.buffer_len, c.d),
         }
+
+
+def _rows_arg(rows):
+    """Host int32 array of row indices (kept alive by the caller's reference)."""
+    import numpy as np
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1))
+    return r, ctypes.c_void_p(r.ctypes.data), int(r.size)
+
+
+class PagedCache:
+    """One compressed tensor in the paged layout: B rows (sequences) of H kv heads
+    whose compressed tokens live in a pool of num_pages pages of page_tokens tokens.
+    The host state (per-row counters, block-table mirror, free pages) is a numpy
+    int32 array this object owns."""
+
+    def __init__(self, params: GearParams, B: int, H: int, page_tokens: int, num_pages: int, pages_per_row: int,
+                 nblk_max: int, dtype: torch.dtype, device="cuda", d: int = 128, stream=None):
+        import numpy as np
+        self.params = params
+        self.dtype = dtype
+        self.device = torch.device(device)
+        nbytes = lib.gear_paged_cache_bytes(ctypes.byref(params), B, H, d, page_tokens, num_pages, pages_per_row,
+                                            nblk_max, _DT[dtype])
+        if nbytes == 0:
+            raise GearError(GEAR_ERR_INVALID_ARG, "gear_paged_cache_bytes")
+        nh = lib.gear_paged_host_ints(B, pages_per_row, num_pages)
+        self.host = np.zeros(nh, dtype=np.int32)
+        self.mem = torch.empty(nbytes + 256, dtype=torch.uint8, device=self.device)
+        base = (self.mem.data_ptr() + 255) & ~255
+        self.c = GearCacheStruct()
+        _check(lib.gear_paged_cache_init(ctypes.byref(self.c), ctypes.byref(params), B, H, d, page_tokens, num_pages,
+                                         pages_per_row, nblk_max, _DT[dtype], ctypes.c_void_p(base), nbytes,
+                                         ctypes.c_void_p(self.host.ctypes.data), nh, _stream_ptr(stream)),
+               "gear_paged_cache_init")
+
+    @property
+    def n_comp(self) -> int:
+        return self.c.n_comp
+
+    @property
+    def n_buf(self) -> int:
+        return self.c.n_buf
+
+    def counters(self):
+        """Copies of the per-row (block-0 length, blocks, buffer fill) and the table mirror."""
+        B, ppr = self.c.B, self.c.pages_per_row
+        h = self.host
+        return h[:B].copy(), h[B:2 * B].copy(), h[2 * B:3 * B].copy(), h[3 * B:3 * B + B * ppr].reshape(B, ppr).copy()
+
+    def free_pages(self) -> int:
+        return int(self.host[-1])
+
+    def encode_rows(self, rows, kv: torch.Tensor, stream=None):
+        """gear_encode_rows: kv [len(rows)][H][n][d] becomes block 0 of the (empty) rows."""
+        assert kv.is_cuda and kv.dtype == self.dtype and kv.is_contiguous()
+        r, rp, nr = _rows_arg(rows)
+        n = kv.shape[2]
+        nbytes = lib.gear_encode_rows_workspace_bytes(ctypes.byref(self.c), nr, n)
+        wp, wn = _ws.get(nbytes, kv.device)
+        _check(lib.gear_encode_rows(ctypes.byref(self.c), rp, nr, ctypes.c_void_p(kv.data_ptr()), n,
+                                    ctypes.c_void_p(wp), wn, _stream_ptr(stream)), "gear_encode_rows")
+
+    def release_rows(self, rows, stream=None):
+        r, rp, nr = _rows_arg(rows)
+        _check(lib.gear_release_rows(ctypes.byref(self.c), rp, nr, _stream_ptr(stream)), "gear_release_rows")
+
+    def _view(self, ptr, count, dtype):
+        off = ptr - self.mem.data_ptr()
+        nbytes = count * torch.empty((), dtype=dtype).element_size()
+        return self.mem[off:off + nbytes].view(dtype)
+
+    def arrays(self) -> dict:
+        """Raw views: pool arrays [num_pages][H][P][...], rfac [U][nblk_max][d][r_pad], buf, table, rows."""
+        c = self.c
+        U = c.B * c.H
+        NP, H, P = c.num_pages, c.H, c.page_tokens
+        R = NP * H * P
+        ld = torch.float32 if self.dtype == torch.float32 else torch.float16
+        k = max(c.k, 1)
+        rp = (c.r_max + 3) // 4 * 4
+        return {
+            "codes": self._view(c.codes, R * c.W, torch.int32).view(NP, H, P, c.W),
+            "meta": self._view(c.meta, R * c.G * 2, torch.float16 if c.p.meta_f16 else torch.float32)
+            .view(NP, H, P, c.G, 2),
+            "oidx": self._view(c.oidx, R * k, torch.uint8).view(NP, H, P, k),
+            "oval": self._view(c.oval, R * k, self.dtype).view(NP, H, P, k),
+            "lfac": self._view(c.lfac, R * c.r_max, ld).view(NP, H, P, c.r_max),
+            "rfac": self._view(c.rfac, U * c.nblk_max * c.d * rp, torch.float32).view(c.B, H, c.nblk_max, c.d, rp),
+            "buf": self._view(c.buf, U * c.p.buffer_len * c.d, self.dtype).view(c.B, H, c.p.buffer_len, c.d),
+            "table": self._view(c.table, c.B * c.pages_per_row, torch.int32).view(c.B, c.pages_per_row),
+            "rows": self._view(c.rows, 3 * c.B, torch.int32).view(3, c.B),
+        }
+
+
+def append_rows(kc: PagedCache, vc: PagedCache, rows, k_new: torch.Tensor, v_new: torch.Tensor, stream=None):
+    """gear_append_rows: one token per listed row, k_new/v_new [len(rows)][H][d]."""
+    assert k_new.is_cuda and k_new.dtype == kc.dtype and k_new.is_contiguous() and v_new.is_contiguous()
+    r, rp, nr = _rows_arg(rows)
+    nbytes = lib.gear_append_rows_workspace_bytes(ctypes.byref(kc.c))
+    wp, wn = _ws.get(nbytes, k_new.device)
+    _check(lib.gear_append_rows(ctypes.byref(kc.c), ctypes.byref(vc.c), rp, nr, ctypes.c_void_p(k_new.data_ptr()),
+                                ctypes.c_void_p(v_new.data_ptr()), ctypes.c_void_p(wp), wn, _stream_ptr(stream)),
+           "gear_append_rows")
 
 
 def encode_batch(caches, kvs, stream=None):

@@ -43,9 +43,10 @@ def test_struct_layout_matches_c(gear):
 #include <stddef.h>
 #include "gear.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu\n", sizeof(gear_params), sizeof(gear_cache),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(gear_params), sizeof(gear_cache),
          offsetof(gear_cache, p), offsetof(gear_cache, codes), offsetof(gear_cache, buf),
-         offsetof(gear_cache, n_comp), offsetof(gear_params, seed));
+         offsetof(gear_cache, n_comp), offsetof(gear_params, seed), offsetof(gear_cache, page_tokens),
+         offsetof(gear_cache, table), offsetof(gear_cache, host));
   return 0;
 }'''
     with tempfile.TemporaryDirectory() as td:
@@ -56,7 +57,7 @@ int main(void) {
         vals = [int(v) for v in subprocess.check_output([exe]).split()]
     G, P = gear.GearCacheStruct, gear.GearParams
     assert vals == [ctypes.sizeof(P), ctypes.sizeof(G), G.p.offset, G.codes.offset, G.buf.offset,
-                    G.n_comp.offset, P.seed.offset]
+                    G.n_comp.offset, P.seed.offset, G.page_tokens.offset, G.table.offset, G.host.offset]
 
 
 def test_num_outliers_and_validation(gear):
@@ -196,3 +197,63 @@ def test_channel_groups_validation_and_layout(gear):
     assert L.gear_cache_init(ctypes.byref(c), ctypes.byref(ok), 1, 4, 128, 1000, 2, 0, fake, nbytes) == 0
     slots = -(-c.n_max // 64) + 1                # n_max is rounded up to 1024
     assert c.n_max == 1024 and c.oidx - c.meta >= 4 * slots * 128 * 8
+
+
+def test_paged_layout_and_host_errors(gear):
+    """The paged layout's sizes, the host state init writes, and the row calls'
+    argument errors, all decided on the host. Without a GPU, init's two memsets
+    fail (GEAR_ERR_CUDA) after the host state is written."""
+    import numpy as np
+    L, E = gear.lib, gear.gear
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.02, rank=4, buffer_len=20, buffer_rank=2)
+    B, H, P, NP, ppr, nblk = 3, 2, 64, 10, 4, 5
+    nb = L.gear_paged_cache_bytes(ctypes.byref(p), B, H, 128, P, NP, ppr, nblk, 0)
+    per_tok = 64 + 16 + 3 + 6 + 8
+    pool = per_tok * NP * H * P
+    assert pool <= nb <= pool + B * H * (nblk * 128 * 4 * 4 + 20 * 256) + 12 * 256
+    assert L.gear_paged_host_ints(B, ppr, NP) == 3 * B + B * ppr + NP + 1
+    for bad in [(B, H, 48, NP, ppr), (B, H, 0, NP, ppr), (0, H, P, NP, ppr), (B, H, P, 0, ppr), (B, H, P, NP, 0)]:
+        assert L.gear_paged_cache_bytes(ctypes.byref(p), bad[0], bad[1], 128, bad[2], bad[3], bad[4], nblk, 0) == 0
+    pk = gear.make_params(channel_groups=True, buffer_len=64)
+    assert L.gear_paged_cache_bytes(ctypes.byref(pk), B, H, 128, P, NP, ppr, nblk, 0) == 0
+    nh = L.gear_paged_host_ints(B, ppr, NP)
+    host = np.full(nh, 7, dtype=np.int32)
+    hp = ctypes.c_void_p(host.ctypes.data)
+    c = gear.GearCacheStruct()
+    fake = ctypes.c_void_p(1 << 40)
+    assert L.gear_paged_cache_init(ctypes.byref(c), ctypes.byref(p), B, H, 128, P, NP, ppr, nblk, 0, fake, nb - 1,
+                                   hp, nh, None) == E.GEAR_ERR_CAPACITY
+    assert L.gear_paged_cache_init(ctypes.byref(c), ctypes.byref(p), B, H, 128, P, NP, ppr, nblk, 0, fake, nb,
+                                   hp, nh - 1, None) == E.GEAR_ERR_CAPACITY
+    assert L.gear_paged_cache_init(ctypes.byref(c), ctypes.byref(p), B, H, 128, 40, NP, ppr, nblk, 0, fake, nb,
+                                   hp, nh, None) == E.GEAR_ERR_INVALID_ARG
+    assert (host == 7).all()   # nothing written on an error
+    st = L.gear_paged_cache_init(ctypes.byref(c), ctypes.byref(p), B, H, 128, P, NP, ppr, nblk, 0, fake, nb,
+                                 hp, nh, None)
+    assert st in (E.GEAR_OK, E.GEAR_ERR_CUDA)
+    assert (c.page_tokens, c.num_pages, c.pages_per_row, c.n_max, c.blk0_rank) == (P, NP, ppr, P * ppr, 4)
+    offs = [c.codes, c.meta, c.oidx, c.oval, c.lfac, c.rfac, c.buf, c.table, c.rows]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert c.rows + 3 * B * 4 <= (1 << 40) + nb
+    assert (host[:3 * B] == 0).all() and (host[3 * B:3 * B + B * ppr] == -1).all()
+    assert list(host[3 * B + B * ppr:-1]) == list(range(NP - 1, -1, -1)) and host[-1] == NP
+    # row-call argument errors: returned before anything is enqueued
+    rows = (ctypes.c_int32 * 2)(0, 0)
+    ws = ctypes.c_void_p(1 << 41)
+    kv = ctypes.c_void_p(1 << 42)
+    assert L.gear_encode_rows(ctypes.byref(c), rows, 2, kv, 10, ws, 1 << 30, None) == E.GEAR_ERR_INVALID_ARG  # repeated
+    rows = (ctypes.c_int32 * 1)(3)
+    assert L.gear_encode_rows(ctypes.byref(c), rows, 1, kv, 10, ws, 1 << 30, None) == E.GEAR_ERR_INVALID_ARG  # range
+    rows = (ctypes.c_int32 * 1)(1)
+    assert L.gear_encode_rows(ctypes.byref(c), rows, 1, kv, 2, ws, 1 << 30, None) == E.GEAR_ERR_INVALID_ARG  # rank > n
+    assert L.gear_encode_rows(ctypes.byref(c), rows, 1, kv, P * ppr + 1, ws, 1 << 30, None) == E.GEAR_ERR_CAPACITY
+    rows3 = (ctypes.c_int32 * 3)(0, 1, 2)
+    assert L.gear_encode_rows(ctypes.byref(c), rows3, 3, kv, 4 * P, ws, 1 << 30, None) == E.GEAR_ERR_CAPACITY  # pages
+    assert L.gear_encode_rows(ctypes.byref(c), rows, 1, kv, 100, None, 0, None) == E.GEAR_ERR_WORKSPACE
+    assert L.gear_append_rows(ctypes.byref(c), ctypes.byref(c), rows, 1, kv, kv, ws, 1 << 30,
+                              None) == E.GEAR_ERR_INVALID_ARG   # one cache as both K and V
+    # the contiguous entry points refuse a paged cache
+    assert L.gear_encode(ctypes.byref(c), kv, 10, ws, 1 << 30, None) == E.GEAR_ERR_UNSUPPORTED
+    assert L.gear_cache_reset(ctypes.byref(c)) == E.GEAR_ERR_UNSUPPORTED
+    assert L.gear_decode_dense(ctypes.byref(c), ctypes.c_void_p(1 << 42), None) == E.GEAR_ERR_UNSUPPORTED
+    assert (host[:3 * B] == 0).all() and host[-1] == NP   # untouched by the refused calls

@@ -1,0 +1,287 @@
+"""GPU parity of the paged layout: rows (sequences) with their own prompt
+lengths join, append and leave independently, each row's buffer flushing when
+that row's buffer is full. The oracle of a batch of independent rows is one
+oracle cache per row (batch 1), driven by the same calls; the stored blocks are
+compared bit for bit (codes, scales, zero points, outliers) and attention within
+the decode tolerance. With equal rows the paged cache must store exactly what
+the contiguous cache stores."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.gpu_helpers import TORCH_DT, compare_unit, oracle_params, seeded_kv, to_dev
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import kv_cache_compression_gear_b200 as gear
+else:
+    gear = None
+
+TAU = 1.0 / math.sqrt(128)
+
+
+def _tol_out(dtype: str) -> float:
+    return 8e-3 if dtype == "bf16" else 1e-3
+
+
+def paged_block(cache, b: int, h: int, t0: int, t1: int, blk: int, rank: int) -> dict:
+    """Stored arrays of tokens [t0, t1) of row b, head h, gathered through the
+    host copy of the block table (numpy; L and Rf unscaled)."""
+    A = cache.arrays()
+    P = cache.c.page_tokens
+    _, _, _, table = cache.counters()
+    t = np.arange(t0, t1)
+    pg = table[b, t // P]
+    assert (pg >= 0).all()
+    off = t % P
+    n = t1 - t0
+    e = 0
+    while (2 << e) <= n:
+        e += 1
+    e //= 2
+    pg_t = torch.from_numpy(pg.astype(np.int64)).cuda()
+    off_t = torch.from_numpy(off.astype(np.int64)).cuda()
+
+    def take(name):
+        return A[name][pg_t, h, off_t].cpu()
+
+    return {
+        "codes": take("codes").numpy(),
+        "meta": take("meta").float().numpy() if A["meta"].dtype == torch.float16 else take("meta").numpy(),
+        "oidx": take("oidx").numpy(),
+        "oval": take("oval").float().numpy(),
+        "L": take("lfac")[:, :rank].float().numpy().astype(np.float64) * 2.0 ** -e,
+        "Rf": A["rfac"][b, h, blk, :, :rank].cpu().numpy().astype(np.float64) * 2.0 ** e,
+    }
+
+
+class RowOracle:
+    """One oracle K and V cache (batch 1) per row of the paged batch."""
+
+    def __init__(self, op, B, H):
+        self.op, self.H = op, H
+        self.k = [None] * B
+        self.v = [None] * B
+
+    def encode(self, b, xk, xv):
+        self.k[b] = oracle.Cache(self.op, 1, self.H, 128)
+        self.v[b] = oracle.Cache(self.op, 1, self.H, 128)
+        self.k[b].encode(xk[None])
+        self.v[b].encode(xv[None])
+
+    def append(self, b, rk, rv):
+        self.k[b].append(rk[None])
+        self.v[b].append(rv[None])
+
+    def release(self, b):
+        self.k[b] = self.v[b] = None
+
+    def attn(self, q):
+        out = np.zeros(q.shape, dtype=np.float64)
+        vmax = 0.0
+        for b in range(q.shape[0]):
+            if self.k[b] is None:
+                continue
+            out[b] = oracle.decode_attn(self.k[b], self.v[b], q[b:b + 1], TAU)[0]
+            vmax = max(vmax, float(np.abs(self.v[b].dense()).max()))
+        return out, vmax
+
+
+def _check_blocks(kc, ro: RowOracle, B, H, p, what):
+    b0, nblk, nbuf, _ = kc.counters()
+    for b in range(B):
+        if ro.k[b] is None:
+            assert nblk[b] == 0 and nbuf[b] == 0
+            continue
+        ok = ro.k[b]
+        assert nblk[b] == len(ok.blocks) and nbuf[b] == len(ok.buffer), (what, b)
+        t0 = 0
+        for bi, blk in enumerate(ok.blocks):
+            n = blk[0].codes.shape[0]
+            rank = p.rank if bi == 0 else p.buffer_rank
+            for h in range(H):
+                compare_unit(paged_block(kc, b, h, t0, t0 + n, bi, rank), blk[h], p, f"{what} row {b} block {bi}")
+            t0 += n
+        assert b0[b] == ok.blocks[0][0].codes.shape[0]
+
+
+PAGED_CASES = [
+    # dtype, H, Hq, bits, g, s, r, n_b, r_buf, P, meta_f16
+    ("f16", 2, 4, 4, 64, 0.02, 4, 24, 2, 64, False),
+    ("bf16", 2, 16, 2, 32, 0.05, 8, 20, 2, 32, False),   # eight query heads per kv head, pages of one tile
+    ("f32", 1, 2, 8, 64, 0.02, 2, 12, 1, 96, False),
+    ("f16", 2, 2, 4, 32, 0.0, 4, 16, 2, 64, True),       # GEAR-L, binary16 metadata
+]
+
+
+@pytest.mark.parametrize("dtype,H,Hq,bits,g,s,r,n_b,r_buf,P,meta_f16", PAGED_CASES)
+def test_paged_rows_match_oracle(dtype, H, Hq, bits, g, s, r, n_b, r_buf, P, meta_f16):
+    B = 4
+    p = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=r, buffer_len=n_b, buffer_rank=r_buf,
+                         power_iters=3, seed=23, meta_f16=meta_f16)
+    op = oracle_params(p)
+    ppr, num_pages = 8, 20
+    kc = gear.PagedCache(p, B, H, P, num_pages, ppr, 8, TORCH_DT[dtype])
+    vc = gear.PagedCache(p, B, H, P, num_pages, ppr, 8, TORCH_DT[dtype])
+    ro = RowOracle(op, B, H)
+    seed = [1000]
+
+    def kv(n, rows):
+        seed[0] += 1
+        xk = seeded_kv(seed[0], 1, (rows, H, n, 128), dtype, channel_scale=True)
+        xv = seeded_kv(seed[0], 2, (rows, H, n, 128), dtype)
+        return xk, xv
+
+    def encode(rows, n):
+        xk, xv = kv(n, len(rows))
+        kc.encode_rows(rows, to_dev(xk, dtype))
+        vc.encode_rows(rows, to_dev(xv, dtype))
+        for i, b in enumerate(rows):
+            ro.encode(b, xk[i], xv[i])
+
+    def append(rows):
+        seed[0] += 1
+        rk = seeded_kv(seed[0], 3, (len(rows), H, 128), dtype)
+        rv = seeded_kv(seed[0], 4, (len(rows), H, 128), dtype)
+        gear.append_rows(kc, vc, rows, to_dev(rk, dtype), to_dev(rv, dtype))
+        for i, b in enumerate(rows):
+            ro.append(b, rk[i], rv[i])
+
+    def check(what):
+        torch.cuda.synchronize()
+        assert gear.device_status() == 0
+        seed[0] += 1
+        q = seeded_kv(seed[0], 5, (B, Hq, 128), dtype)
+        od, vmax = ro.attn(q)
+        out = gear.decode_attn(kc, vc, to_dev(q, dtype), TAU, out_dtype=torch.float32).cpu().numpy()
+        err = np.abs(out - od).max()
+        assert err <= _tol_out(dtype) * vmax, f"{what}: attention error {err:.3e} vs {_tol_out(dtype) * vmax:.3e}"
+        for b in range(B):
+            if ro.k[b] is None:
+                assert not out[b].any(), f"{what}: row {b} has no tokens"
+        _check_blocks(kc, ro, B, H, p, what)
+        assert np.array_equal(kc.host, vc.host)
+
+    # rows 0 and 2 join with 100 tokens, row 1 with 37; row 3 stays empty
+    encode([0, 2], 100)
+    encode([1], 37)
+    check("after prefill")
+    for step in range(60):
+        rows = [0] + ([1] if step % 2 == 0 else []) + ([2] if step % 3 == 0 else []) + ([3] if step >= 21 else [])
+        if step == 20:
+            encode([3], 70)
+        if step == 40:   # row 1 leaves; its pages go back to the pool and a new sequence takes the row
+            kc.release_rows([1])
+            vc.release_rows([1])
+            ro.release(1)
+            check("after release")
+            encode([1], 50)
+        append(rows)
+        if step in (25, 49, 59):
+            check(f"step {step}")
+    b0, nblk, nbuf, _ = kc.counters()
+    assert nblk.max() >= 3   # some row flushed twice
+    assert len(set(nblk.tolist())) > 1   # rows at different block counts
+    # every page is accounted for
+    _, _, _, table = kc.counters()
+    used = table[table >= 0]
+    assert len(set(used.tolist())) == used.size
+    assert used.size + kc.free_pages() == num_pages
+
+
+@pytest.mark.parametrize("dtype,Hq", [("f16", 4), ("bf16", 2)])
+def test_paged_equal_rows_match_contiguous_exactly(dtype, Hq):
+    """Equal rows: the paged cache runs the same encoder launches (same unit
+    count and tiling) and the same decode plan, so every stored value is
+    bit-identical to the contiguous cache's, and attention agrees up to the
+    order of the value-outlier atomics (fp32 sums in either order)."""
+    B, H, n0, n_b = 3, 2, 150, 20
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.02, rank=4, buffer_len=n_b, buffer_rank=2,
+                         power_iters=3, seed=5)
+    xk = seeded_kv(71, 1, (B, H, n0, 128), dtype, channel_scale=True)
+    xv = seeded_kv(71, 2, (B, H, n0, 128), dtype)
+    kc = gear.Cache(p, B, H, 256, 6, TORCH_DT[dtype])
+    vc = gear.Cache(p, B, H, 256, 6, TORCH_DT[dtype])
+    pk = gear.PagedCache(p, B, H, 64, 16, 4, 6, TORCH_DT[dtype])
+    pv = gear.PagedCache(p, B, H, 64, 16, 4, 6, TORCH_DT[dtype])
+    kc.encode(to_dev(xk, dtype))
+    vc.encode(to_dev(xv, dtype))
+    pk.encode_rows([0, 1, 2], to_dev(xk, dtype))
+    pv.encode_rows([0, 1, 2], to_dev(xv, dtype))
+    for i in range(45):
+        rk = to_dev(seeded_kv(300 + i, 3, (B, H, 128), dtype), dtype)
+        rv = to_dev(seeded_kv(300 + i, 4, (B, H, 128), dtype), dtype)
+        gear.append_buffer(kc, vc, rk, rv)
+        gear.append_rows(pk, pv, [0, 1, 2], rk, rv)
+        if i in (0, 20, 44):
+            q = to_dev(seeded_kv(900 + i, 5, (B, Hq, 128), dtype), dtype)
+            a = gear.decode_attn(kc, vc, q, TAU, out_dtype=torch.float32)
+            b = gear.decode_attn(pk, pv, q, TAU, out_dtype=torch.float32)
+            assert (a - b).abs().max().item() <= 1e-5 * a.abs().max().item() + 1e-30, i
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    assert (pk.n_comp, pk.n_buf, pk.c.n_blk) == (kc.n_comp, kc.n_buf, kc.n_blk)
+    A, Pa = kc.arrays(), pk.arrays()
+    _, _, _, table = pk.counters()
+    P = pk.c.page_tokens
+    t = np.arange(kc.n_comp)
+    for b in range(B):
+        pg = torch.from_numpy(table[b, t // P].astype(np.int64)).cuda()
+        off = torch.from_numpy((t % P).astype(np.int64)).cuda()
+        for h in range(H):
+            u = b * H + h
+            for name in ("codes", "meta", "oidx", "oval", "lfac"):
+                assert torch.equal(A[name][u, :kc.n_comp], Pa[name][pg, h, off]), (name, b, h)
+            assert torch.equal(A["rfac"][u, :kc.n_blk], Pa["rfac"][b, h, :kc.n_blk]), (b, h)
+            assert torch.equal(A["buf"][u], Pa["buf"][b, h])
+
+
+def test_paged_pool_exhaustion_and_reuse():
+    B, H = 3, 1
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.02, rank=2, buffer_len=8, buffer_rank=1)
+    kc = gear.PagedCache(p, B, H, 32, 5, 4, 8, torch.float16)
+    vc = gear.PagedCache(p, B, H, 32, 5, 4, 8, torch.float16)
+    x = to_dev(seeded_kv(3, 1, (1, H, 64, 128), "f16"), "f16")
+    kc.encode_rows([0], x)      # 2 pages
+    vc.encode_rows([0], x)
+    kc.encode_rows([1], x)      # 2 pages
+    vc.encode_rows([1], x)
+    assert kc.free_pages() == 1
+    with pytest.raises(gear.GearError) as ei:
+        kc.encode_rows([2], x)  # needs 2, 1 left
+    assert ei.value.status == gear.gear.GEAR_ERR_CAPACITY
+    with pytest.raises(gear.GearError) as ei:
+        kc.encode_rows([0], x)  # row 0 is not empty
+    assert ei.value.status == gear.gear.GEAR_ERR_INVALID_ARG
+    with pytest.raises(gear.GearError) as ei:
+        gear.append_rows(kc, vc, [2], x[0, :, 0].contiguous(), x[0, :, 0].contiguous())   # row 2 never encoded
+    assert ei.value.status == gear.gear.GEAR_ERR_INVALID_ARG
+    # fill row 0's buffer (8 tokens), then the ninth append flushes into the last free page
+    r = x[0, :, :1].reshape(1, H, 128).contiguous()
+    for _ in range(9):
+        gear.append_rows(kc, vc, [0], r, r)
+    assert kc.free_pages() == 0
+    # row 1's flush would need a page: nothing is enqueued and the counters stay
+    for _ in range(8):
+        gear.append_rows(kc, vc, [1], r, r)
+    before = kc.host.copy()
+    with pytest.raises(gear.GearError) as ei:
+        gear.append_rows(kc, vc, [1], r, r)
+    assert ei.value.status == gear.gear.GEAR_ERR_CAPACITY
+    assert np.array_equal(kc.host, before)
+    kc.release_rows([0])
+    vc.release_rows([0])
+    assert kc.free_pages() == 3
+    gear.append_rows(kc, vc, [1], r, r)   # the flush takes a page row 0 gave back
+    kc.encode_rows([2], x)
+    vc.encode_rows([2], x)
+    assert kc.free_pages() == 0
+    q = to_dev(seeded_kv(4, 5, (B, H, 128), "f16"), "f16")
+    out = gear.decode_attn(kc, vc, q, TAU, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    assert not out[0].any() and out[1].abs().max() > 0 and out[2].abs().max() > 0
