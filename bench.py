@@ -624,6 +624,7 @@ def run_gpu(args, rank: int, world: int):
                                            meta_f16=True)
         line["kivi_keys"] = variant_measure(gear, wl, we, wd, dev, max(3, args.steps // 2), hbm, s=we.s,
                                             kivi=True)
+        line["paged"] = paged_measure(gear, wl, wl.WORKLOADS[DEC], dev, max(3, args.steps // 2), hbm)
         line["cpu_baseline"] = cpu_baseline(HEADLINE)
         for sc in BESIDE:
             line["configs"][sc.name]["cpu_baseline"] = cpu_baseline(sc)
@@ -709,6 +710,94 @@ def variant_measure(gear, wl, we, wd, dev, reps, hbm, s, meta_f16=False, kivi=Fa
             "decode_ms": round(dec_ms, 4), "decode_tokens_per_s": round(w0d.B / dec_ms * 1e3, 1),
             "decode_hbm_frac": round(dec_alg / dec_ms / 1e6 / hbm, 4),
             "bytes_per_token": ptb}
+
+
+def paged_measure(gear, wl, wd, dev, reps, hbm, page_tokens=256):
+    """The decode workload in the paged layout (gear_encode_rows, gear_append_rows,
+    decode through the block table): first with every row at the full context, the
+    case the contiguous decode stage times, then with the rows' prompts spread evenly
+    over [n/2, n] (each row encoded at its own length). Timed like the main stages
+    (CUDA events, L2 flushed before each timed launch sequence). The decode split
+    covers the longest row, so the ragged batch's fraction (counted on the tokens
+    the rows hold) shows what the idle share of the shorter rows costs."""
+    import torch
+    dt = wl.torch_dtype(wd.dtype)
+    p = _gparams(gear, wd)
+    P = page_tokens
+    ppr = -(-(wd.n + 2 * wd.buffer_len) // P)
+    nblk = 4
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    esz = 4 if wd.dtype == "f32" else 2
+    rows = list(range(wd.B))
+    xs = {which: wl.kv_tensor_torch(wd, which, 0, dev) for which in ("k", "v")}
+    q = wl.rows_torch(wd, wl.S_Q, 0, 0, wd.Hq, dev)
+    out = torch.empty((wd.B, wd.Hq, 128), dtype=dt, device=dev)
+    tau = 1.0 / math.sqrt(128)
+    kc = gear.PagedCache(p, wd.B, wd.H, P, wd.B * ppr, ppr, nblk, dt, dev)
+    vc = gear.PagedCache(p, wd.B, wd.H, P, wd.B * ppr, ppr, nblk, dt, dev)
+
+    def fill(lengths):
+        for c in (kc, vc):
+            c.release_rows(rows)
+        by_len = {}
+        for b, n in enumerate(lengths):
+            by_len.setdefault(n, []).append(b)
+        for n, rs in by_len.items():
+            for c, which in ((kc, "k"), (vc, "v")):
+                c.encode_rows(rs, xs[which][rs][:, :, :n].contiguous())
+        for i in range(wd.buffer_fill):
+            gear.append_rows(kc, vc, rows, wl.rows_torch(wd, wl.S_KBUF, 0, i, wd.H, dev),
+                             wl.rows_torch(wd, wl.S_VBUF, 0, i, wd.H, dev))
+
+    def time_decode():
+        ts = []
+        for it in range(reps + 3):
+            flush.fill_(it & 0xFF)
+            a, b = ev(), ev()
+            a.record()
+            gear.decode_attn(kc, vc, q, tau, out=out)
+            b.record()
+            torch.cuda.synchronize()
+            if it >= 3:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def alg_bytes(lengths):
+        rp = (max(wd.rank, wd.buffer_rank) + 3) // 4 * 4
+        return sum(2 * wd.H * (n * per_token_bytes(wd) + rp * 128 * 4 + wd.buffer_fill * 128 * esz)
+                   for n in lengths) + 2 * wd.B * wd.Hq * 128 * esz
+
+    # encode_rows of the whole batch (K and V): the codec on a staging copy, then the scatter into pages
+    enc = []
+    for it in range(reps + 3):
+        for c in (kc, vc):
+            c.release_rows(rows)
+        flush.fill_(it & 0xFF)
+        a, b = ev(), ev()
+        a.record()
+        kc.encode_rows(rows, xs["k"])
+        vc.encode_rows(rows, xs["v"])
+        b.record()
+        torch.cuda.synchronize()
+        if it >= 3:
+            enc.append(a.elapsed_time(b))
+    full = [wd.n] * wd.B
+    fill(full)
+    dec_full = time_decode()
+    ragged = [wd.n // 2 + (wd.n // 2) * b // max(1, wd.B - 1) // 32 * 32 for b in range(wd.B)]
+    fill(ragged)
+    dec_rag = time_decode()
+    assert gear.device_status() == 0, "device-side error word set"
+    enc_ms = statistics.median(enc)
+    enc_in = 2 * wd.B * wd.H * wd.n * wd.d * esz
+    af, ar = alg_bytes(full), alg_bytes(ragged)
+    return {"page_tokens": P, "pages_per_row": ppr, "encode_rows_ms": round(enc_ms, 4),
+            "encode_rows_gbs": round(enc_in / enc_ms / 1e6, 3),
+            "decode_ms": round(dec_full, 4), "decode_tokens_per_s": round(wd.B / dec_full * 1e3, 1),
+            "decode_hbm_frac": round(af / dec_full / 1e6 / hbm, 4),
+            "ragged": {"prefill_lengths": [min(ragged), max(ragged)], "decode_ms": round(dec_rag, 4),
+                       "decode_hbm_frac": round(ar / dec_rag / 1e6 / hbm, 4)}}
 
 
 def main():
