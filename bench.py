@@ -718,8 +718,7 @@ def paged_measure(gear, wl, wd, dev, reps, hbm, page_tokens=256):
     case the contiguous decode stage times, then with the rows' prompts spread evenly
     over [n/2, n] (each row encoded at its own length). Timed like the main stages
     (CUDA events, L2 flushed before each timed launch sequence). The decode split
-    covers the longest row, so the ragged batch's fraction (counted on the tokens
-    the rows hold) shows what the idle share of the shorter rows costs."""
+    runs over the tokens the rows hold, so both fractions count the tokens read."""
     import torch
     dt = wl.torch_dtype(wd.dtype)
     p = _gparams(gear, wd)

@@ -317,8 +317,9 @@ gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream)
  * paged caches (both K and V paged, built by the same calls on the same rows,
  * so that their counters and tables agree; INVALID_ARG otherwise): each row
  * attends over its own tokens, a row without tokens gets an output of 0.
- * The work split covers the longest row, so rows shorter than it leave part
- * of their share idle. gear_encode, gear_encode_batch, gear_append_buffer,
+ * The decode work split runs over the tokens the rows hold (rows laid end to
+ * end at their own lengths), so a ragged batch costs what its tokens cost.
+ * gear_encode, gear_encode_batch, gear_append_buffer,
  * gear_cache_reset and gear_decode_dense return UNSUPPORTED on a paged cache.
  * Limits: channel_groups = 0; P a multiple of 32 (a decode tile of 32 tokens
  * never spans two pages). */

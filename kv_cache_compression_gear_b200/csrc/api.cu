@@ -537,6 +537,11 @@ static gear_status decode_args(const gear_cache* k, const gear_cache* v, int32_t
     a.page_tokens = k->page_tokens;
     a.ppr = k->pages_per_row;
     a.num_pages = k->num_pages;
+    // the split runs over the tokens the rows hold, not over B * H * max length
+    const HostView h = host_view(k);
+    int64_t tot = 0;
+    for (int b = 0; b < k->B; ++b) tot += (int64_t)k->H * row_ncomp(k, h, b);
+    a.tot_tokens = tot;
   }
   decode_plan(a, current_sm_count());
   return GEAR_OK;

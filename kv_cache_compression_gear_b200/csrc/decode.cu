@@ -28,7 +28,19 @@ __global__ void __launch_bounds__(128) decode_combine(const DecodeArgs a) {
   const float* p = a.part + (size_t)bj * a.nsplit * 130;
   // the warps that met this query head's unit wrote partial rows 0 .. nseg-1
   int nseg = 1;
-  if (a.n_comp > 0) {
+  if (a.rows && a.tot_tokens > 0) {
+    // paged layout: the unit's start in the rows' token space (see decode_warp)
+    const int b = bj / a.Hq, h = (bj % a.Hq) / a.hq;
+    auto len_of = [&](int r) {
+      const int nb = __ldg(a.rows + a.B + r);
+      return nb > 0 ? __ldg(a.rows + r) + (nb - 1) * a.n_b : 0;
+    };
+    int64_t start = 0;
+    for (int r = 0; r < b; ++r) start += (int64_t)a.H * len_of(r);
+    const int len = len_of(b);
+    start += (int64_t)h * len;
+    nseg = len > 0 ? (int)((start + len - 1) / a.seg_tokens - start / a.seg_tokens + 1) : 0;
+  } else if (a.n_comp > 0) {
     const int64_t u = (int64_t)(bj / a.Hq) * a.H + (bj % a.Hq) / a.hq, n = a.n_comp;
     nseg = (int)(((u + 1) * n - 1) / a.seg_tokens - (u * n) / a.seg_tokens + 1);
   }
@@ -78,8 +90,8 @@ void decode_plan(DecodeArgs& a, int num_sms) {
   const int by_smem = 233472 / (smem_cta + 1024);   // 228 KiB per SM, 1 KiB reserved per CTA
   const int by_regs = hq <= 2 ? 4 : (hq == 4 ? 2 : 1);
   const long long resident = (long long)num_sms * (by_smem < by_regs ? (by_smem > 0 ? by_smem : 1) : by_regs) * 4;
-  if (a.n_comp > 0) {
-    const long long tot = (long long)a.n_comp * units;
+  const long long tot = a.rows ? (long long)a.tot_tokens : (long long)a.n_comp * units;
+  if (tot > 0) {
     long long seg = (tot + resident - 1) / resident;
     seg = (seg + kDTile - 1) / kDTile * kDTile;
     a.seg_tokens = (int)seg;

@@ -71,6 +71,7 @@ struct DecodeArgs {
   const int32_t* table;
   const int32_t* rows;
   int32_t page_tokens, ppr, num_pages;
+  int64_t tot_tokens;     // paged layout: compressed tokens of all units (H * sum of the rows' lengths)
   int32_t seg_tokens;     // compressed tokens per warp (a multiple of 32); 0 without any
   int32_t nsplit;         // partial rows per unit: at most ceil(n_comp / seg_tokens) + 1 warps meet a unit
   int32_t total_splits;   // warps: ceil(units * n_comp / seg_tokens), or units without compressed tokens

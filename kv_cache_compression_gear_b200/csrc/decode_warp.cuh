@@ -998,23 +998,66 @@ __global__ void __launch_bounds__(kDThreads, HQ <= 2 ? 4 : (HQ == 4 ? 2 : 1)) de
   // units' compressed tokens, cut at unit boundaries; the warp that ends a unit
   // also takes its buffer. Without compressed tokens, warp gs takes unit gs's
   // buffer.
+  // Paged layout: units hold their rows' own lengths, laid end to end row by
+  // row (unit b*H + h starts at H * (lengths of rows < b) + h * length of b).
   const int64_t n = a.n_comp;
-  int64_t gpos = n > 0 ? (int64_t)gs * a.seg_tokens : 0;
-  const int64_t gend = n > 0 ? min(gpos + (int64_t)a.seg_tokens, (int64_t)a.B * a.H * n) : 1;
+  const int64_t tot = a.rows ? a.tot_tokens : (int64_t)a.B * a.H * n;
+  int64_t gpos = tot > 0 ? (int64_t)gs * a.seg_tokens : 0;
+  const int64_t gend = tot > 0 ? min(gpos + (int64_t)a.seg_tokens, tot) : 1;
   while (gpos < gend) {
     int unit, c0, c1, sp;
-    if (n > 0) {
+    bool with_buf;
+    if (a.rows && tot > 0) {
+      // the row holding position gpos: 32 rows per pass, lane = row, running
+      // sums of the rows' token counts (H units each)
+      int row = -1, rlen = 0;
+      int64_t rstart = 0, base = 0;
+      for (int bc = 0; bc < a.B && row < 0; bc += 32) {
+        const int bl = bc + lane;
+        int len = 0;
+        if (bl < a.B) {
+          const int nb = __ldg(a.rows + a.B + bl);
+          len = nb > 0 ? __ldg(a.rows + bl) + (nb - 1) * a.n_b : 0;
+        }
+        int64_t incl = (int64_t)a.H * len;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int64_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int64_t end = base + incl;
+        const unsigned hit = __ballot_sync(0xFFFFFFFFu, bl < a.B && end > gpos);
+        if (hit) {
+          const int l = __ffs(hit) - 1;
+          row = bc + l;
+          rlen = __shfl_sync(0xFFFFFFFFu, len, l);
+          rstart = __shfl_sync(0xFFFFFFFFu, end, l) - (int64_t)a.H * rlen;
+        }
+        base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      if (row < 0) break;   // past the last token (not reached: gend <= tot)
+      const int hh = (int)((gpos - rstart) / rlen);
+      const int64_t ustart = rstart + (int64_t)hh * rlen;
+      unit = row * a.H + hh;
+      c0 = (int)(gpos - ustart);
+      c1 = (int)min((int64_t)rlen, gend - ustart);
+      sp = gs - (int)(ustart / a.seg_tokens);
+      gpos = ustart + c1;
+      with_buf = c1 == rlen;
+    } else if (n > 0) {
       unit = (int)(gpos / n);
       c0 = (int)(gpos - unit * n);
       c1 = (int)min(n, gend - unit * n);
       sp = gs - (int)((unit * n) / a.seg_tokens);
       gpos = unit * n + c1;
+      with_buf = c1 == (int)n && a.n_buf > 0;
     } else {
       unit = gs;
       c0 = c1 = sp = 0;
       gpos = gend;
+      with_buf = a.n_buf > 0;
     }
-    if (!segment(unit, c0, c1, sp, c1 == (int)n && a.n_buf > 0)) return;
+    if (!segment(unit, c0, c1, sp, with_buf)) return;
   }
 }
 

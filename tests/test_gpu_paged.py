@@ -285,3 +285,45 @@ def test_paged_pool_exhaustion_and_reuse():
     torch.cuda.synchronize()
     assert gear.device_status() == 0
     assert not out[0].any() and out[1].abs().max() > 0 and out[2].abs().max() > 0
+
+
+def test_paged_many_ragged_rows_match_oracle():
+    """More rows than a warp has lanes (the decoder's row search runs in passes of
+    32 rows), lengths from 1 to a few hundred tokens, empty rows between them, and
+    buffers at different fills: every row against its own oracle caches."""
+    B, H, Hq, dtype = 45, 1, 2, "f16"
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.02, rank=1, buffer_len=8, buffer_rank=1,
+                         power_iters=2, seed=9)
+    op = oracle_params(p)
+    kc = gear.PagedCache(p, B, H, 32, 400, 12, 6, torch.float16)
+    vc = gear.PagedCache(p, B, H, 32, 400, 12, 6, torch.float16)
+    ro = RowOracle(op, B, H)
+    lengths = [0 if b % 7 == 3 else 1 + (b * 37) % 300 for b in range(B)]
+    for b, n in enumerate(lengths):
+        if n == 0:
+            continue
+        xk = seeded_kv(500 + b, 1, (1, H, n, 128), dtype, channel_scale=True)
+        xv = seeded_kv(500 + b, 2, (1, H, n, 128), dtype)
+        kc.encode_rows([b], to_dev(xk, dtype))
+        vc.encode_rows([b], to_dev(xv, dtype))
+        ro.encode(b, xk[0], xv[0])
+    live = [b for b in range(B) if lengths[b]]
+    for step in range(20):
+        rows = [b for b in live if (b + step) % 3 != 0]
+        rk = seeded_kv(700 + step, 3, (len(rows), H, 128), dtype)
+        rv = seeded_kv(700 + step, 4, (len(rows), H, 128), dtype)
+        gear.append_rows(kc, vc, rows, to_dev(rk, dtype), to_dev(rv, dtype))
+        for i, b in enumerate(rows):
+            ro.append(b, rk[i], rv[i])
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    q = seeded_kv(901, 5, (B, Hq, 128), dtype)
+    od, vmax = ro.attn(q)
+    for _ in range(2):   # twice: nothing depends on what the workspace held before
+        out = gear.decode_attn(kc, vc, to_dev(q, dtype), TAU, out_dtype=torch.float32).cpu().numpy()
+        err = np.abs(out - od).max()
+        assert err <= 1e-3 * vmax, f"attention error {err:.3e} vs {1e-3 * vmax:.3e}"
+    for b in range(B):
+        if not lengths[b]:
+            assert not out[b].any()
+    _check_blocks(kc, ro, B, H, p, "many rows")
