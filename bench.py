@@ -499,8 +499,8 @@ class Runner:
 TRAFFIC_BYTES = {
     # encode stage: E1 539145984 + 175796224, E2 26292736, E3 723998208 + 30295040 bytes at batch 4
     ("twobit_b64_ctx8192", "encode"): 16 * (539145984 + 175796224 + 26292736 + 723998208 + 30295040),
-    # decode_warp 213756928 + 757504 bytes at batch 4
-    ("twobit_b64_ctx8192", "decode"): 16 * (213756928 + 757504),
+    # decode_warp 213735424 + 463360 bytes at batch 4
+    ("twobit_b64_ctx8192", "decode"): 16 * (213735424 + 463360),
 }
 
 
