@@ -933,11 +933,13 @@ __host__ __device__ constexpr int zimg_offset(int N, int n, int c) {
 // Per unit: M = sym(sum of partial Grams), then T power steps with
 // Cholesky-QR on the r x r Gram. Outputs Rf (cache, scaled 2^-e) and
 // Z = Q_{T-1} C_T^-1 scaled 2^e (workspace) so that E3's R Z is the stored L.
-// The partials arrive by 64 KiB bulk asynchronous copies, two in flight, and
-// are summed in a fixed order (deterministic); M is kept in fp32 (the
+// The partials are read by 16-byte loads, all of a partial's in flight at
+// once, and summed in a fixed order (deterministic); M is kept in fp32 (the
 // partials carry about 17 significant bits), products accumulate in fp64.
-constexpr int kE2Threads = 512;
-constexpr int kE2Parts = kE2Threads / 128;   // threads per row of W = M Q
+// NT threads per CTA: 512 when the units fit in one wave (more threads per
+// unit), else 256 with two CTAs per SM (about 95 KB of shared memory at
+// r <= 8), so that one unit's serial steps (the r x r factorization on one
+// thread) overlap another unit's products.
 constexpr int kMStride = 132;  // padded fp32 row of M
 
 __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t i) {
@@ -956,19 +958,15 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
       : "memory");
 }
 
-template <int RM>
+template <int RM, int NT>
 struct E2Smem {
   float M[128 * kMStride];
   double Q[128 * RM];
-  uint64_t bar[2];
-  union {
-    float stage[2][16384];   // partial Grams in flight (phase 1)
-    struct {                 // power-iteration scratch (phase 2)
-      double Wp[kE2Parts * 128 * RM];
-      double red[4 * RM * RM];
-      double Xi[RM * RM];
-    } it;
-  } u;
+  struct {   // power-iteration scratch
+    double Wp[NT / 128 * 128 * RM];
+    double red[4 * RM * RM];
+    double Xi[RM * RM];
+  } it;
 };
 
 // The unit's slab for E3 (see kZSlab): fp32 Z rows, then for 16-bit inputs
@@ -1057,10 +1055,12 @@ __device__ void write_z_slab(const EncodeArgs& a, int u, const float* Zf, float*
   }
 }
 
-template <int RM>
-__global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a) {
+template <int RM, int NT>
+__global__ void __launch_bounds__(NT, 512 / NT) encode_power(const EncodeArgs a) {
+  constexpr int kE2Threads = NT;
+  constexpr int kE2Parts = NT / 128;   // threads per row of W = M Q
   extern __shared__ __align__(128) uint8_t sm2raw[];
-  E2Smem<RM>& S = *reinterpret_cast<E2Smem<RM>*>(sm2raw);
+  E2Smem<RM, NT>& S = *reinterpret_cast<E2Smem<RM, NT>*>(sm2raw);
   const int u = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = a.r;
@@ -1070,15 +1070,6 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
   const int nseg = (int)(c1 - c0 + 1);
   const float* part = a.gram + (int64_t)u * a.maxc * 16384;
 
-  if (tid == 0) {
-    mbar_init(&S.bar[0], 1);
-    mbar_init(&S.bar[1], 1);
-    fence_mbarrier_init();
-    for (int sg = 0; sg < 2 && sg < nseg; ++sg) {
-      mbar_arrive_expect_tx(&S.bar[sg], 65536);
-      bulk_load(S.u.stage[sg], part + (int64_t)sg * 16384, 65536, &S.bar[sg]);
-    }
-  }
   // Q0 from the seed (columns r .. RM-1 stay zero)
   for (int e = tid; e < 128 * RM; e += kE2Threads) {
     const int i = e / RM, j = e % RM;
@@ -1089,33 +1080,26 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
     }
     S.Q[e] = v;
   }
-  __syncthreads();
+  // M = the partials summed in segment order; each thread owns the same 16
+  // float4 slots of every partial, so no barrier is needed between partials
   for (int sg = 0; sg < nseg; ++sg) {
-    const int b = sg & 1;
-    // a wait that gives up (error word set) ends the unit: no factors are
-    // computed from an incomplete Gram; the other stage's copy, if one was
-    // issued, is given its own bounded wait so that nothing lands after exit
-    if (!__syncthreads_and(mbar_wait(&S.bar[b], (sg >> 1) & 1))) {
-      if (tid == 0 && sg + 1 < nseg) mbar_wait(&S.bar[b ^ 1], ((sg + 1) >> 1) & 1);
-      __syncthreads();
-      return;
-    }
-    for (int e4 = tid; e4 < 4096; e4 += kE2Threads) {
-      const float4 v = reinterpret_cast<const float4*>(S.u.stage[b])[e4];
+    const float4* src = reinterpret_cast<const float4*>(part + (int64_t)sg * 16384);
+    float4 v[4096 / kE2Threads];
+#pragma unroll
+    for (int m = 0; m < 4096 / kE2Threads; ++m) v[m] = __ldcs(src + tid + m * kE2Threads);
+#pragma unroll
+    for (int m = 0; m < 4096 / kE2Threads; ++m) {
+      const int e4 = tid + m * kE2Threads;
       float4* dst = reinterpret_cast<float4*>(&S.M[(e4 >> 5) * kMStride + ((e4 & 31) << 2)]);   // 16-byte aligned rows
       if (sg == 0) {
-        *dst = v;
+        *dst = v[m];
       } else {
         const float4 o = *dst;
-        *dst = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+        *dst = make_float4(o.x + v[m].x, o.y + v[m].y, o.z + v[m].z, o.w + v[m].w);
       }
     }
-    __syncthreads();
-    if (tid == 0 && sg + 2 < nseg) {
-      mbar_arrive_expect_tx(&S.bar[b], 65536);
-      bulk_load(S.u.stage[b], part + (int64_t)(sg + 2) * 16384, 65536, &S.bar[b]);
-    }
   }
+  __syncthreads();
   for (int e = tid; e < 128 * 128; e += kE2Threads) {
     const int i = e >> 7, j = e & 127;
     if (i < j) {
@@ -1140,7 +1124,7 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
         for (int j = 0; j < RM; ++j) w[j] = fma(mv, S.Q[c * RM + j], w[j]);
       }
 #pragma unroll
-      for (int j = 0; j < RM; ++j) S.u.it.Wp[(wpart * 128 + i) * RM + j] = w[j];
+      for (int j = 0; j < RM; ++j) S.it.Wp[(wpart * 128 + i) * RM + j] = w[j];
     }
     __syncthreads();
     // G = Q^T W (upper triangle), reduced by warp then across warps
@@ -1148,21 +1132,21 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
       double w[RM], qv[RM];
 #pragma unroll
       for (int j = 0; j < RM; ++j) {
-        double v = S.u.it.Wp[i * RM + j];
+        double v = S.it.Wp[i * RM + j];
 #pragma unroll
-        for (int pp = 1; pp < kE2Parts; ++pp) v += S.u.it.Wp[(pp * 128 + i) * RM + j];
+        for (int pp = 1; pp < kE2Parts; ++pp) v += S.it.Wp[(pp * 128 + i) * RM + j];
         w[j] = v;
         qv[j] = S.Q[i * RM + j];
       }
 #pragma unroll
-      for (int j = 0; j < RM; ++j) S.u.it.Wp[i * RM + j] = w[j];
+      for (int j = 0; j < RM; ++j) S.it.Wp[i * RM + j] = w[j];
 #pragma unroll
       for (int p = 0; p < RM; ++p)
 #pragma unroll
         for (int q = p; q < RM; ++q) {
           double v = qv[p] * w[q];
           for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-          if (lane == 0) S.u.it.red[(warp * RM + p) * RM + q] = v;
+          if (lane == 0) S.it.red[(warp * RM + p) * RM + q] = v;
         }
     }
     __syncthreads();
@@ -1177,8 +1161,8 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
 #pragma unroll
         for (int q = 0; q < RM; ++q) {
           double g = 0.0;
-          if (p <= q) g = S.u.it.red[p * RM + q] + S.u.it.red[(RM + p) * RM + q] + S.u.it.red[(2 * RM + p) * RM + q] +
-                          S.u.it.red[(3 * RM + p) * RM + q];
+          if (p <= q) g = S.it.red[p * RM + q] + S.it.red[(RM + p) * RM + q] + S.it.red[(2 * RM + p) * RM + q] +
+                          S.it.red[(3 * RM + p) * RM + q];
           C[p][q] = g;
           X[p][q] = 0.0;
         }
@@ -1215,7 +1199,7 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
 #pragma unroll
       for (int p = 0; p < RM; ++p)
 #pragma unroll
-        for (int q = 0; q < RM; ++q) S.u.it.Xi[p * RM + q] = X[p][q];
+        for (int q = 0; q < RM; ++q) S.it.Xi[p * RM + q] = X[p][q];
     }
     __syncthreads();
     const bool last = (step + 1 == a.T);
@@ -1226,8 +1210,8 @@ __global__ void __launch_bounds__(kE2Threads, 1) encode_power(const EncodeArgs a
         double sq = 0.0, swv = 0.0;
 #pragma unroll
         for (int m2 = 0; m2 < RM; ++m2) {
-          sq = fma(S.Q[i * RM + m2], S.u.it.Xi[m2 * RM + j], sq);
-          swv = fma(S.u.it.Wp[i * RM + m2], S.u.it.Xi[m2 * RM + j], swv);
+          sq = fma(S.Q[i * RM + m2], S.it.Xi[m2 * RM + j], sq);
+          swv = fma(S.it.Wp[i * RM + m2], S.it.Xi[m2 * RM + j], swv);
         }
         zq[j] = sq;
         wq[j] = swv;
@@ -2032,12 +2016,22 @@ cudaError_t encode_launch(EncodeArgs a, int num_sms, cudaStream_t st) {
 
   {
     const int RM = a.r <= 4 ? 4 : (a.r <= 8 ? 8 : 16);
-    const size_t sm2 = RM == 4 ? sizeof(E2Smem<4>) : (RM == 8 ? sizeof(E2Smem<8>) : sizeof(E2Smem<16>));
-    auto kern = RM == 4 ? encode_power<4> : (RM == 8 ? encode_power<8> : encode_power<16>);
-    static std::atomic<int> smem_set[3][kMaxDevices];
-    e = ensure_smem_limit(kern, (int)sm2, smem_set[RM == 4 ? 0 : (RM == 8 ? 1 : 2)]);
-    if (e != cudaSuccess) return e;
-    kern<<<a.U, kE2Threads, sm2, st>>>(a);
+    const bool wide = a.U <= num_sms;   // one wave: 512 threads per unit
+    const int ri = RM == 4 ? 0 : (RM == 8 ? 1 : 2);
+    static std::atomic<int> smem_set[2][3][kMaxDevices];
+    if (wide) {
+      const size_t sm2 = RM == 4 ? sizeof(E2Smem<4, 512>) : (RM == 8 ? sizeof(E2Smem<8, 512>) : sizeof(E2Smem<16, 512>));
+      auto kern = RM == 4 ? encode_power<4, 512> : (RM == 8 ? encode_power<8, 512> : encode_power<16, 512>);
+      e = ensure_smem_limit(kern, (int)sm2, smem_set[0][ri]);
+      if (e != cudaSuccess) return e;
+      kern<<<a.U, 512, sm2, st>>>(a);
+    } else {
+      const size_t sm2 = RM == 4 ? sizeof(E2Smem<4, 256>) : (RM == 8 ? sizeof(E2Smem<8, 256>) : sizeof(E2Smem<16, 256>));
+      auto kern = RM == 4 ? encode_power<4, 256> : (RM == 8 ? encode_power<8, 256> : encode_power<16, 256>);
+      e = ensure_smem_limit(kern, (int)sm2, smem_set[1][ri]);
+      if (e != cudaSuccess) return e;
+      kern<<<a.U, 256, sm2, st>>>(a);
+    }
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
