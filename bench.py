@@ -497,8 +497,8 @@ class Runner:
 # The 2-bit batch-64 workload's traffic comes from a capture of the same step at
 # batch 4 (1/16 of the units), scaled by 16: every kernel's traffic is per unit.
 TRAFFIC_BYTES = {
-    # encode stage: E1 539145984 + 175796224, E2 26292736, E3 723998208 + 30295040 bytes at batch 4
-    ("twobit_b64_ctx8192", "encode"): 16 * (539145984 + 175796224 + 26292736 + 723998208 + 30295040),
+    # encode stage: E1 539130624 + 175976960, E2 26284032, E3 723844864 + 30014208 bytes at batch 4
+    ("twobit_b64_ctx8192", "encode"): 16 * (539130624 + 175976960 + 26284032 + 723844864 + 30014208),
     # decode_warp 213735424 + 463360 bytes at batch 4
     ("twobit_b64_ctx8192", "decode"): 16 * (213735424 + 463360),
 }
