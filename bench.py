@@ -41,6 +41,9 @@ ENC = "llama7b_layer_encode"
 DEC = "decode_b16_ctx8192"
 
 
+NOMINAL_HBM_GBS = 8000.0   # the B200's nominal HBM3e bandwidth, beside the measured copy bandwidth
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -555,9 +558,11 @@ def measure(gear, wl, sc: Scenario, dev, rank, world, steps, warmup, hbm, peak_k
     oth = "encode" if dom == "decode" else "decode"
     roof = {"bound": "hbm", "kernel": stages[dom][2], "achieved": round(stages[dom][1], 2), "peak": hbm,
             "unit": "GB/s", "frac": round(stages[dom][1] / hbm, 4), "peak_kind": peak_kind,
+            "frac_nominal": round(stages[dom][1] / NOMINAL_HBM_GBS, 4),
             "traffic": TRAFFIC_BYTES.get((sc.name, dom)),
             "algorithmic_bytes": enc_alg if dom == "encode" else dec_alg}
     other = {"kernel": stages[oth][2], "achieved": round(stages[oth][1], 2), "frac": round(stages[oth][1] / hbm, 4),
+             "frac_nominal": round(stages[oth][1] / NOMINAL_HBM_GBS, 4),
              "traffic": TRAFFIC_BYTES.get((sc.name, oth)),
              "algorithmic_bytes": enc_alg if oth == "encode" else dec_alg}
     res = {
