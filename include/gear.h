@@ -22,7 +22,9 @@
  *    *_bytes() queries.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued asynchronously on it. Argument validation runs on the
- *    host before any launch; on any non-OK status nothing was enqueued.
+ *    host before any launch; on any status other than GEAR_ERR_CUDA nothing
+ *    was enqueued. GEAR_ERR_CUDA means a launch or runtime call failed part
+ *    way through; the caches the call was given are then undefined.
  *  - Element types: GEAR_F16 / GEAR_BF16 / GEAR_F32 for KV, queries, buffer
  *    and outlier values. Quantization metadata is fp32. Low-rank factors L are
  *    fp16 for 16-bit caches and fp32 for fp32 caches; Rf is always fp32.

@@ -209,13 +209,24 @@ static bool paged_ok(const gear_cache* c) {
 }
 
 // K and V caches built by the same calls: same geometry, parameters and host
-// state (counters, tables and free pages), so that one table serves both.
+// state, so that one table serves both. Compared: the row counters, the table
+// entries in use (a row holds exactly the pages its tokens reach) and the free
+// stack, O(B + num_pages) per call.
 static bool paged_pair(const gear_cache* k, const gear_cache* v) {
-  return k->B == v->B && k->H == v->H && k->dtype == v->dtype && k->page_tokens == v->page_tokens &&
-         k->num_pages == v->num_pages && k->pages_per_row == v->pages_per_row && k->nblk_max == v->nblk_max &&
-         k->n_comp == v->n_comp && k->n_buf == v->n_buf && k->n_blk == v->n_blk &&
-         memcmp(&k->p, &v->p, sizeof(gear_params)) == 0 &&
-         memcmp(k->host, v->host, paged_host_ints(k->B, k->pages_per_row, k->num_pages) * sizeof(int32_t)) == 0;
+  if (!(k->B == v->B && k->H == v->H && k->dtype == v->dtype && k->page_tokens == v->page_tokens &&
+        k->num_pages == v->num_pages && k->pages_per_row == v->pages_per_row && k->nblk_max == v->nblk_max &&
+        k->n_comp == v->n_comp && k->n_buf == v->n_buf && k->n_blk == v->n_blk &&
+        memcmp(&k->p, &v->p, sizeof(gear_params)) == 0))
+    return false;
+  const int B = k->B;
+  if (memcmp(k->host, v->host, (size_t)3 * B * sizeof(int32_t)) != 0) return false;
+  const HostView hk = host_view(k), hv = host_view(v);
+  for (int b = 0; b < B; ++b) {
+    const size_t used = (size_t)((row_ncomp(k, hk, b) + k->page_tokens - 1) / k->page_tokens);
+    const size_t off = (size_t)b * k->pages_per_row;
+    if (used && memcmp(hk.table + off, hv.table + off, used * sizeof(int32_t)) != 0) return false;
+  }
+  return *hk.top == *hv.top && memcmp(hk.stack, hv.stack, (size_t)*hk.top * sizeof(int32_t)) == 0;
 }
 
 // rows[0 .. nrows) are distinct rows of c

@@ -327,3 +327,30 @@ def test_paged_many_ragged_rows_match_oracle():
         if not lengths[b]:
             assert not out[b].any()
     _check_blocks(kc, ro, B, H, p, "many rows")
+
+
+def test_paged_pair_must_agree():
+    """K and V caches whose pages were handed out in different orders are
+    refused by decode and append (one table serves both tensors)."""
+    B, H = 2, 1
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.02, rank=2, buffer_len=8, buffer_rank=1)
+    kc = gear.PagedCache(p, B, H, 32, 8, 4, 4, torch.float16)
+    vc = gear.PagedCache(p, B, H, 32, 8, 4, 4, torch.float16)
+    x = to_dev(seeded_kv(8, 1, (1, H, 40, 128), "f16"), "f16")
+    kc.encode_rows([0], x)
+    kc.encode_rows([1], x)
+    vc.encode_rows([1], x)   # the other order: same counters, other pages
+    vc.encode_rows([0], x)
+    b0k, nbk, nfk, tk = kc.counters()
+    b0v, nbv, nfv, tv = vc.counters()
+    assert (b0k == b0v).all() and (nbk == nbv).all() and (nfk == nfv).all() and not (tk == tv).all()
+    q = to_dev(seeded_kv(9, 5, (B, H, 128), "f16"), "f16")
+    with pytest.raises(gear.GearError) as ei:
+        gear.decode_attn(kc, vc, q, TAU)
+    assert ei.value.status == gear.gear.GEAR_ERR_INVALID_ARG
+    r = x[0, :, :1].reshape(1, H, 128).contiguous()
+    with pytest.raises(gear.GearError) as ei:
+        gear.append_rows(kc, vc, [0], r, r)
+    assert ei.value.status == gear.gear.GEAR_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
