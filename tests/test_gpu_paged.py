@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import oracle
-from tests.gpu_helpers import TORCH_DT, compare_unit, oracle_params, seeded_kv, to_dev
+import workloads as wl
+from tests.gpu_helpers import TORCH_DT, compare_unit, oracle_params, pmap, seeded_kv, spread_units, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -354,3 +355,68 @@ def test_paged_pair_must_agree():
     assert ei.value.status == gear.gear.GEAR_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert gear.device_status() == 0
+
+
+def test_full_paged_decode_b16_ragged():
+    """The batch-16 decode workload in the launch configuration the benchmark's
+    paged line times (pages of 256 tokens): rows' prompts spread over 4096..8192
+    tokens, a full 20-token buffer, decode; then one more token per row, which
+    flushes every row's buffer as its block 1 (mid-page), and decode again. 16
+    sampled (row, head) units against the oracle built from the same tokens."""
+    w = wl.WORKLOADS["decode_b16_ctx8192"]
+    p = gear.make_params(bits=w.bits, group_size=w.group, outlier_frac=w.s, rank=w.rank, power_iters=w.iters,
+                         buffer_len=w.buffer_len, buffer_rank=w.buffer_rank, seed=w.seed)
+    op = oracle_params(p)
+    dt = TORCH_DT[w.dtype]
+    P = 256
+    ppr = -(-(w.n + 2 * w.buffer_len) // P)
+    kc = gear.PagedCache(p, w.B, w.H, P, w.B * ppr, ppr, 4, dt)
+    vc = gear.PagedCache(p, w.B, w.H, P, w.B * ppr, ppr, 4, dt)
+    lengths = [w.n // 2 + (w.n // 2) * b // (w.B - 1) // 32 * 32 for b in range(w.B)]
+    xs = {which: wl.kv_tensor_torch(w, which, 0, "cuda") for which in ("k", "v")}
+    by_len = {}
+    for b, n in enumerate(lengths):
+        by_len.setdefault(n, []).append(b)
+    for n, rs in by_len.items():
+        kc.encode_rows(rs, xs["k"][rs][:, :, :n].contiguous())
+        vc.encode_rows(rs, xs["v"][rs][:, :, :n].contiguous())
+    del xs
+    rows = list(range(w.B))
+    for i in range(w.buffer_fill):
+        gear.append_rows(kc, vc, rows, wl.rows_torch(w, wl.S_KBUF, 0, i, w.H, "cuda"),
+                         wl.rows_torch(w, wl.S_VBUF, 0, i, w.H, "cuda"))
+    q = wl.rows_torch(w, wl.S_Q, 0, 0, w.Hq, "cuda")
+    out = gear.decode_attn(kc, vc, q, TAU, out_dtype=torch.float32).cpu().numpy()
+    gear.append_rows(kc, vc, rows, wl.rows_torch(w, wl.S_KNEW, 0, 0, w.H, "cuda"),
+                     wl.rows_torch(w, wl.S_VNEW, 0, 0, w.H, "cuda"))
+    out2 = gear.decode_attn(kc, vc, q, TAU, out_dtype=torch.float32).cpu().numpy()
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    _, nblk, nbuf, _ = kc.counters()
+    assert (nblk == 2).all() and (nbuf == 1).all()
+    qn = wl.rows_np(w, wl.S_Q, 0, 0, w.Hq)
+    units = [(u // w.H, u % w.H) for u in spread_units(w.B * w.H, 16)]
+
+    def refs(bh):
+        b, h = bh
+        n = lengths[b]
+        ok, ov = oracle.Cache(op, 1, 1, 128), oracle.Cache(op, 1, 1, 128)
+        ok.encode(wl.kv_unit_np(w, "k", 0, b, h)[:n][None, None])
+        ov.encode(wl.kv_unit_np(w, "v", 0, b, h)[:n][None, None])
+        for i in range(w.buffer_fill):
+            ok.append(wl.rows_np(w, wl.S_KBUF, 0, i, w.H)[b:b + 1, h:h + 1])
+            ov.append(wl.rows_np(w, wl.S_VBUF, 0, i, w.H)[b:b + 1, h:h + 1])
+        r1 = oracle.decode_attn(ok, ov, qn[b:b + 1, h:h + 1], TAU)[0, 0]
+        v1 = np.abs(ov.dense()).max()
+        ok.append(wl.rows_np(w, wl.S_KNEW, 0, 0, w.H)[b:b + 1, h:h + 1])
+        ov.append(wl.rows_np(w, wl.S_VNEW, 0, 0, w.H)[b:b + 1, h:h + 1])
+        r2 = oracle.decode_attn(ok, ov, qn[b:b + 1, h:h + 1], TAU)[0, 0]
+        return r1, v1, r2, np.abs(ov.dense()).max(), ok.blocks[0][0], ok.blocks[1][0]
+
+    for (b, h), (r1, v1, r2, v2, blk0, blk1) in zip(units, pmap(refs, units)):
+        n = lengths[b]
+        assert np.abs(out[b, h] - r1).max() <= 1e-3 * v1, (b, h)
+        assert np.abs(out2[b, h] - r2).max() <= 1e-3 * v2, (b, h)
+        compare_unit(paged_block(kc, b, h, 0, n, 0, w.rank), blk0, p, f"paged K block 0 ({b},{h})")
+        compare_unit(paged_block(kc, b, h, n, n + w.buffer_len, 1, w.buffer_rank), blk1, p,
+                     f"paged K block 1 ({b},{h})")
