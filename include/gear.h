@@ -323,8 +323,11 @@ gear_status gear_decode_dense(const gear_cache* c, float* out_f32, void* stream)
  * end at their own lengths), so a ragged batch costs what its tokens cost.
  * gear_encode, gear_encode_batch, gear_append_buffer,
  * gear_cache_reset and gear_decode_dense return UNSUPPORTED on a paged cache.
- * Limits: channel_groups = 0; P a multiple of 32 (a decode tile of 32 tokens
- * never spans two pages). */
+ * Per-channel key groups (channel_groups = 1, a K cache of 16-bit values): the
+ * meta slots stay per unit, [U][S][d][2] fp32 with S = ceil(P * pages_per_row /
+ * g) + 1, numbered per row as in a contiguous cache with that row's block-0
+ * length; the V cache beside it has channel_groups = 0.
+ * Limits: P a multiple of 32 (a decode tile of 32 tokens never spans two pages). */
 
 /* Host int32 entries a paged cache keeps in caller memory:
  * 3*B counters (block-0 length, blocks, buffer fill per row), the table
@@ -341,9 +344,9 @@ size_t gear_paged_cache_bytes(const gear_params* p, int32_t B, int32_t H, int32_
 /* Lays a paged cache out in [dev, dev + bytes) (256-byte aligned) with host
  * state in host[0 .. host_ints). Every row starts empty and every page free.
  * Enqueues two memsets on `stream` (counters to 0, table to -1).
- * Errors: INVALID_ARG (null, misaligned, bad geometry, P % 32 != 0,
- * channel_groups), UNSUPPORTED (d != 128, pool rows >= 2^31), CAPACITY (bytes
- * or host_ints too small), CUDA. */
+ * Errors: INVALID_ARG (null, misaligned, bad geometry, P % 32 != 0),
+ * UNSUPPORTED (d != 128, pool rows >= 2^31, per-channel key groups of fp32),
+ * CAPACITY (bytes or host_ints too small), CUDA. */
 gear_status gear_paged_cache_init(gear_cache* c, const gear_params* p, int32_t B, int32_t H, int32_t d,
                                   int32_t page_tokens, int32_t num_pages, int32_t pages_per_row, int32_t nblk_max,
                                   gear_dtype dtype, void* dev, size_t bytes, int32_t* host, size_t host_ints,

@@ -215,8 +215,7 @@ static bool paged_ok(const gear_cache* c) {
 static bool paged_pair(const gear_cache* k, const gear_cache* v) {
   if (!(k->B == v->B && k->H == v->H && k->dtype == v->dtype && k->page_tokens == v->page_tokens &&
         k->num_pages == v->num_pages && k->pages_per_row == v->pages_per_row && k->nblk_max == v->nblk_max &&
-        k->n_comp == v->n_comp && k->n_buf == v->n_buf && k->n_blk == v->n_blk &&
-        memcmp(&k->p, &v->p, sizeof(gear_params)) == 0))
+        k->n_comp == v->n_comp && k->n_buf == v->n_buf && k->n_blk == v->n_blk && kv_params_match(k, v)))
     return false;
   const int B = k->B;
   if (memcmp(k->host, v->host, (size_t)3 * B * sizeof(int32_t)) != 0) return false;
@@ -289,7 +288,7 @@ static cudaError_t enqueue_set(const gear_cache* c, const std::vector<std::pair<
 // batch rows i) into the pages of c: row rows[i] at token offset t0[i], block
 // blk[i]. The device table must already map every page these tokens reach.
 static cudaError_t scatter_rows(const gear_cache* c, const gear_cache* stg, const int32_t* rows, const int* t0,
-                                const int* blk, int nrows, int n, cudaStream_t st) {
+                                const int* blk, const int* s0, int nrows, int n, cudaStream_t st) {
   ScatterArgs s;
   memset(&s, 0, sizeof(s));
   s.s_codes = reinterpret_cast<const uint8_t*>(stg->codes);
@@ -313,7 +312,11 @@ static cudaError_t scatter_rows(const gear_cache* c, const gear_cache* stg, cons
   s.nmax_s = stg->n_max;
   s.n = n;
   s.wb = c->W * 4;
-  s.mb = meta_row_bytes(c->G, c->p.meta_f16);
+  s.ch = c->p.channel_groups;
+  s.mb = s.ch ? 0 : meta_row_bytes(c->G, c->p.meta_f16);
+  s.g = c->p.group_size;
+  s.ch_slots_s = s.ch ? channel_group_slots(stg->n_max, s.g) : 0;
+  s.ch_slots_d = s.ch ? channel_group_slots(c->n_max, s.g) : 0;
   s.kb = c->k;
   s.ob = c->k * esize(c->dtype);
   s.lb = c->r_max * (c->dtype == GEAR_F32 ? 4 : 2);
@@ -327,6 +330,7 @@ static cudaError_t scatter_rows(const gear_cache* c, const gear_cache* stg, cons
       r.row[j] = rows[i0 + j];
       r.t0[j] = t0[i0 + j];
       r.blk[j] = blk[i0 + j];
+      r.s0[j] = s0[i0 + j];
     }
     cudaError_t e = paged_scatter_launch(s, r, st);
     if (e != cudaSuccess) return e;
@@ -348,10 +352,13 @@ static size_t rows_encode_ws(const gear_cache* c, int nt, int nrows, int n) {
 
 // workspace of a flush of nf rows (K and V): two staging caches, the gathered
 // buffers and the batched encode
+// (V's parameters are K's with channel_groups = 0: kv_params_match)
 static size_t flush_ws_bytes(const gear_cache* k, int nf) {
   const int n_b = k->p.buffer_len;
   const size_t in = align256((size_t)nf * k->H * n_b * k->d * esize(k->dtype));
-  return 2 * staging_bytes(k, nf, n_b) + 2 * in + rows_encode_ws(k, 2, nf, n_b);
+  gear_cache v = *k;
+  v.p.channel_groups = 0;
+  return staging_bytes(k, nf, n_b) + staging_bytes(&v, nf, n_b) + 2 * in + rows_encode_ws(k, 2, nf, n_b);
 }
 
 // ------------------------------------------------------------------ append
@@ -681,8 +688,8 @@ static gear_status paged_geometry(const gear_params* p, int32_t B, int32_t H, in
   if (B <= 0 || H <= 0 || P <= 0 || P % 32 != 0 || num_pages <= 0 || ppr <= 0 || nblk_max <= 0 ||
       dtype < GEAR_F16 || dtype > GEAR_F32)
     return GEAR_ERR_INVALID_ARG;
-  if (p->channel_groups) return GEAR_ERR_INVALID_ARG;   // per-channel key groups stay contiguous
   if (p->meta_f16 && dtype != GEAR_F16) return GEAR_ERR_UNSUPPORTED;
+  if (p->channel_groups && dtype == GEAR_F32) return GEAR_ERR_UNSUPPORTED;   // per-channel keys of 16-bit caches
   if ((int64_t)num_pages * H * P >= ((int64_t)1 << 31) || (int64_t)P * ppr >= ((int64_t)1 << 31) ||
       (int64_t)B * ppr >= ((int64_t)1 << 31))
     return GEAR_ERR_UNSUPPORTED;
@@ -691,7 +698,9 @@ static gear_status paged_geometry(const gear_params* p, int32_t B, int32_t H, in
 
 static size_t paged_total(const gear_params* p, int B, int H, int d, int P, int num_pages, int ppr, int nblk_max,
                           int dt, Layout* L, size_t* table_off, size_t* rows_off) {
-  *L = layout_rows(p, (size_t)B * H, (size_t)num_pages * H * P, 0, d, nblk_max, dt);
+  // per-channel key groups: the meta slots stay per unit, for a row's whole capacity
+  const size_t slots = p->channel_groups ? (size_t)channel_group_slots(P * ppr, p->group_size) : 0;
+  *L = layout_rows(p, (size_t)B * H, (size_t)num_pages * H * P, slots, d, nblk_max, dt);
   *table_off = L->total;
   *rows_off = *table_off + align256((size_t)B * ppr * 4);
   return *rows_off + align256((size_t)3 * B * 4);
@@ -783,7 +792,7 @@ gear_status gear_encode_rows(gear_cache* c, const int32_t* rows, int32_t nrows, 
   // pages for tokens [0, n) of every row, then the move into them
   std::vector<std::pair<int, int>> tab;
   std::vector<RowState> rs;
-  std::vector<int> t0((size_t)nrows, 0), blk((size_t)nrows, 0);
+  std::vector<int> t0((size_t)nrows, 0), blk((size_t)nrows, 0), s0((size_t)nrows, 0);
   for (int i = 0; i < nrows; ++i) {
     const int b = rows[i];
     for (int lp = 0; lp < per; ++lp) {
@@ -798,7 +807,7 @@ gear_status gear_encode_rows(gear_cache* c, const int32_t* rows, int32_t nrows, 
   }
   update_maxima(c);
   cudaError_t e = enqueue_set(c, tab, rs, st);
-  if (e == cudaSuccess) e = scatter_rows(c, &stg, rows, t0.data(), blk.data(), nrows, n, st);
+  if (e == cudaSuccess) e = scatter_rows(c, &stg, rows, t0.data(), blk.data(), s0.data(), nrows, n, st);
   return cuda_status(e);
 }
 
@@ -820,7 +829,7 @@ gear_status gear_append_rows(gear_cache* k, gear_cache* v, const int32_t* rows, 
   HostView hk = host_view(k), hv = host_view(v);
   const int n_b = k->p.buffer_len, P = k->page_tokens;
   std::vector<int32_t> fr;   // rows whose buffer is flushed first
-  std::vector<int> ft0, fblk;
+  std::vector<int> ft0, fblk, fs0;   // token offset, block and (per-channel keys) first slot of each
   int need = 0;
   for (int i = 0; i < nrows; ++i) {
     const int b = rows[i];
@@ -832,6 +841,9 @@ gear_status gear_append_rows(gear_cache* k, gear_cache* v, const int32_t* rows, 
       fr.push_back(b);
       ft0.push_back(nc);
       fblk.push_back(hk.nblk[b]);
+      // block j >= 1 starts at group slot ceil(b0 / g) + (j - 1) * n_b / g
+      const int g = k->p.group_size;
+      fs0.push_back(ceil_div(hk.b0[b], g) + (hk.nblk[b] - 1) * (n_b / g));
     }
   }
   if (need > *hk.top) return GEAR_ERR_CAPACITY;
@@ -842,16 +854,16 @@ gear_status gear_append_rows(gear_cache* k, gear_cache* v, const int32_t* rows, 
   cudaError_t e = cudaSuccess;
   if (nf > 0) {
     // gather the full buffers, encode them as one block per row (both tensors
-    // in one pass), then move the blocks into fresh pages
+    // in one pass when their parameters agree), then move the blocks into fresh pages
     uint8_t* w = reinterpret_cast<uint8_t*>(workspace);
-    const size_t sb = staging_bytes(k, nf, n_b);
+    const size_t sbk = staging_bytes(k, nf, n_b), sbv = staging_bytes(v, nf, n_b);
     const size_t ub = (size_t)k->H * n_b * k->d * esize(k->dtype);   // buffer bytes per row
     const size_t in = align256((size_t)nf * ub);
     gear_cache stk, stv;
-    gear_status s = gear_cache_init(&stk, &k->p, nf, k->H, k->d, n_b, 1, (gear_dtype)k->dtype, w, sb);
-    if (s == GEAR_OK) s = gear_cache_init(&stv, &v->p, nf, v->H, v->d, n_b, 1, (gear_dtype)v->dtype, w + sb, sb);
+    gear_status s = gear_cache_init(&stk, &k->p, nf, k->H, k->d, n_b, 1, (gear_dtype)k->dtype, w, sbk);
+    if (s == GEAR_OK) s = gear_cache_init(&stv, &v->p, nf, v->H, v->d, n_b, 1, (gear_dtype)v->dtype, w + sbk, sbv);
     if (s != GEAR_OK) return s;
-    uint8_t* ink = w + 2 * sb;
+    uint8_t* ink = w + sbk + sbv;
     uint8_t* inv = ink + in;
     for (int i0 = 0; i0 < nf && e == cudaSuccess; i0 += kRowsMax) {
       PagedRows r;
@@ -864,7 +876,13 @@ gear_status gear_append_rows(gear_cache* k, gear_cache* v, const int32_t* rows, 
     if (e != cudaSuccess) return GEAR_ERR_CUDA;
     gear_cache* cs[2] = {&stk, &stv};
     const void* ins[2] = {ink, inv};
-    s = encode_block(cs, ins, 2, n_b, 0, 0, k->p.buffer_rank, inv + in, ws_bytes - (2 * sb + 2 * in), st);
+    const size_t used = sbk + sbv + 2 * in;
+    if (memcmp(&k->p, &v->p, sizeof(gear_params)) == 0) {
+      s = encode_block(cs, ins, 2, n_b, 0, 0, k->p.buffer_rank, inv + in, ws_bytes - used, st);
+    } else {   // per-channel key groups on K only: one encode per tensor
+      s = encode_block(&cs[0], &ins[0], 1, n_b, 0, 0, k->p.buffer_rank, inv + in, ws_bytes - used, st);
+      if (s == GEAR_OK) s = encode_block(&cs[1], &ins[1], 1, n_b, 0, 0, v->p.buffer_rank, inv + in, ws_bytes - used, st);
+    }
     if (s != GEAR_OK) return s;
     std::vector<std::pair<int, int>> tab;
     for (int i = 0; i < nf; ++i) {
@@ -883,8 +901,8 @@ gear_status gear_append_rows(gear_cache* k, gear_cache* v, const int32_t* rows, 
     const std::vector<RowState> none;
     e = enqueue_set(k, tab, none, st);
     if (e == cudaSuccess) e = enqueue_set(v, tab, none, st);
-    if (e == cudaSuccess) e = scatter_rows(k, &stk, fr.data(), ft0.data(), fblk.data(), nf, n_b, st);
-    if (e == cudaSuccess) e = scatter_rows(v, &stv, fr.data(), ft0.data(), fblk.data(), nf, n_b, st);
+    if (e == cudaSuccess) e = scatter_rows(k, &stk, fr.data(), ft0.data(), fblk.data(), fs0.data(), nf, n_b, st);
+    if (e == cudaSuccess) e = scatter_rows(v, &stv, fr.data(), ft0.data(), fblk.data(), fs0.data(), nf, n_b, st);
     if (e != cudaSuccess) return GEAR_ERR_CUDA;
   }
   // the new tokens, and every listed row's counters

@@ -78,6 +78,12 @@ __global__ void __launch_bounds__(128) paged_scatter(const ScatterArgs s, const 
     float* d = s.d_rfac + (du * s.nblk_max + r.blk[i]) * s.rf_floats;
     const float* src = s.s_rfac + su * s.rf_floats;   // the staging copy holds one block
     for (int e = threadIdx.x; e < s.rf_floats; e += blockDim.x) d[e] = src[e];
+    if (s.ch) {   // the block's token-group slots (1 KB each)
+      const int nf = (s.n + s.g - 1) / s.g * 256;
+      const float* ms = reinterpret_cast<const float*>(s.s_meta) + su * s.ch_slots_s * 256;
+      float* md = reinterpret_cast<float*>(s.d_meta) + (du * s.ch_slots_d + r.s0[i]) * 256;
+      for (int e = threadIdx.x; e < nf; e += blockDim.x) md[e] = ms[e];
+    }
   }
 }
 

@@ -25,11 +25,12 @@ struct PagedSet {
 };
 
 // Rows of one gather / scatter launch: entry i is batch row row[i], whose
-// tokens land at row offset t0[i] as block blk[i]; its units are unit
-// (i0 + i) * H + h of the contiguous staging copy.
+// tokens land at row offset t0[i] as block blk[i] (per-channel key groups: its
+// first token group at slot s0[i]); its units are unit (i0 + i) * H + h of the
+// contiguous staging copy.
 struct PagedRows {
   int32_t n, i0;
-  int32_t row[kRowsMax], t0[kRowsMax], blk[kRowsMax];
+  int32_t row[kRowsMax], t0[kRowsMax], blk[kRowsMax], s0[kRowsMax];
 };
 
 // One tensor's staging copy (contiguous, one block) and its paged destination.
@@ -50,8 +51,11 @@ struct ScatterArgs {
   int32_t H, P, ppr, num_pages, nblk_max;
   int32_t nmax_s;                 // token rows per unit of the staging copy
   int32_t n;                      // tokens per unit
-  int32_t wb, mb, kb, ob, lb;     // bytes per token: codes, meta, oidx, oval, lfac
+  int32_t wb, mb, kb, ob, lb;     // bytes per token: codes, meta, oidx, oval, lfac (mb = 0 with ch)
   int32_t rf_floats;              // Rf floats per unit and block (128 * r_pad)
+  // per-channel key groups: meta is [unit][slot][128][2] floats; the block's
+  // ceil(n / g) slots move from slot 0 of the staging unit to slot s0 of the row's unit
+  int32_t ch, g, ch_slots_s, ch_slots_d;
 };
 
 // Per-row append: token i of k_new/v_new goes to buffer slot slot[i] of row

@@ -296,8 +296,11 @@ class PagedCache:
         rp = (c.r_max + 3) // 4 * 4
         return {
             "codes": self._view(c.codes, R * c.W, torch.int32).view(NP, H, P, c.W),
-            "meta": self._view(c.meta, R * c.G * 2, torch.float16 if c.p.meta_f16 else torch.float32)
-            .view(NP, H, P, c.G, 2),
+            # per-channel key groups: per unit [U][ceil(P * pages_per_row / g) + 1 slots][d][2]
+            "meta": (self._view(c.meta, U * (-(-(P * c.pages_per_row) // c.p.group_size) + 1) * c.d * 2,
+                                torch.float32).view(c.B, H, -1, c.d, 2) if c.p.channel_groups else
+                     self._view(c.meta, R * c.G * 2, torch.float16 if c.p.meta_f16 else torch.float32)
+                     .view(NP, H, P, c.G, 2)),
             "oidx": self._view(c.oidx, R * k, torch.uint8).view(NP, H, P, k),
             "oval": self._view(c.oval, R * k, self.dtype).view(NP, H, P, k),
             "lfac": self._view(c.lfac, R * c.r_max, ld).view(NP, H, P, c.r_max),

@@ -214,8 +214,14 @@ def test_paged_layout_and_host_errors(gear):
     assert L.gear_paged_host_ints(B, ppr, NP) == 3 * B + B * ppr + NP + 1
     for bad in [(B, H, 48, NP, ppr), (B, H, 0, NP, ppr), (0, H, P, NP, ppr), (B, H, P, 0, ppr), (B, H, P, NP, 0)]:
         assert L.gear_paged_cache_bytes(ctypes.byref(p), bad[0], bad[1], 128, bad[2], bad[3], bad[4], nblk, 0) == 0
+    # per-channel key groups: the pool loses its per-token meta rows, and each unit
+    # keeps ceil(P * ppr / g) + 1 slots of 1 KB; fp32 caches are refused
     pk = gear.make_params(channel_groups=True, buffer_len=64)
-    assert L.gear_paged_cache_bytes(ctypes.byref(pk), B, H, 128, P, NP, ppr, nblk, 0) == 0
+    nk = L.gear_paged_cache_bytes(ctypes.byref(pk), B, H, 128, P, NP, ppr, nblk, 0)
+    slots = -(-(P * ppr) // 64) + 1
+    buf_more = B * H * (64 - 20) * 128 * 2   # the larger buffer (64 tokens, not 20)
+    assert abs(nk - (nb - 16 * NP * H * P + B * H * slots * 1024 + buf_more)) <= 4 * 256
+    assert L.gear_paged_cache_bytes(ctypes.byref(pk), B, H, 128, P, NP, ppr, nblk, 2) == 0
     nh = L.gear_paged_host_ints(B, ppr, NP)
     host = np.full(nh, 7, dtype=np.int32)
     hp = ctypes.c_void_p(host.ctypes.data)

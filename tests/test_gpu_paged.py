@@ -44,15 +44,22 @@ def paged_block(cache, b: int, h: int, t0: int, t1: int, blk: int, rank: int) ->
     while (2 << e) <= n:
         e += 1
     e //= 2
+    # host-side bounds first: a bad index fails here, not in a device-side check
+    assert pg.max() < A["codes"].shape[0] and h < A["codes"].shape[1] and off.max() < A["codes"].shape[2]
+    assert blk < A["rfac"].shape[2] and b < A["rfac"].shape[0]
     pg_t = torch.from_numpy(pg.astype(np.int64)).cuda()
     off_t = torch.from_numpy(off.astype(np.int64)).cuda()
 
     def take(name):
         return A[name][pg_t, h, off_t].cpu()
 
+    if cache.c.p.channel_groups:
+        meta = None   # per-unit token-group slots, not per-token rows: see paged_ch_block
+    else:
+        meta = take("meta").float().numpy() if A["meta"].dtype == torch.float16 else take("meta").numpy()
     return {
         "codes": take("codes").numpy(),
-        "meta": take("meta").float().numpy() if A["meta"].dtype == torch.float16 else take("meta").numpy(),
+        "meta": meta,
         "oidx": take("oidx").numpy(),
         "oval": take("oval").float().numpy(),
         "L": take("lfac")[:, :rank].float().numpy().astype(np.float64) * 2.0 ** -e,
@@ -61,16 +68,17 @@ def paged_block(cache, b: int, h: int, t0: int, t1: int, blk: int, rank: int) ->
 
 
 class RowOracle:
-    """One oracle K and V cache (batch 1) per row of the paged batch."""
+    """One oracle K and V cache (batch 1) per row of the paged batch (opv: the
+    V parameters when they differ from K's)."""
 
-    def __init__(self, op, B, H):
-        self.op, self.H = op, H
+    def __init__(self, op, B, H, opv=None):
+        self.op, self.opv, self.H = op, opv or op, H
         self.k = [None] * B
         self.v = [None] * B
 
     def encode(self, b, xk, xv):
         self.k[b] = oracle.Cache(self.op, 1, self.H, 128)
-        self.v[b] = oracle.Cache(self.op, 1, self.H, 128)
+        self.v[b] = oracle.Cache(self.opv, 1, self.H, 128)
         self.k[b].encode(xk[None])
         self.v[b].encode(xv[None])
 
@@ -420,3 +428,124 @@ def test_full_paged_decode_b16_ragged():
         compare_unit(paged_block(kc, b, h, 0, n, 0, w.rank), blk0, p, f"paged K block 0 ({b},{h})")
         compare_unit(paged_block(kc, b, h, n, n + w.buffer_len, 1, w.buffer_rank), blk1, p,
                      f"paged K block 1 ({b},{h})")
+
+
+def paged_ch_block(cache, b, h, t0, t1, blk, rank, slot0):
+    """Like paged_block, for a K cache with per-channel key groups: the block's
+    token-group slots from slot0 (per unit) instead of per-token meta rows."""
+    g = paged_block(cache, b, h, t0, t1, blk, rank)
+    gs = cache.c.p.group_size
+    ng = (t1 - t0 + gs - 1) // gs
+    m = cache.arrays()["meta"][b, h, slot0:slot0 + ng].cpu().numpy()
+    g["scale"], g["zero"] = m[..., 0], m[..., 1]
+    return g
+
+
+@pytest.mark.parametrize("dtype,bits,g,s", [("f16", 4, 32, 0.02), ("bf16", 2, 64, 0.05)])
+def test_paged_kivi_keys_match_oracle(dtype, bits, g, s):
+    """Per-channel key groups (the KIVI-combined quantizer) on the paged K cache,
+    per-token groups on V: ragged prompts (block 0 ending in a short group),
+    ragged appends and flushes of whole groups at different steps per row."""
+    from tests.test_gpu_kivi import compare_ch
+    B, H, Hq, n_b, P = 3, 2, 4, 2 * g, 64
+    pk = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=4, buffer_len=n_b, buffer_rank=2,
+                          power_iters=3, seed=31, channel_groups=True)
+    pv = gear.make_params(bits=bits, group_size=g, outlier_frac=s, rank=4, buffer_len=n_b, buffer_rank=2,
+                          power_iters=3, seed=31)
+    kc = gear.PagedCache(pk, B, H, P, 40, 8, 6, TORCH_DT[dtype])
+    vc = gear.PagedCache(pv, B, H, P, 40, 8, 6, TORCH_DT[dtype])
+    ro = RowOracle(oracle_params(pk), B, H, oracle_params(pv))
+    for rows, n in (([0, 1], 100), ([2], 45)):
+        xk = seeded_kv(40 + n, 1, (len(rows), H, n, 128), dtype, channel_scale=True)
+        xv = seeded_kv(40 + n, 2, (len(rows), H, n, 128), dtype)
+        kc.encode_rows(rows, to_dev(xk, dtype))
+        vc.encode_rows(rows, to_dev(xv, dtype))
+        for i, b in enumerate(rows):
+            ro.encode(b, xk[i], xv[i])
+    for step in range(2 * n_b + 10):
+        rows = [0] + ([1] if step % 2 == 0 else []) + ([2] if step >= 5 else [])
+        rk = seeded_kv(600 + step, 3, (len(rows), H, 128), dtype)
+        rv = seeded_kv(600 + step, 4, (len(rows), H, 128), dtype)
+        gear.append_rows(kc, vc, rows, to_dev(rk, dtype), to_dev(rv, dtype))
+        for i, b in enumerate(rows):
+            ro.append(b, rk[i], rv[i])
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    _, nblk, nbuf, _ = kc.counters()
+    assert nblk[0] >= 3 and len(set(nblk.tolist())) > 1
+    for b in range(B):
+        ok, ov = ro.k[b], ro.v[b]
+        assert nblk[b] == len(ok.blocks) and nbuf[b] == len(ok.buffer)
+        t0, slot = 0, 0
+        for bi, (kb, vb) in enumerate(zip(ok.blocks, ov.blocks)):
+            n = kb[0].codes.shape[0]
+            rank = 4 if bi == 0 else 2
+            for h in range(H):
+                compare_ch(paged_ch_block(kc, b, h, t0, t0 + n, bi, rank, slot), kb[h], bi,
+                           f"K row {b} block {bi} head {h}")
+                compare_unit(paged_block(vc, b, h, t0, t0 + n, bi, rank), vb[h], pv, f"V row {b} block {bi}")
+            t0 += n
+            slot += (n + g - 1) // g
+    q = seeded_kv(77, 5, (B, Hq, 128), dtype)
+    od, vmax = ro.attn(q)
+    out = gear.decode_attn(kc, vc, to_dev(q, dtype), TAU, out_dtype=torch.float32).cpu().numpy()
+    err = np.abs(out - od).max()
+    assert err <= _tol_out(dtype) * vmax, f"attention error {err:.3e} vs {_tol_out(dtype) * vmax:.3e}"
+
+
+def _poison(cache, names=("codes", "meta", "oidx", "oval", "lfac", "rfac", "buf")):
+    """Every byte of the cache's data arrays set to 0xFF (NaN for floats), so that
+    a read of anything the library did not write shows in the result."""
+    A = cache.arrays()
+    for n in names:
+        A[n].view(torch.uint8).fill_(255)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_decode_reads_only_written_memory(paged):
+    """Caches whose memory starts as NaN bytes: 4..8 outliers per token with rank
+    <= 4 (Rf rows of four floats) take the decoder's eight-rank outlier path,
+    which must not read past a row's own Rf floats (past channel 127's row lies
+    the next block, never written). Attention against the oracle."""
+    B, H, Hq, dtype, n0, n_b = 2, 2, 4, "f16", 150, 16
+    p = gear.make_params(bits=4, group_size=64, outlier_frac=0.05, rank=4, buffer_len=n_b, buffer_rank=2,
+                         power_iters=3, seed=3)
+    op = oracle_params(p)
+    xk = seeded_kv(51, 1, (B, H, n0, 128), dtype, channel_scale=True)
+    xv = seeded_kv(51, 2, (B, H, n0, 128), dtype)
+    if paged:
+        kc = gear.PagedCache(p, B, H, 64, 16, 6, 6, TORCH_DT[dtype])
+        vc = gear.PagedCache(p, B, H, 64, 16, 6, 6, TORCH_DT[dtype])
+    else:
+        kc = gear.Cache(p, B, H, 320, 6, TORCH_DT[dtype])
+        vc = gear.Cache(p, B, H, 320, 6, TORCH_DT[dtype])
+    _poison(kc)
+    _poison(vc)
+    if paged:
+        kc.encode_rows([0, 1], to_dev(xk, dtype))
+        vc.encode_rows([0, 1], to_dev(xv, dtype))
+    else:
+        kc.encode(to_dev(xk, dtype))
+        vc.encode(to_dev(xv, dtype))
+    ok, ov = oracle.Cache(op, B, H, 128), oracle.Cache(op, B, H, 128)
+    ok.encode(xk)
+    ov.encode(xv)
+    for i in range(n_b + 3):   # one flush
+        rk = seeded_kv(900 + i, 3, (B, H, 128), dtype)
+        rv = seeded_kv(900 + i, 4, (B, H, 128), dtype)
+        if paged:
+            gear.append_rows(kc, vc, [0, 1], to_dev(rk, dtype), to_dev(rv, dtype))
+        else:
+            gear.append_buffer(kc, vc, to_dev(rk, dtype), to_dev(rv, dtype))
+        ok.append(rk)
+        ov.append(rv)
+    # the case that matters is there: channel 127 is an outlier in the last block
+    assert any((u.oidx == 127).any() for u in ok.blocks[-1] + ov.blocks[-1])
+    q = seeded_kv(71, 5, (B, Hq, 128), dtype)
+    out = gear.decode_attn(kc, vc, to_dev(q, dtype), TAU, out_dtype=torch.float32).cpu().numpy()
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    od = oracle.decode_attn(ok, ov, q, TAU)
+    vmax = np.abs(ov.dense()).max()
+    assert np.isfinite(out).all()
+    assert np.abs(out - od).max() <= 1e-3 * vmax
