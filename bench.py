@@ -502,8 +502,8 @@ class Runner:
 TRAFFIC_BYTES = {
     # encode stage: E1 539130624 + 175976960, E2 26284032, E3 723844864 + 30014208 bytes at batch 4
     ("twobit_b64_ctx8192", "encode"): 16 * (539130624 + 175976960 + 26284032 + 723844864 + 30014208),
-    # decode_warp 213735424 + 463360 bytes at batch 4
-    ("twobit_b64_ctx8192", "decode"): 16 * (213735424 + 463360),
+    # decode_warp 213763840 + 762624 bytes at batch 4
+    ("twobit_b64_ctx8192", "decode"): 16 * (213763840 + 762624),
 }
 
 

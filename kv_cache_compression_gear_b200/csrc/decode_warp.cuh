@@ -208,11 +208,12 @@ __device__ __forceinline__ void outlier_fixes(const uint8_t* rest, int oval_off,
     // the zero point at the outlier's channel: per channel (ZC) or of its group
     zr[i] = on ? (ZC ? zc[cix[i]] : meta_at<MF>(mrow, cix[i] >> lg, mx).y) : 0.0f;
     // only the row's own rp floats: past them lies the next channel's row, or
-    // for channel 127 the next block's, which may never have been written
+    // for channel 127 the next block's, which may never have been written (the
+    // first float4 is always inside the row, rp >= 4)
 #pragma unroll
     for (int q = 0; q < NR / 4; ++q)
-      rv[i][q] = (on && 4 * q < rp) ? __ldg(reinterpret_cast<const float4*>(rf + cix[i] * rp) + q)
-                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      rv[i][q] = (on && (q == 0 || 4 * q < rp)) ? __ldg(reinterpret_cast<const float4*>(rf + cix[i] * rp) + q)
+                                               : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
 #pragma unroll
   for (int i = 0; i < NS; ++i) {
