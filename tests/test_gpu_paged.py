@@ -549,3 +549,59 @@ def test_decode_reads_only_written_memory(paged):
     vmax = np.abs(ov.dense()).max()
     assert np.isfinite(out).all()
     assert np.abs(out - od).max() <= 1e-3 * vmax
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_workspace_reads_only_what_it_wrote(paged):
+    """The shared workspace filled with 0xFF bytes (NaN) before every encode,
+    flush and decode: the encoder's Gram partials and Z slabs, the staging
+    copies of the paged layout and the decode partials must all be written
+    before they are read."""
+    B, H, Hq, dtype, n0, n_b = 2, 2, 4, "bf16", 300, 20
+    p = gear.make_params(bits=2, group_size=32, outlier_frac=0.05, rank=8, buffer_len=n_b, buffer_rank=2,
+                         power_iters=3, seed=13)
+    op = oracle_params(p)
+    xk = seeded_kv(61, 1, (B, H, n0, 128), dtype, channel_scale=True)
+    xv = seeded_kv(61, 2, (B, H, n0, 128), dtype)
+
+    def poison():
+        torch.cuda.synchronize()
+        ws = gear.gear._ws
+        ws.get(64 << 20, "cuda")
+        ws.buf.fill_(255)
+
+    if paged:
+        kc = gear.PagedCache(p, B, H, 128, 16, 4, 4, TORCH_DT[dtype])
+        vc = gear.PagedCache(p, B, H, 128, 16, 4, 4, TORCH_DT[dtype])
+        poison()
+        kc.encode_rows([0, 1], to_dev(xk, dtype))
+        poison()
+        vc.encode_rows([0, 1], to_dev(xv, dtype))
+    else:
+        kc = gear.Cache(p, B, H, 400, 4, TORCH_DT[dtype])
+        vc = gear.Cache(p, B, H, 400, 4, TORCH_DT[dtype])
+        poison()
+        kc.encode(to_dev(xk, dtype))
+        poison()
+        vc.encode(to_dev(xv, dtype))
+    ok, ov = oracle.Cache(op, B, H, 128), oracle.Cache(op, B, H, 128)
+    ok.encode(xk)
+    ov.encode(xv)
+    for i in range(n_b + 2):   # one flush
+        rk = seeded_kv(700 + i, 3, (B, H, 128), dtype)
+        rv = seeded_kv(700 + i, 4, (B, H, 128), dtype)
+        poison()
+        if paged:
+            gear.append_rows(kc, vc, [0, 1], to_dev(rk, dtype), to_dev(rv, dtype))
+        else:
+            gear.append_buffer(kc, vc, to_dev(rk, dtype), to_dev(rv, dtype))
+        ok.append(rk)
+        ov.append(rv)
+    q = seeded_kv(81, 5, (B, Hq, 128), dtype)
+    poison()
+    out = gear.decode_attn(kc, vc, to_dev(q, dtype), TAU, out_dtype=torch.float32).cpu().numpy()
+    torch.cuda.synchronize()
+    assert gear.device_status() == 0
+    od = oracle.decode_attn(ok, ov, q, TAU)
+    assert np.isfinite(out).all()
+    assert np.abs(out - od).max() <= _tol_out(dtype) * np.abs(ov.dense()).max()
